@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the CLSA decode step (indexer scan + exact top-k + gather +
+L-layer sparse GQA attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode128k]
+                    [--impl {clsa,reference}] [--no-graph] [--no-cpu-baseline]
+
+One JSON line on rank 0.  A step is one decode token per sequence through the
+whole path; the default workload is the 128K-context decode (batch 1, n=131072,
+d_idx=128, k=2048, L=24, 32 query / 8 KV heads, d=128, bf16, 1% planted tokens).
+Device time is measured with CUDA events around each step on the stream the
+library launches on, with L2 flushed (a 512 MiB write) before every step
+outside the timed events.  With N > 1 every rank runs its own sequences (weak
+scaling, no collective on the data path); the step time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on the host cores on a
+bounded sample of the same workload and prints the same line with
+``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CLSA decode step µs & tokens/s at 128K ctx; achieved HBM GB/s vs roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode128k")
+    ap.add_argument("--impl", default="clsa", choices=["clsa", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-steps", type=int, default=2)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ algorithmic bytes
+
+def step_bytes(w, lens):
+    """K_idx scan + gathered K/V rows once + Q/O + q_idx (per step, all sequences)."""
+    e = w.elem_bytes
+    kidx = sum(int(n) for n in lens) * w.d_idx * e
+    kv = sum(min(w.k, int(n)) for n in lens) * w.Hkv * w.d * e * 2
+    qo = 2 * w.L * w.B * w.Hq * w.d * e
+    qi = w.B * w.d_idx * e
+    return {"kidx": kidx, "kv": kv, "qo": qo, "qidx": qi, "total": kidx + kv + qo + qi}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def profile_traffic(kernel: str, workload: str, src_files):
+    """dram bytes per launch recorded in profiles/<kernel>__<workload>.txt, or None
+    when the kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    for f in src_files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if vals.get("source_sha256") != h.hexdigest():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 5 + i and s[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def time_oracle(inp, w, steps: int):
+    """Run the oracle's decode step on the host cores; returns (s per step, threads, note)."""
+    from oracle import clsa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    # the cache is upcast once (state a real decoder keeps resident); each sample step
+    # re-scores, re-selects and attends
+    qf = inp.f32("q_idx").astype(np.float64)
+    kf = inp.f32("k_idx").astype(np.float64)
+    Kf = inp.f32("K").astype(np.float64)
+    Vf = inp.f32("V").astype(np.float64)
+    Qf = inp.f32("Q").astype(np.float64)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.decode_step(qf, kf, Kf, Vf, Qf, inp.seq_lens, w.k)
+    dt = (time.perf_counter() - t0) / steps
+    return dt, threads, f"{steps} full decode step(s) of {w.name} (B={w.B}, n={w.n_max})"
+
+
+# ------------------------------------------------------------------ main paths
+
+def dist_init(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def run_reference(args):
+    rank, world, _ = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return
+    from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    steps = max(1, min(args.steps, args.cpu_sample_steps))
+    for _ in range(min(args.warmup, 1)):
+        time_oracle(inp, w, 1)
+    dt, threads, note = time_oracle(inp, w, steps)
+    v = w.B / dt
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
+            "warmup": min(args.warmup, 1), "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "n": w.n_max, "k": w.k, "L": w.L, "Hq": w.Hq,
+                       "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_clsa(args):
+    import torch
+    rank, world, local = dist_init(args.gpus)
+    torch.cuda.set_device(local)
+    from long_context_sparse_clsa_b200 import clsa
+    from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs, replace
+    clsa.load_library()
+    w = WORKLOADS[args.workload]
+    if world > 1:  # each rank its own sequences: a different seed per rank
+        w = replace(w, seed=w.seed + rank)
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    L, B, Hq, d, k = w.L, w.B, w.Hq, w.d, w.k
+    out = {"O": torch.empty_like(dv["Q"]), "idx": torch.empty(B, k, dtype=torch.int32, device=dev),
+           "count": torch.empty(B, dtype=torch.int32, device=dev)}
+    a = clsa.decode_args(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], k, out["O"],
+                         out["idx"], out["count"])
+    ws = clsa.Workspace(clsa.decode_workspace_size(a))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        clsa.decode_step_args(a, ws)
+
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = clsa.last_launch_count()
+    graph = None
+    if not args.no_graph:
+        try:
+            s2 = torch.cuda.Stream()
+            s2.wait_stream(stream)
+            with torch.cuda.stream(s2):
+                step()
+            stream.wait_stream(s2)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+        except Exception as ex:  # graph capture unsupported: time eager launches
+            graph = None
+            print(f"# graph capture failed, timing eager launches: {ex}", file=sys.stderr)
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        run_step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local) as clk:
+        for e0, e1 in evs:
+            flush.fill_(1)
+            e0.record(stream)
+            run_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    st = ws.status()
+    if st[0] != "CLSA_OK":
+        raise RuntimeError(f"device error during timing: {st}")
+    times = [e0.elapsed_time(e1) for e0, e1 in evs]  # ms
+    total_ms = sum(times)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * B / (ms_per_step / 1e3)
+
+    # ---- per-kernel timing (each C-ABI stage alone, same stream, L2 flushed) -----------
+    sc = torch.empty(B, w.n_max, dtype=torch.float32, device=dev)
+    tws = clsa.Workspace(max(256, clsa.load_library().clsa_topk_workspace_size(B, w.n_max, k)))
+    KS = torch.empty(B, k, w.Hkv, d, dtype=dv["K"].dtype, device=dev)
+    VS = torch.empty_like(KS)
+
+    def timed(fn, reps=50):
+        fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / reps * 1e3  # us
+
+    by = step_bytes(w, inp.seq_lens)
+    kern = {}
+    kern["index_scores"] = timed(lambda: clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"], sc))
+    kern["topk"] = timed(lambda: clsa.topk(sc, dv["seq_lens"], k, tws, out["idx"], out["count"]))
+    kern["gather_kv"] = timed(lambda: clsa.gather_kv(dv["K"], dv["V"], out["idx"], out["count"], tws, KS, VS))
+    attn_ws = clsa.Workspace(clsa.load_library().clsa_sparse_attn_workspace_size(B, k, L, Hq, w.Hkv, d))
+    kern["sparse_attn_all_layers"] = timed(
+        lambda: clsa.sparse_attn(dv["Q"], KS, VS, out["count"], ws=attn_ws, O=out["O"], want_lse=False))
+    Q1 = dv["Q"][:1].contiguous()
+    O1 = torch.empty_like(Q1)
+    kern["sparse_attn_one_layer"] = timed(
+        lambda: clsa.sparse_attn(Q1, KS, VS, out["count"], ws=attn_ws, O=O1, want_lse=False))
+
+    hbm, bf16, peak_kind = peaks()
+    # dominant kernel of the step among the fused-path stages
+    stage_bytes = {"index_scores": by["kidx"] + by["qidx"] + 4 * sum(int(n) for n in inp.seq_lens)}
+    dom = "index_scores"
+    dom_us = kern[dom]
+    achieved = stage_bytes[dom] / (dom_us * 1e-6) / 1e9
+    traffic = profile_traffic("index_scores", w.name, ["long_context_sparse_clsa_b200/csrc/index_scores.cu",
+                                                       "long_context_sparse_clsa_b200/csrc/common.cuh"])
+    step_gbs = by["total"] / (ms_per_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers --------------------------
+    q_idx_h = dv["q_idx"].cpu().pin_memory()
+    Q_h = dv["Q"].cpu().pin_memory()
+    O_h = torch.empty(out["O"].shape, dtype=out["O"].dtype).pin_memory()
+    idx_h = torch.empty(B, k, dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty(B, dtype=torch.int32).pin_memory()
+    h2d = q_idx_h.numel() * q_idx_h.element_size() + Q_h.numel() * Q_h.element_size()
+    d2h = O_h.numel() * O_h.element_size() + idx_h.numel() * 4 + cnt_h.numel() * 4
+    e2e_steps = min(args.steps, 50)
+    tot = 0.0
+    for i in range(e2e_steps + 3):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dv["q_idx"].copy_(q_idx_h, non_blocking=True)
+        dv["Q"].copy_(Q_h, non_blocking=True)
+        clsa.decode_step_args(a, ws)
+        O_h.copy_(out["O"], non_blocking=True)
+        idx_h.copy_(out["idx"], non_blocking=True)
+        cnt_h.copy_(out["count"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            tot += e0.elapsed_time(e1)
+    e2e_ms = tot / e2e_steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, threads, note = time_oracle(inp, w, args.cpu_sample_steps)
+        cpu = {"value": w.B / dt, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1), 1% planted index keys)",
+        "config": {"workload": w.name, "B": w.B, "n": w.n_max, "d_idx": w.d_idx, "k": w.k, "L": w.L,
+                   "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step (512 MiB write, outside the timed events)",
+                   "launch": "cuda graph" if graph is not None else "eager"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": stage_bytes[dom], "us_per_launch": dom_us},
+        "step_roofline": {"algorithmic_bytes": by["total"], "achieved_gbs": step_gbs, "peak": hbm,
+                          "frac": step_gbs / hbm, "peak_kind": peak_kind},
+        "kernels_us": kern,
+        "e2e": {"value": world * B / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_clsa(args)
+
+
+if __name__ == "__main__":
+    main()

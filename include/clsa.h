@@ -1,0 +1,189 @@
+/*
+ * clsa.h -- C ABI of libclsa.so, the B200 (sm_100a) implementation of the
+ * Cross-Layer Sparse Attention (CLSA) shared-routing hot path.
+ *
+ * The method ("You Only Index Once: Cross-Layer Sparse Attention with Shared
+ * Routing"; picx.dev summary, Methodology > Architecture Overview):
+ *   routing equation    I = Q_idx K_idx^T ,  S_t = TopK(I_t, k)     -- once per token
+ *   per-layer equation  O_t^(l) = Attn(Q_t^(l), K_{S_t}, V_{S_t})    -- every layer l
+ * with Attn(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V (zhichai.net post "CLSA
+ * Explained", Background: Attention and Its Limits), K/V one shared (YOCO) cache,
+ * and the selected rows gathered by the shared index ("Selector", zhichai.net
+ * post, CLSA: Sharing the Index Across Layers).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.    Every tensor pointer is a DEVICE pointer (cudaMalloc'd or
+ *              equivalent) unless stated otherwise, 16-byte aligned, dense,
+ *              row-major in the layout given.  The caller owns every buffer;
+ *              the library never allocates device memory and keeps no state
+ *              between calls other than what lives in the caller's workspace.
+ * Streams.     `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *              stream).  Every call is asynchronous on that stream.
+ * dtype.       CLSA_F32 or CLSA_BF16 for every floating input of one call;
+ *              outputs O are written in the same dtype (bf16 rounded to nearest
+ *              even from fp32); scores and lse are always fp32.  All scoring,
+ *              softmax and accumulation are fp32.
+ * Shapes.      d, d_idx in {64, 128}; Hq % Hkv == 0; 1 <= k <= 4096;
+ *              B >= 1; 0 <= seq_lens[b] <= n_max (seq_lens is device int32).
+ *              Other shapes return CLSA_ERR_UNSUPPORTED before any launch.
+ * scale.       Attention scale; a value <= 0 selects 1/sqrt(d).
+ * TopK order.  Largest score first; equal scores go to the lower token index;
+ *              -0.0 equals +0.0.  The selected indices of a row are written in
+ *              ascending token order, k_eff = min(k, len) of them, and the rest
+ *              of the row is -1.  count[b] = k_eff.  Scores must not be NaN.
+ * GQA.         Query head h reads KV head h / (Hq / Hkv).
+ * Workspace.   `ws` is a caller-owned device buffer of at least the size the
+ *              matching *_workspace_size function returns.  It must be zeroed
+ *              once before first use (clsa_workspace_init) and again after any
+ *              call reported CLSA_ERR_TIMEOUT; the kernels leave it clean after
+ *              a successful call.  One workspace must not be used by two calls
+ *              that can run at the same time.
+ * Errors.      Argument errors return before anything is launched.  Errors the
+ *              kernels detect (an out-of-range index, a wait that ran out)
+ *              are recorded in the workspace and read with
+ *              clsa_read_device_status.  A failed launch returns CLSA_ERR_CUDA.
+ *              No kernel traps or asserts.
+ */
+#ifndef CLSA_H_
+#define CLSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CLSA_API __attribute__((visibility("default")))
+#else
+#define CLSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum clsa_status {
+  CLSA_OK = 0,
+  CLSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer     */
+  CLSA_ERR_UNSUPPORTED = 2,  /* shape outside the supported set               */
+  CLSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required     */
+  CLSA_ERR_CUDA = 4,         /* a CUDA launch or copy failed                   */
+  CLSA_ERR_TIMEOUT = 5,      /* an inter-CTA wait ran out (device-detected)    */
+  CLSA_ERR_BAD_INDEX = 6     /* a gather index outside [0, n_max) (device)     */
+} clsa_status;
+
+typedef enum clsa_dtype { CLSA_F32 = 0, CLSA_BF16 = 1 } clsa_dtype;
+
+/* ------------------------------------------------------------------------ */
+/* Routing equation, scores: I[b, j] = q_idx[b] . k_idx[b, j]                */
+/* ------------------------------------------------------------------------ */
+/* q_idx [B][d_idx], k_idx [B][n_max][d_idx] (dtype dt); scores [B][n_max]
+ * fp32 out: entries j < seq_lens[b] hold the dot product (fp32 accumulation of
+ * exact products), entries j >= seq_lens[b] are -inf.  No scale or activation
+ * (the indexer is a single head with a bare product).  Needs no workspace. */
+CLSA_API clsa_status clsa_index_scores(const void* q_idx, const void* k_idx, const int32_t* seq_lens,
+                              int B, int n_max, int d_idx, clsa_dtype dt, float* scores,
+                              void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Routing equation, selection: S_b = TopK(I_b, k)  (exact radix select)     */
+/* ------------------------------------------------------------------------ */
+/* scores [B][n_max] fp32 (only j < seq_lens[b] are read); idx [B][k] int32 and
+ * count [B] int32 out, ordered as in "TopK order" above.  The result is exact:
+ * bit-identical to a stable sort of the same fp32 scores. */
+CLSA_API size_t clsa_topk_workspace_size(int B, int n_max, int k);
+CLSA_API clsa_status clsa_topk(const float* scores, const int32_t* seq_lens, int B, int n_max, int k,
+                      int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Selector: gather the selected K/V rows once into a compact buffer          */
+/* ------------------------------------------------------------------------ */
+/* K, V [B][n_max][Hkv][d]; idx [B][k], count [B] as written by clsa_topk.
+ * K_S, V_S [B][k][Hkv][d] out: row i < count[b] is the cache row idx[b][i];
+ * rows i >= count[b] are left untouched.  An index outside [0, n_max) is not
+ * read: its row is zero-filled and CLSA_ERR_BAD_INDEX is recorded in ws. */
+CLSA_API size_t clsa_gather_kv_workspace_size(void);
+CLSA_API clsa_status clsa_gather_kv(const void* K, const void* V, const int32_t* idx, const int32_t* count,
+                           int B, int n_max, int k, int Hkv, int d, clsa_dtype dt,
+                           void* K_S, void* V_S, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Per-layer equation: O^(l) = softmax(Q^(l) K_S^T * scale) V_S               */
+/* ------------------------------------------------------------------------ */
+/* Q [L][B][Hq][d]: the queries of L >= 1 layers that share one selection (L = 1
+ * is the per-layer call a model makes layer by layer).  K_S, V_S [B][k][Hkv][d]
+ * compact rows, count [B] valid rows per sequence.  O [L][B][Hq][d] out;
+ * lse [L][B][Hq] fp32 out (natural-log sum of exp of the scaled scores), may
+ * be NULL.  A sequence with count 0 gets O = 0 and lse = -inf.
+ * Split-k flash decoding with an online softmax; fp32 accumulation. */
+CLSA_API size_t clsa_sparse_attn_workspace_size(int B, int k, int L, int Hq, int Hkv, int d);
+CLSA_API clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void* V_S, const int32_t* count,
+                             int B, int k, int L, int Hq, int Hkv, int d, float scale,
+                             clsa_dtype dt, void* O, float* lse, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* One decode step: score once, select once, gather once, attend in L layers */
+/* ------------------------------------------------------------------------ */
+typedef struct clsa_decode_args {
+  clsa_dtype dtype;
+  int B, n_max, d_idx, k, L, Hq, Hkv, d;
+  float scale;               /* <= 0: 1/sqrt(d)                                   */
+  const void* q_idx;         /* [B][d_idx]                                        */
+  const void* k_idx;         /* [B][n_max][d_idx]                                 */
+  const void* K;             /* [B][n_max][Hkv][d]  shared by every layer         */
+  const void* V;             /* [B][n_max][Hkv][d]                                */
+  const void* Q;             /* [L][B][Hq][d]       one query per layer           */
+  const int32_t* seq_lens;   /* [B]                                               */
+  void* O;                   /* out [L][B][Hq][d]                                 */
+  int32_t* idx;              /* out [B][k]  the shared S, ascending, -1 padded    */
+  int32_t* count;            /* out [B]                                           */
+  float* scores;             /* out [B][n_max] or NULL (kept in the workspace)    */
+  float* lse;                /* out [L][B][Hq] or NULL                            */
+  void* K_S;                 /* out [B][k][Hkv][d] compact gathered rows, or NULL */
+  void* V_S;                 /* out, NULL exactly when K_S is NULL                */
+} clsa_decode_args;
+/* With K_S/V_S NULL the attention kernel reads each selected cache row once
+ * straight from K/V for all L layers (the gather is fused); with them set,
+ * the rows are first compacted there and attention reads the compact copy. */
+CLSA_API size_t clsa_decode_workspace_size(const clsa_decode_args* a);
+CLSA_API clsa_status clsa_decode_step(const clsa_decode_args* a, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Prefill chunk: T new rows at cache positions n-T .. n-1, causal            */
+/* ------------------------------------------------------------------------ */
+typedef struct clsa_prefill_args {
+  clsa_dtype dtype;          /* CLSA_BF16 (the scores GEMM runs on tcgen05)       */
+  int n, T, d_idx, k, L, Hq, Hkv, d;
+  float scale;
+  const void* q_idx;         /* [T][d_idx]  index queries of the new rows         */
+  const void* k_idx;         /* [n][d_idx]  index keys of the whole cache         */
+  const void* K;             /* [n][Hkv][d]                                       */
+  const void* V;             /* [n][Hkv][d]                                       */
+  const void* Q;             /* [L][T][Hq][d]                                     */
+  void* O;                   /* out [L][T][Hq][d]                                 */
+  int32_t* idx;              /* out [T][k]: row i selects among tokens j <= n-T+i */
+  int32_t* count;            /* out [T]: min(k, n-T+i+1)                          */
+  float* lse;                /* out [L][T][Hq] or NULL                            */
+} clsa_prefill_args;
+CLSA_API size_t clsa_prefill_workspace_size(const clsa_prefill_args* a);
+CLSA_API clsa_status clsa_prefill_chunk(const clsa_prefill_args* a, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Helpers                                                                    */
+/* ------------------------------------------------------------------------ */
+/* Zero `bytes` of workspace on `stream` (asynchronous). */
+CLSA_API clsa_status clsa_workspace_init(void* ws, size_t bytes, void* stream);
+/* Synchronise `stream`, return the first device-detected error recorded in
+ * `ws` (CLSA_OK if none) and clear it.  `detail`, if not NULL, receives a
+ * kernel-specific code (the offending index, or the wait site). */
+CLSA_API clsa_status clsa_read_device_status(void* ws, void* stream, int64_t* detail);
+CLSA_API const char* clsa_status_string(clsa_status s);
+/* Library version as major*10000 + minor*100 + patch. */
+CLSA_API int clsa_version(void);
+/* Number of kernel launches the last call made on this host thread. */
+CLSA_API int clsa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CLSA_H_ */

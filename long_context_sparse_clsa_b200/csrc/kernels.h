@@ -1,0 +1,66 @@
+// Internal launchers used by the C ABI layer (api.cu).  Host code only.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/clsa.h"
+
+namespace clsa {
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int max_smem_optin = 0;
+};
+const DeviceInfo& device_info();
+
+// per-host-thread count of kernel launches in the current API call
+void launches_reset();
+void launches_add(int n);
+int launches_get();
+
+// ----- indexer scan (routing equation, scores) ------------------------------
+cudaError_t launch_index_scores(const void* q_idx, const void* k_idx, const int32_t* seq_lens, int B,
+                                int n_max, int d_idx, clsa_dtype dt, float* scores, cudaStream_t s);
+
+// ----- exact radix top-k -----------------------------------------------------
+size_t topk_ws_bytes(int B, int n_max, int k);
+// causal_base >= 0: row b has length causal_base + b + 1 and seq_lens is ignored
+cudaError_t launch_topk(const float* scores, const int32_t* seq_lens, int B, int n_max, int k,
+                        int32_t* idx, int32_t* count, void* ws_header, void* topk_ws, cudaStream_t s,
+                        int causal_base = -1);
+
+// ----- selector gather --------------------------------------------------------
+cudaError_t launch_gather_kv(const void* K, const void* V, const int32_t* idx, const int32_t* count, int B,
+                             int n_max, int k, int Hkv, int d, clsa_dtype dt, void* K_S, void* V_S,
+                             void* ws_header, cudaStream_t s);
+
+// ----- sparse attention (split-k flash decoding) ----------------------------
+struct AttnShape {
+  int B, k, L, Hq, Hkv, d;
+  clsa_dtype dt;
+  // gather mode: rows come from the full cache through idx
+  bool gather;
+  int n_max;
+  // cache rows per sequence in gather mode (n_max; 0 = one cache shared by every b)
+  long long kv_bstride;
+};
+struct AttnPlan {
+  int Lg;       // layers per CTA row-group
+  int nlg;      // layer groups
+  int rows;     // Lg * G rows per CTA
+  int nsplit;   // token splits per (b, kv head, layer group)
+  int chunk;    // tokens per split (multiple of 64)
+};
+AttnPlan plan_attention(const AttnShape& sh);
+size_t attn_ws_bytes(const AttnShape& sh);
+cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
+                               const int32_t* idx, const int32_t* count, float scale, void* O, float* lse,
+                               void* ws_header, void* attn_ws, cudaStream_t s);
+
+// ----- prefill ------------------------------------------------------------------
+size_t prefill_ws_bytes(const clsa_prefill_args* a);
+clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_body, cudaStream_t s);
+
+}  // namespace clsa

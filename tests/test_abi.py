@@ -1,0 +1,103 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol include/clsa.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_sparse_clsa_b200 import clsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "clsa.h")
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"CLSA_API\s+[\w\s\*]+?\b(clsa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_sparse_clsa_b200.build import build
+    build()
+    return clsa.load_library()
+
+
+def test_header_declares_the_six_calls():
+    syms = header_symbols()
+    for name in ("clsa_index_scores", "clsa_topk", "clsa_gather_kv", "clsa_sparse_attn",
+                 "clsa_decode_step", "clsa_prefill_chunk"):
+        assert name in syms
+
+
+def test_library_exports_every_header_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+    assert sorted(clsa.EXPORTS) == header_symbols()
+
+
+def test_status_strings_and_version(lib):
+    for code, name in clsa.STATUS.items():
+        assert lib.clsa_status_string(code).decode() == name
+    assert lib.clsa_version() >= 100
+
+
+NULL = None
+
+
+def test_index_scores_rejects_bad_args(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.clsa_index_scores(NULL, p, p, 1, 16, 64, 0, p, NULL) == 1
+    assert lib.clsa_index_scores(p, p, p, 0, 16, 64, 0, p, NULL) == 1
+    assert lib.clsa_index_scores(p, p, p, 1, 16, 96, 0, p, NULL) == 2       # d_idx not 64/128
+    assert lib.clsa_index_scores(ctypes.c_void_p(18), p, p, 1, 16, 64, 0, p, NULL) == 1  # misaligned
+
+
+def test_topk_rejects_bad_args(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.clsa_topk(p, p, 1, 16, 0, p, p, p, 1 << 20, NULL) == 1      # k = 0
+    assert lib.clsa_topk(p, p, 1, 16, 5000, p, p, p, 1 << 20, NULL) == 2   # k > 4096
+    assert lib.clsa_topk(p, p, 1, 16, 4, p, p, NULL, 0, NULL) == 3         # no workspace
+
+
+def test_sparse_attn_rejects_bad_shapes(lib):
+    p = ctypes.c_void_p(16)
+    ws = ctypes.c_void_p(256)
+    args = dict(B=1, k=8, L=1, Hq=8, Hkv=3, d=64)
+    assert lib.clsa_sparse_attn(p, p, p, p, 1, 8, 1, 8, 3, 64, 0.0, 1, p, NULL, ws, 1 << 30, NULL) == 2
+    assert lib.clsa_sparse_attn(p, p, p, p, 1, 8, 1, 8, 2, 80, 0.0, 1, p, NULL, ws, 1 << 30, NULL) == 2
+    assert lib.clsa_sparse_attn(p, p, p, p, 1, 8, 1, 8, 2, 64, 0.0, 7, p, NULL, ws, 1 << 30, NULL) == 1
+    # fp32 path holds at most 32 query heads per KV head
+    assert lib.clsa_sparse_attn(p, p, p, p, 1, 8, 1, 64, 1, 64, 0.0, 0, p, NULL, ws, 1 << 30, NULL) == 2
+    del args
+
+
+def test_decode_step_rejects_bad_args(lib):
+    p = ctypes.c_void_p(16)
+    a = clsa.DecodeArgs(1, 1, 1024, 128, 64, 2, 8, 2, 128, 0.0, p, p, p, p, p, p, p, p, p, NULL, NULL,
+                        p, NULL)  # K_S without V_S
+    assert lib.clsa_decode_step(ctypes.byref(a), p, 1 << 30, NULL) == 1
+    a.V_S = p
+    a.d = 96
+    assert lib.clsa_decode_step(ctypes.byref(a), p, 1 << 30, NULL) == 2
+    assert lib.clsa_decode_workspace_size(ctypes.byref(a)) == 0
+    assert lib.clsa_decode_step(None, p, 0, NULL) == 1
+
+
+def test_prefill_rejects_bad_args(lib):
+    p = ctypes.c_void_p(16)
+    a = clsa.PrefillArgs(1, 100, 200, 128, 16, 1, 8, 2, 64, 0.0, p, p, p, p, p, p, p, p, NULL)  # T > n
+    assert lib.clsa_prefill_chunk(ctypes.byref(a), p, 1 << 30, NULL) == 1
+    a.T, a.dtype = 50, 0
+    assert lib.clsa_prefill_chunk(ctypes.byref(a), p, 1 << 30, NULL) == 2   # fp32 prefill unsupported
+
+
+def test_oracle_is_not_imported_by_the_product():
+    pkg = os.path.join(ROOT, "long_context_sparse_clsa_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle|clsa_oracle|#include.*oracle",
+                                     text, re.M), f

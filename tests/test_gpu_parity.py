@@ -1,0 +1,262 @@
+"""GPU parity: every C-ABI call against the CPU oracle on the same seeded inputs.
+
+Acceptance (stated for this path): TopK index sets bit-exact on identical fp32
+scores; end-to-end sets may differ only at near-ties (|I_j - I_(k)| <= 1e-4 max|I|);
+attention max-abs <= 2e-2 for bf16 inputs (fp32 accumulation) and <= 1e-4 in fp32
+mode, against the oracle evaluated on the GPU's own selection.  Scores are held
+to the fp32 forward-error bound of a d-term dot product.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import clsa_oracle as O
+from long_context_sparse_clsa_b200 import clsa
+from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs, scaled
+from parity_util import check_near_tie_sets, max_abs, score_tol, tensor_f64
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+LSE_TOL = {"f32": 1e-4, "bf16": 2e-3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_sparse_clsa_b200.build import build
+    build()
+    clsa.load_library()
+
+
+CASES = {
+    "tiny": WORKLOADS["tiny"],
+    "d32k_small": scaled("decode32k", n_max=8192 + 77, k=512, L=3),
+    "ragged_small": scaled("ragged16", B=5, n_max=6000, lens=(0, 6000), k=700, L=2, seed=3),
+    "bf16_d64": scaled("decode32k", n_max=3000, d_idx=64, d=64, k=300, L=2, Hq=8, Hkv=2, plant=0.0),
+    "f32_d128": scaled("tiny", n_max=2500, d_idx=128, d=128, k=333, L=2, Hq=6, Hkv=3, seed=5),
+}
+
+
+def _inputs(name):
+    inp = make_inputs(CASES[name])
+    return inp, clsa.to_device(inp)
+
+
+# ----------------------------------------------------------------------- A1 scores
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_index_scores(name):
+    inp, dv = _inputs(name)
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    torch.cuda.synchronize()
+    got = tensor_f64(sc)
+    want = O.index_scores(inp.q_idx, inp.k_idx, inp.seq_lens)
+    tol = score_tol(inp.f32("q_idx"), inp.f32("k_idx"), inp.seq_lens)
+    for b, n in enumerate(inp.seq_lens):
+        assert np.all(np.abs(got[b, :n] - want[b, :n]) <= tol[b, :n])
+        assert np.isneginf(got[b, n:]).all()
+
+
+# ----------------------------------------------------------------------- A2 top-k
+
+def _topk_case(scores, lens, k):
+    s = torch.tensor(scores, dtype=torch.float32, device="cuda")
+    L = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    idx, cnt = clsa.topk(s, L, k)
+    torch.cuda.synchronize()
+    want_idx, want_cnt = O.topk_select(scores.astype(np.float64), lens, k)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), want_cnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+
+
+@pytest.mark.parametrize("B,n,k,kind", [
+    (1, 131072, 2048, "normal"), (1, 131072, 2048, "ties"), (1, 32768, 2048, "normal"),
+    (3, 5000, 4096, "normal"), (16, 40000, 2048, "ragged"), (2, 777, 1, "ties"),
+    (1, 4096, 256, "allequal"), (1, 1000, 999, "signedzero"), (200, 3000, 100, "normal"),
+    (4, 100, 200, "normal"),
+])
+def test_topk_bit_exact(B, n, k, kind):
+    rng = np.random.default_rng(B * 7 + n + k)
+    if kind == "ties":
+        scores = rng.integers(-20, 20, size=(B, n)).astype(np.float32)
+    elif kind == "allequal":
+        scores = np.full((B, n), 1.5, dtype=np.float32)
+    elif kind == "signedzero":
+        scores = rng.choice(np.array([-0.0, 0.0, 1.0, -1.0], dtype=np.float32), size=(B, n))
+    else:
+        scores = (rng.standard_normal((B, n)) * 11).astype(np.float32)
+    lens = np.full(B, n, dtype=np.int32)
+    if kind == "ragged":
+        lens = rng.integers(0, n + 1, size=B).astype(np.int32)
+        lens[0] = 0
+        lens[1] = 1
+    _topk_case(scores, lens, k)
+
+
+def test_topk_on_gpu_scores_bit_exact():
+    inp, dv = _inputs("d32k_small")
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    torch.cuda.synchronize()
+    _topk_case(sc.cpu().numpy(), inp.seq_lens, CASES["d32k_small"].k)
+
+
+# ----------------------------------------------------------------------- A3 gather
+
+def test_gather_bit_exact_and_bad_index():
+    inp, dv = _inputs("ragged_small")
+    w = CASES["ragged_small"]
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    idx, cnt = clsa.topk(sc, dv["seq_lens"], w.k)
+    KS, VS = clsa.gather_kv(dv["K"], dv["V"], idx, cnt)
+    torch.cuda.synchronize()
+    i_np, c_np = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(w.B):
+        c = int(c_np[b])
+        sel = torch.tensor(i_np[b, :c], dtype=torch.long, device="cuda")
+        assert torch.equal(KS[b, :c], dv["K"][b].index_select(0, sel))
+        assert torch.equal(VS[b, :c], dv["V"][b].index_select(0, sel))
+    bad = idx.clone()
+    bad[0, 0] = w.n_max + 5
+    cnt1 = cnt.clone()
+    cnt1[0] = max(int(c_np[0]), 1)
+    ws = clsa.Workspace(256)
+    clsa.gather_kv(dv["K"], dv["V"], bad, cnt1, ws=ws)
+    status, detail = ws.status()
+    assert status == "CLSA_ERR_BAD_INDEX" and detail == 0
+    assert ws.status()[0] == "CLSA_OK"   # reading clears it
+
+
+# ----------------------------------------------------------------------- A4 attention
+
+@pytest.mark.parametrize("name,L", [("tiny", None), ("tiny", 1), ("d32k_small", None), ("d32k_small", 1),
+                                    ("ragged_small", None), ("bf16_d64", None), ("f32_d128", None)])
+def test_sparse_attn(name, L):
+    w = CASES[name]
+    inp, dv = _inputs(name)
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    idx, cnt = clsa.topk(sc, dv["seq_lens"], w.k)
+    KS, VS = clsa.gather_kv(dv["K"], dv["V"], idx, cnt)
+    Q = dv["Q"] if L is None else dv["Q"][:1].contiguous()
+    out, lse = clsa.sparse_attn(Q, KS, VS, cnt)
+    torch.cuda.synchronize()
+    i_np, c_np = idx.cpu().numpy(), cnt.cpu().numpy()
+    Qh = inp.Q if L is None else inp.Q[:1]
+    want, want_lse = O.sparse_attention(Qh, inp.K, inp.V, i_np, c_np)
+    assert max_abs(tensor_f64(out), want) <= TOL[w.dtype]
+    got_lse = tensor_f64(lse)
+    fin = np.isfinite(want_lse)
+    assert (np.isneginf(got_lse) == ~fin).all()
+    assert max_abs(got_lse[fin], want_lse[fin]) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse[fin]).max())
+
+
+# ----------------------------------------------------------------------- A5 decode step
+
+@pytest.mark.parametrize("name", list(CASES))
+@pytest.mark.parametrize("compact", [False, True])
+def test_decode_step(name, compact):
+    w = CASES[name]
+    inp, dv = _inputs(name)
+    r = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k,
+                         compact=compact, want_scores=True)
+    torch.cuda.synchronize()
+    assert r["ws"].status()[0] == "CLSA_OK"
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    ora_scores = O.index_scores(inp.q_idx, inp.k_idx, inp.seq_lens)
+    check_near_tie_sets(i_np, c_np, ora_scores, inp.seq_lens, w.k)
+    # the selection the GPU made is exactly TopK of the scores it computed
+    gi, gc = O.topk_select(tensor_f64(r["scores"]), inp.seq_lens, w.k)
+    np.testing.assert_array_equal(gi, i_np)
+    want, want_lse = O.sparse_attention(inp.Q, inp.K, inp.V, i_np, c_np)
+    assert max_abs(tensor_f64(r["O"]), want) <= TOL[w.dtype]
+    fin = np.isfinite(want_lse)
+    assert max_abs(tensor_f64(r["lse"])[fin], want_lse[fin]) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse[fin]).max())
+
+
+def test_decode_step_deterministic():
+    w = CASES["d32k_small"]
+    _, dv = _inputs("d32k_small")
+    a = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k)
+    b = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k, ws=a["ws"])
+    torch.cuda.synchronize()
+    assert torch.equal(a["O"], b["O"]) and torch.equal(a["idx"], b["idx"]) and torch.equal(a["lse"], b["lse"])
+
+
+@pytest.mark.parametrize("name", ["decode128k", "decode32k"])
+def test_decode_step_full_size(name):
+    """Full-size workloads in the launch configuration the benchmark times:
+    selection bit-exact against TopK of the GPU scores, near-tie rule against the
+    oracle's float64 scores, and attention against the oracle on sampled heads."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    r = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k,
+                         want_scores=True)
+    torch.cuda.synchronize()
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    gi, _ = O.topk_select(tensor_f64(r["scores"]), inp.seq_lens, w.k)
+    np.testing.assert_array_equal(gi, i_np)
+    ora_scores = O.index_scores(inp.q_idx, inp.k_idx, inp.seq_lens)
+    check_near_tie_sets(i_np, c_np, ora_scores, inp.seq_lens, w.k)
+    # planted salient tokens are all selected (1% of n < k)
+    assert set(inp.planted[0].tolist()) <= set(i_np[0, : c_np[0]].tolist())
+    rng = np.random.default_rng(0)
+    heads = sorted(set(rng.choice(w.Hq, 6, replace=False).tolist()) | {0, w.Hq - 1})
+    layers = sorted({0, w.L - 1, int(rng.integers(w.L))})
+    got = tensor_f64(r["O"])
+    for l in layers:
+        for h in heads:
+            want, _ = O.sparse_attention(inp.Q[l:l + 1, :, h:h + 1], inp.K[:, :, h // w.G: h // w.G + 1],
+                                         inp.V[:, :, h // w.G: h // w.G + 1], i_np, c_np)
+            assert max_abs(got[l, :, h], want[0, :, 0]) <= TOL[w.dtype]
+
+
+def test_ragged16_full_size_sampled():
+    w = WORKLOADS["ragged16"]
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    r = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k,
+                         want_scores=True)
+    torch.cuda.synchronize()
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    gi, _ = O.topk_select(tensor_f64(r["scores"]), inp.seq_lens, w.k)
+    np.testing.assert_array_equal(gi, i_np)
+    got = tensor_f64(r["O"])
+    for b in (0, 7, 15):
+        ora_scores = O.index_scores(inp.q_idx[b:b + 1], inp.k_idx[b:b + 1], inp.seq_lens[b:b + 1])
+        check_near_tie_sets(i_np[b:b + 1], c_np[b:b + 1], ora_scores, inp.seq_lens[b:b + 1], w.k)
+        for l, h in ((0, 0), (w.L - 1, w.Hq - 1), (11, 13)):
+            g = h // w.G
+            want, _ = O.sparse_attention(inp.Q[l:l + 1, b:b + 1, h:h + 1], inp.K[b:b + 1, :, g:g + 1],
+                                         inp.V[b:b + 1, :, g:g + 1], i_np[b:b + 1], c_np[b:b + 1])
+            assert max_abs(got[l, b, h], want[0, 0, 0]) <= TOL[w.dtype]
+
+
+# ----------------------------------------------------------------------- A6-A8 prefill
+
+def _prefill_check(w, rows):
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    r = clsa.prefill_chunk(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], w.k)
+    torch.cuda.synchronize()
+    assert r["ws"].status()[0] == "CLSA_OK"
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    n, T = w.n_max, w.T
+    assert c_np.tolist() == [min(w.k, n - T + i + 1) for i in range(T)]
+    ora_scores = O.prefill_scores(inp.q_idx, inp.k_idx, n, rows)
+    lens = [n - T + i + 1 for i in rows]
+    check_near_tie_sets(i_np[rows], c_np[rows], ora_scores, lens, w.k)
+    want, want_lse = O.prefill_attention(inp.Q, inp.K, inp.V, i_np[rows], c_np[rows], rows)
+    got = tensor_f64(r["O"])[:, rows]
+    assert max_abs(got, want) <= TOL[w.dtype]
+
+
+def test_prefill_small():
+    w = scaled("prefill4k", n_max=3000, T=300, k=256, L=2)
+    _prefill_check(w, list(range(300)))
+
+
+def test_prefill_full_size_sampled():
+    w = WORKLOADS["prefill4k"]
+    _prefill_check(w, [0, 1, 2047, 2048, 4095])
