@@ -9,7 +9,7 @@ One JSON line on rank 0.  A step is one decode token per sequence through the
 whole path; the default workload is the 128K-context decode (batch 1, n=131072,
 d_idx=128, k=2048, L=24, 32 query / 8 KV heads, d=128, bf16, 1% planted tokens).
 Device time is measured with CUDA events around each step on the stream the
-library launches on, with L2 flushed (a 512 MiB write) before every step
+library launches on, with L2 flushed (a 512 MiB write and read-back) before every step
 outside the timed events.  With N > 1 every rank runs its own sequences (weak
 scaling, no collective on the data path); the step time is the max over ranks.
 
@@ -41,7 +41,7 @@ UNIT = "tokens/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="decode128k")
     ap.add_argument("--impl", default="clsa", choices=["clsa", "reference"])
@@ -96,6 +96,7 @@ def profile_traffic(kernel: str, workload: str, src_files):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """nvidia-smi streaming its clocks every 100 ms while the timed region runs."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -103,40 +104,50 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.samples = []
-        self._stop = threading.Event()
+        self._p = None
         self._t = None
 
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                out = subprocess.run(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                                     timeout=5).stdout.strip()
-                if out:
-                    self.samples.append([x.strip() for x in out.split(",")])
-            except Exception:
-                pass
-            self._stop.wait(0.2)
+    def _read(self):
+        for line in self._p.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
 
     def __enter__(self):
-        self._t = threading.Thread(target=self._run, daemon=True)
-        self._t.start()
+        try:
+            self._p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                        "--format=csv,noheader,nounits", "-lms", "100"],
+                                       stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)
+        except Exception:
+            self._p = None
         return self
 
     def __exit__(self, *a):
-        self._stop.set()
-        if self._t:
-            self._t.join(timeout=10)
+        if self._p is not None:
+            time.sleep(0.15)
+            self._p.terminate()
+            try:
+                self._p.wait(timeout=5)
+            except Exception:
+                self._p.kill()
+            self._t.join(timeout=5)
 
     def summary(self):
-        if not self.samples:
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [v for v in (num(s[1]) for s in self.samples) if v is not None]
+        mx = [v for v in (num(s[2]) for s in self.samples) if v is not None]
+        if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if len(s) > 5 + i and s[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(self.samples)}
 
 
@@ -145,11 +156,6 @@ class ClockSampler:
 def time_oracle(inp, w, steps: int):
     """Run the oracle's decode step on the host cores; returns (s per step, threads, note)."""
     from oracle import clsa_oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
     # the cache is upcast once (state a real decoder keeps resident); each sample step
     # re-scores, re-selects and attends
     qf = inp.f32("q_idx").astype(np.float64)
@@ -161,6 +167,11 @@ def time_oracle(inp, w, steps: int):
     for _ in range(steps):
         O.decode_step(qf, kf, Kf, Vf, Qf, inp.seq_lens, w.k)
     dt = (time.perf_counter() - t0) / steps
+    try:  # threads of the BLAS pool the oracle's matrix products ran on
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
     return dt, threads, f"{steps} full decode step(s) of {w.name} (B={w.B}, n={w.n_max})"
 
 
@@ -221,6 +232,13 @@ def run_clsa(args):
                          out["idx"], out["count"])
     ws = clsa.Workspace(clsa.decode_workspace_size(a))
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_view = flush.view(torch.int32)
+
+    def flush_l2():
+        # write 512 MiB, then read 512 MiB back: every line the step may touch is evicted
+        # and the dirty lines of the write are written back before the timed events
+        flush.fill_(1)
+        flush_view.max()
 
     def step():
         clsa.decode_step_args(a, ws)
@@ -252,7 +270,7 @@ def run_clsa(args):
             step()
 
     for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
+        flush_l2()
         run_step()
     torch.cuda.synchronize()
 
@@ -266,7 +284,7 @@ def run_clsa(args):
     barrier()
     with ClockSampler(local) as clk:
         for e0, e1 in evs:
-            flush.fill_(1)
+            flush_l2()
             e0.record(stream)
             run_step()
             e1.record(stream)
@@ -296,7 +314,7 @@ def run_clsa(args):
         torch.cuda.synchronize()
         tot = 0.0
         for _ in range(reps):
-            flush.fill_(1)
+            flush_l2()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -339,7 +357,7 @@ def run_clsa(args):
     e2e_steps = min(args.steps, 50)
     tot = 0.0
     for i in range(e2e_steps + 3):
-        flush.fill_(1)
+        flush_l2()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         dv["q_idx"].copy_(q_idx_h, non_blocking=True)
@@ -377,7 +395,7 @@ def run_clsa(args):
         "data": "synthetic (seeded N(0,1), 1% planted index keys)",
         "config": {"workload": w.name, "B": w.B, "n": w.n_max, "d_idx": w.d_idx, "k": w.k, "L": w.L,
                    "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every step (512 MiB write, outside the timed events)",
+                   "l2": "flushed before every step (512 MiB write + read-back, outside the timed events)",
                    "launch": "cuda graph" if graph is not None else "eager"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
