@@ -94,6 +94,26 @@ CLSA_API size_t clsa_topk_workspace_size(int B, int n_max, int k);
 CLSA_API clsa_status clsa_topk(const float* scores, const int32_t* seq_lens, int B, int n_max, int k,
                       int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free TopK.  The paper has no counterpart for this entry point; it
+ * exists for callers that cannot call cudaMalloc: code that runs inside another
+ * runtime's memory pool and gets no allocator handle, or a path that must not
+ * risk the device synchronisation cudaMalloc/cudaFree can cause.  It computes
+ * exactly what clsa_topk computes (same kernel, same result) but takes no
+ * workspace: its scratch is a fixed 2 MiB array inside the library, held on
+ * every GPU that loads the library until the process exits.
+ *   - The first call on a device looks up that array's device address; make
+ *     that first call before any stream capture.
+ *   - Each call clears the part of the array it uses on `stream` before the
+ *     kernel runs.  Calls that overlap on the GPU (other streams, other host
+ *     threads) share the array and race: serialise them.
+ *   - Sizes whose scratch would exceed 2 MiB (many rows that each need several
+ *     CTAs, about B > 55 at n_max = 128K) return CLSA_ERR_UNSUPPORTED.
+ *   - Errors the kernel records on the device are not reported (there is no
+ *     caller workspace to hold them); argument errors are returned as usual.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+CLSA_API clsa_status clsa_topk_noalloc(const float* scores, const int32_t* seq_lens, int B, int n_max,
+                                       int k, int32_t* idx, int32_t* count, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Selector: gather the selected K/V rows once into a compact buffer          */
 /* ------------------------------------------------------------------------ */

@@ -23,7 +23,8 @@ STATUS = {0: "CLSA_OK", 1: "CLSA_ERR_INVALID_ARG", 2: "CLSA_ERR_UNSUPPORTED", 3:
 
 # every symbol include/clsa.h declares
 EXPORTS = [
-    "clsa_index_scores", "clsa_topk_workspace_size", "clsa_topk", "clsa_gather_kv_workspace_size",
+    "clsa_index_scores", "clsa_topk_workspace_size", "clsa_topk", "clsa_topk_noalloc",
+    "clsa_gather_kv_workspace_size",
     "clsa_gather_kv", "clsa_sparse_attn_workspace_size", "clsa_sparse_attn",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
     "clsa_prefill_chunk", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
@@ -73,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_index_scores": (S, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
         "clsa_topk_workspace_size": (_sz, [_i, _i, _i]),
         "clsa_topk": (S, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+        "clsa_topk_noalloc": (S, [_vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
         "clsa_gather_kv_workspace_size": (_sz, []),
         "clsa_gather_kv": (S, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
         "clsa_sparse_attn_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -172,6 +174,17 @@ def topk(scores, seq_lens, k, ws: Optional[Workspace] = None, idx=None, count=No
     count = count if count is not None else torch.empty(B, dtype=torch.int32, device=scores.device)
     _check(lib.clsa_topk(_p(scores), _p(seq_lens), B, n_max, k, _p(idx), _p(count), ws.ptr, ws.nbytes,
                          _stream()), "clsa_topk")
+    return idx, count
+
+
+def topk_noalloc(scores, seq_lens, k, idx=None, count=None):
+    """clsa_topk without a workspace (scratch inside the library; see clsa.h)."""
+    lib = load_library()
+    B, n_max = scores.shape
+    idx = idx if idx is not None else torch.empty(B, k, dtype=torch.int32, device=scores.device)
+    count = count if count is not None else torch.empty(B, dtype=torch.int32, device=scores.device)
+    _check(lib.clsa_topk_noalloc(_p(scores), _p(seq_lens), B, n_max, k, _p(idx), _p(count), _stream()),
+           "clsa_topk_noalloc")
     return idx, count
 
 
