@@ -2,6 +2,7 @@
 // The operations are defined in include/clsa.h; every step of the path runs in
 // the kernels of this directory.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -49,11 +50,23 @@ clsa_status check_attn(int B, int k, int L, int Hq, int Hkv, int d, clsa_dtype d
 }
 
 struct DecodeLayout {
+  bool fused = false;
   size_t scores = 0, topk = 0, attn = 0, total = 0;
 };
 
+// CLSA_DECODE_PLAN=unfused forces the four-kernel path (scan, top-k, attention, combine)
+bool fused_allowed() {
+  const char* v = std::getenv("CLSA_DECODE_PLAN");
+  return !(v && std::strcmp(v, "unfused") == 0);
+}
+
 DecodeLayout decode_layout(const clsa_decode_args* a) {
   DecodeLayout l;
+  if (fused_allowed() && fused_decode_supported(a)) {
+    l.fused = true;
+    l.total = kWsHeader + fused_decode_ws_bytes(a);
+    return l;
+  }
   size_t off = kWsHeader;
   if (!a->scores) {
     l.scores = off;
@@ -225,6 +238,7 @@ clsa_status clsa_decode_step(const clsa_decode_args* a, void* ws, size_t ws_byte
   if (!ws || ws_bytes < lay.total || !aligned16(ws)) return CLSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
+  if (lay.fused) return from_cuda(launch_decode_fused(a, resolve_scale(a->scale, a->d), w, w + kWsHeader, s));
   float* scores = a->scores ? a->scores : reinterpret_cast<float*>(w + lay.scores);
   cudaError_t e = launch_index_scores(a->q_idx, a->k_idx, a->seq_lens, a->B, a->n_max, a->d_idx, a->dtype,
                                       scores, s);

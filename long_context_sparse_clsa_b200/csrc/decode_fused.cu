@@ -1,0 +1,971 @@
+// Fused CLSA decode step: one persistent cooperative launch that scores, selects,
+// gathers and attends.
+//
+//   routing equation   I = q_idx . K_idx^T ,  S = TopK(I, k)      (once per token)
+//   per-layer equation O^(l) = softmax(Q^(l) K_S^T / sqrt(d)) V_S  (every layer)
+// (picx.dev CLSA summary, Methodology > Architecture Overview; scale from the
+// zhichai.net post, Background; gather by the shared index from its "Selector").
+//
+// One CTA per SM.  Each sequence b gets a group of C_b CTAs, in proportion to its
+// length; CTA c of the group owns the contiguous token slice [r0, r1).
+//
+//  1. Scan.  The slice's K_idx rows stream into a 4-stage shared-memory ring
+//     through 1-D bulk copies (TMA engine, mbarrier completion, no multicast);
+//     16 lanes per 256-byte row compute the fp32 dot product.  Scores go to
+//     global memory (L2-resident).  The first half of the slice also feeds a
+//     12-bit histogram that is added to the group's global histogram.
+//  2. Candidate bound.  After its slice, a CTA reads the group histogram as it
+//     stands: whatever subset of tokens it counts, its k-th largest bin is a lower
+//     bound on the true k-th largest score, so every token of the true TopK scores
+//     at least the bin's lower edge tau.  The CTA writes its tokens with
+//     key >= tau, in token order, to its own segment of the candidate list.
+//  3. One barrier for the group.  Every CTA then resolves the exact TopK from the
+//     candidate list by itself (12+12+8-bit radix select over the candidate keys,
+//     ties to the earlier list position = lower token index), ranks the selected
+//     tokens in ascending token order, writes its share of idx, and keeps the
+//     tokens of its attention unit.  If the candidates do not fit in shared
+//     memory, the same selection runs over the whole row of scores instead.
+//  4. Attention.  A unit is (KV head g, split s of the selected ranks); its rows
+//     are all L*G (layer, query head) pairs of head g, so every selected K/V row is
+//     read once for all layers.  mma.sync m16n8k16 bf16 -> fp32, online softmax in
+//     exp2, two warp sets per 16-row tile over alternating 64-token blocks,
+//     merged in shared memory.
+//  5. Splits of one head meet at a barrier and merge with the log-sum-exp rule.
+//
+// Every wait is bounded (kWaitLimitNs); running out records CLSA_ERR_TIMEOUT.
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace clsa {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kStages = 4;
+constexpr int kStageBytes = 32 * 1024;
+constexpr int kBins = 4096;
+constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
+constexpr int kD = 128;               // head dim of the fused path
+constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
+constexpr int kTokBlk = 64;           // tokens per attention block
+constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096)
+constexpr int kCandCap = 16384;       // candidates kept in shared memory (key + index)
+constexpr int kMaxGroups = 256;       // CTAs per launch
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// per-row global state (u32 words)
+constexpr int kRowHist = 0;                       // [kBins] partial histogram (self-clearing)
+constexpr int kRowArrive = kBins;                 // CTAs that published their first half
+constexpr int kRowBar = kBins + 32;               // row-group barrier state [2]
+constexpr int kRowCnt = kBins + 64;               // [kMaxGroups] candidate count per CTA
+constexpr int kRowHeadBar = kRowCnt + kMaxGroups; // [Hkv][2] head-group barrier states (<= 64 heads)
+constexpr int kRowWords = kRowHeadBar + 128;
+
+struct FusedParams {
+  const __nv_bfloat16* q_idx;
+  const __nv_bfloat16* k_idx;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const __nv_bfloat16* Q;
+  const int32_t* seq_lens;
+  __nv_bfloat16* O;
+  int32_t* idx;
+  int32_t* count;
+  float* lse;
+  float* scores;       // [B][n_max]
+  uint32_t* row_ws;    // [B][kRowWords]
+  uint32_t* cand_key;  // [B][n_max]
+  int32_t* cand_tok;   // [B][n_max]
+  float* Op;           // [gridDim][rows][D]  split partials, one slot per CTA
+  float* Ml;           // [gridDim][rows][2]
+  void* ws_header;
+  int B, n_max, k, L, Hq, Hkv, G, rows, nsplit_max;
+  float scale_log2;
+};
+
+struct Plan {
+  int b, c, Cb, start;   // sequence, index in its group, group size, group's first CTA (b < 0: idle)
+  int len, keff, r0, r1;
+  int nsplit;            // token splits per KV head in this group
+  int unit_g0, unit_step, nunits_here;  // heads this CTA attends: g0, g0+step, ... (count)
+  int split;             // split index of this CTA's units
+  int tok0, tok1;        // selected-rank range of the unit
+};
+
+struct Smem {
+  uint64_t bar[kStages];
+  Plan plan;
+  int abort_flag;
+  uint32_t tau_key;
+  int all_selected;
+  int ctot, fast;        // candidate count; candidates held in shared memory
+  uint32_t theta, ties_needed;
+  int sel_bin;
+  uint32_t sel_above;
+  uint32_t warp_tot[kWarps];
+  uint32_t warp_tot2[kWarps];
+  int seg_off[kMaxGroups + 1];
+  uint32_t hist[kBins];
+  int unit_tok[kMaxUnitTok];
+};
+// dynamic shared memory: [Smem][sQ: kMaxRows x kSTR bf16][big: kStages x kStageBytes]
+constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
+constexpr size_t kSmemBig = (size_t)kStages * kStageBytes;
+constexpr size_t smem_bytes() { return align_up(sizeof(Smem), 128) + kSmemQ + kSmemBig; }
+
+// ---------------------------------------------------------------------------
+// small block-wide helpers (512 threads)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* warp_tot, uint32_t* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    uint32_t t = lane < kWarps ? warp_tot[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kWarps) warp_tot[lane] = t;
+  }
+  __syncthreads();
+  const uint32_t before = (w > 0 ? warp_tot[w - 1] : 0u) + x - v;
+  *total = warp_tot[kWarps - 1];
+  __syncthreads();
+  return before;
+}
+
+// bin T with sum(hist[>T]) < need <= sum(hist[>=T]); sm.sel_bin = -1 if the total is below need
+__device__ void select_bin(Smem& sm, int nbins, uint32_t need) {
+  const int per = (nbins + kThreads - 1) / kThreads;
+  const int hi = nbins - threadIdx.x * per;
+  const int lo = max(hi - per, 0);
+  uint32_t local = 0;
+  for (int i = lo; i < hi; ++i) local += sm.hist[i];
+  if (threadIdx.x == 0) sm.sel_bin = -1;
+  uint32_t total;
+  const uint32_t before = block_scan(hi > 0 ? local : 0u, sm.warp_tot, &total);
+  if (hi > 0 && before < need && need <= before + local) {
+    uint32_t acc = before;
+    for (int i = hi - 1; i >= lo; --i) {
+      const uint32_t c = sm.hist[i];
+      if (acc + c >= need) {
+        sm.sel_bin = i;
+        sm.sel_above = acc;
+        break;
+      }
+      acc += c;
+    }
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// work partition (computed identically by every CTA from seq_lens)
+// ---------------------------------------------------------------------------
+__device__ void make_plan(const FusedParams& p, Plan& pl) {
+  const int ncta = gridDim.x;
+  long long total = 0;
+  int nb = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const int len = max(0, min(p.seq_lens[b], p.n_max));
+    total += len;
+    nb += len > 0;
+  }
+  pl.b = -1;
+  if (nb == 0) return;
+  const int spare = ncta - nb;
+  int start = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const int len = max(0, min(p.seq_lens[b], p.n_max));
+    if (len == 0) continue;
+    const int Cb = 1 + (int)((long long)spare * len / total);
+    if ((int)blockIdx.x < start + Cb) {
+      pl.b = b;
+      pl.start = start;
+      pl.c = blockIdx.x - start;
+      pl.Cb = Cb;
+      pl.len = len;
+      pl.keff = min(p.k, len);
+      const int chunk = (len + Cb - 1) / Cb;
+      pl.r0 = min(len, pl.c * chunk);
+      pl.r1 = min(len, pl.r0 + chunk);
+      break;
+    }
+    start += Cb;
+  }
+  if (pl.b < 0) return;
+  if (pl.Cb >= p.Hkv) {
+    pl.nsplit = pl.Cb / p.Hkv;
+    const bool active = pl.c < p.Hkv * pl.nsplit;
+    pl.unit_g0 = active ? pl.c / pl.nsplit : 0;
+    pl.unit_step = p.Hkv;
+    pl.nunits_here = active ? 1 : 0;
+    pl.split = active ? pl.c % pl.nsplit : 0;
+  } else {
+    pl.nsplit = 1;
+    pl.unit_g0 = pl.c;
+    pl.unit_step = pl.Cb;
+    pl.nunits_here = (p.Hkv - pl.c + pl.Cb - 1) / pl.Cb;
+    pl.split = 0;
+  }
+  const int per = (pl.keff + pl.nsplit - 1) / pl.nsplit;
+  pl.tok0 = min(pl.keff, pl.split * per);
+  pl.tok1 = min(pl.keff, pl.tok0 + per);
+}
+
+__device__ __forceinline__ void abort_cta(Smem& sm, const FusedParams& p, int site) {
+  record_error(p.ws_header, CLSA_ERR_TIMEOUT, site);
+  sm.abort_flag = 1;
+}
+
+// ---------------------------------------------------------------------------
+// phase 1: streaming scan of the slice (bulk-copy ring)
+// ---------------------------------------------------------------------------
+template <int DIDX>
+__device__ bool scan_slice(const FusedParams& p, Smem& sm, unsigned char* ring, bool publish) {
+  constexpr int RB = DIDX * 2;                 // row bytes
+  constexpr int RPC = kStageBytes / RB;        // rows per chunk
+  constexpr int LPR = RB / 16;                 // lanes per row
+  constexpr int RPI = 32 / LPR;                // rows per warp instruction
+  const Plan& pl = sm.plan;
+  const int nrows = pl.r1 - pl.r0;
+  const int nchunks = (nrows + RPC - 1) / RPC;
+  const int half = publish ? (nchunks + 1) / 2 : 0;  // chunks [0, half) feed the histogram
+  const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
+  float* sc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % LPR, rsub = lane / LPR;
+
+  float q[8];
+  {
+    const uint4 qv = *reinterpret_cast<const uint4*>(p.q_idx + (size_t)pl.b * DIDX + sub * 8);
+    unpack_bf16x2(qv.x, q[0], q[1]);
+    unpack_bf16x2(qv.y, q[2], q[3]);
+    unpack_bf16x2(qv.z, q[4], q[5]);
+    unpack_bf16x2(qv.w, q[6], q[7]);
+  }
+  for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int ch) {  // thread 0 only
+    const int s = ch % kStages;
+    const int rows = min(RPC, nrows - ch * RPC);
+    const uint32_t bytes = (uint32_t)rows * RB;
+    mbar_arrive_expect_tx(&sm.bar[s], bytes);
+    bulk_g2s(ring + s * kStageBytes, src + (size_t)ch * RPC * DIDX, bytes, &sm.bar[s]);
+  };
+  if (threadIdx.x == 0)
+    for (int ch = 0; ch < min(kStages, nchunks); ++ch) issue(ch);
+
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int s = ch % kStages;
+    const uint32_t parity = (ch / kStages) & 1;
+    if (!mbar_wait(&sm.bar[s], parity)) {
+      if (threadIdx.x == 0) abort_cta(sm, p, 100 + ch);
+    }
+    __syncthreads();
+    if (sm.abort_flag) return false;
+    const int rows = min(RPC, nrows - ch * RPC);
+    const unsigned char* buf = ring + s * kStageBytes;
+    for (int r = warp * RPI + rsub; r < RPC; r += kWarps * RPI) {
+      // every lane of the warp runs the shuffle; rows past the chunk contribute nothing
+      float acc = 0.f;
+      if (r < rows) {
+        const uint4 v = *reinterpret_cast<const uint4*>(buf + r * RB + sub * 16);
+        float a0, a1, a2, a3, a4, a5, a6, a7;
+        unpack_bf16x2(v.x, a0, a1);
+        unpack_bf16x2(v.y, a2, a3);
+        unpack_bf16x2(v.z, a4, a5);
+        unpack_bf16x2(v.w, a6, a7);
+        acc = q[0] * a0;
+        acc = fmaf(q[1], a1, acc);
+        acc = fmaf(q[2], a2, acc);
+        acc = fmaf(q[3], a3, acc);
+        acc = fmaf(q[4], a4, acc);
+        acc = fmaf(q[5], a5, acc);
+        acc = fmaf(q[6], a6, acc);
+        acc = fmaf(q[7], a7, acc);
+      }
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (sub == 0 && r < rows) {
+        const int j = ch * RPC + r;
+        sc[j] = acc;
+        if (ch < half) atomicAdd(&sm.hist[float_key(acc) >> 20], 1u);
+      }
+    }
+    __syncthreads();  // stage s fully read
+    if (threadIdx.x == 0 && ch + kStages < nchunks) {
+      fence_proxy_async_smem();
+      issue(ch + kStages);
+    }
+    if (ch == half - 1) {  // first half done: publish its histogram to the group
+      uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
+      for (int i = threadIdx.x; i < kBins; i += kThreads)
+        if (sm.hist[i]) atomicAdd(gh + i, sm.hist[i]);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
+      }
+    }
+  }
+  if (publish && nchunks == 0 && threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
+  }
+  __syncthreads();
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// phase 2: candidate bound tau from the group histogram, candidate segment
+// ---------------------------------------------------------------------------
+__device__ void write_candidates(const FusedParams& p, Smem& sm) {
+  const Plan& pl = sm.plan;
+  uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
+  // wait briefly for half of the group's first halves (tau stays valid without it)
+  if (threadIdx.x == 0) {
+    const unsigned long long t0 = globaltimer_ns();
+    const uint32_t want = (uint32_t)(pl.Cb + 1) / 2;
+    while (ld_acquire_gpu(rw + kRowArrive) < want && globaltimer_ns() - t0 < 20000ull) __nanosleep(64);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = __ldcg(rw + kRowHist + i);
+  __syncthreads();
+  select_bin(sm, kBins, (uint32_t)pl.keff);
+  if (threadIdx.x == 0) sm.tau_key = sm.sel_bin >= 0 ? ((uint32_t)sm.sel_bin << 20) : 0u;
+  __syncthreads();
+  const uint32_t tau = sm.tau_key;
+  // this CTA's tokens with key >= tau, in token order, to its segment
+  const float* sc = p.scores + (size_t)pl.b * p.n_max;
+  const int n = pl.r1 - pl.r0;
+  const int run = (n + kThreads - 1) / kThreads;
+  const int a = pl.r0 + threadIdx.x * run, e = min(pl.r1, a + run);
+  uint32_t mine = 0;
+  for (int j = a; j < e; ++j) mine += float_key(__ldcg(sc + j)) >= tau;
+  uint32_t total;
+  uint32_t pos = block_scan(mine, sm.warp_tot, &total);
+  uint32_t* ck = p.cand_key + (size_t)pl.b * p.n_max + pl.r0;
+  int32_t* ct = p.cand_tok + (size_t)pl.b * p.n_max + pl.r0;
+  for (int j = a; j < e; ++j) {
+    const uint32_t key = float_key(__ldcg(sc + j));
+    if (key >= tau) {
+      __stcg(ck + pos, key);
+      __stcg(ct + pos, j);
+      ++pos;
+    }
+  }
+  if (threadIdx.x == 0) __stcg(rw + kRowCnt + pl.c, total);
+}
+
+// ---------------------------------------------------------------------------
+// phase 3: exact TopK over the candidate positions p in [0, P)
+//   fast: keys/tokens in shared memory (concatenated segments, token order)
+//   slow: the whole row of scores (position = token)
+// ---------------------------------------------------------------------------
+struct CandSrc {
+  const uint32_t* skey;
+  const int32_t* stok;
+  const float* row_scores;
+  bool fast;
+  __device__ __forceinline__ uint32_t key(int i) const {
+    return fast ? skey[i] : float_key(__ldcg(row_scores + i));
+  }
+  __device__ __forceinline__ int tok(int i) const { return fast ? stok[i] : i; }
+};
+
+// digit histograms; leaves theta and ties_needed in sm
+__device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff, void* ws_header) {
+  const int run = (P + kThreads - 1) / kThreads;
+  const int a = threadIdx.x * run, e = min(P, a + run);
+  for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
+  __syncthreads();
+  for (int i = a; i < e; ++i) atomicAdd(&sm.hist[src.key(i) >> 20], 1u);
+  __syncthreads();
+  select_bin(sm, kBins, keff);
+  if (sm.sel_bin < 0) {  // fewer candidates than k_eff: cannot happen for a clean workspace
+    if (threadIdx.x == 0) {
+      record_error(ws_header, CLSA_ERR_BAD_INDEX, -1);
+      sm.theta = 0xFFFFFFFFu;
+      sm.ties_needed = 0;
+    }
+    __syncthreads();
+    return;
+  }
+  const uint32_t t1 = (uint32_t)sm.sel_bin;
+  uint32_t need = keff - sm.sel_above;
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
+  __syncthreads();
+  for (int i = a; i < e; ++i) {
+    const uint32_t k = src.key(i);
+    if ((k >> 20) == t1) atomicAdd(&sm.hist[(k >> 8) & 0xFFFu], 1u);
+  }
+  __syncthreads();
+  select_bin(sm, kBins, need);
+  const uint32_t p2 = (t1 << 12) | (uint32_t)sm.sel_bin;
+  need -= sm.sel_above;
+  __syncthreads();
+  for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[i] = 0;
+  __syncthreads();
+  for (int i = a; i < e; ++i) {
+    const uint32_t k = src.key(i);
+    if ((k >> 8) == p2) atomicAdd(&sm.hist[k & 0xFFu], 1u);
+  }
+  __syncthreads();
+  select_bin(sm, 256, need);
+  if (threadIdx.x == 0) {
+    sm.theta = (p2 << 8) | (uint32_t)sm.sel_bin;
+    sm.ties_needed = need - sm.sel_above;
+  }
+  __syncthreads();
+}
+
+// rank the selected positions in order; keep the unit's tokens, write this CTA's share of idx
+__device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& src, int P) {
+  const Plan& pl = sm.plan;
+  const uint32_t theta = sm.theta, ties = sm.ties_needed;
+  const int run = (P + kThreads - 1) / kThreads;
+  const int a = threadIdx.x * run, e = min(P, a + run);
+  uint32_t eq = 0;
+  for (int i = a; i < e; ++i) eq += src.key(i) == theta;
+  uint32_t tot;
+  uint32_t eq_rank = block_scan(eq, sm.warp_tot, &tot);
+  uint32_t sel = 0;
+  {
+    uint32_t r = eq_rank;
+    for (int i = a; i < e; ++i) {
+      const uint32_t k = src.key(i);
+      if (k > theta) ++sel;
+      else if (k == theta) sel += (r++ < ties);
+    }
+  }
+  uint32_t rank = block_scan(sel, sm.warp_tot, &tot);
+  int32_t* out = p.idx + (size_t)pl.b * p.k;
+  uint32_t r = eq_rank;
+  for (int i = a; i < e; ++i) {
+    const uint32_t k = src.key(i);
+    bool s = k > theta;
+    if (k == theta) s = (r++ < ties);
+    if (!s) continue;
+    const int t = src.tok(i);
+    if ((int)rank >= pl.tok0 && (int)rank < pl.tok1) sm.unit_tok[rank - pl.tok0] = t;
+    if (t >= pl.r0 && t < pl.r1 && (int)rank < pl.keff) out[rank] = t;
+    ++rank;
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// phase 4: attention of one unit (head g, tokens sm.unit_tok[0..ntok))
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, __nv_bfloat16* sQ, int mt_rows) {
+  constexpr int VPR = kD * 2 / 16;
+  for (int v = threadIdx.x; v < mt_rows * VPR; v += kThreads) {
+    const int r = v / VPR, c = v % VPR;
+    __nv_bfloat16* dst = sQ + r * kSTR + c * 8;
+    if (r < p.rows) {
+      const int l = r / p.G, h = g * p.G + r % p.G;
+      cp_async_16(dst, p.Q + (((size_t)l * p.B + b) * p.Hq + h) * kD + c * 8, 16);
+    } else {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void load_kv_block(const FusedParams& p, const Smem& sm, int b, int g, int blk0, int ntok,
+                                              __nv_bfloat16* dk, __nv_bfloat16* dv) {
+  constexpr int VPR = kD * 2 / 16;
+  for (int v = threadIdx.x; v < kTokBlk * VPR; v += kThreads) {
+    const int r = v / VPR, c = v % VPR;
+    const int i = blk0 + r;
+    const __nv_bfloat16* sk = p.K;
+    const __nv_bfloat16* sv = p.V;
+    int bytes = 0;
+    if (i < ntok) {
+      const int t = sm.unit_tok[i];
+      if ((unsigned)t < (unsigned)sm.plan.len) {
+        const size_t off = (((size_t)b * p.n_max + t) * p.Hkv + g) * kD + c * 8;
+        sk += off;
+        sv += off;
+        bytes = 16;
+      } else if (c == 0) {
+        record_error(p.ws_header, CLSA_ERR_BAD_INDEX, ((long long)b << 32) | (unsigned)i);
+      }
+    }
+    cp_async_16(dk + r * kSTR + c * 8, sk, bytes);
+    cp_async_16(dv + r * kSTR + c * 8, sv, bytes);
+  }
+  cp_async_commit();
+}
+
+// NT = n-tiles (8 tokens each) one warp set handles per 64-token block; NS = 64 / (8 NT) sets
+template <int NT>
+__device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, unsigned char* big, int g,
+                            int ntok, bool q_loaded, int unit_split) {
+  constexpr int NS = kTokBlk / (8 * NT);
+  const Plan& pl = sm.plan;
+  const int b = pl.b;
+  const int MT = (p.rows + 15) / 16;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const bool active = warp < MT * NS;
+  const int mt = warp % MT, set = warp / MT;
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(big);  // [2][kTokBlk][kSTR]
+  __nv_bfloat16* sV = sK + 2 * kTokBlk * kSTR;
+  if (!q_loaded) load_q_tile(p, b, g, sQ, MT * 16);
+  const int nblk = (ntok + kTokBlk - 1) / kTokBlk;
+  if (nblk > 0) {
+    load_kv_block(p, sm, b, g, 0, ntok, sK, sV);
+    cp_async_wait<1>();  // the Q tile (older group) has landed
+  } else {
+    cp_async_wait<0>();
+  }
+  __syncthreads();
+
+  // Q fragments are re-read from shared memory per k-step (keeps the register budget of 512 threads)
+  const __nv_bfloat16* qrow = sQ + (mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * kSTR + 8 * (lane >> 4);
+  float o[kD / 8][4];
+#pragma unroll
+  for (int i = 0; i < kD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  for (int bi = 0; bi < nblk; ++bi) {
+    const int stage = bi & 1;
+    const int blk0 = bi * kTokBlk;
+    if (bi + 1 < nblk) {
+      load_kv_block(p, sm, b, g, blk0 + kTokBlk, ntok, sK + (stage ^ 1) * kTokBlk * kSTR,
+                    sV + (stage ^ 1) * kTokBlk * kSTR);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (active) {
+      const __nv_bfloat16* tk = sK + stage * kTokBlk * kSTR + set * NT * 8 * kSTR;
+      const __nv_bfloat16* tv = sV + stage * kTokBlk * kSTR + set * NT * 8 * kSTR;
+      const int tbase = blk0 + set * NT * 8;
+      float s[NT][4];
+#pragma unroll
+      for (int i = 0; i < NT; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        uint32_t qa[4];
+        ldmatrix_x4(qa[0], qa[1], qa[2], qa[3], qrow + ks * 16);
+#pragma unroll
+        for (int nt2 = 0; nt2 < NT / 2; ++nt2) {
+          const int mi = lane >> 3;
+          const int tok = nt2 * 16 + 8 * (mi >> 1) + (lane & 7);
+          const int col = ks * 16 + 8 * (mi & 1);
+          uint32_t r0, r1, r2, r3;
+          ldmatrix_x4(r0, r1, r2, r3, tk + tok * kSTR + col);
+          mma_bf16_16816(s[2 * nt2], qa, r0, r1);
+          mma_bf16_16816(s[2 * nt2 + 1], qa, r2, r3);
+        }
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = tbase + nt * 8 + 2 * tig + (e & 1);
+          s[nt][e] = tok < ntok ? s[nt][e] * p.scale_log2 : -INFINITY;
+        }
+        mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
+        mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
+      const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float c0 = exp2f(m0 - ref0), c1 = exp2f(m1 - ref1);
+      m0 = mn0;
+      m1 = mn1;
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        s[nt][0] = exp2f(s[nt][0] - ref0);
+        s[nt][1] = exp2f(s[nt][1] - ref0);
+        s[nt][2] = exp2f(s[nt][2] - ref1);
+        s[nt][3] = exp2f(s[nt][3] - ref1);
+        rs0 += s[nt][0] + s[nt][1];
+        rs1 += s[nt][2] + s[nt][3];
+      }
+      l0 = l0 * c0 + rs0;
+      l1 = l1 * c1 + rs1;
+#pragma unroll
+      for (int nd = 0; nd < kD / 8; ++nd) {
+        o[nd][0] *= c0;
+        o[nd][1] *= c0;
+        o[nd][2] *= c1;
+        o[nd][3] *= c1;
+      }
+#pragma unroll
+      for (int kk = 0; kk < NT / 2; ++kk) {
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+        pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+        pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+        pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+        for (int nd2 = 0; nd2 < kD / 16; ++nd2) {
+          const int mi = lane >> 3;
+          const int tok = kk * 16 + 8 * (mi & 1) + (lane & 7);
+          const int col = nd2 * 16 + 8 * (mi >> 1);
+          uint32_t r0, r1, r2, r3;
+          ldmatrix_x4_trans(r0, r1, r2, r3, tv + tok * kSTR + col);
+          mma_bf16_16816(o[2 * nd2], pa, r0, r1);
+          mma_bf16_16816(o[2 * nd2 + 1], pa, r2, r3);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- merge the NS token sets of each m-tile (thread-private slots in shared memory)
+  float* xo = reinterpret_cast<float*>(big);                  // [NS-1][MT][64][32]
+  float* xm = xo + (size_t)(NS - 1) * MT * 64 * 32;           // [NS-1][MT][4][32]
+  if (active && set > 0) {
+    float* d = xo + ((size_t)(set - 1) * MT + mt) * 64 * 32;
+#pragma unroll
+    for (int nd = 0; nd < kD / 8; ++nd)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[(nd * 4 + e) * 32 + lane] = o[nd][e];
+    float* dm = xm + ((size_t)(set - 1) * MT + mt) * 4 * 32;
+    dm[0 * 32 + lane] = m0;
+    dm[1 * 32 + lane] = m1;
+    dm[2 * 32 + lane] = l0;
+    dm[3 * 32 + lane] = l1;
+  }
+  __syncthreads();
+  if (active && set == 0) {
+    for (int s2 = 1; s2 < NS; ++s2) {
+      const float* d = xo + ((size_t)(s2 - 1) * MT + mt) * 64 * 32;
+      const float* dm = xm + ((size_t)(s2 - 1) * MT + mt) * 4 * 32;
+      const float om0 = dm[lane], om1 = dm[32 + lane], ol0 = dm[64 + lane], ol1 = dm[96 + lane];
+      const float nm0 = fmaxf(m0, om0), nm1 = fmaxf(m1, om1);
+      const float r0 = nm0 == -INFINITY ? 0.f : nm0, r1 = nm1 == -INFINITY ? 0.f : nm1;
+      const float a0 = exp2f(m0 - r0), b0 = exp2f(om0 - r0);
+      const float a1 = exp2f(m1 - r1), b1 = exp2f(om1 - r1);
+#pragma unroll
+      for (int nd = 0; nd < kD / 8; ++nd) {
+        o[nd][0] = o[nd][0] * a0 + d[(nd * 4 + 0) * 32 + lane] * b0;
+        o[nd][1] = o[nd][1] * a0 + d[(nd * 4 + 1) * 32 + lane] * b0;
+        o[nd][2] = o[nd][2] * a1 + d[(nd * 4 + 2) * 32 + lane] * b1;
+        o[nd][3] = o[nd][3] * a1 + d[(nd * 4 + 3) * 32 + lane] * b1;
+      }
+      l0 = l0 * a0 + ol0 * b0;
+      l1 = l1 * a1 + ol1 * b1;
+      m0 = nm0;
+      m1 = nm1;
+    }
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int r = mt * 16 + gid + 8 * half;
+      if (r >= p.rows) continue;
+      const int l = r / p.G, h = g * p.G + r % p.G;
+      const float m = half ? m1 : m0;
+      const float ls = half ? l1 : l0;
+      if (pl.nsplit == 1) {
+        const float inv = ls > 0.f ? 1.f / ls : 0.f;
+        __nv_bfloat16* out = p.O + (((size_t)l * p.B + b) * p.Hq + h) * kD;
+#pragma unroll
+        for (int nd = 0; nd < kD / 8; ++nd)
+          *reinterpret_cast<uint32_t*>(out + nd * 8 + 2 * tig) =
+              pack_bf16x2(o[nd][2 * half] * inv, o[nd][2 * half + 1] * inv);
+        if (p.lse && tig == 0)
+          p.lse[((size_t)l * p.B + b) * p.Hq + h] = ls > 0.f ? (m + log2f(ls)) * kLn2 : -INFINITY;
+      } else {
+        const size_t pi = (size_t)blockIdx.x * p.rows + r;  // partial slot of this CTA
+        float* op = p.Op + pi * kD;
+#pragma unroll
+        for (int nd = 0; nd < kD / 8; ++nd)
+          __stcg(reinterpret_cast<float2*>(op + nd * 8 + 2 * tig), make_float2(o[nd][2 * half], o[nd][2 * half + 1]));
+        if (tig == 0) __stcg(reinterpret_cast<float2*>(p.Ml + pi * 2), make_float2(m, ls));
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// phase 5: merge the nsplit partials of head g (rows r with r % nsplit == split)
+// ---------------------------------------------------------------------------
+__device__ void combine_head(const FusedParams& p, const Plan& pl, int g) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // split s of head g is CTA start + g * nsplit + s; its partial rows start at that CTA's slot
+  const size_t base = ((size_t)pl.start + (size_t)g * pl.nsplit) * p.rows;
+  for (int r = pl.split + warp * pl.nsplit; r < p.rows; r += kWarps * pl.nsplit) {
+    float M = -INFINITY;
+    for (int s = lane; s < pl.nsplit; s += 32) M = fmaxf(M, __ldcg(p.Ml + (base + (size_t)s * p.rows + r) * 2));
+    M = warp_max(M);
+    float den = 0.f;
+    float acc[kD / 32];
+#pragma unroll
+    for (int c = 0; c < kD / 32; ++c) acc[c] = 0.f;
+    if (M != -INFINITY) {
+      for (int s0 = 0; s0 < pl.nsplit; s0 += 32) {
+        const int s = s0 + lane;
+        float w = 0.f;
+        if (s < pl.nsplit) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + (base + (size_t)s * p.rows + r) * 2));
+          w = exp2f(ml.x - M);
+          den = fmaf(w, ml.y, den);
+        }
+        const int cnt = min(32, pl.nsplit - s0);
+#pragma unroll 4
+        for (int j = 0; j < cnt; ++j) {
+          const float wj = __shfl_sync(0xffffffffu, w, j);
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(p.Op + (base + (size_t)(s0 + j) * p.rows + r) * kD) + lane);
+          acc[0] = fmaf(wj, v.x, acc[0]);
+          acc[1] = fmaf(wj, v.y, acc[1]);
+          acc[2] = fmaf(wj, v.z, acc[2]);
+          acc[3] = fmaf(wj, v.w, acc[3]);
+        }
+      }
+      den = warp_sum(den);
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const int l = r / p.G, h = g * p.G + r % p.G;
+    __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
+    uint2 wv;
+    wv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    wv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(out) = wv;
+    if (p.lse && lane == 0)
+      p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <int DIDX>
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem);
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + align_up(sizeof(Smem), 128));
+  unsigned char* big = smem + align_up(sizeof(Smem), 128) + kSmemQ;
+
+  if (threadIdx.x == 0) {
+    make_plan(p, sm.plan);
+    sm.abort_flag = 0;
+  }
+  __syncthreads();
+  const Plan pl = sm.plan;
+  if (blockIdx.x == 0) {  // sequences with no tokens: count 0, idx -1, O = 0, lse = -inf
+    for (int b = 0; b < p.B; ++b) {
+      if (max(0, min(p.seq_lens[b], p.n_max)) > 0) continue;
+      for (int i = threadIdx.x; i < p.k; i += kThreads) p.idx[(size_t)b * p.k + i] = -1;
+      if (threadIdx.x == 0) p.count[b] = 0;
+      for (int i = threadIdx.x; i < p.L * p.Hq * kD; i += kThreads) {
+        const int l = i / (p.Hq * kD), rem = i % (p.Hq * kD);
+        p.O[((size_t)l * p.B + b) * p.Hq * kD + rem] = __float2bfloat16_rn(0.f);
+      }
+      if (p.lse)
+        for (int i = threadIdx.x; i < p.L * p.Hq; i += kThreads)
+          p.lse[((size_t)(i / p.Hq) * p.B + b) * p.Hq + i % p.Hq] = -INFINITY;
+    }
+  }
+  if (pl.b < 0) return;
+  const int MT = (p.rows + 15) / 16;
+  if (pl.c == 0) {
+    for (int i = pl.keff + threadIdx.x; i < p.k; i += kThreads) p.idx[(size_t)pl.b * p.k + i] = -1;
+    if (threadIdx.x == 0) p.count[pl.b] = pl.keff;
+  }
+  if (pl.c == pl.Cb - 1)  // score tail beyond the sequence
+    for (int j = pl.len + threadIdx.x; j < p.n_max; j += kThreads) p.scores[(size_t)pl.b * p.n_max + j] = -INFINITY;
+  if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQ, MT * 16);  // lands during the scan
+
+  const bool all_sel = pl.keff == pl.len;
+  if (!scan_slice<DIDX>(p, sm, big, !all_sel)) return;
+
+  if (all_sel) {  // every token is selected: rank = token index
+    int32_t* out = p.idx + (size_t)pl.b * p.k;
+    for (int j = pl.r0 + threadIdx.x; j < pl.r1; j += kThreads) out[j] = j;
+    for (int i = threadIdx.x; i < pl.tok1 - pl.tok0; i += kThreads) sm.unit_tok[i] = pl.tok0 + i;
+    __syncthreads();
+  } else {
+    write_candidates(p, sm);
+    uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
+    if (!group_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
+    // everyone has read the partial histogram: clear this CTA's share for the next call
+    {
+      const int per = (kBins + pl.Cb - 1) / pl.Cb;
+      for (int i = pl.c * per + threadIdx.x; i < min(kBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
+      if (pl.c == 0 && threadIdx.x == 0) rw[kRowArrive] = 0u;
+    }
+    // segment offsets of the concatenated candidate list
+    const int chunk = (pl.len + pl.Cb - 1) / pl.Cb;
+    {
+      const uint32_t v = threadIdx.x < pl.Cb ? __ldcg(rw + kRowCnt + threadIdx.x) : 0u;
+      uint32_t total;
+      const uint32_t before = block_scan(v, sm.warp_tot, &total);
+      if (threadIdx.x < pl.Cb) sm.seg_off[threadIdx.x] = (int)before;
+      if (threadIdx.x == 0) {
+        sm.seg_off[pl.Cb] = (int)total;
+        sm.ctot = (int)total;
+        sm.fast = total <= (uint32_t)kCandCap;
+      }
+      __syncthreads();
+    }
+    uint32_t* skey = reinterpret_cast<uint32_t*>(big);
+    int32_t* stok = reinterpret_cast<int32_t*>(big + kCandCap * 4);
+    if (sm.fast) {
+      const uint32_t* gk = p.cand_key + (size_t)pl.b * p.n_max;
+      const int32_t* gt = p.cand_tok + (size_t)pl.b * p.n_max;
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+      for (int c = warp; c < pl.Cb; c += kWarps) {
+        const int o = sm.seg_off[c], n = sm.seg_off[c + 1] - o;
+        const size_t src = (size_t)min(pl.len, c * chunk);
+        for (int i = lane; i < n; i += 32) {
+          skey[o + i] = __ldcg(gk + src + i);
+          stok[o + i] = __ldcg(gt + src + i);
+        }
+      }
+      __syncthreads();
+    }
+    CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
+    const int P = sm.fast ? sm.ctot : pl.len;
+    resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
+    compact_selected(p, sm, src, P);
+  }
+
+  // ---- attention units
+  const int ntok = pl.tok1 - pl.tok0;
+  const int NS = min(4, kWarps / MT) >= 4 ? 4 : 2;
+  for (int u = 0; u < pl.nunits_here; ++u) {
+    const int g = pl.unit_g0 + u * pl.unit_step;
+    if (NS == 4) attend_unit<2>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
+    else attend_unit<4>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
+  }
+  if (pl.nsplit > 1 && pl.nunits_here > 0) {
+    uint32_t* hb = p.row_ws + (size_t)pl.b * kRowWords + kRowHeadBar + 2 * pl.unit_g0;
+    if (!group_barrier(hb, pl.nsplit, p.ws_header, 2)) return;
+    combine_head(p, pl, pl.unit_g0);
+  }
+}
+
+struct FusedCfg {
+  int ncta = 0;
+  bool ok = false;
+};
+
+FusedCfg fused_cfg() {
+  static FusedCfg cfg;
+  static bool done = false;
+  if (!done) {
+    done = true;
+    const DeviceInfo& di = device_info();
+    if (di.sm_count > 0 && (size_t)di.max_smem_optin >= smem_bytes()) {
+      cfg.ncta = std::min(di.sm_count, kMaxGroups);
+      cfg.ok = true;
+    }
+  }
+  return cfg;
+}
+
+}  // namespace
+
+bool fused_decode_supported(const clsa_decode_args* a) {
+  if (a->dtype != CLSA_BF16 || a->d != kD || (a->d_idx != 64 && a->d_idx != 128)) return false;
+  if (a->K_S != nullptr) return false;
+  if (a->Hkv > 64 || a->L * (a->Hq / a->Hkv) > kMaxRows || a->k > kMaxUnitTok) return false;
+  const FusedCfg cfg = fused_cfg();
+  if (!cfg.ok || a->B > cfg.ncta / 2) return false;
+  return true;
+}
+
+size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
+  const FusedCfg cfg = fused_cfg();
+  const size_t rows = (size_t)a->L * (a->Hq / a->Hkv);
+  size_t off = 0;
+  off += align_up((size_t)a->B * a->n_max * 4, 256);           // scores (when not an output)
+  off += align_up((size_t)a->B * kRowWords * 4, 256);          // row state
+  off += 2 * align_up((size_t)a->B * a->n_max * 4, 256);       // candidate keys + tokens
+  off += align_up((size_t)cfg.ncta * rows * kD * 4, 256);      // split partials
+  off += align_up((size_t)cfg.ncta * rows * 2 * 4, 256);
+  return off;
+}
+
+cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws_header, void* ws_body,
+                                cudaStream_t s) {
+  const FusedCfg cfg = fused_cfg();
+  FusedParams p{};
+  p.q_idx = static_cast<const __nv_bfloat16*>(a->q_idx);
+  p.k_idx = static_cast<const __nv_bfloat16*>(a->k_idx);
+  p.K = static_cast<const __nv_bfloat16*>(a->K);
+  p.V = static_cast<const __nv_bfloat16*>(a->V);
+  p.Q = static_cast<const __nv_bfloat16*>(a->Q);
+  p.seq_lens = a->seq_lens;
+  p.O = static_cast<__nv_bfloat16*>(a->O);
+  p.idx = a->idx;
+  p.count = a->count;
+  p.lse = a->lse;
+  p.B = a->B;
+  p.n_max = a->n_max;
+  p.k = a->k;
+  p.L = a->L;
+  p.Hq = a->Hq;
+  p.Hkv = a->Hkv;
+  p.G = a->Hq / a->Hkv;
+  p.rows = a->L * p.G;
+  p.nsplit_max = std::max(1, cfg.ncta / a->Hkv);
+  p.scale_log2 = scale * kLog2e;
+  p.ws_header = ws_header;
+  char* w = static_cast<char*>(ws_body);
+  float* ws_scores = reinterpret_cast<float*>(w);
+  w += align_up((size_t)a->B * a->n_max * 4, 256);
+  p.scores = a->scores ? a->scores : ws_scores;
+  p.row_ws = reinterpret_cast<uint32_t*>(w);
+  w += align_up((size_t)a->B * kRowWords * 4, 256);
+  p.cand_key = reinterpret_cast<uint32_t*>(w);
+  w += align_up((size_t)a->B * a->n_max * 4, 256);
+  p.cand_tok = reinterpret_cast<int32_t*>(w);
+  w += align_up((size_t)a->B * a->n_max * 4, 256);
+  p.Op = reinterpret_cast<float*>(w);
+  w += align_up((size_t)cfg.ncta * p.rows * kD * 4, 256);
+  p.Ml = reinterpret_cast<float*>(w);
+  const size_t smem = smem_bytes();
+  void* args[] = {(void*)&p};
+  cudaError_t e;
+  if (a->d_idx == 128) {
+    e = cudaFuncSetAttribute(decode_fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaLaunchCooperativeKernel((const void*)decode_fused_kernel<128>, dim3(cfg.ncta), dim3(kThreads), args,
+                                      smem, s);
+  } else {
+    e = cudaFuncSetAttribute(decode_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaLaunchCooperativeKernel((const void*)decode_fused_kernel<64>, dim3(cfg.ncta), dim3(kThreads), args,
+                                      smem, s);
+  }
+  launches_add(1);
+  return e;
+}
+
+}  // namespace clsa

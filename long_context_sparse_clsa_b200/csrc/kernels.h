@@ -59,6 +59,12 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
                                const int32_t* idx, const int32_t* count, float scale, void* O, float* lse,
                                void* ws_header, void* attn_ws, cudaStream_t s);
 
+// ----- fused decode step (one cooperative launch) -------------------------------
+bool fused_decode_supported(const clsa_decode_args* a);
+size_t fused_decode_ws_bytes(const clsa_decode_args* a);
+cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws_header, void* ws_body,
+                                cudaStream_t s);
+
 // ----- prefill ------------------------------------------------------------------
 size_t prefill_ws_bytes(const clsa_prefill_args* a);
 clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_body, cudaStream_t s);

@@ -262,3 +262,47 @@ def test_prefill_small():
 def test_prefill_full_size_sampled():
     w = WORKLOADS["prefill4k"]
     _prefill_check(w, [0, 1, 2047, 2048, 4095])
+
+
+# ----------------------------------------------------------------------- fused vs four-kernel plan
+
+def _decode(dv, w, plan, monkeypatch, **kw):
+    monkeypatch.setenv("CLSA_DECODE_PLAN", plan)
+    r = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k,
+                         want_scores=True, **kw)
+    torch.cuda.synchronize()
+    assert r["ws"].status()[0] == "CLSA_OK"
+    return r
+
+
+@pytest.mark.parametrize("name", ["d32k_small", "ragged_small"])
+def test_fused_matches_unfused(name, monkeypatch):
+    w = CASES[name]
+    _, dv = _inputs(name)
+    a = _decode(dv, w, "fused", monkeypatch)
+    b = _decode(dv, w, "unfused", monkeypatch)
+    assert torch.equal(a["scores"], b["scores"])      # same fp32 arithmetic order
+    assert torch.equal(a["idx"], b["idx"]) and torch.equal(a["count"], b["count"])
+    assert max_abs(tensor_f64(a["O"]), tensor_f64(b["O"])) <= TOL[w.dtype]
+
+
+@pytest.mark.parametrize("n,k,mode", [(10000, 2048, "equal"), (40000, 2048, "equal"), (20000, 3000, "blocks"),
+                                      (5000, 4096, "equal"), (3000, 4000, "normal")])
+def test_decode_step_adversarial_selection(n, k, mode, monkeypatch):
+    """Ties everywhere (every index key equal, or a few distinct values): the
+    candidate list of the fused plan overflows shared memory (n > 16384) or holds
+    every token; selection must still be the exact TopK with lower-index ties."""
+    w = scaled("decode32k", n_max=n, k=k, L=2, plant=0.0)
+    inp = make_inputs(w)
+    if mode == "equal":
+        inp.k_idx[:] = inp.k_idx[:, :1, :]
+    elif mode == "blocks":
+        inp.k_idx[:] = inp.k_idx[:, (np.arange(n) % 7)[None, :].repeat(1, 0)[0], :][None]
+    dv = clsa.to_device(inp)
+    r = _decode(dv, w, "fused", monkeypatch)
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    gi, gc = O.topk_select(tensor_f64(r["scores"]), inp.seq_lens, w.k)
+    np.testing.assert_array_equal(gi, i_np)
+    np.testing.assert_array_equal(gc, c_np)
+    want, _ = O.sparse_attention(inp.Q, inp.K, inp.V, i_np, c_np)
+    assert max_abs(tensor_f64(r["O"]), want) <= TOL[w.dtype]
