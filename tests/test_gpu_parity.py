@@ -297,7 +297,7 @@ def test_decode_step_adversarial_selection(n, k, mode, monkeypatch):
     if mode == "equal":
         inp.k_idx[:] = inp.k_idx[:, :1, :]
     elif mode == "blocks":
-        inp.k_idx[:] = inp.k_idx[:, (np.arange(n) % 7)[None, :].repeat(1, 0)[0], :][None]
+        inp.k_idx[0] = inp.k_idx[0][np.arange(n) % 7]
     dv = clsa.to_device(inp)
     r = _decode(dv, w, "fused", monkeypatch)
     i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
