@@ -34,6 +34,7 @@
 //
 // Every wait is bounded (kWaitLimitNs); running out records CLSA_ERR_TIMEOUT.
 #include <cmath>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -83,9 +84,14 @@ struct FusedParams {
   float* Op;           // [gridDim][rows][D]  split partials, one slot per CTA
   float* Ml;           // [gridDim][rows][2]
   void* ws_header;
+  unsigned long long* trace;  // [gridDim][16] globaltimer stamps per phase, or null
   int B, n_max, k, L, Hq, Hkv, G, rows, nsplit_max;
   float scale_log2;
 };
+
+__device__ __forceinline__ void stamp(const FusedParams& p, int phase) {
+  if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * 16 + phase] = globaltimer_ns();
+}
 
 struct Plan {
   int b, c, Cb, start;   // sequence, index in its group, group size, group's first CTA (b < 0: idle)
@@ -771,6 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + align_up(sizeof(Smem), 128));
   unsigned char* big = smem + align_up(sizeof(Smem), 128) + kSmemQ;
 
+  stamp(p, 0);
   if (threadIdx.x == 0) {
     make_plan(p, sm.plan);
     sm.abort_flag = 0;
@@ -803,6 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
 
   const bool all_sel = pl.keff == pl.len;
   if (!scan_slice<DIDX>(p, sm, big, !all_sel)) return;
+  stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
     int32_t* out = p.idx + (size_t)pl.b * p.k;
@@ -811,8 +819,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     __syncthreads();
   } else {
     write_candidates(p, sm);
+    stamp(p, 2);
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!group_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
+    stamp(p, 3);
     // everyone has read the partial histogram: clear this CTA's share for the next call
     {
       const int per = (kBins + pl.Cb - 1) / pl.Cb;
@@ -851,9 +861,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     }
     CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
     const int P = sm.fast ? sm.ctot : pl.len;
+    stamp(p, 4);
     resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
+    stamp(p, 5);
     compact_selected(p, sm, src, P);
+    if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * 16 + 15] = (unsigned long long)sm.ctot | ((unsigned long long)sm.fast << 32);
   }
+  stamp(p, 6);
 
   // ---- attention units
   const int ntok = pl.tok1 - pl.tok0;
@@ -863,11 +877,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     if (NS == 4) attend_unit<2>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
     else attend_unit<4>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
   }
+  stamp(p, 7);
   if (pl.nsplit > 1 && pl.nunits_here > 0) {
     uint32_t* hb = p.row_ws + (size_t)pl.b * kRowWords + kRowHeadBar + 2 * pl.unit_g0;
     if (!group_barrier(hb, pl.nsplit, p.ws_header, 2)) return;
+    stamp(p, 8);
     combine_head(p, pl, pl.unit_g0);
   }
+  stamp(p, 9);
 }
 
 struct FusedCfg {
@@ -904,6 +921,7 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   const FusedCfg cfg = fused_cfg();
   const size_t rows = (size_t)a->L * (a->Hq / a->Hkv);
   size_t off = 0;
+  off += (size_t)kMaxGroups * 16 * 8;                           // phase stamps (CLSA_TRACE=1)
   off += align_up((size_t)a->B * a->n_max * 4, 256);           // scores (when not an output)
   off += align_up((size_t)a->B * kRowWords * 4, 256);          // row state
   off += 2 * align_up((size_t)a->B * a->n_max * 4, 256);       // candidate keys + tokens
@@ -938,6 +956,9 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   p.scale_log2 = scale * kLog2e;
   p.ws_header = ws_header;
   char* w = static_cast<char*>(ws_body);
+  const char* tr = std::getenv("CLSA_TRACE");
+  p.trace = (tr && tr[0] == '1') ? reinterpret_cast<unsigned long long*>(w) : nullptr;
+  w += (size_t)kMaxGroups * 16 * 8;
   float* ws_scores = reinterpret_cast<float*>(w);
   w += align_up((size_t)a->B * a->n_max * 4, 256);
   p.scores = a->scores ? a->scores : ws_scores;
