@@ -88,6 +88,44 @@ __device__ __forceinline__ bool group_barrier(uint32_t* state, uint32_t nblocks,
   return s_ok != 0;
 }
 
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Count-up barrier among `n` co-resident CTAs: state[0] counts arrivals (a
+// fire-and-forget release add), every CTA polls it until it reaches n, then
+// counts itself in state[1]; the last CTA to pass returns both words to zero, off
+// the critical path, so the state is clean for the next use.  Bounded wait:
+// false (and CLSA_ERR_TIMEOUT with `site`) if it runs out.
+__device__ __forceinline__ bool count_barrier(uint32_t* state, uint32_t n, void* ws, int site) {
+  __shared__ int s_ok2;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    if (n > 1) {
+      __threadfence();
+      red_add_release_gpu(state, 1u);
+      if (ld_acquire_gpu(state) < n) {
+        const unsigned long long t0 = globaltimer_ns();
+        while (ld_acquire_gpu(state) < n) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_error(ws, CLSA_ERR_TIMEOUT, site);
+            ok = 0;
+            break;
+          }
+        }
+      }
+      if (ok && atomicAdd(state + 1, 1u) == n - 1) {  // everyone has seen n: reset
+        state[0] = 0u;
+        state[1] = 0u;
+      }
+    }
+    s_ok2 = ok;
+  }
+  __syncthreads();
+  return s_ok2 != 0;
+}
+
 // ---------------------------------------------------------------------------
 // order-preserving key: larger float -> larger unsigned key; -0.0 == +0.0
 // ---------------------------------------------------------------------------
@@ -139,6 +177,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ void cp_async_16(void* smem, const void* gmem, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
                "r"(src_bytes) : "memory");
+}
+// 4-byte async copy global -> shared (through L1)
+__device__ __forceinline__ void cp_async_4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>

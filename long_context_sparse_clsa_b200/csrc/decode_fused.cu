@@ -52,7 +52,7 @@ constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token 
 constexpr int kD = 128;               // head dim of the fused path
 constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
 constexpr int kTokBlk = 64;           // tokens per attention block
-constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096)
+constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096); also slice scores kept on chip
 constexpr int kCandCap = 16384;       // candidates kept in shared memory (key + index)
 constexpr int kMaxGroups = 256;       // CTAs per launch
 constexpr float kLog2e = 1.4426950408889634f;
@@ -89,8 +89,9 @@ struct FusedParams {
   float scale_log2;
 };
 
+constexpr int kTraceSlots = 32;
 __device__ __forceinline__ void stamp(const FusedParams& p, int phase) {
-  if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * 16 + phase] = globaltimer_ns();
+  if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + phase] = globaltimer_ns();
 }
 
 struct Plan {
@@ -113,10 +114,14 @@ struct Smem {
   int sel_bin;
   uint32_t sel_above;
   uint32_t warp_tot[kWarps];
-  uint32_t warp_tot2[kWarps];
+  uint32_t warp_tot2[kWarps + 1];
   int seg_off[kMaxGroups + 1];
   uint32_t hist[kBins];
-  int unit_tok[kMaxUnitTok];
+  union {                          // slice scores until the candidates are out, then unit tokens
+    float score[kMaxUnitTok];
+    int unit_tok[kMaxUnitTok];
+  };
+  float cm[512], cl[512];          // split-combine staging (m, l per row x split)
 };
 // dynamic shared memory: [Smem][sQ: kMaxRows x kSTR bf16][big: kStages x kStageBytes]
 constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
@@ -175,6 +180,36 @@ __device__ void select_bin(Smem& sm, int nbins, uint32_t need) {
     }
   }
   __syncthreads();
+}
+
+// exclusive prefix of a 0/1 flag in thread order (ballots); *total = block total
+__device__ __forceinline__ uint32_t block_flag_scan(bool flag, uint32_t* warp_tot, uint32_t* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const uint32_t bal = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) warp_tot[w] = __popc(bal);
+  __syncthreads();
+  if (w == 0) {
+    const uint32_t t = lane < kWarps ? warp_tot[lane] : 0u;
+    uint32_t x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < kWarps) warp_tot[lane] = x - t;
+    if (lane == 31) warp_tot[kWarps] = x;
+  }
+  __syncthreads();
+  const uint32_t before = warp_tot[w] + __popc(bal & ((1u << lane) - 1u));
+  *total = warp_tot[kWarps];
+  __syncthreads();
+  return before;
+}
+
+// histogram increment, aggregated over the lanes of a warp that hit the same bin
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
+  const uint32_t m = __match_any_sync(__activemask(), bin);
+  if ((threadIdx.x & 31) == __ffs(m) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(m));
 }
 
 // ---------------------------------------------------------------------------
@@ -312,6 +347,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, unsigned char* ring, 
       if (sub == 0 && r < rows) {
         const int j = ch * RPC + r;
         sc[j] = acc;
+        if (nrows <= kMaxUnitTok) sm.score[j] = acc;
         if (ch < half) atomicAdd(&sm.hist[float_key(acc) >> 20], 1u);
       }
     }
@@ -359,25 +395,29 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm) {
   __syncthreads();
   const uint32_t tau = sm.tau_key;
   // this CTA's tokens with key >= tau, in token order, to its segment
-  const float* sc = p.scores + (size_t)pl.b * p.n_max;
+  const float* gsc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
   const int n = pl.r1 - pl.r0;
-  const int run = (n + kThreads - 1) / kThreads;
-  const int a = pl.r0 + threadIdx.x * run, e = min(pl.r1, a + run);
-  uint32_t mine = 0;
-  for (int j = a; j < e; ++j) mine += float_key(__ldcg(sc + j)) >= tau;
-  uint32_t total;
-  uint32_t pos = block_scan(mine, sm.warp_tot, &total);
+  const bool on_chip = n <= kMaxUnitTok;
   uint32_t* ck = p.cand_key + (size_t)pl.b * p.n_max + pl.r0;
   int32_t* ct = p.cand_tok + (size_t)pl.b * p.n_max + pl.r0;
-  for (int j = a; j < e; ++j) {
-    const uint32_t key = float_key(__ldcg(sc + j));
-    if (key >= tau) {
-      __stcg(ck + pos, key);
-      __stcg(ct + pos, j);
-      ++pos;
+  uint32_t written = 0;
+  for (int base = 0; base < n; base += kThreads) {
+    const int j = base + threadIdx.x;
+    uint32_t key = 0;
+    bool f = false;
+    if (j < n) {
+      key = float_key(on_chip ? sm.score[j] : __ldcg(gsc + j));
+      f = key >= tau;
     }
+    uint32_t tot;
+    const uint32_t pos = written + block_flag_scan(f, sm.warp_tot2, &tot);
+    if (f) {
+      __stcg(ck + pos, key);
+      __stcg(ct + pos, pl.r0 + j);
+    }
+    written += tot;
   }
-  if (threadIdx.x == 0) __stcg(rw + kRowCnt + pl.c, total);
+  if (threadIdx.x == 0) __stcg(rw + kRowCnt + pl.c, written);
 }
 
 // ---------------------------------------------------------------------------
@@ -398,11 +438,9 @@ struct CandSrc {
 
 // digit histograms; leaves theta and ties_needed in sm
 __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff, void* ws_header) {
-  const int run = (P + kThreads - 1) / kThreads;
-  const int a = threadIdx.x * run, e = min(P, a + run);
   for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
-  for (int i = a; i < e; ++i) atomicAdd(&sm.hist[src.key(i) >> 20], 1u);
+  for (int i = threadIdx.x; i < P; i += kThreads) hist_add(sm.hist, src.key(i) >> 20);
   __syncthreads();
   select_bin(sm, kBins, keff);
   if (sm.sel_bin < 0) {  // fewer candidates than k_eff: cannot happen for a clean workspace
@@ -419,9 +457,9 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
   __syncthreads();
   for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
-  for (int i = a; i < e; ++i) {
+  for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = src.key(i);
-    if ((k >> 20) == t1) atomicAdd(&sm.hist[(k >> 8) & 0xFFFu], 1u);
+    if ((k >> 20) == t1) hist_add(sm.hist, (k >> 8) & 0xFFFu);
   }
   __syncthreads();
   select_bin(sm, kBins, need);
@@ -430,9 +468,9 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
   __syncthreads();
   for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
-  for (int i = a; i < e; ++i) {
+  for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = src.key(i);
-    if ((k >> 8) == p2) atomicAdd(&sm.hist[k & 0xFFu], 1u);
+    if ((k >> 8) == p2) hist_add(sm.hist, k & 0xFFu);
   }
   __syncthreads();
   select_bin(sm, 256, need);
@@ -447,33 +485,24 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
 __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& src, int P) {
   const Plan& pl = sm.plan;
   const uint32_t theta = sm.theta, ties = sm.ties_needed;
-  const int run = (P + kThreads - 1) / kThreads;
-  const int a = threadIdx.x * run, e = min(P, a + run);
-  uint32_t eq = 0;
-  for (int i = a; i < e; ++i) eq += src.key(i) == theta;
-  uint32_t tot;
-  uint32_t eq_rank = block_scan(eq, sm.warp_tot, &tot);
-  uint32_t sel = 0;
-  {
-    uint32_t r = eq_rank;
-    for (int i = a; i < e; ++i) {
-      const uint32_t k = src.key(i);
-      if (k > theta) ++sel;
-      else if (k == theta) sel += (r++ < ties);
-    }
-  }
-  uint32_t rank = block_scan(sel, sm.warp_tot, &tot);
   int32_t* out = p.idx + (size_t)pl.b * p.k;
-  uint32_t r = eq_rank;
-  for (int i = a; i < e; ++i) {
-    const uint32_t k = src.key(i);
-    bool s = k > theta;
-    if (k == theta) s = (r++ < ties);
-    if (!s) continue;
-    const int t = src.tok(i);
-    if ((int)rank >= pl.tok0 && (int)rank < pl.tok1) sm.unit_tok[rank - pl.tok0] = t;
-    if (t >= pl.r0 && t < pl.r1 && (int)rank < pl.keff) out[rank] = t;
-    ++rank;
+  uint32_t eq_seen = 0, sel_seen = 0;
+  for (int base = 0; base < P; base += kThreads) {
+    const int i = base + threadIdx.x;
+    const bool valid = i < P;
+    const uint32_t k = valid ? src.key(i) : 0u;
+    const bool gt = valid && k > theta, eq = valid && k == theta;
+    uint32_t eq_tot, s_tot;
+    const uint32_t er = eq_seen + block_flag_scan(eq, sm.warp_tot2, &eq_tot);
+    const bool s = gt || (eq && er < ties);
+    const uint32_t rank = sel_seen + block_flag_scan(s, sm.warp_tot2, &s_tot);
+    if (s) {
+      const int t = src.tok(i);
+      if ((int)rank >= pl.tok0 && (int)rank < pl.tok1) sm.unit_tok[rank - pl.tok0] = t;
+      if (t >= pl.r0 && t < pl.r1 && (int)rank < pl.keff) out[rank] = t;
+    }
+    eq_seen += eq_tot;
+    sel_seen += s_tot;
   }
   __syncthreads();
 }
@@ -564,6 +593,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
       cp_async_wait<0>();
     }
     __syncthreads();
+    if (bi == 0) stamp(p, 10);
     if (active) {
       const __nv_bfloat16* tk = sK + stage * kTokBlk * kSTR + set * NT * 8 * kSTR;
       const __nv_bfloat16* tv = sV + stage * kTokBlk * kSTR + set * NT * 8 * kSTR;
@@ -648,6 +678,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
     __syncthreads();
   }
 
+  stamp(p, 11);
   // ---- merge the NS token sets of each m-tile (thread-private slots in shared memory)
   float* xo = reinterpret_cast<float*>(big);                  // [NS-1][MT][64][32]
   float* xm = xo + (size_t)(NS - 1) * MT * 64 * 32;           // [NS-1][MT][4][32]
@@ -719,51 +750,91 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
 }
 
 // ---------------------------------------------------------------------------
-// phase 5: merge the nsplit partials of head g (rows r with r % nsplit == split)
+// phase 5: merge the nsplit partials of head g for rows r = split, split + nsplit, ...
+// Every (m, l) is staged first (one round trip), then each row's partial
+// vectors are fetched six at a time by up to kWarps / rows warps.
 // ---------------------------------------------------------------------------
-__device__ void combine_head(const FusedParams& p, const Plan& pl, int g) {
+__device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan& pl, int g) {
+  const int ns = pl.nsplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // split s of head g is CTA start + g * nsplit + s; its partial rows start at that CTA's slot
-  const size_t base = ((size_t)pl.start + (size_t)g * pl.nsplit) * p.rows;
-  for (int r = pl.split + warp * pl.nsplit; r < p.rows; r += kWarps * pl.nsplit) {
-    float M = -INFINITY;
-    for (int s = lane; s < pl.nsplit; s += 32) M = fmaxf(M, __ldcg(p.Ml + (base + (size_t)s * p.rows + r) * 2));
-    M = warp_max(M);
-    float den = 0.f;
-    float acc[kD / 32];
+  const int nr = (p.rows - pl.split + ns - 1) / ns;
+  if (nr <= 0) return;
+  const size_t cta0 = (size_t)pl.start + (size_t)g * ns;  // CTA holding split 0 of head g
+  for (int t = threadIdx.x; t < nr * ns; t += kThreads) {
+    const int ri = t / ns, s2 = t % ns;
+    const float2 ml =
+        __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
+    sm.cm[t] = ml.x;
+    sm.cl[t] = ml.y;
+  }
+  __syncthreads();
+  const int parts = nr >= kWarps ? 1 : kWarps / nr;
+  const int rows_per_pass = kWarps / parts;
+  float* stage = reinterpret_cast<float*>(big);  // [(parts-1) * rows_per_pass][kD]
+  const int part = warp % parts;
+  for (int rbase = 0; rbase < nr; rbase += rows_per_pass) {
+    const int slot = warp / parts;
+    const int ri = rbase + slot;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float M = -INFINITY, den = 0.f;
+    const bool live = ri < nr;
+    const int r = pl.split + ri * ns;
+    if (live) {
+      for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, sm.cm[ri * ns + s2]);
+      M = warp_max(M);
+      if (M != -INFINITY) {
+        for (int s2 = lane; s2 < ns; s2 += 32) den = fmaf(exp2f(sm.cm[ri * ns + s2] - M), sm.cl[ri * ns + s2], den);
+        den = warp_sum(den);
+        for (int s0 = part; s0 < ns; s0 += 6 * parts) {
+          float4 v[6];
+          float w[6];
 #pragma unroll
-    for (int c = 0; c < kD / 32; ++c) acc[c] = 0.f;
-    if (M != -INFINITY) {
-      for (int s0 = 0; s0 < pl.nsplit; s0 += 32) {
-        const int s = s0 + lane;
-        float w = 0.f;
-        if (s < pl.nsplit) {
-          const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + (base + (size_t)s * p.rows + r) * 2));
-          w = exp2f(ml.x - M);
-          den = fmaf(w, ml.y, den);
-        }
-        const int cnt = min(32, pl.nsplit - s0);
-#pragma unroll 4
-        for (int j = 0; j < cnt; ++j) {
-          const float wj = __shfl_sync(0xffffffffu, w, j);
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(p.Op + (base + (size_t)(s0 + j) * p.rows + r) * kD) + lane);
-          acc[0] = fmaf(wj, v.x, acc[0]);
-          acc[1] = fmaf(wj, v.y, acc[1]);
-          acc[2] = fmaf(wj, v.z, acc[2]);
-          acc[3] = fmaf(wj, v.w, acc[3]);
+          for (int u = 0; u < 6; ++u) {
+            const int s2 = s0 + u * parts;
+            if (s2 < ns) {
+              w[u] = exp2f(sm.cm[ri * ns + s2] - M);
+              v[u] = __ldcg(reinterpret_cast<const float4*>(p.Op + ((cta0 + s2) * p.rows + r) * kD) + lane);
+            } else {
+              w[u] = 0.f;
+              v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 6; ++u) {
+            acc[0] = fmaf(w[u], v[u].x, acc[0]);
+            acc[1] = fmaf(w[u], v[u].y, acc[1]);
+            acc[2] = fmaf(w[u], v[u].z, acc[2]);
+            acc[3] = fmaf(w[u], v[u].w, acc[3]);
+          }
         }
       }
-      den = warp_sum(den);
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const int l = r / p.G, h = g * p.G + r % p.G;
-    __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
-    uint2 wv;
-    wv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    wv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out) = wv;
-    if (p.lse && lane == 0)
-      p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+    if (parts > 1) {
+      if (live && part > 0)
+        *reinterpret_cast<float4*>(stage + ((size_t)(part - 1) * rows_per_pass + slot) * kD + lane * 4) =
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
+      __syncthreads();
+      if (live && part == 0)
+        for (int pp = 1; pp < parts; ++pp) {
+          const float4 o = *reinterpret_cast<const float4*>(stage + ((size_t)(pp - 1) * rows_per_pass + slot) * kD + lane * 4);
+          acc[0] += o.x;
+          acc[1] += o.y;
+          acc[2] += o.z;
+          acc[3] += o.w;
+        }
+    }
+    if (live && part == 0) {
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const int l = r / p.G, h = g * p.G + r % p.G;
+      __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
+      uint2 wv;
+      wv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      wv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      *reinterpret_cast<uint2*>(out) = wv;
+      if (p.lse && lane == 0)
+        p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+    }
+    __syncthreads();
   }
 }
 
@@ -821,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     write_candidates(p, sm);
     stamp(p, 2);
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
-    if (!group_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
+    if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
     stamp(p, 3);
     // everyone has read the partial histogram: clear this CTA's share for the next call
     {
@@ -845,18 +916,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     }
     uint32_t* skey = reinterpret_cast<uint32_t*>(big);
     int32_t* stok = reinterpret_cast<int32_t*>(big + kCandCap * 4);
-    if (sm.fast) {
+    if (sm.fast) {  // all candidates in flight at once: one round trip
       const uint32_t* gk = p.cand_key + (size_t)pl.b * p.n_max;
       const int32_t* gt = p.cand_tok + (size_t)pl.b * p.n_max;
-      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-      for (int c = warp; c < pl.Cb; c += kWarps) {
-        const int o = sm.seg_off[c], n = sm.seg_off[c + 1] - o;
-        const size_t src = (size_t)min(pl.len, c * chunk);
-        for (int i = lane; i < n; i += 32) {
-          skey[o + i] = __ldcg(gk + src + i);
-          stok[o + i] = __ldcg(gt + src + i);
+      const int ctot = sm.ctot;
+      for (int q = threadIdx.x; q < ctot; q += kThreads) {
+        int lo = 0, hi = pl.Cb - 1;  // last segment starting at or before q
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (sm.seg_off[mid] <= q) lo = mid;
+          else hi = mid - 1;
         }
+        const size_t src = (size_t)min(pl.len, lo * chunk) + (size_t)(q - sm.seg_off[lo]);
+        cp_async_4(skey + q, gk + src);
+        cp_async_4(stok + q, gt + src);
       }
+      cp_async_commit();
+      cp_async_wait<0>();
       __syncthreads();
     }
     CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
@@ -865,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
     stamp(p, 5);
     compact_selected(p, sm, src, P);
-    if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * 16 + 15] = (unsigned long long)sm.ctot | ((unsigned long long)sm.fast << 32);
+    if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + 31] = (unsigned long long)sm.ctot | ((unsigned long long)sm.fast << 32);
   }
   stamp(p, 6);
 
@@ -880,9 +956,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   stamp(p, 7);
   if (pl.nsplit > 1 && pl.nunits_here > 0) {
     uint32_t* hb = p.row_ws + (size_t)pl.b * kRowWords + kRowHeadBar + 2 * pl.unit_g0;
-    if (!group_barrier(hb, pl.nsplit, p.ws_header, 2)) return;
+    if (!count_barrier(hb, pl.nsplit, p.ws_header, 2)) return;
     stamp(p, 8);
-    combine_head(p, pl, pl.unit_g0);
+    combine_head(p, sm, big, pl, pl.unit_g0);
   }
   stamp(p, 9);
 }
@@ -921,7 +997,7 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   const FusedCfg cfg = fused_cfg();
   const size_t rows = (size_t)a->L * (a->Hq / a->Hkv);
   size_t off = 0;
-  off += (size_t)kMaxGroups * 16 * 8;                           // phase stamps (CLSA_TRACE=1)
+  off += (size_t)kMaxGroups * kTraceSlots * 8;                  // phase stamps (CLSA_TRACE=1)
   off += align_up((size_t)a->B * a->n_max * 4, 256);           // scores (when not an output)
   off += align_up((size_t)a->B * kRowWords * 4, 256);          // row state
   off += 2 * align_up((size_t)a->B * a->n_max * 4, 256);       // candidate keys + tokens
@@ -958,7 +1034,7 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   char* w = static_cast<char*>(ws_body);
   const char* tr = std::getenv("CLSA_TRACE");
   p.trace = (tr && tr[0] == '1') ? reinterpret_cast<unsigned long long*>(w) : nullptr;
-  w += (size_t)kMaxGroups * 16 * 8;
+  w += (size_t)kMaxGroups * kTraceSlots * 8;
   float* ws_scores = reinterpret_cast<float*>(w);
   w += align_up((size_t)a->B * a->n_max * 4, 256);
   p.scores = a->scores ? a->scores : ws_scores;
