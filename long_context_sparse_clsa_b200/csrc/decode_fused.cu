@@ -9,11 +9,12 @@
 // One CTA per SM.  Each sequence b gets a group of C_b CTAs, in proportion to its
 // length; CTA c of the group owns the contiguous token slice [r0, r1).
 //
-//  1. Scan.  The slice's K_idx rows stream into a 4-stage shared-memory ring
-//     through 1-D bulk copies (TMA engine, mbarrier completion, no multicast);
-//     16 lanes per 256-byte row compute the fp32 dot product.  Scores go to
-//     global memory (L2-resident).  The first half of the slice also feeds a
-//     12-bit histogram that is added to the group's global histogram.
+//  1. Scan.  16 lanes per 256-byte K_idx row, 16-byte non-allocating loads with
+//     8 rows in flight per lane group, fp32 dot product, shuffle reduce.  (Measured
+//     on B200: deep plain loads stream a 32 MiB slice set faster than a 1-D bulk-copy
+//     ring with one CTA per SM.)  Scores stay on chip and go to global memory
+//     (L2-resident).  The first half of the slice feeds a 12-bit histogram that is
+//     added to the group's global histogram before the second half is read.
 //  2. Candidate bound.  After its slice, a CTA reads the group histogram as it
 //     stands: whatever subset of tokens it counts, its k-th largest bin is a lower
 //     bound on the true k-th largest score, so every token of the true TopK scores
@@ -45,15 +46,14 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kStages = 4;
-constexpr int kStageBytes = 32 * 1024;
 constexpr int kBins = 4096;
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
 constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
 constexpr int kTokBlk = 64;           // tokens per attention block
 constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096); also slice scores kept on chip
-constexpr int kCandCap = 16384;       // candidates kept in shared memory (key + index)
+constexpr int kCandCap = 16384;       // candidate slots kept in shared memory (key + index)
+constexpr int kWin = 64;              // candidate window per CTA (more: the group takes the whole-row path)
 constexpr int kMaxGroups = 256;       // CTAs per launch
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -79,8 +79,8 @@ struct FusedParams {
   float* lse;
   float* scores;       // [B][n_max]
   uint32_t* row_ws;    // [B][kRowWords]
-  uint32_t* cand_key;  // [B][n_max]
-  int32_t* cand_tok;   // [B][n_max]
+  uint32_t* cand_key;  // [B][kMaxGroups][kWin]  candidate keys per CTA window (0 = empty slot)
+  int32_t* cand_tok;   // [B][kMaxGroups][kWin]
   float* Op;           // [gridDim][rows][D]  split partials, one slot per CTA
   float* Ml;           // [gridDim][rows][2]
   void* ws_header;
@@ -104,7 +104,6 @@ struct Plan {
 };
 
 struct Smem {
-  uint64_t bar[kStages];
   Plan plan;
   int abort_flag;
   uint32_t tau_key;
@@ -116,16 +115,23 @@ struct Smem {
   uint32_t warp_tot[kWarps];
   uint32_t warp_tot2[kWarps + 1];
   int seg_off[kMaxGroups + 1];
-  uint32_t hist[kBins];
-  union {                          // slice scores until the candidates are out, then unit tokens
-    float score[kMaxUnitTok];
+  __align__(16) uint32_t hist[kBins];
+  uint32_t red_min[kWarps], red_max[kWarps];
+  uint32_t theta_key, theta_pos;
+  int list_n;
+  union {                          // slice scores until the candidates are out, then the
+    float score[kMaxUnitTok];      // boundary-bin list of the selection, then unit tokens
     int unit_tok[kMaxUnitTok];
+    struct {
+      uint32_t list_key[1024];
+      int list_pos[1024];
+    };
   };
   float cm[512], cl[512];          // split-combine staging (m, l per row x split)
 };
-// dynamic shared memory: [Smem][sQ: kMaxRows x kSTR bf16][big: kStages x kStageBytes]
+// dynamic shared memory: [Smem][sQ: kMaxRows x kSTR bf16][big: 128 KiB, reused by phase]
 constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
-constexpr size_t kSmemBig = (size_t)kStages * kStageBytes;
+constexpr size_t kSmemBig = 128 * 1024;
 constexpr size_t smem_bytes() { return align_up(sizeof(Smem), 128) + kSmemQ + kSmemBig; }
 
 // ---------------------------------------------------------------------------
@@ -206,10 +212,53 @@ __device__ __forceinline__ uint32_t block_flag_scan(bool flag, uint32_t* warp_to
   return before;
 }
 
-// histogram increment, aggregated over the lanes of a warp that hit the same bin
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
-  const uint32_t m = __match_any_sync(__activemask(), bin);
-  if ((threadIdx.x & 31) == __ffs(m) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(m));
+// histogram increment (plain shared atomics measured ~9x faster here than warp aggregation)
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) { atomicAdd(&hist[bin], 1u); }
+
+// Find bin T with sum(hist[>T]) < need <= sum(hist[>=T]) for nbins in {2048, 4096}.
+// Warp w covers a contiguous range from the top, each lane a run of nbins/512 bins read
+// with 16-byte loads; two block syncs.  Writes sm.sel_bin (-1 if the total is below
+// need) and sm.sel_above.
+__device__ void select_bin_wide(Smem& sm, int nbins, uint32_t need) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int per_lane = nbins / kThreads;  // 4 or 8
+  const int hi = nbins - (w * 32 + lane) * per_lane;
+  uint32_t v[8];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    if (q * 4 < per_lane) {
+      const uint4 x = *reinterpret_cast<const uint4*>(&sm.hist[hi - per_lane + q * 4]);
+      v[q * 4 + 0] = x.x; v[q * 4 + 1] = x.y; v[q * 4 + 2] = x.z; v[q * 4 + 3] = x.w;
+    } else {
+      v[q * 4 + 0] = v[q * 4 + 1] = v[q * 4 + 2] = v[q * 4 + 3] = 0u;
+    }
+  }
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) local += v[i];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sm.warp_tot[w] = incl;
+  if (threadIdx.x == 0) sm.sel_bin = -1;
+  __syncthreads();
+  uint32_t before = incl - local;
+  for (int u = 0; u < w; ++u) before += sm.warp_tot[u];
+  if (before < need && need <= before + local) {
+    uint32_t acc = before;
+    for (int i = per_lane - 1; i >= 0; --i) {  // bins hi-1 down to hi-per_lane
+      if (acc + v[i] >= need) {
+        sm.sel_bin = hi - per_lane + i;
+        sm.sel_above = acc;
+        break;
+      }
+      acc += v[i];
+    }
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -271,24 +320,63 @@ __device__ __forceinline__ void abort_cta(Smem& sm, const FusedParams& p, int si
   sm.abort_flag = 1;
 }
 
+template <int DIDX>
+__device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, const __nv_bfloat16* src, float* sc,
+                                          const float (&q)[8], int j0, int j1, int nrows, bool hist) {
+  constexpr int LPR = DIDX / 8;                 // lanes per row (16-byte loads)
+  constexpr int GROUPS = kThreads / LPR;        // row groups per CTA
+  constexpr int U = 8;                          // rows in flight per group
+  const int grp = threadIdx.x / LPR, sub = threadIdx.x % LPR;
+  // the trip count is the same for every thread (the shuffles below need whole warps)
+  for (int base0 = j0; base0 < j1; base0 += GROUPS * U) {
+    const int base = base0 + grp;
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = base + u * GROUPS;
+      v[u] = j < j1 ? ld_stream_v4(src + (size_t)j * DIDX + sub * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = base + u * GROUPS;
+      float a0, a1, a2, a3, a4, a5, a6, a7;
+      unpack_bf16x2(v[u].x, a0, a1);
+      unpack_bf16x2(v[u].y, a2, a3);
+      unpack_bf16x2(v[u].z, a4, a5);
+      unpack_bf16x2(v[u].w, a6, a7);
+      float acc = q[0] * a0;
+      acc = fmaf(q[1], a1, acc);
+      acc = fmaf(q[2], a2, acc);
+      acc = fmaf(q[3], a3, acc);
+      acc = fmaf(q[4], a4, acc);
+      acc = fmaf(q[5], a5, acc);
+      acc = fmaf(q[6], a6, acc);
+      acc = fmaf(q[7], a7, acc);
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (sub == 0 && j < j1) {
+        __stcg(sc + j, acc);
+        if (nrows <= kMaxUnitTok) sm.score[j] = acc;
+        if (hist) atomicAdd(&sm.hist[float_key(acc) >> 20], 1u);
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
-// phase 1: streaming scan of the slice (bulk-copy ring)
+// phase 1: streaming scan of the slice.  Groups of DIDX/8 lanes own a row each
+// (16-byte non-allocating loads, 8 rows in flight per group), fp32 dot product,
+// shuffle reduce.  The first half of the slice feeds the 12-bit histogram, which
+// is published to the group before the second half is read.
 // ---------------------------------------------------------------------------
 template <int DIDX>
-__device__ bool scan_slice(const FusedParams& p, Smem& sm, unsigned char* ring, bool publish) {
-  constexpr int RB = DIDX * 2;                 // row bytes
-  constexpr int RPC = kStageBytes / RB;        // rows per chunk
-  constexpr int LPR = RB / 16;                 // lanes per row
-  constexpr int RPI = 32 / LPR;                // rows per warp instruction
+__device__ bool scan_slice(const FusedParams& p, Smem& sm, bool publish) {
   const Plan& pl = sm.plan;
   const int nrows = pl.r1 - pl.r0;
-  const int nchunks = (nrows + RPC - 1) / RPC;
-  const int half = publish ? (nchunks + 1) / 2 : 0;  // chunks [0, half) feed the histogram
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
   float* sc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = lane % LPR, rsub = lane / LPR;
-
+  constexpr int LPR = DIDX / 8;
+  const int sub = threadIdx.x % LPR;
   float q[8];
   {
     const uint4 qv = *reinterpret_cast<const uint4*>(p.q_idx + (size_t)pl.b * DIDX + sub * 8);
@@ -298,79 +386,23 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, unsigned char* ring, 
     unpack_bf16x2(qv.w, q[6], q[7]);
   }
   for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
-    fence_mbar_init();
-  }
   __syncthreads();
-  auto issue = [&](int ch) {  // thread 0 only
-    const int s = ch % kStages;
-    const int rows = min(RPC, nrows - ch * RPC);
-    const uint32_t bytes = (uint32_t)rows * RB;
-    mbar_arrive_expect_tx(&sm.bar[s], bytes);
-    bulk_g2s(ring + s * kStageBytes, src + (size_t)ch * RPC * DIDX, bytes, &sm.bar[s]);
-  };
-  if (threadIdx.x == 0)
-    for (int ch = 0; ch < min(kStages, nchunks); ++ch) issue(ch);
-
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const int s = ch % kStages;
-    const uint32_t parity = (ch / kStages) & 1;
-    if (!mbar_wait(&sm.bar[s], parity)) {
-      if (threadIdx.x == 0) abort_cta(sm, p, 100 + ch);
+  const int half = publish ? nrows / 2 : 0;
+  scan_rows<DIDX>(p, sm, src, sc, q, 0, half, nrows, true);
+  if (publish) {
+    __syncthreads();
+    uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) {
+      const uint32_t c = sm.hist[i];
+      if (c) atomicAdd(gh + i, c);  // relaxed reduction; ordered by the fence below
     }
     __syncthreads();
-    if (sm.abort_flag) return false;
-    const int rows = min(RPC, nrows - ch * RPC);
-    const unsigned char* buf = ring + s * kStageBytes;
-    for (int r = warp * RPI + rsub; r < RPC; r += kWarps * RPI) {
-      // every lane of the warp runs the shuffle; rows past the chunk contribute nothing
-      float acc = 0.f;
-      if (r < rows) {
-        const uint4 v = *reinterpret_cast<const uint4*>(buf + r * RB + sub * 16);
-        float a0, a1, a2, a3, a4, a5, a6, a7;
-        unpack_bf16x2(v.x, a0, a1);
-        unpack_bf16x2(v.y, a2, a3);
-        unpack_bf16x2(v.z, a4, a5);
-        unpack_bf16x2(v.w, a6, a7);
-        acc = q[0] * a0;
-        acc = fmaf(q[1], a1, acc);
-        acc = fmaf(q[2], a2, acc);
-        acc = fmaf(q[3], a3, acc);
-        acc = fmaf(q[4], a4, acc);
-        acc = fmaf(q[5], a5, acc);
-        acc = fmaf(q[6], a6, acc);
-        acc = fmaf(q[7], a7, acc);
-      }
-#pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (sub == 0 && r < rows) {
-        const int j = ch * RPC + r;
-        sc[j] = acc;
-        if (nrows <= kMaxUnitTok) sm.score[j] = acc;
-        if (ch < half) atomicAdd(&sm.hist[float_key(acc) >> 20], 1u);
-      }
-    }
-    __syncthreads();  // stage s fully read
-    if (threadIdx.x == 0 && ch + kStages < nchunks) {
-      fence_proxy_async_smem();
-      issue(ch + kStages);
-    }
-    if (ch == half - 1) {  // first half done: publish its histogram to the group
-      uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
-      for (int i = threadIdx.x; i < kBins; i += kThreads)
-        if (sm.hist[i]) atomicAdd(gh + i, sm.hist[i]);
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
-      }
+    if (threadIdx.x == 0) {
+      __threadfence();
+      red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
     }
   }
-  if (publish && nchunks == 0 && threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
-  }
+  scan_rows<DIDX>(p, sm, src, sc, q, half, nrows, nrows, false);
   __syncthreads();
   return true;
 }
@@ -387,19 +419,24 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm) {
     const uint32_t want = (uint32_t)(pl.Cb + 1) / 2;
     while (ld_acquire_gpu(rw + kRowArrive) < want && globaltimer_ns() - t0 < 20000ull) __nanosleep(64);
   }
+  stamp(p, 13);
   __syncthreads();
-  for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = __ldcg(rw + kRowHist + i);
+  for (int i = threadIdx.x; i < kBins / 4; i += kThreads) cp_async_16(&sm.hist[i * 4], rw + kRowHist + i * 4, 16);
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
-  select_bin(sm, kBins, (uint32_t)pl.keff);
+  stamp(p, 14);
+  select_bin_wide(sm, kBins, (uint32_t)pl.keff);
+  stamp(p, 16);
   if (threadIdx.x == 0) sm.tau_key = sm.sel_bin >= 0 ? ((uint32_t)sm.sel_bin << 20) : 0u;
   __syncthreads();
   const uint32_t tau = sm.tau_key;
-  // this CTA's tokens with key >= tau, in token order, to its segment
+  // this CTA's tokens with key >= tau, in token order, to its window of kWin slots
   const float* gsc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
   const int n = pl.r1 - pl.r0;
   const bool on_chip = n <= kMaxUnitTok;
-  uint32_t* ck = p.cand_key + (size_t)pl.b * p.n_max + pl.r0;
-  int32_t* ct = p.cand_tok + (size_t)pl.b * p.n_max + pl.r0;
+  uint32_t* ck = p.cand_key + ((size_t)pl.b * kMaxGroups + pl.c) * kWin;
+  int32_t* ct = p.cand_tok + ((size_t)pl.b * kMaxGroups + pl.c) * kWin;
   uint32_t written = 0;
   for (int base = 0; base < n; base += kThreads) {
     const int j = base + threadIdx.x;
@@ -411,13 +448,14 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm) {
     }
     uint32_t tot;
     const uint32_t pos = written + block_flag_scan(f, sm.warp_tot2, &tot);
-    if (f) {
+    if (f && pos < (uint32_t)kWin) {
       __stcg(ck + pos, key);
       __stcg(ct + pos, pl.r0 + j);
     }
     written += tot;
   }
-  if (threadIdx.x == 0) __stcg(rw + kRowCnt + pl.c, written);
+  for (int i = (int)written + threadIdx.x; i < kWin; i += kThreads) __stcg(ck + i, 0u);  // empty slots
+  if (threadIdx.x == 0) __stcg(rw + kRowCnt + pl.c, written);  // > kWin: overflow
 }
 
 // ---------------------------------------------------------------------------
@@ -442,7 +480,7 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
   __syncthreads();
   for (int i = threadIdx.x; i < P; i += kThreads) hist_add(sm.hist, src.key(i) >> 20);
   __syncthreads();
-  select_bin(sm, kBins, keff);
+  select_bin_wide(sm, kBins, keff);
   if (sm.sel_bin < 0) {  // fewer candidates than k_eff: cannot happen for a clean workspace
     if (threadIdx.x == 0) {
       record_error(ws_header, CLSA_ERR_BAD_INDEX, -1);
@@ -462,7 +500,7 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
     if ((k >> 20) == t1) hist_add(sm.hist, (k >> 8) & 0xFFFu);
   }
   __syncthreads();
-  select_bin(sm, kBins, need);
+  select_bin_wide(sm, kBins, need);
   const uint32_t p2 = (t1 << 12) | (uint32_t)sm.sel_bin;
   need -= sm.sel_above;
   __syncthreads();
@@ -503,6 +541,107 @@ __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& 
     }
     eq_seen += eq_tot;
     sel_seen += s_tot;
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// phase 3 (fast path): candidates on chip.  One histogram over 2048 bins that are
+// linear in key space between the smallest and the largest candidate key, a
+// two-sync search for the boundary bin, then an exact rank count inside that bin
+// (key descending, list position = token order ascending).  theta is the
+// (key, position) pair of the k_eff-th candidate.  False if the boundary bin holds
+// more than 1024 candidates (then the generic digit-by-digit path runs).
+// ---------------------------------------------------------------------------
+__device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_t keff) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = threadIdx.x; i < P; i += kThreads) {
+    const uint32_t k = skey[i];
+    if (k == 0u) continue;  // empty window slot
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sm.red_min[w] = kmin;
+    sm.red_max[w] = kmax;
+  }
+  for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0;
+  if (threadIdx.x == 0) sm.list_n = 0;
+  __syncthreads();
+  kmin = sm.red_min[0];
+  kmax = sm.red_max[0];
+  for (int u = 1; u < kWarps; ++u) {
+    kmin = min(kmin, sm.red_min[u]);
+    kmax = max(kmax, sm.red_max[u]);
+  }
+  int shift = 0;
+  while (((kmax - kmin) >> shift) >= 2048u) ++shift;
+  for (int i = threadIdx.x; i < P; i += kThreads) {
+    const uint32_t k = skey[i];
+    if (k != 0u) atomicAdd(&sm.hist[(k - kmin) >> shift], 1u);
+  }
+  __syncthreads();
+  select_bin_wide(sm, 2048, keff);
+  const int T = sm.sel_bin;
+  if (T < 0) return false;
+  const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
+  const uint32_t m = sm.hist[T];
+  if (m > 1024u) return false;
+  for (int i = threadIdx.x; i < P; i += kThreads) {
+    const uint32_t k = skey[i];
+    if (k != 0u && (int)((k - kmin) >> shift) == T) {
+      const int q = atomicAdd(&sm.list_n, 1);
+      sm.list_key[q] = k;
+      sm.list_pos[q] = i;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < (int)m; e += kThreads) {
+    const uint32_t ke = sm.list_key[e];
+    const int pe = sm.list_pos[e];
+    uint32_t r = 0;
+    for (int f = 0; f < (int)m; ++f) {
+      const uint32_t kf = sm.list_key[f];
+      r += kf > ke || (kf == ke && sm.list_pos[f] < pe);
+    }
+    if (r == need - 1) {
+      sm.theta_key = ke;
+      sm.theta_pos = (uint32_t)pe;
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+// selected iff key > theta_key, or key == theta_key at a position <= theta_pos
+__device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, const int32_t* stok,
+                                   int P) {
+  const Plan& pl = sm.plan;
+  const uint32_t tk = sm.theta_key, tp = sm.theta_pos;
+  int run = (P + kThreads - 1) / kThreads;
+  run += (run & 1) ^ 1;  // odd stride: the per-thread runs do not collide on shared-memory banks
+  const int a = threadIdx.x * run, e = min(P, a + run);
+  uint32_t mine = 0;
+  for (int i = a; i < e; ++i) {
+    const uint32_t k = skey[i];
+    mine += k > tk || (k == tk && (uint32_t)i <= tp);
+  }
+  uint32_t tot;
+  uint32_t rank = block_scan(mine, sm.warp_tot, &tot);
+  int32_t* out = p.idx + (size_t)pl.b * p.k;
+  for (int i = a; i < e; ++i) {
+    const uint32_t k = skey[i];
+    if (!(k > tk || (k == tk && (uint32_t)i <= tp))) continue;
+    const int t = stok[i];
+    if ((int)rank >= pl.tok0 && (int)rank < pl.tok1) sm.unit_tok[rank - pl.tok0] = t;
+    if (t >= pl.r0 && t < pl.r1 && (int)rank < pl.keff) out[rank] = t;
+    ++rank;
   }
   __syncthreads();
 }
@@ -880,7 +1019,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQ, MT * 16);  // lands during the scan
 
   const bool all_sel = pl.keff == pl.len;
-  if (!scan_slice<DIDX>(p, sm, big, !all_sel)) return;
+  if (!scan_slice<DIDX>(p, sm, !all_sel)) return;
   stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
@@ -900,47 +1039,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
       for (int i = pl.c * per + threadIdx.x; i < min(kBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
       if (pl.c == 0 && threadIdx.x == 0) rw[kRowArrive] = 0u;
     }
-    // segment offsets of the concatenated candidate list
-    const int chunk = (pl.len + pl.Cb - 1) / pl.Cb;
+    // candidate windows: every count (one load each), then every window (16-byte copies)
     {
       const uint32_t v = threadIdx.x < pl.Cb ? __ldcg(rw + kRowCnt + threadIdx.x) : 0u;
+      const bool over = __syncthreads_or(v > (uint32_t)kWin);
       uint32_t total;
-      const uint32_t before = block_scan(v, sm.warp_tot, &total);
-      if (threadIdx.x < pl.Cb) sm.seg_off[threadIdx.x] = (int)before;
+      block_scan(v, sm.warp_tot, &total);
       if (threadIdx.x == 0) {
-        sm.seg_off[pl.Cb] = (int)total;
         sm.ctot = (int)total;
-        sm.fast = total <= (uint32_t)kCandCap;
+        sm.fast = !over && pl.Cb * kWin <= kCandCap;
       }
       __syncthreads();
     }
     uint32_t* skey = reinterpret_cast<uint32_t*>(big);
     int32_t* stok = reinterpret_cast<int32_t*>(big + kCandCap * 4);
-    if (sm.fast) {  // all candidates in flight at once: one round trip
-      const uint32_t* gk = p.cand_key + (size_t)pl.b * p.n_max;
-      const int32_t* gt = p.cand_tok + (size_t)pl.b * p.n_max;
-      const int ctot = sm.ctot;
-      for (int q = threadIdx.x; q < ctot; q += kThreads) {
-        int lo = 0, hi = pl.Cb - 1;  // last segment starting at or before q
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (sm.seg_off[mid] <= q) lo = mid;
-          else hi = mid - 1;
-        }
-        const size_t src = (size_t)min(pl.len, lo * chunk) + (size_t)(q - sm.seg_off[lo]);
-        cp_async_4(skey + q, gk + src);
-        cp_async_4(stok + q, gt + src);
+    if (sm.fast) {
+      const uint4* gk = reinterpret_cast<const uint4*>(p.cand_key + (size_t)pl.b * kMaxGroups * kWin);
+      const uint4* gt = reinterpret_cast<const uint4*>(p.cand_tok + (size_t)pl.b * kMaxGroups * kWin);
+      const int nvec = pl.Cb * kWin / 4;
+      for (int i = threadIdx.x; i < nvec; i += kThreads) {
+        cp_async_16(skey + i * 4, gk + i, 16);
+        cp_async_16(stok + i * 4, gt + i, 16);
       }
       cp_async_commit();
       cp_async_wait<0>();
       __syncthreads();
     }
-    CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
-    const int P = sm.fast ? sm.ctot : pl.len;
     stamp(p, 4);
-    resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
-    stamp(p, 5);
-    compact_selected(p, sm, src, P);
+    bool done = false;
+    if (sm.fast) {
+      done = select_candidates(sm, skey, pl.Cb * kWin, (uint32_t)pl.keff);
+      stamp(p, 5);
+      if (done) compact_candidates(p, sm, skey, stok, pl.Cb * kWin);
+    }
+    if (!done) {  // a window overflowed, or a boundary bin of heavy ties: digit-by-digit select
+      CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
+      const int P = sm.fast ? pl.Cb * kWin : pl.len;
+      resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
+      stamp(p, 5);
+      compact_selected(p, sm, src, P);
+    }
     if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + 31] = (unsigned long long)sm.ctot | ((unsigned long long)sm.fast << 32);
   }
   stamp(p, 6);
@@ -1000,7 +1138,7 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   off += (size_t)kMaxGroups * kTraceSlots * 8;                  // phase stamps (CLSA_TRACE=1)
   off += align_up((size_t)a->B * a->n_max * 4, 256);           // scores (when not an output)
   off += align_up((size_t)a->B * kRowWords * 4, 256);          // row state
-  off += 2 * align_up((size_t)a->B * a->n_max * 4, 256);       // candidate keys + tokens
+  off += 2 * align_up((size_t)a->B * kMaxGroups * kWin * 4, 256);  // candidate windows
   off += align_up((size_t)cfg.ncta * rows * kD * 4, 256);      // split partials
   off += align_up((size_t)cfg.ncta * rows * 2 * 4, 256);
   return off;
@@ -1041,9 +1179,9 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   p.row_ws = reinterpret_cast<uint32_t*>(w);
   w += align_up((size_t)a->B * kRowWords * 4, 256);
   p.cand_key = reinterpret_cast<uint32_t*>(w);
-  w += align_up((size_t)a->B * a->n_max * 4, 256);
+  w += align_up((size_t)a->B * kMaxGroups * kWin * 4, 256);
   p.cand_tok = reinterpret_cast<int32_t*>(w);
-  w += align_up((size_t)a->B * a->n_max * 4, 256);
+  w += align_up((size_t)a->B * kMaxGroups * kWin * 4, 256);
   p.Op = reinterpret_cast<float*>(w);
   w += align_up((size_t)cfg.ncta * p.rows * kD * 4, 256);
   p.Ml = reinterpret_cast<float*>(w);
