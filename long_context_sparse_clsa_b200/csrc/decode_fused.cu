@@ -556,6 +556,7 @@ __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& 
 __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_t keff) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll 8
   for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = skey[i];
     if (k == 0u) continue;  // empty window slot
@@ -582,6 +583,7 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
   }
   int shift = 0;
   while (((kmax - kmin) >> shift) >= 2048u) ++shift;
+#pragma unroll 8
   for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = skey[i];
     if (k != 0u) atomicAdd(&sm.hist[(k - kmin) >> shift], 1u);
@@ -593,6 +595,7 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
   const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
   const uint32_t m = sm.hist[T];
   if (m > 1024u) return false;
+#pragma unroll 8
   for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = skey[i];
     if (k != 0u && (int)((k - kmin) >> shift) == T) {
@@ -619,26 +622,36 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
   return true;
 }
 
-// selected iff key > theta_key, or key == theta_key at a position <= theta_pos
+// selected iff key > theta_key, or key == theta_key at a position <= theta_pos.
+// Each thread owns a contiguous odd-length run (bank-conflict free), reads its keys
+// eight at a time into registers, keeps a bitmask of its selected slots, and after
+// one block scan visits only the selected ones.
 __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, const int32_t* stok,
                                    int P) {
   const Plan& pl = sm.plan;
   const uint32_t tk = sm.theta_key, tp = sm.theta_pos;
   int run = (P + kThreads - 1) / kThreads;
-  run += (run & 1) ^ 1;  // odd stride: the per-thread runs do not collide on shared-memory banks
-  const int a = threadIdx.x * run, e = min(P, a + run);
-  uint32_t mine = 0;
-  for (int i = a; i < e; ++i) {
-    const uint32_t k = skey[i];
-    mine += k > tk || (k == tk && (uint32_t)i <= tp);
+  run += (run & 1) ^ 1;
+  const int a = threadIdx.x * run;
+  uint64_t sel = 0;
+  for (int c0 = 0; c0 < run; c0 += 8) {
+    uint32_t k[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = a + c0 + u;
+      k[u] = (c0 + u < run && i < P) ? skey[i] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (k[u] > tk || (k[u] == tk && (uint32_t)(a + c0 + u) <= tp)) sel |= 1ull << (c0 + u);
   }
   uint32_t tot;
-  uint32_t rank = block_scan(mine, sm.warp_tot, &tot);
+  uint32_t rank = block_scan((uint32_t)__popcll(sel), sm.warp_tot, &tot);
   int32_t* out = p.idx + (size_t)pl.b * p.k;
-  for (int i = a; i < e; ++i) {
-    const uint32_t k = skey[i];
-    if (!(k > tk || (k == tk && (uint32_t)i <= tp))) continue;
-    const int t = stok[i];
+  while (sel) {
+    const int bit = __ffsll((long long)sel) - 1;
+    sel &= sel - 1;
+    const int t = stok[a + bit];
     if ((int)rank >= pl.tok0 && (int)rank < pl.tok1) sm.unit_tok[rank - pl.tok0] = t;
     if (t >= pl.r0 && t < pl.r1 && (int)rank < pl.keff) out[rank] = t;
     ++rank;
