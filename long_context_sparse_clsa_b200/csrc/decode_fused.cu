@@ -46,7 +46,9 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 4096;
+constexpr int kBins = 4096;          // digit histograms of the selection
+constexpr int kTauBits = 14;          // key bits of the candidate-bound histogram
+constexpr int kTauBins = 1 << kTauBits;
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
 constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
@@ -59,10 +61,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // per-row global state (u32 words)
-constexpr int kRowHist = 0;                       // [kBins] partial histogram (self-clearing)
-constexpr int kRowArrive = kBins;                 // CTAs that published their first half
-constexpr int kRowBar = kBins + 32;               // row-group barrier state [2]
-constexpr int kRowCnt = kBins + 64;               // [kMaxGroups] candidate count per CTA
+constexpr int kRowHist = 0;                       // [kTauBins] partial histogram (self-clearing)
+constexpr int kRowArrive = kTauBins;              // CTAs that published their first half
+constexpr int kRowBar = kTauBins + 32;            // row-group barrier state [2]
+constexpr int kRowCnt = kTauBins + 64;            // [kMaxGroups] candidate count per CTA
 constexpr int kRowHeadBar = kRowCnt + kMaxGroups; // [Hkv][2] head-group barrier states (<= 64 heads)
 constexpr int kRowWords = kRowHeadBar + 128;
 
@@ -215,27 +217,20 @@ __device__ __forceinline__ uint32_t block_flag_scan(bool flag, uint32_t* warp_to
 // histogram increment (plain shared atomics measured ~9x faster here than warp aggregation)
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) { atomicAdd(&hist[bin], 1u); }
 
-// Find bin T with sum(hist[>T]) < need <= sum(hist[>=T]) for nbins in {2048, 4096}.
-// Warp w covers a contiguous range from the top, each lane a run of nbins/512 bins read
-// with 16-byte loads; two block syncs.  Writes sm.sel_bin (-1 if the total is below
-// need) and sm.sel_above.
-__device__ void select_bin_wide(Smem& sm, int nbins, uint32_t need) {
+// Find bin T with sum(hist[>T]) < need <= sum(hist[>=T]) over hist[0, nbins), nbins a
+// multiple of 2048.  Warp w covers a contiguous range from the top, each lane a run of
+// nbins/512 bins read with 16-byte loads; two block syncs.  Writes sm.sel_bin (-1 if
+// the total is below need) and sm.sel_above.
+// With scale > 0 the target is max(1, floor(need * total * scale)), total = the histogram sum.
+__device__ void select_bin_wide(Smem& sm, const uint32_t* hist, int nbins, uint32_t need, float scale = 0.f) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int per_lane = nbins / kThreads;  // 4 or 8
+  const int per_lane = nbins / kThreads;
   const int hi = nbins - (w * 32 + lane) * per_lane;
-  uint32_t v[8];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    if (q * 4 < per_lane) {
-      const uint4 x = *reinterpret_cast<const uint4*>(&sm.hist[hi - per_lane + q * 4]);
-      v[q * 4 + 0] = x.x; v[q * 4 + 1] = x.y; v[q * 4 + 2] = x.z; v[q * 4 + 3] = x.w;
-    } else {
-      v[q * 4 + 0] = v[q * 4 + 1] = v[q * 4 + 2] = v[q * 4 + 3] = 0u;
-    }
-  }
   uint32_t local = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) local += v[i];
+  for (int q = 0; q < per_lane; q += 4) {
+    const uint4 x = *reinterpret_cast<const uint4*>(hist + hi - per_lane + q);
+    local += x.x + x.y + x.z + x.w;
+  }
   uint32_t incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -247,15 +242,21 @@ __device__ void select_bin_wide(Smem& sm, int nbins, uint32_t need) {
   __syncthreads();
   uint32_t before = incl - local;
   for (int u = 0; u < w; ++u) before += sm.warp_tot[u];
+  if (scale > 0.f) {
+    uint32_t total = 0;
+    for (int u = 0; u < kWarps; ++u) total += sm.warp_tot[u];
+    need = max(1u, (uint32_t)((float)need * (float)total * scale));
+  }
   if (before < need && need <= before + local) {
     uint32_t acc = before;
-    for (int i = per_lane - 1; i >= 0; --i) {  // bins hi-1 down to hi-per_lane
-      if (acc + v[i] >= need) {
-        sm.sel_bin = hi - per_lane + i;
+    for (int i = hi - 1; i >= hi - per_lane; --i) {
+      const uint32_t c = hist[i];
+      if (acc + c >= need) {
+        sm.sel_bin = i;
         sm.sel_above = acc;
         break;
       }
-      acc += v[i];
+      acc += c;
     }
   }
   __syncthreads();
@@ -321,8 +322,8 @@ __device__ __forceinline__ void abort_cta(Smem& sm, const FusedParams& p, int si
 }
 
 template <int DIDX>
-__device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, const __nv_bfloat16* src, float* sc,
-                                          const float (&q)[8], int j0, int j1, int nrows, bool hist) {
+__device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32_t* th, const __nv_bfloat16* src,
+                                          float* sc, const float (&q)[8], int j0, int j1, int nrows, bool hist) {
   constexpr int LPR = DIDX / 8;                 // lanes per row (16-byte loads)
   constexpr int GROUPS = kThreads / LPR;        // row groups per CTA
   constexpr int U = 8;                          // rows in flight per group
@@ -357,7 +358,7 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, const 
       if (sub == 0 && j < j1) {
         __stcg(sc + j, acc);
         if (nrows <= kMaxUnitTok) sm.score[j] = acc;
-        if (hist) atomicAdd(&sm.hist[float_key(acc) >> 20], 1u);
+        if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
       }
     }
   }
@@ -370,7 +371,7 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, const 
 // is published to the group before the second half is read.
 // ---------------------------------------------------------------------------
 template <int DIDX>
-__device__ bool scan_slice(const FusedParams& p, Smem& sm, bool publish) {
+__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool publish) {
   const Plan& pl = sm.plan;
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
@@ -385,15 +386,15 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, bool publish) {
     unpack_bf16x2(qv.z, q[4], q[5]);
     unpack_bf16x2(qv.w, q[6], q[7]);
   }
-  for (int i = threadIdx.x; i < kBins; i += kThreads) sm.hist[i] = 0;
+  for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
   const int half = publish ? nrows / 2 : 0;
-  scan_rows<DIDX>(p, sm, src, sc, q, 0, half, nrows, true);
+  scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
   if (publish) {
     __syncthreads();
     uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
-    for (int i = threadIdx.x; i < kBins; i += kThreads) {
-      const uint32_t c = sm.hist[i];
+    for (int i = threadIdx.x; i < kTauBins; i += kThreads) {
+      const uint32_t c = th[i];
       if (c) atomicAdd(gh + i, c);  // relaxed reduction; ordered by the fence below
     }
     __syncthreads();
@@ -402,7 +403,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, bool publish) {
       red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
     }
   }
-  scan_rows<DIDX>(p, sm, src, sc, q, half, nrows, nrows, false);
+  scan_rows<DIDX>(p, sm, th, src, sc, q, half, nrows, nrows, false);
   __syncthreads();
   return true;
 }
@@ -410,7 +411,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, bool publish) {
 // ---------------------------------------------------------------------------
 // phase 2: candidate bound tau from the group histogram, candidate segment
 // ---------------------------------------------------------------------------
-__device__ void write_candidates(const FusedParams& p, Smem& sm) {
+__device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   const Plan& pl = sm.plan;
   uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
   // wait briefly for half of the group's first halves (tau stays valid without it)
@@ -421,14 +422,16 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm) {
   }
   stamp(p, 13);
   __syncthreads();
-  for (int i = threadIdx.x; i < kBins / 4; i += kThreads) cp_async_16(&sm.hist[i * 4], rw + kRowHist + i * 4, 16);
+  for (int i = threadIdx.x; i < kTauBins / 4; i += kThreads) cp_async_16(th + i * 4, rw + kRowHist + i * 4, 16);
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
   stamp(p, 14);
-  select_bin_wide(sm, kBins, (uint32_t)pl.keff);
+  // aim at 80% of k_eff scaled to the share of the row the histogram has counted: the
+  // candidates then hold about 1.25 k_eff tokens; too few is caught after the barrier
+  select_bin_wide(sm, th, kTauBins, (uint32_t)pl.keff, 0.8f / (float)pl.len);
   stamp(p, 16);
-  if (threadIdx.x == 0) sm.tau_key = sm.sel_bin >= 0 ? ((uint32_t)sm.sel_bin << 20) : 0u;
+  if (threadIdx.x == 0) sm.tau_key = sm.sel_bin >= 0 ? ((uint32_t)sm.sel_bin << (32 - kTauBits)) : 0u;
   __syncthreads();
   const uint32_t tau = sm.tau_key;
   // this CTA's tokens with key >= tau, in token order, to its window of kWin slots
@@ -480,7 +483,7 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
   __syncthreads();
   for (int i = threadIdx.x; i < P; i += kThreads) hist_add(sm.hist, src.key(i) >> 20);
   __syncthreads();
-  select_bin_wide(sm, kBins, keff);
+  select_bin_wide(sm, sm.hist, kBins, keff);
   if (sm.sel_bin < 0) {  // fewer candidates than k_eff: cannot happen for a clean workspace
     if (threadIdx.x == 0) {
       record_error(ws_header, CLSA_ERR_BAD_INDEX, -1);
@@ -500,7 +503,7 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
     if ((k >> 20) == t1) hist_add(sm.hist, (k >> 8) & 0xFFFu);
   }
   __syncthreads();
-  select_bin_wide(sm, kBins, need);
+  select_bin_wide(sm, sm.hist, kBins, need);
   const uint32_t p2 = (t1 << 12) | (uint32_t)sm.sel_bin;
   need -= sm.sel_above;
   __syncthreads();
@@ -589,7 +592,7 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
     if (k != 0u) atomicAdd(&sm.hist[(k - kmin) >> shift], 1u);
   }
   __syncthreads();
-  select_bin_wide(sm, 2048, keff);
+  select_bin_wide(sm, sm.hist, 2048, keff);
   const int T = sm.sel_bin;
   if (T < 0) return false;
   const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
@@ -1032,7 +1035,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQ, MT * 16);  // lands during the scan
 
   const bool all_sel = pl.keff == pl.len;
-  if (!scan_slice<DIDX>(p, sm, !all_sel)) return;
+  if (!scan_slice<DIDX>(p, sm, reinterpret_cast<uint32_t*>(big), !all_sel)) return;
   stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
@@ -1041,38 +1044,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     for (int i = threadIdx.x; i < pl.tok1 - pl.tok0; i += kThreads) sm.unit_tok[i] = pl.tok0 + i;
     __syncthreads();
   } else {
-    write_candidates(p, sm);
+    write_candidates(p, sm, reinterpret_cast<uint32_t*>(big));
     stamp(p, 2);
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
     stamp(p, 3);
     // everyone has read the partial histogram: clear this CTA's share for the next call
     {
-      const int per = (kBins + pl.Cb - 1) / pl.Cb;
-      for (int i = pl.c * per + threadIdx.x; i < min(kBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
+      const int per = (kTauBins + pl.Cb - 1) / pl.Cb;
+      for (int i = pl.c * per + threadIdx.x; i < min(kTauBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
       if (pl.c == 0 && threadIdx.x == 0) rw[kRowArrive] = 0u;
     }
-    // candidate windows: every count (one load each), then every window (16-byte copies)
+    // candidate windows: every count (one load each), then every valid slot copied to a
+    // dense list in window order (= token order), all copies in flight at once
     {
       const uint32_t v = threadIdx.x < pl.Cb ? __ldcg(rw + kRowCnt + threadIdx.x) : 0u;
       const bool over = __syncthreads_or(v > (uint32_t)kWin);
       uint32_t total;
-      block_scan(v, sm.warp_tot, &total);
+      const uint32_t before = block_scan(v, sm.warp_tot, &total);
+      if (threadIdx.x < pl.Cb) sm.seg_off[threadIdx.x] = (int)before;
       if (threadIdx.x == 0) {
+        sm.seg_off[pl.Cb] = (int)total;
         sm.ctot = (int)total;
-        sm.fast = !over && pl.Cb * kWin <= kCandCap;
+        // too few candidates (the scaled bound overshot) or a full window: whole-row path
+        sm.fast = !over && total >= (uint32_t)pl.keff && total <= (uint32_t)kCandCap;
       }
       __syncthreads();
     }
     uint32_t* skey = reinterpret_cast<uint32_t*>(big);
     int32_t* stok = reinterpret_cast<int32_t*>(big + kCandCap * 4);
     if (sm.fast) {
-      const uint4* gk = reinterpret_cast<const uint4*>(p.cand_key + (size_t)pl.b * kMaxGroups * kWin);
-      const uint4* gt = reinterpret_cast<const uint4*>(p.cand_tok + (size_t)pl.b * kMaxGroups * kWin);
-      const int nvec = pl.Cb * kWin / 4;
-      for (int i = threadIdx.x; i < nvec; i += kThreads) {
-        cp_async_16(skey + i * 4, gk + i, 16);
-        cp_async_16(stok + i * 4, gt + i, 16);
+      const uint32_t* gk = p.cand_key + (size_t)pl.b * kMaxGroups * kWin;
+      const int32_t* gt = p.cand_tok + (size_t)pl.b * kMaxGroups * kWin;
+      for (int slot = threadIdx.x; slot < pl.Cb * kWin; slot += kThreads) {
+        const int c = slot / kWin, i = slot % kWin;
+        const int o = sm.seg_off[c];
+        if (i < sm.seg_off[c + 1] - o) {
+          cp_async_4(skey + o + i, gk + slot);
+          cp_async_4(stok + o + i, gt + slot);
+        }
       }
       cp_async_commit();
       cp_async_wait<0>();
@@ -1081,13 +1091,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     stamp(p, 4);
     bool done = false;
     if (sm.fast) {
-      done = select_candidates(sm, skey, pl.Cb * kWin, (uint32_t)pl.keff);
+      done = select_candidates(sm, skey, sm.ctot, (uint32_t)pl.keff);
       stamp(p, 5);
-      if (done) compact_candidates(p, sm, skey, stok, pl.Cb * kWin);
+      if (done) compact_candidates(p, sm, skey, stok, sm.ctot);
     }
     if (!done) {  // a window overflowed, or a boundary bin of heavy ties: digit-by-digit select
       CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
-      const int P = sm.fast ? pl.Cb * kWin : pl.len;
+      const int P = sm.fast ? sm.ctot : pl.len;
       resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
       stamp(p, 5);
       compact_selected(p, sm, src, P);
