@@ -62,9 +62,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 // per-row global state (u32 words)
 constexpr int kRowHist = 0;                       // [kTauBins] partial histogram (self-clearing)
-constexpr int kRowArrive = kTauBins;              // CTAs that published their first half
-constexpr int kRowBar = kTauBins + 32;            // row-group barrier state [2]
-constexpr int kRowCnt = kTauBins + 64;            // [kMaxGroups] candidate count per CTA
+constexpr int kRowCoarse = kTauBins;              // [256] the same histogram, 64 fine bins per bin
+constexpr int kRowArrive = kTauBins + 256;        // CTAs that published their first half
+constexpr int kRowBar = kTauBins + 256 + 32;      // row-group barrier state [2]
+constexpr int kRowCnt = kTauBins + 256 + 64;      // [kMaxGroups] candidate count per CTA
 constexpr int kRowHeadBar = kRowCnt + kMaxGroups; // [Hkv][2] head-group barrier states (<= 64 heads)
 constexpr int kRowWords = kRowHeadBar + 128;
 
@@ -358,7 +359,11 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
       if (sub == 0 && j < j1) {
         __stcg(sc + j, acc);
         if (nrows <= kMaxUnitTok) sm.score[j] = acc;
-        if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
+        if (hist) {
+          const uint32_t fb = float_key(acc) >> (32 - kTauBits);
+          atomicAdd(&th[fb], 1u);
+          atomicAdd(&sm.hist[fb >> 6], 1u);
+        }
       }
     }
   }
@@ -387,6 +392,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
     unpack_bf16x2(qv.w, q[6], q[7]);
   }
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
+  for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
   const int half = publish ? nrows / 2 : 0;
   scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
@@ -396,6 +402,10 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
     for (int i = threadIdx.x; i < kTauBins; i += kThreads) {
       const uint32_t c = th[i];
       if (c) atomicAdd(gh + i, c);  // relaxed reduction; ordered by the fence below
+    }
+    for (int i = threadIdx.x; i < 256; i += kThreads) {
+      const uint32_t c = sm.hist[i];
+      if (c) atomicAdd(gh + kRowCoarse + i, c);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -422,16 +432,69 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   }
   stamp(p, 13);
   __syncthreads();
-  for (int i = threadIdx.x; i < kTauBins / 4; i += kThreads) cp_async_16(th + i * 4, rw + kRowHist + i * 4, 16);
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
+  // The bound: the bin where the count from the top reaches 1.25 k_eff scaled to the share
+  // of the row counted so far (then the candidates hold about 1.25 k_eff tokens; too few is
+  // caught after the barrier).  Warp 0 finds the coarse bin, then the fine bin inside it.
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    uint32_t c8[8];
+    {
+      const uint4 x = __ldcg(reinterpret_cast<const uint4*>(rw + kRowCoarse + 256 - 8 * (lane + 1)));
+      const uint4 y = __ldcg(reinterpret_cast<const uint4*>(rw + kRowCoarse + 256 - 8 * (lane + 1) + 4));
+      c8[0] = x.x; c8[1] = x.y; c8[2] = x.z; c8[3] = x.w; c8[4] = y.x; c8[5] = y.y; c8[6] = y.z; c8[7] = y.w;
+    }
+    uint32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) local += c8[i];
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t need = max(1u, (uint32_t)(1.25f * (float)pl.keff * (float)total / (float)pl.len));
+    const uint32_t before = incl - local;
+    int tc = -1;
+    uint32_t above = 0;
+    if (before < need && need <= incl) {
+      uint32_t acc = before;
+      for (int i = 7; i >= 0; --i) {  // bins from the top of this lane's run
+        if (acc + c8[i] >= need) {
+          tc = 256 - 8 * (lane + 1) + i;
+          above = acc;
+          break;
+        }
+        acc += c8[i];
+      }
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, tc >= 0);
+    uint32_t tau = 0u;  // everything is a candidate when too few tokens were counted
+    if (hit) {
+      const int src_lane = __ffs(hit) - 1;
+      tc = __shfl_sync(0xffffffffu, tc, src_lane);
+      above = __shfl_sync(0xffffffffu, above, src_lane);
+      // the 64 fine bins of coarse bin tc, two per lane from the top
+      const uint2 f2 = __ldcg(reinterpret_cast<const uint2*>(rw + kRowHist + tc * 64 + 62 - 2 * lane));
+      const uint32_t fl = f2.x + f2.y;
+      uint32_t fi = fl;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, fi, o);
+        if (lane >= o) fi += y;
+      }
+      const uint32_t fb = above + fi - fl;
+      int tf = -1;
+      if (fb < need && need <= fb + fl) tf = (fb + f2.y >= need) ? 63 - 2 * lane : 62 - 2 * lane;
+      const uint32_t fh = __ballot_sync(0xffffffffu, tf >= 0);
+      if (fh) tf = __shfl_sync(0xffffffffu, tf, __ffs(fh) - 1);
+      else tf = 0;
+      tau = ((uint32_t)(tc * 64 + tf)) << (32 - kTauBits);
+    }
+    if (lane == 0) sm.tau_key = tau;
+  }
   stamp(p, 14);
-  // aim at 80% of k_eff scaled to the share of the row the histogram has counted: the
-  // candidates then hold about 1.25 k_eff tokens; too few is caught after the barrier
-  select_bin_wide(sm, th, kTauBins, (uint32_t)pl.keff, 0.8f / (float)pl.len);
   stamp(p, 16);
-  if (threadIdx.x == 0) sm.tau_key = sm.sel_bin >= 0 ? ((uint32_t)sm.sel_bin << (32 - kTauBits)) : 0u;
   __syncthreads();
   const uint32_t tau = sm.tau_key;
   // this CTA's tokens with key >= tau, in token order, to its window of kWin slots
@@ -1053,6 +1116,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     {
       const int per = (kTauBins + pl.Cb - 1) / pl.Cb;
       for (int i = pl.c * per + threadIdx.x; i < min(kTauBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
+      if (pl.c == 0 && threadIdx.x < 256) rw[kRowCoarse + threadIdx.x] = 0u;
       if (pl.c == 0 && threadIdx.x == 0) rw[kRowArrive] = 0u;
     }
     // candidate windows: every count (one load each), then every valid slot copied to a
