@@ -242,11 +242,16 @@ __device__ void select_bin_wide(Smem& sm, const uint32_t* hist, int nbins, uint3
   if (threadIdx.x == 0) sm.sel_bin = -1;
   __syncthreads();
   uint32_t before = incl - local;
-  for (int u = 0; u < w; ++u) before += sm.warp_tot[u];
-  if (scale > 0.f) {
-    uint32_t total = 0;
-    for (int u = 0; u < kWarps; ++u) total += sm.warp_tot[u];
-    need = max(1u, (uint32_t)((float)need * (float)total * scale));
+  {
+    const uint32_t wt = lane < kWarps ? sm.warp_tot[lane] : 0u;
+    uint32_t pre = lane < w ? wt : 0u, total = wt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      pre += __shfl_xor_sync(0xffffffffu, pre, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+    }
+    before += pre;
+    if (scale > 0.f) need = max(1u, (uint32_t)((float)need * (float)total * scale));
   }
   if (before < need && need <= before + local) {
     uint32_t acc = before;
@@ -323,58 +328,64 @@ __device__ __forceinline__ void abort_cta(Smem& sm, const FusedParams& p, int si
 }
 
 template <int DIDX>
+__device__ __forceinline__ float row_dot(const uint4 v, const float (&q)[8]) {
+  float a0, a1, a2, a3, a4, a5, a6, a7;
+  unpack_bf16x2(v.x, a0, a1);
+  unpack_bf16x2(v.y, a2, a3);
+  unpack_bf16x2(v.z, a4, a5);
+  unpack_bf16x2(v.w, a6, a7);
+  float acc = q[0] * a0;
+  acc = fmaf(q[1], a1, acc);
+  acc = fmaf(q[2], a2, acc);
+  acc = fmaf(q[3], a3, acc);
+  acc = fmaf(q[4], a4, acc);
+  acc = fmaf(q[5], a5, acc);
+  acc = fmaf(q[6], a6, acc);
+  acc = fmaf(q[7], a7, acc);
+  return acc;
+}
+
+// Rows [j0, j1) of the slice; the loads of the next batch of U rows per group are in
+// flight while the current batch is reduced.
+template <int DIDX>
 __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32_t* th, const __nv_bfloat16* src,
                                           float* sc, const float (&q)[8], int j0, int j1, int nrows, bool hist) {
   constexpr int LPR = DIDX / 8;                 // lanes per row (16-byte loads)
   constexpr int GROUPS = kThreads / LPR;        // row groups per CTA
   constexpr int U = 8;                          // rows in flight per group
   const int grp = threadIdx.x / LPR, sub = threadIdx.x % LPR;
-  // the trip count is the same for every thread (the shuffles below need whole warps)
-  for (int base0 = j0; base0 < j1; base0 += GROUPS * U) {
-    const int base = base0 + grp;
-    uint4 v[U];
+  auto load = [&](uint4 (&v)[U], int base0) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int j = base + u * GROUPS;
+      const int j = base0 + grp + u * GROUPS;
       v[u] = j < j1 ? ld_stream_v4(src + (size_t)j * DIDX + sub * 8) : make_uint4(0, 0, 0, 0);
     }
+  };
+  uint4 cur[U], nxt[U];
+  if (j0 < j1) load(cur, j0);
+  // the trip count is the same for every thread (the shuffles below need whole warps)
+  for (int base0 = j0; base0 < j1; base0 += GROUPS * U) {
+    const bool more = base0 + GROUPS * U < j1;
+    if (more) load(nxt, base0 + GROUPS * U);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int j = base + u * GROUPS;
-      float a0, a1, a2, a3, a4, a5, a6, a7;
-      unpack_bf16x2(v[u].x, a0, a1);
-      unpack_bf16x2(v[u].y, a2, a3);
-      unpack_bf16x2(v[u].z, a4, a5);
-      unpack_bf16x2(v[u].w, a6, a7);
-      float acc = q[0] * a0;
-      acc = fmaf(q[1], a1, acc);
-      acc = fmaf(q[2], a2, acc);
-      acc = fmaf(q[3], a3, acc);
-      acc = fmaf(q[4], a4, acc);
-      acc = fmaf(q[5], a5, acc);
-      acc = fmaf(q[6], a6, acc);
-      acc = fmaf(q[7], a7, acc);
+      const int j = base0 + grp + u * GROUPS;
+      float acc = row_dot<DIDX>(cur[u], q);
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (sub == 0 && j < j1) {
         __stcg(sc + j, acc);
         if (nrows <= kMaxUnitTok) sm.score[j] = acc;
-        if (hist) {
-          const uint32_t fb = float_key(acc) >> (32 - kTauBits);
-          atomicAdd(&th[fb], 1u);
-          atomicAdd(&sm.hist[fb >> 6], 1u);
-        }
+        if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
       }
+    }
+    if (more) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) cur[u] = nxt[u];
     }
   }
 }
 
-// ---------------------------------------------------------------------------
-// phase 1: streaming scan of the slice.  Groups of DIDX/8 lanes own a row each
-// (16-byte non-allocating loads, 8 rows in flight per group), fp32 dot product,
-// shuffle reduce.  The first half of the slice feeds the 12-bit histogram, which
-// is published to the group before the second half is read.
-// ---------------------------------------------------------------------------
 template <int DIDX>
 __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool publish) {
   const Plan& pl = sm.plan;
@@ -392,25 +403,33 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
     unpack_bf16x2(qv.w, q[6], q[7]);
   }
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
-  for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
   const int half = publish ? nrows / 2 : 0;
   scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
   if (publish) {
     __syncthreads();
-    uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
-    for (int i = threadIdx.x; i < kTauBins; i += kThreads) {
-      const uint32_t c = th[i];
-      if (c) atomicAdd(gh + i, c);  // relaxed reduction; ordered by the fence below
-    }
-    for (int i = threadIdx.x; i < 256; i += kThreads) {
-      const uint32_t c = sm.hist[i];
-      if (c) atomicAdd(gh + kRowCoarse + i, c);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
+    // the last warp publishes the first-half histogram (fine bins and 64-bin coarse
+    // sums) while the other warps read the second half
+    if ((threadIdx.x >> 5) == kWarps - 1) {
+      const int lane = threadIdx.x & 31;
+      uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
+      for (int cb = lane; cb < kTauBins / 64; cb += 32) {
+        uint32_t sum = 0;
+        for (int i = 0; i < 64; i += 4) {
+          const uint4 x = *reinterpret_cast<const uint4*>(th + cb * 64 + i);
+          if (x.x) atomicAdd(gh + cb * 64 + i, x.x);
+          if (x.y) atomicAdd(gh + cb * 64 + i + 1, x.y);
+          if (x.z) atomicAdd(gh + cb * 64 + i + 2, x.z);
+          if (x.w) atomicAdd(gh + cb * 64 + i + 3, x.w);
+          sum += x.x + x.y + x.z + x.w;
+        }
+        if (sum) atomicAdd(gh + kRowCoarse + cb, sum);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
+      }
     }
   }
   scan_rows<DIDX>(p, sm, th, src, sc, q, half, nrows, nrows, false);
@@ -641,11 +660,12 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
   for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0;
   if (threadIdx.x == 0) sm.list_n = 0;
   __syncthreads();
-  kmin = sm.red_min[0];
-  kmax = sm.red_max[0];
-  for (int u = 1; u < kWarps; ++u) {
-    kmin = min(kmin, sm.red_min[u]);
-    kmax = max(kmax, sm.red_max[u]);
+  kmin = lane < kWarps ? sm.red_min[lane] : 0xFFFFFFFFu;
+  kmax = lane < kWarps ? sm.red_max[lane] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
   int shift = 0;
   while (((kmax - kmin) >> shift) >= 2048u) ++shift;
@@ -964,6 +984,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
       }
     }
   }
+  stamp(p, 12);
   __syncthreads();
 }
 
@@ -973,6 +994,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
 // vectors are fetched six at a time by up to kWarps / rows warps.
 // ---------------------------------------------------------------------------
 __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan& pl, int g) {
+  stamp(p, 18);
   const int ns = pl.nsplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nr = (p.rows - pl.split + ns - 1) / ns;
@@ -986,6 +1008,7 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
     sm.cl[t] = ml.y;
   }
   __syncthreads();
+  stamp(p, 17);
   const int parts = nr >= kWarps ? 1 : kWarps / nr;
   const int rows_per_pass = kWarps / parts;
   float* stage = reinterpret_cast<float*>(big);  // [(parts-1) * rows_per_pass][kD]
@@ -1140,12 +1163,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     if (sm.fast) {
       const uint32_t* gk = p.cand_key + (size_t)pl.b * kMaxGroups * kWin;
       const int32_t* gt = p.cand_tok + (size_t)pl.b * kMaxGroups * kWin;
-      for (int slot = threadIdx.x; slot < pl.Cb * kWin; slot += kThreads) {
-        const int c = slot / kWin, i = slot % kWin;
-        const int o = sm.seg_off[c];
-        if (i < sm.seg_off[c + 1] - o) {
-          cp_async_4(skey + o + i, gk + slot);
-          cp_async_4(stok + o + i, gt + slot);
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+      for (int c = warp; c < pl.Cb; c += kWarps) {  // one warp per window
+        const int o = sm.seg_off[c], n = sm.seg_off[c + 1] - o;
+        for (int i = lane; i < n; i += 32) {
+          cp_async_4(skey + o + i, gk + c * kWin + i);
+          cp_async_4(stok + o + i, gt + c * kWin + i);
         }
       }
       cp_async_commit();
