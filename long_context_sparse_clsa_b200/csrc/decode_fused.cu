@@ -406,30 +406,26 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
   __syncthreads();
   const int half = publish ? nrows / 2 : 0;
   scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
-  if (publish) {
+  if (publish) {  // first-half histogram (fine bins, and coarse sums of 64) to the group
+    for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[i] = 0;
     __syncthreads();
-    // the last warp publishes the first-half histogram (fine bins and 64-bin coarse
-    // sums) while the other warps read the second half
-    if ((threadIdx.x >> 5) == kWarps - 1) {
-      const int lane = threadIdx.x & 31;
-      uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
-      for (int cb = lane; cb < kTauBins / 64; cb += 32) {
-        uint32_t sum = 0;
-        for (int i = 0; i < 64; i += 4) {
-          const uint4 x = *reinterpret_cast<const uint4*>(th + cb * 64 + i);
-          if (x.x) atomicAdd(gh + cb * 64 + i, x.x);
-          if (x.y) atomicAdd(gh + cb * 64 + i + 1, x.y);
-          if (x.z) atomicAdd(gh + cb * 64 + i + 2, x.z);
-          if (x.w) atomicAdd(gh + cb * 64 + i + 3, x.w);
-          sum += x.x + x.y + x.z + x.w;
-        }
-        if (sum) atomicAdd(gh + kRowCoarse + cb, sum);
-      }
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence();
-        red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
-      }
+    uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
+    for (int v = threadIdx.x; v < kTauBins / 4; v += kThreads) {  // consecutive threads, consecutive bins
+      const uint4 x = *reinterpret_cast<const uint4*>(th + v * 4);
+      if (x.x) atomicAdd(gh + v * 4, x.x);
+      if (x.y) atomicAdd(gh + v * 4 + 1, x.y);
+      if (x.z) atomicAdd(gh + v * 4 + 2, x.z);
+      if (x.w) atomicAdd(gh + v * 4 + 3, x.w);
+      const uint32_t sum = x.x + x.y + x.z + x.w;
+      if (sum) atomicAdd(&sm.hist[(v * 4) >> 6], sum);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += kThreads)
+      if (sm.hist[i]) atomicAdd(gh + kRowCoarse + i, sm.hist[i]);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
     }
   }
   scan_rows<DIDX>(p, sm, th, src, sc, q, half, nrows, nrows, false);
@@ -443,11 +439,12 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
 __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   const Plan& pl = sm.plan;
   uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
-  // wait briefly for half of the group's first halves (tau stays valid without it)
+  // wait briefly for a quarter of the group's first halves: the bound is scaled to the
+  // share it has counted, so a smaller sample only widens the candidate count's spread
   if (threadIdx.x == 0) {
     const unsigned long long t0 = globaltimer_ns();
-    const uint32_t want = (uint32_t)(pl.Cb + 1) / 2;
-    while (ld_acquire_gpu(rw + kRowArrive) < want && globaltimer_ns() - t0 < 20000ull) __nanosleep(64);
+    const uint32_t want = (uint32_t)(pl.Cb + 3) / 4;
+    while (ld_acquire_gpu(rw + kRowArrive) < want && globaltimer_ns() - t0 < 5000ull) __nanosleep(32);
   }
   stamp(p, 13);
   __syncthreads();
