@@ -416,8 +416,11 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
       if (x.y) atomicAdd(gh + v * 4 + 1, x.y);
       if (x.z) atomicAdd(gh + v * 4 + 2, x.z);
       if (x.w) atomicAdd(gh + v * 4 + 3, x.w);
-      const uint32_t sum = x.x + x.y + x.z + x.w;
-      if (sum) atomicAdd(&sm.hist[(v * 4) >> 6], sum);
+      // the 16 threads of a half-warp hold the 64 fine bins of one coarse bin: sum first
+      uint32_t sum = x.x + x.y + x.z + x.w;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if ((threadIdx.x & 15) == 0 && sum) atomicAdd(&sm.hist[(v * 4) >> 6], sum);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < 256; i += kThreads)
