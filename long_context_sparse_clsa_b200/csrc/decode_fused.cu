@@ -407,7 +407,6 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
   const int half = publish ? nrows / 2 : 0;
   scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
   if (publish) {  // first-half histogram (fine bins, and coarse sums of 64) to the group
-    for (int i = threadIdx.x; i < 256; i += kThreads) sm.hist[i] = 0;
     __syncthreads();
     uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
     for (int v = threadIdx.x; v < kTauBins / 4; v += kThreads) {  // consecutive threads, consecutive bins
@@ -416,15 +415,12 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
       if (x.y) atomicAdd(gh + v * 4 + 1, x.y);
       if (x.z) atomicAdd(gh + v * 4 + 2, x.z);
       if (x.w) atomicAdd(gh + v * 4 + 3, x.w);
-      // the 16 threads of a half-warp hold the 64 fine bins of one coarse bin: sum first
+      // the 16 threads of a half-warp hold exactly the 64 fine bins of one coarse bin
       uint32_t sum = x.x + x.y + x.z + x.w;
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if ((threadIdx.x & 15) == 0 && sum) atomicAdd(&sm.hist[(v * 4) >> 6], sum);
+      if ((threadIdx.x & 15) == 0 && sum) atomicAdd(gh + kRowCoarse + ((v * 4) >> 6), sum);
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += kThreads)
-      if (sm.hist[i]) atomicAdd(gh + kRowCoarse + i, sm.hist[i]);
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
