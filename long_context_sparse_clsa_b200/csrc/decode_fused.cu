@@ -406,25 +406,32 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
   __syncthreads();
   const int half = publish ? nrows / 2 : 0;
   scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
-  if (publish) {  // first-half histogram (fine bins, and coarse sums of 64) to the group
+  if (publish) {
+    // First-half histogram (fine bins, and coarse sums of 64) to the group.  The last four
+    // warps publish (named barrier 1 among them) while the other warps start the second
+    // half; the publishers join the scan afterwards.
     __syncthreads();
-    uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
-    for (int v = threadIdx.x; v < kTauBins / 4; v += kThreads) {  // consecutive threads, consecutive bins
-      const uint4 x = *reinterpret_cast<const uint4*>(th + v * 4);
-      if (x.x) atomicAdd(gh + v * 4, x.x);
-      if (x.y) atomicAdd(gh + v * 4 + 1, x.y);
-      if (x.z) atomicAdd(gh + v * 4 + 2, x.z);
-      if (x.w) atomicAdd(gh + v * 4 + 3, x.w);
-      // the 16 threads of a half-warp hold exactly the 64 fine bins of one coarse bin
-      uint32_t sum = x.x + x.y + x.z + x.w;
+    constexpr int kPubThreads = 128;
+    const int pt = threadIdx.x - (kThreads - kPubThreads);
+    if (pt >= 0) {
+      uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
+      for (int v = pt; v < kTauBins / 4; v += kPubThreads) {  // consecutive threads, consecutive bins
+        const uint4 x = *reinterpret_cast<const uint4*>(th + v * 4);
+        if (x.x) atomicAdd(gh + v * 4, x.x);
+        if (x.y) atomicAdd(gh + v * 4 + 1, x.y);
+        if (x.z) atomicAdd(gh + v * 4 + 2, x.z);
+        if (x.w) atomicAdd(gh + v * 4 + 3, x.w);
+        // the 16 threads of a half-warp hold exactly the 64 fine bins of one coarse bin
+        uint32_t sum = x.x + x.y + x.z + x.w;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if ((threadIdx.x & 15) == 0 && sum) atomicAdd(gh + kRowCoarse + ((v * 4) >> 6), sum);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if ((pt & 15) == 0 && sum) atomicAdd(gh + kRowCoarse + ((v * 4) >> 6), sum);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kPubThreads) : "memory");
+      if (pt == 0) {
+        __threadfence();
+        red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
+      }
     }
   }
   scan_rows<DIDX>(p, sm, th, src, sc, q, half, nrows, nrows, false);
