@@ -47,7 +47,8 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 4096;          // digit histograms of the selection
-constexpr int kTauBits = 14;          // key bits of the candidate-bound histogram
+constexpr int kTauBits = 12;          // key bits of the candidate-bound histogram
+constexpr int kCoarse = (1 << kTauBits) / 64;  // coarse bins of 64 fine bins
 constexpr int kTauBins = 1 << kTauBits;
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
@@ -62,7 +63,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 // per-row global state (u32 words)
 constexpr int kRowHist = 0;                       // [kTauBins] partial histogram (self-clearing)
-constexpr int kRowCoarse = kTauBins;              // [256] the same histogram, 64 fine bins per bin
+constexpr int kRowCoarse = kTauBins;              // [kCoarse] the same histogram, 64 fine bins per bin
 constexpr int kRowArrive = kTauBins + 256;        // CTAs that published their first half
 constexpr int kRowBar = kTauBins + 256 + 32;      // row-group barrier state [2]
 constexpr int kRowCnt = kTauBins + 256 + 64;      // [kMaxGroups] candidate count per CTA
@@ -459,15 +460,13 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   // caught after the barrier).  Warp 0 finds the coarse bin, then the fine bin inside it.
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    uint32_t c8[8];
-    {
-      const uint4 x = __ldcg(reinterpret_cast<const uint4*>(rw + kRowCoarse + 256 - 8 * (lane + 1)));
-      const uint4 y = __ldcg(reinterpret_cast<const uint4*>(rw + kRowCoarse + 256 - 8 * (lane + 1) + 4));
-      c8[0] = x.x; c8[1] = x.y; c8[2] = x.z; c8[3] = x.w; c8[4] = y.x; c8[5] = y.y; c8[6] = y.z; c8[7] = y.w;
-    }
+    constexpr int CPL = kCoarse / 32;  // coarse bins per lane, lane 0 holding the top ones
+    uint32_t cc[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) cc[i] = __ldcg(rw + kRowCoarse + kCoarse - CPL * (lane + 1) + i);
     uint32_t local = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) local += c8[i];
+    for (int i = 0; i < CPL; ++i) local += cc[i];
     uint32_t incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -481,13 +480,13 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
     uint32_t above = 0;
     if (before < need && need <= incl) {
       uint32_t acc = before;
-      for (int i = 7; i >= 0; --i) {  // bins from the top of this lane's run
-        if (acc + c8[i] >= need) {
-          tc = 256 - 8 * (lane + 1) + i;
+      for (int i = CPL - 1; i >= 0; --i) {  // bins from the top of this lane's run
+        if (acc + cc[i] >= need) {
+          tc = kCoarse - CPL * (lane + 1) + i;
           above = acc;
           break;
         }
-        acc += c8[i];
+        acc += cc[i];
       }
     }
     const uint32_t hit = __ballot_sync(0xffffffffu, tc >= 0);
@@ -1142,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     {
       const int per = (kTauBins + pl.Cb - 1) / pl.Cb;
       for (int i = pl.c * per + threadIdx.x; i < min(kTauBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
-      if (pl.c == 0 && threadIdx.x < 256) rw[kRowCoarse + threadIdx.x] = 0u;
+      if (pl.c == 0 && threadIdx.x < kCoarse) rw[kRowCoarse + threadIdx.x] = 0u;
       if (pl.c == 0 && threadIdx.x == 0) rw[kRowArrive] = 0u;
     }
     // candidate windows: every count (one load each), then every valid slot copied to a
