@@ -4,88 +4,121 @@
 // k_eff = min(k, t + 1).
 //
 // Stages:
-//   1. index scores  I[i, j] = q_idx[i] . k_idx[j]   (dense contraction, bf16
-//      tensor cores, fp32 accumulate; tiles wholly above the diagonal skipped)
+//   1. index scores  I[i, j] = q_idx[i] . k_idx[j]   (dense contraction on the
+//      tcgen05 tensor cores, fp32 accumulate in TMEM; tiles wholly above the diagonal
+//      skipped)
 //   2. per-row exact radix TopK (the decode top-k kernel with causal lengths)
 //   3. per-row sparse attention of every layer (the decode attention kernel in
 //      gather mode, each row its own sequence over the one shared cache)
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace clsa {
 
 namespace {
 
-constexpr int kTM = 64;   // query rows per CTA
-constexpr int kTN = 128;  // keys per CTA
+constexpr int kTcM = 128;  // query rows per tile (TMEM lanes)
+constexpr int kTcN = 256;  // keys per tile (TMEM columns, fp32)
 
-// S tile = Q_idx[64 rows] . K_idx[128 keys]^T with mma.sync m16n8k16; 4 warps x 16 rows.
+// Score tiles I[i0:i0+128, j0:j0+256] = Q_idx[rows] . K_idx[keys]^T on the 5th-generation
+// tensor cores.  Operands are staged with 16-byte cp.async into 128B-swizzled K-major
+// tiles; one thread issues DI/16 tcgen05.mma (M=128, N=256, K=16, bf16 -> fp32) into a
+// 256-column TMEM accumulator and commits to an mbarrier; the four warps read their 32
+// TMEM lanes (one query row per thread), apply the causal mask and store the row.
+// Tiles whose keys all lie beyond every row's position are skipped.  Persistent: each
+// CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...
 template <int DI>
-__global__ void __launch_bounds__(128) prefill_scores_kernel(const __nv_bfloat16* __restrict__ q_idx,
-                                                             const __nv_bfloat16* __restrict__ k_idx, int n,
-                                                             int T, float* __restrict__ scores) {
-  constexpr int STR = DI + 8;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16* sA = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [kTM][STR]
-  __nv_bfloat16* sB = sA + kTM * STR;                               // [kTN][STR]
-  const int j0 = blockIdx.x * kTN;
-  const int i0 = blockIdx.y * kTM;
-  const int base = n - T;
-  // rows i0..i0+63 see keys j <= base + i; skip tiles with every key beyond every row
-  if (j0 > base + min(i0 + kTM - 1, T - 1)) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  constexpr int VPR = DI * 2 / 16;
-  for (int v = threadIdx.x; v < kTM * VPR; v += blockDim.x) {
-    const int r = v / VPR, c = v % VPR;
-    const int i = i0 + r;
-    cp_async_16(sA + r * STR + c * 8, i < T ? q_idx + (size_t)i * DI + c * 8 : q_idx, i < T ? 16 : 0);
+__global__ void __launch_bounds__(128) prefill_scores_tc_kernel(const __nv_bfloat16* __restrict__ q_idx,
+                                                                const __nv_bfloat16* __restrict__ k_idx, int n,
+                                                                int T, float* __restrict__ scores,
+                                                                void* ws_header) {
+  constexpr int KAT = DI / 64;                 // 128-byte K atoms
+  constexpr uint32_t A_ATOM = kTcM * 128;      // bytes of one K atom of the A tile
+  constexpr uint32_t B_ATOM = kTcN * 128;
+  constexpr int CPR = DI / 8;                  // 16-byte chunks per row
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + KAT * A_ATOM;
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_base;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp == 0) {
+    tc::tmem_alloc(&tmem_base, kTcN);
+    tc::tmem_relinquish();
   }
-  for (int v = threadIdx.x; v < kTN * VPR; v += blockDim.x) {
-    const int r = v / VPR, c = v % VPR;
-    const int j = j0 + r;
-    cp_async_16(sB + r * STR + c * 8, j < n ? k_idx + (size_t)j * DI + c * 8 : k_idx, j < n ? 16 : 0);
+  if (tid == 0) {
+    mbar_init(&mbar, 1);
+    fence_mbar_init();
   }
-  cp_async_commit();
-  cp_async_wait<0>();
+  tc::fence_before_sync();
   __syncthreads();
-
-  float acc[kTN / 8][4];
-#pragma unroll
-  for (int t = 0; t < kTN / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < DI / 16; ++ks) {
-    uint32_t a[4];
-    {
-      const int mi = lane >> 3;
-      const int row = warp * 16 + (lane & 7) + 8 * (mi & 1);
-      const int col = ks * 16 + 8 * (mi >> 1);
-      ldmatrix_x4(a[0], a[1], a[2], a[3], sA + row * STR + col);
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_base;
+  const int base = n - T;
+  const int nqb = (T + kTcM - 1) / kTcM, nkt = (n + kTcN - 1) / kTcN;
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcM, kTcN);
+  uint32_t phase = 0;
+  for (int item = blockIdx.x; item < nqb * nkt; item += gridDim.x) {
+    const int qb = item / nkt, kt = item % nkt;
+    const int i0 = qb * kTcM, j0 = kt * kTcN;
+    if (j0 > base + min(i0 + kTcM - 1, T - 1)) continue;  // every key beyond every row
+    for (int v = tid; v < kTcM * CPR; v += 128) {
+      const int r = v / CPR, c = v % CPR;
+      const bool in = i0 + r < T;
+      cp_async_16(sA + (c >> 3) * A_ATOM + tc::sw128_offset(r, c & 7),
+                  in ? q_idx + (size_t)(i0 + r) * DI + c * 8 : q_idx, in ? 16 : 0);
     }
-#pragma unroll
-    for (int nt2 = 0; nt2 < kTN / 16; ++nt2) {
-      const int mi = lane >> 3;
-      const int tok = nt2 * 16 + 8 * (mi >> 1) + (lane & 7);
-      const int col = ks * 16 + 8 * (mi & 1);
-      uint32_t r0, r1, r2, r3;
-      ldmatrix_x4(r0, r1, r2, r3, sB + tok * STR + col);
-      mma_bf16_16816(acc[2 * nt2], a, r0, r1);
-      mma_bf16_16816(acc[2 * nt2 + 1], a, r2, r3);
+    for (int v = tid; v < kTcN * CPR; v += 128) {
+      const int r = v / CPR, c = v % CPR;
+      const bool in = j0 + r < n;
+      cp_async_16(sB + (c >> 3) * B_ATOM + tc::sw128_offset(r, c & 7),
+                  in ? k_idx + (size_t)(j0 + r) * DI + c * 8 : k_idx, in ? 16 : 0);
     }
-  }
+    cp_async_commit();
+    cp_async_wait<0>();
+    fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core's reads
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int i = i0 + warp * 16 + gid + 8 * half;
-    if (i >= T) continue;
+      for (int ks = 0; ks < DI / 16; ++ks) {
+        const uint32_t koff = (uint32_t)(ks & 3) * 32u;
+        const uint64_t a = tc::sw128_desc(smem_u32(sA) + (ks >> 2) * A_ATOM + koff);
+        const uint64_t b = tc::sw128_desc(smem_u32(sB) + (ks >> 2) * B_ATOM + koff);
+        tc::mma_bf16(tmem, a, b, idesc, ks > 0);
+      }
+      tc::mma_commit(&mbar);
+    }
+    const bool ok = __syncthreads_and(mbar_wait(&mbar, phase));
+    phase ^= 1u;
+    if (!ok) {
+      if (tid == 0) record_error(ws_header, CLSA_ERR_TIMEOUT, 300);
+      break;
+    }
+    tc::fence_after_sync();
+    const int i = i0 + warp * 32 + lane;  // this thread's query row = its TMEM lane
     const int t = base + i;
     float* row = scores + (size_t)i * n;
+#pragma unroll 1
+    for (int cb = 0; cb < kTcN; cb += 32) {
+      uint32_t v[32];
+      tc::ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)cb, v);
+      tc::ld_wait();
+      if (i < T) {
 #pragma unroll
-    for (int nt = 0; nt < kTN / 8; ++nt) {
-      const int j = j0 + nt * 8 + 2 * tig;
-      if (j < n) row[j] = j <= t ? acc[nt][2 * half] : -INFINITY;
-      if (j + 1 < n) row[j + 1] = j + 1 <= t ? acc[nt][2 * half + 1] : -INFINITY;
+        for (int q = 0; q < 32; ++q) {
+          const int j = j0 + cb + q;
+          if (j < n) row[j] = j <= t ? __uint_as_float(v[q]) : -INFINITY;
+        }
+      }
     }
+    tc::fence_before_sync();
+    __syncthreads();  // TMEM and the operand tiles are reused by the next tile
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, kTcN);
 }
 
 struct PrefillLayout {
@@ -117,16 +150,16 @@ clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_bo
   const PrefillLayout lay = prefill_layout(a);
   char* w = static_cast<char*>(ws_body);
   float* scores = reinterpret_cast<float*>(w + lay.scores);
-  dim3 grid((a->n + kTN - 1) / kTN, (a->T + kTM - 1) / kTM);
+  const int nsm = std::max(1, device_info().sm_count);
   const auto* q = static_cast<const __nv_bfloat16*>(a->q_idx);
   const auto* kx = static_cast<const __nv_bfloat16*>(a->k_idx);
-  const int smem = (kTM + kTN) * (a->d_idx + 8) * 2;
+  const int smem = (a->d_idx / 64) * (kTcM + kTcN) * 128;
   if (a->d_idx == 128) {
-    cudaFuncSetAttribute(prefill_scores_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_scores_kernel<128><<<grid, 128, smem, s>>>(q, kx, a->n, a->T, scores);
+    cudaFuncSetAttribute(prefill_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    prefill_scores_tc_kernel<128><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header);
   } else {
-    cudaFuncSetAttribute(prefill_scores_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_scores_kernel<64><<<grid, 128, smem, s>>>(q, kx, a->n, a->T, scores);
+    cudaFuncSetAttribute(prefill_scores_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    prefill_scores_tc_kernel<64><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header);
   }
   launches_add(1);
   if (cudaGetLastError() != cudaSuccess) return CLSA_ERR_CUDA;
