@@ -26,10 +26,14 @@ cudaError_t launch_index_scores(const void* q_idx, const void* k_idx, const int3
 
 // ----- exact radix top-k -----------------------------------------------------
 size_t topk_ws_bytes(int B, int n_max, int k);
-// causal_base >= 0: row b has length causal_base + b + 1 and seq_lens is ignored
+// causal_base >= 0: row b has length causal_base + b + 1 and seq_lens is ignored.
+// row_skip: rows with row_skip[b] == skip_val are left untouched.  idx_map: the row's
+// selected positions j are written as idx_map[b * ld_map + j] (positions are ascending,
+// so ascending maps stay ascending).
 cudaError_t launch_topk(const float* scores, const int32_t* seq_lens, int B, int n_max, int k,
                         int32_t* idx, int32_t* count, void* ws_header, void* topk_ws, cudaStream_t s,
-                        int causal_base = -1);
+                        int causal_base = -1, const int32_t* row_skip = nullptr, int skip_val = 0,
+                        const int32_t* idx_map = nullptr, int ld_map = 0);
 
 // ----- selector gather --------------------------------------------------------
 cudaError_t launch_gather_kv(const void* K, const void* V, const int32_t* idx, const int32_t* count, int B,
@@ -66,6 +70,19 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
                                 cudaStream_t s);
 
 // ----- prefill ------------------------------------------------------------------
+struct PrefillRouteBufs {
+  uint32_t* dval;     // [T][ldd] dense candidate scores (fp32 bits)
+  int32_t* dtok;      // [T][ldd] their token indices (ascending per row)
+  int32_t* dlen;      // [T] candidates per row (0 for a flagged row)
+  int32_t* flag;      // [T] 1: the row needs the exact fallback
+  uint32_t* any_flag; // some row is flagged
+  int ldd;
+};
+bool prefill_route_supported(const clsa_prefill_args* a);
+int prefill_route_ldd(const clsa_prefill_args* a);  // dense candidate row length
+size_t prefill_route_ws_bytes(const clsa_prefill_args* a);
+cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, void* ws, cudaStream_t s,
+                                 PrefillRouteBufs* out);
 size_t prefill_ws_bytes(const clsa_prefill_args* a);
 clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_body, cudaStream_t s);
 

@@ -32,7 +32,9 @@ template <int DI>
 __global__ void __launch_bounds__(128) prefill_scores_tc_kernel(const __nv_bfloat16* __restrict__ q_idx,
                                                                 const __nv_bfloat16* __restrict__ k_idx, int n,
                                                                 int T, float* __restrict__ scores,
-                                                                void* ws_header) {
+                                                                void* ws_header,
+                                                                const int32_t* __restrict__ only_rows,
+                                                                const uint32_t* __restrict__ any_flag) {
   constexpr int KAT = DI / 64;                 // 128-byte K atoms
   constexpr uint32_t A_ATOM = kTcM * 128;      // bytes of one K atom of the A tile
   constexpr uint32_t B_ATOM = kTcN * 128;
@@ -43,6 +45,7 @@ __global__ void __launch_bounds__(128) prefill_scores_tc_kernel(const __nv_bfloa
   __shared__ uint64_t mbar;
   __shared__ uint32_t tmem_base;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (any_flag && *any_flag == 0u) return;  // fallback use: nothing to recompute
   if (warp == 0) {
     tc::tmem_alloc(&tmem_base, kTcN);
     tc::tmem_relinquish();
@@ -63,6 +66,10 @@ __global__ void __launch_bounds__(128) prefill_scores_tc_kernel(const __nv_bfloa
     const int qb = item / nkt, kt = item % nkt;
     const int i0 = qb * kTcM, j0 = kt * kTcN;
     if (j0 > base + min(i0 + kTcM - 1, T - 1)) continue;  // every key beyond every row
+    if (only_rows) {  // fallback use: only row blocks holding a flagged row
+      const int r = i0 + tid;
+      if (!__syncthreads_or(r < T && only_rows[r] != 0)) continue;
+    }
     for (int v = tid; v < kTcM * CPR; v += 128) {
       const int r = v / CPR, c = v % CPR;
       const bool in = i0 + r < T;
@@ -97,21 +104,25 @@ __global__ void __launch_bounds__(128) prefill_scores_tc_kernel(const __nv_bfloa
       break;
     }
     tc::fence_after_sync();
-    const int i = i0 + warp * 32 + lane;  // this thread's query row = its TMEM lane
-    const int t = base + i;
-    float* row = scores + (size_t)i * n;
+    // Epilogue: each thread pulls its row's next 32 columns from TMEM (its lane) and
+    // parks them in the free B tile; then each warp writes its 32 rows as 128-byte
+    // row segments (lane = column), causal mask applied on the way out.
+    float* stage = reinterpret_cast<float*>(sB) + warp * 32 * 33;  // [32 rows][33] per warp
 #pragma unroll 1
     for (int cb = 0; cb < kTcN; cb += 32) {
       uint32_t v[32];
       tc::ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)cb, v);
       tc::ld_wait();
-      if (i < T) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int j = j0 + cb + q;
-          if (j < n) row[j] = j <= t ? __uint_as_float(v[q]) : -INFINITY;
-        }
+      for (int q = 0; q < 32; ++q) stage[lane * 33 + q] = __uint_as_float(v[q]);
+      __syncwarp();
+      const int j = j0 + cb + lane;
+#pragma unroll 4
+      for (int rr = 0; rr < 32; ++rr) {
+        const int i = i0 + warp * 32 + rr;
+        if (i < T && j < n) scores[(size_t)i * n + j] = j <= base + i ? stage[rr * 33 + lane] : -INFINITY;
       }
+      __syncwarp();
     }
     tc::fence_before_sync();
     __syncthreads();  // TMEM and the operand tiles are reused by the next tile
@@ -122,19 +133,26 @@ __global__ void __launch_bounds__(128) prefill_scores_tc_kernel(const __nv_bfloa
 }
 
 struct PrefillLayout {
-  size_t scores = 0, topk = 0, attn = 0, total = 0;
+  bool route = false;
+  size_t scores = 0, topk = 0, attn = 0, route_ws = 0, total = 0;
 };
 
 PrefillLayout prefill_layout(const clsa_prefill_args* a) {
   PrefillLayout l;
+  l.route = prefill_route_supported(a);
   size_t off = 0;
-  l.scores = off;
+  l.scores = off;  // fp32 scores of the exact path (the fallback when routing is on)
   off += align_up((size_t)a->T * a->n * sizeof(float), 256);
-  l.topk = off;
-  off += topk_ws_bytes(a->T, a->n, a->k);
+  l.topk = off;  // shared by the top-k over score rows and over dense candidate rows
+  off += std::max(topk_ws_bytes(a->T, a->n, a->k),
+                  l.route ? topk_ws_bytes(a->T, prefill_route_ldd(a), a->k) : (size_t)0);
   AttnShape sh{a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype, true, a->n, 0};
   l.attn = off;
   off += attn_ws_bytes(sh);
+  if (l.route) {
+    l.route_ws = off;
+    off += prefill_route_ws_bytes(a);
+  }
   l.total = off;
   return l;
 }
@@ -154,18 +172,37 @@ clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_bo
   const auto* q = static_cast<const __nv_bfloat16*>(a->q_idx);
   const auto* kx = static_cast<const __nv_bfloat16*>(a->k_idx);
   const int smem = (a->d_idx / 64) * (kTcM + kTcN) * 128;
-  if (a->d_idx == 128) {
-    cudaFuncSetAttribute(prefill_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_scores_tc_kernel<128><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header);
+  auto scores_kernel = [&](const int32_t* only_rows, const uint32_t* any_flag) {
+    if (a->d_idx == 128) {
+      cudaFuncSetAttribute(prefill_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      prefill_scores_tc_kernel<128><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header, only_rows,
+                                                                 any_flag);
+    } else {
+      cudaFuncSetAttribute(prefill_scores_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      prefill_scores_tc_kernel<64><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header, only_rows,
+                                                                any_flag);
+    }
+    launches_add(1);
+    return cudaGetLastError();
+  };
+  cudaError_t e;
+  if (lay.route) {
+    // routing from on-chip candidates, then the exact path for any flagged row
+    PrefillRouteBufs rb{};
+    e = launch_prefill_route(a, ws_header, w + lay.route_ws, s, &rb);
+    if (e != cudaSuccess) return CLSA_ERR_CUDA;
+    e = launch_topk(reinterpret_cast<const float*>(rb.dval), rb.dlen, a->T, rb.ldd, a->k, a->idx, a->count,
+                    ws_header, w + lay.topk, s, -1, rb.flag, 1, rb.dtok, rb.ldd);
+    if (e != cudaSuccess) return CLSA_ERR_CUDA;
+    if (scores_kernel(rb.flag, rb.any_flag) != cudaSuccess) return CLSA_ERR_CUDA;
+    e = launch_topk(scores, nullptr, a->T, a->n, a->k, a->idx, a->count, ws_header, w + lay.topk, s, a->n - a->T,
+                    rb.flag, 0);
+    if (e != cudaSuccess) return CLSA_ERR_CUDA;
   } else {
-    cudaFuncSetAttribute(prefill_scores_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_scores_tc_kernel<64><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header);
+    if (scores_kernel(nullptr, nullptr) != cudaSuccess) return CLSA_ERR_CUDA;
+    e = launch_topk(scores, nullptr, a->T, a->n, a->k, a->idx, a->count, ws_header, w + lay.topk, s, a->n - a->T);
+    if (e != cudaSuccess) return CLSA_ERR_CUDA;
   }
-  launches_add(1);
-  if (cudaGetLastError() != cudaSuccess) return CLSA_ERR_CUDA;
-  cudaError_t e = launch_topk(scores, nullptr, a->T, a->n, a->k, a->idx, a->count, ws_header, w + lay.topk, s,
-                              a->n - a->T);
-  if (e != cudaSuccess) return CLSA_ERR_CUDA;
   const float scale = a->scale > 0.f ? a->scale : 1.0f / sqrtf((float)a->d);
   AttnShape sh{a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype, true, a->n, 0};
   e = launch_sparse_attn(sh, a->Q, a->K, a->V, a->idx, a->count, scale, a->O, a->lse, ws_header, w + lay.attn, s);

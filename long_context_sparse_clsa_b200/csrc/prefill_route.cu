@@ -1,0 +1,409 @@
+// Prefill routing without materialising the T x n score matrix.
+//
+// Routing equation for T new rows at cache positions t = n - T + i (picx.dev CLSA
+// summary, Methodology > Architecture Overview): I[i, j] = q_idx[i] . K_idx[j] for
+// j <= t, S_t = TopK(I_t, min(k, t + 1)).
+//
+// prefill_route_kernel: persistent, one CTA per SM, warp-specialised tcgen05 GEMM.
+//   unit     = two 128-row query blocks x one slice of the key range (so every CTA has
+//              work; the two blocks share each K_idx tile, halving its L2 traffic)
+//   warp 0   TMA producer: the unit's two Q_idx blocks once, then 128-key K_idx tiles
+//            into a 4-stage ring (128-byte swizzle, the UMMA K-major layout)
+//   warp 1   MMA issuer: per tile, 2 x 8 tcgen05.mma (M=128, N=128, K=16) into one of
+//            two TMEM buffers; commits free the ring stage and publish the buffer
+//   warps 2-9 epilogue, one query row per thread (TMEM lane): tcgen05.ld 128 scores,
+//            causal mask, then
+//              warm-up tiles: keep the row's 16 largest scores;
+//              threshold:     tau = the m-th largest of the warm-up sample, m chosen so
+//                             that ~1.4 k_eff tokens of the whole row score >= tau;
+//              every tile:    append (key, token) of scores >= tau to the row's slice
+//                             buffer, in token order.
+//   The warm-up tiles are spread over the slice and scored a second time in the main
+//   pass (about 4 extra tiles per ~100).
+// prefill_densify_kernel: per row, concatenate the slice buffers (token order) into a
+//   dense candidate row; a row whose slice buffer overflowed or whose candidates number
+//   fewer than k_eff is flagged for the exact fallback (score the whole row, select).
+// The exact TopK over each dense candidate row is the radix-select kernel of topk.cu.
+#include <cmath>
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+#include "tma.h"
+
+namespace clsa {
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                       uint32_t box_rows, uint32_t box_cols) {
+  using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return false;
+    fn = reinterpret_cast<EncodeFn>(p);
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+constexpr int kRM = 128;        // rows per query block (TMEM lanes)
+constexpr int kRN = 128;        // keys per tile
+constexpr int kRStages = 4;     // K tile ring
+constexpr int kRThreads = 320;  // 10 warps
+constexpr int kWarm = 4;        // warm-up tiles per unit
+constexpr int kTrack = 16;      // largest warm-up scores kept per row
+constexpr uint32_t kABlock = kRM * 128 * 2;  // one query block, both 64-column atoms: 32 KiB
+constexpr uint32_t kBTile = kRN * 128 * 2;   // one key tile, both atoms: 32 KiB
+constexpr uint32_t kAtomA = kRM * 128;       // 16 KiB
+constexpr uint32_t kAtomB = kRN * 128;
+
+struct RouteParams {
+  int n, T, k, S, cap, nunits;
+  uint32_t* cand_val;  // [T][S][cap] candidate scores (fp32 bits)
+  int32_t* cand_tok;   // [T][S][cap]
+  int32_t* cand_cnt;   // [T][S]  (> cap: overflow)
+  uint32_t* any_flag;  // set by the densify step when some row needs the exact fallback
+  void* ws_header;
+};
+
+struct RouteSmem {
+  uint64_t full[kRStages], empty[kRStages];
+  uint64_t tfull[2], tempty[2];
+  uint64_t afull, aempty;
+  uint32_t tmem;
+  int abort_flag;
+};
+constexpr size_t kRouteSmem = 1024 /*align slack*/ + 2 * kABlock + kRStages * kBTile + sizeof(RouteSmem);
+
+// the unit's tiles: main pass = [t_lo, t_hi); warm-up = kWarm tiles spread over it
+struct UnitTiles {
+  int r0, t_lo, t_hi, nwarm;
+  __device__ int count() const { return nwarm + (t_hi - t_lo); }
+  __device__ int tile(int it) const {  // tile index of step it
+    if (it < nwarm) return t_lo + (int)(((long long)it * (t_hi - t_lo)) / nwarm);
+    return t_lo + (it - nwarm);
+  }
+};
+
+__device__ __forceinline__ UnitTiles unit_tiles(const RouteParams& p, int u) {
+  UnitTiles ut;
+  const int pair = u / p.S, s = u % p.S;
+  ut.r0 = pair * 2 * kRM;
+  const int tmax = p.n - p.T + min(ut.r0 + 2 * kRM, p.T) - 1;  // largest position of the pair
+  const int ntile = tmax / kRN + 1;
+  ut.t_lo = (int)(((long long)s * ntile) / p.S);
+  ut.t_hi = (int)(((long long)(s + 1) * ntile) / p.S);
+  ut.nwarm = min(kWarm, ut.t_hi - ut.t_lo);
+  return ut;
+}
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    prefill_route_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                         const RouteParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~uintptr_t(1023));
+  unsigned char* sA = smem;                    // [2 blocks][2 atoms][128 rows][128 B]
+  unsigned char* sB = smem + 2 * kABlock;      // [stage][2 atoms][128 keys][128 B]
+  RouteSmem& sm = *reinterpret_cast<RouteSmem*>(sB + kRStages * kBTile);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRStages; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.tfull[i], 1);
+      mbar_init(&sm.tempty[i], 8);
+    }
+    mbar_init(&sm.afull, 1);
+    mbar_init(&sm.aempty, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+    if (blockIdx.x == 0) *p.any_flag = 0u;  // the densify step runs after this kernel
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm.tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph_empty = 1, ph_aempty = 1;
+      for (int u = blockIdx.x; u < p.nunits && !*(volatile int*)&sm.abort_flag; u += gridDim.x) {
+        const UnitTiles ut = unit_tiles(p, u);
+        if (!mbar_wait(&sm.aempty, ph_aempty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 400); sm.abort_flag = 1; break; }
+        ph_aempty ^= 1u;
+        mbar_arrive_expect_tx(&sm.afull, 2 * kABlock);
+        for (int h = 0; h < 2; ++h)
+          for (int a = 0; a < 2; ++a)
+            tma_load_2d(sA + h * kABlock + a * kAtomA, &tq, a * 64, ut.r0 + h * kRM, &sm.afull);
+        for (int it = 0; it < ut.count(); ++it) {
+          if (!mbar_wait(&sm.empty[stage], ph_empty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 401); sm.abort_flag = 1; break; }
+          const int j0 = ut.tile(it) * kRN;
+          mbar_arrive_expect_tx(&sm.full[stage], kBTile);
+          for (int a = 0; a < 2; ++a) tma_load_2d(sB + stage * kBTile + a * kAtomB, &tk, a * 64, j0, &sm.full[stage]);
+          if (++stage == kRStages) { stage = 0; ph_empty ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(kRM, kRN);
+      int stage = 0, buf = 0;
+      uint32_t ph_full = 0, ph_tempty = 1, ph_afull = 0;
+      for (int u = blockIdx.x; u < p.nunits && !*(volatile int*)&sm.abort_flag; u += gridDim.x) {
+        const UnitTiles ut = unit_tiles(p, u);
+        if (!mbar_wait(&sm.afull, ph_afull)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 410); sm.abort_flag = 1; break; }
+        ph_afull ^= 1u;
+        for (int it = 0; it < ut.count(); ++it) {
+          if (!mbar_wait(&sm.full[stage], ph_full) || !mbar_wait(&sm.tempty[buf], ph_tempty)) {
+            record_error(p.ws_header, CLSA_ERR_TIMEOUT, 411);
+            sm.abort_flag = 1;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t b_base = smem_u32(sB + stage * kBTile);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t a_base = smem_u32(sA + h * kABlock);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t koff = (uint32_t)(ks & 3) * 32u;
+              tc::mma_bf16(tmem + (uint32_t)(buf * 256 + h * kRN),
+                           tc::sw128_desc(a_base + (ks >> 2) * kAtomA + koff),
+                           tc::sw128_desc(b_base + (ks >> 2) * kAtomB + koff), idesc, ks > 0);
+            }
+          }
+          tc::mma_commit(&sm.empty[stage]);
+          tc::mma_commit(&sm.tfull[buf]);
+          if (++stage == kRStages) { stage = 0; ph_full ^= 1u; }
+          if (++buf == 2) { buf = 0; ph_tempty ^= 1u; }
+        }
+        tc::mma_commit(&sm.aempty);  // the A blocks are free once this unit's MMAs finish
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (one row per thread)
+    const int q = warp & 3;             // TMEM lane quarter this warp may read
+    const int h = (warp - 2) >> 2;      // query block of this warpgroup
+    int buf = 0;
+    uint32_t ph_tfull = 0;
+    for (int u = blockIdx.x; u < p.nunits && !*(volatile int*)&sm.abort_flag; u += gridDim.x) {
+      const UnitTiles ut = unit_tiles(p, u);
+      const int s = u % p.S;
+      const int i = ut.r0 + h * kRM + q * 32 + lane;  // query row
+      const bool row_ok = i < p.T;
+      const int t = p.n - p.T + i;                    // its cache position
+      const int keff = min(p.k, t + 1);
+      float top[kTrack];
+#pragma unroll
+      for (int x = 0; x < kTrack; ++x) top[x] = -INFINITY;
+      int seen = 0, cnt = 0;
+      float tau = -INFINITY;
+      const size_t slot = ((size_t)(row_ok ? i : 0) * p.S + s) * p.cap;
+      for (int it = 0; it < ut.count(); ++it) {
+        if (!mbar_wait(&sm.tfull[buf], ph_tfull)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 420); sm.abort_flag = 1; break; }
+        tc::fence_after_sync();
+        const int j0 = ut.tile(it) * kRN;
+        const bool warm = it < ut.nwarm;
+#pragma unroll 1
+        for (int cb = 0; cb < kRN; cb += 32) {
+          uint32_t v[32];
+          tc::ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + h * kRN + cb), v);
+          tc::ld_wait();
+          if (!row_ok) continue;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int j = j0 + cb + c;
+            const float val = __uint_as_float(v[c]);
+            if (j > t) continue;
+            if (warm) {
+              ++seen;
+              if (val > top[kTrack - 1]) {  // insert into the descending list
+                float x = val;
+#pragma unroll
+                for (int y = 0; y < kTrack; ++y) {
+                  const float hi = fmaxf(top[y], x), lo = fminf(top[y], x);
+                  top[y] = hi;
+                  x = lo;
+                }
+              }
+            } else if (val >= tau) {
+              if (cnt < p.cap) {
+                p.cand_val[slot + cnt] = __float_as_uint(val);
+                p.cand_tok[slot + cnt] = j;
+              }
+              ++cnt;
+            }
+          }
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+        if (++buf == 2) { buf = 0; ph_tfull ^= 1u; }
+        if (it + 1 == ut.nwarm && row_ok) {
+          // m-th largest warm-up score, m = expected count of the sample above the k_eff
+          // boundary, inflated 1.4x; no usable bound (tau = -inf, every token a candidate)
+          // when all tokens are selected or the sample is too small for m <= kTrack
+          const float m_f = 1.4f * (float)keff * (float)seen / (float)(t + 1);
+          const int m = (int)ceilf(m_f);
+          tau = -INFINITY;
+          if (keff < t + 1 && m >= 1 && m <= kTrack && seen >= m) {
+#pragma unroll
+            for (int y = 0; y < kTrack; ++y)
+              if (y == m - 1) tau = top[y];
+          }
+        }
+      }
+      if (row_ok) p.cand_cnt[(size_t)i * p.S + s] = cnt;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+// One CTA per row: concatenate the row's slice buffers (slices in key order, tokens
+// ascending inside a slice) into a dense candidate row, or flag the row for the exact
+// fallback when a slice overflowed or the candidates number fewer than k_eff.
+__global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams p, uint32_t* __restrict__ dval,
+                                                              int32_t* __restrict__ dtok,
+                                                              int32_t* __restrict__ dlen,
+                                                              int32_t* __restrict__ flag, int ldd) {
+  __shared__ int off[65];
+  __shared__ int bad;
+  const int i = blockIdx.x;
+  const int t = p.n - p.T + i;
+  const int keff = min(p.k, t + 1);
+  if (threadIdx.x == 0) {
+    int acc = 0, over = 0;
+    for (int s2 = 0; s2 < p.S; ++s2) {
+      const int c = p.cand_cnt[(size_t)i * p.S + s2];
+      off[s2] = acc;
+      over |= c > p.cap;
+      acc += min(c, p.cap);
+    }
+    off[p.S] = acc;
+    bad = over || acc < keff;
+    flag[i] = bad;
+    dlen[i] = bad ? 0 : acc;
+    if (bad) atomicOr(p.any_flag, 1u);
+  }
+  __syncthreads();
+  if (bad) return;
+  for (int s2 = 0; s2 < p.S; ++s2) {
+    const int o = off[s2], c = off[s2 + 1] - o;
+    const size_t src = ((size_t)i * p.S + s2) * p.cap;
+    for (int e = threadIdx.x; e < c; e += blockDim.x) {
+      dval[(size_t)i * ldd + o + e] = p.cand_val[src + e];
+      dtok[(size_t)i * ldd + o + e] = p.cand_tok[src + e];
+    }
+  }
+}
+
+struct RoutePlan {
+  int S, cap, nunits, grid, ldd;
+};
+
+RoutePlan route_plan(int n, int T, int k) {
+  RoutePlan rp{};
+  const int sms = std::max(1, device_info().sm_count);
+  const int npairs = (T + 2 * kRM - 1) / (2 * kRM);
+  rp.S = std::max(1, std::min(64, sms / npairs));
+  rp.nunits = npairs * rp.S;
+  rp.grid = std::min(rp.nunits, sms);
+  const int expect = (int)std::ceil(1.4 * std::min(k, n) / rp.S);
+  rp.cap = std::max(256, std::min(16384, (4 * expect + 63) / 64 * 64));
+  rp.ldd = rp.S * rp.cap;
+  return rp;
+}
+
+}  // namespace
+
+int prefill_route_ldd(const clsa_prefill_args* a) { return route_plan(a->n, a->T, a->k).ldd; }
+
+bool prefill_route_supported(const clsa_prefill_args* a) {
+  return a->d_idx == 128 && device_info().max_smem_optin >= (int)kRouteSmem && a->T >= 1;
+}
+
+size_t prefill_route_ws_bytes(const clsa_prefill_args* a) {
+  const RoutePlan rp = route_plan(a->n, a->T, a->k);
+  const size_t T = (size_t)a->T;
+  size_t off = 0;
+  off += 2 * align_up(T * rp.S * rp.cap * 4, 256);  // slice buffers (values, tokens)
+  off += align_up(T * rp.S * 4, 256);               // slice counts
+  off += 2 * align_up(T * rp.ldd * 4, 256);         // dense candidate rows
+  off += 2 * align_up(T * 4, 256);                  // dense lengths, fallback flags
+  off += 256;                                       // any-flag word
+  return off;
+}
+
+cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, void* ws, cudaStream_t s,
+                                 PrefillRouteBufs* out) {
+  const RoutePlan rp = route_plan(a->n, a->T, a->k);
+  const size_t T = (size_t)a->T;
+  char* w = static_cast<char*>(ws);
+  RouteParams p{};
+  p.n = a->n;
+  p.T = a->T;
+  p.k = a->k;
+  p.S = rp.S;
+  p.cap = rp.cap;
+  p.nunits = rp.nunits;
+  p.ws_header = ws_header;
+  p.cand_val = reinterpret_cast<uint32_t*>(w);
+  w += align_up(T * rp.S * rp.cap * 4, 256);
+  p.cand_tok = reinterpret_cast<int32_t*>(w);
+  w += align_up(T * rp.S * rp.cap * 4, 256);
+  p.cand_cnt = reinterpret_cast<int32_t*>(w);
+  w += align_up(T * rp.S * 4, 256);
+  out->dval = reinterpret_cast<uint32_t*>(w);
+  w += align_up(T * rp.ldd * 4, 256);
+  out->dtok = reinterpret_cast<int32_t*>(w);
+  w += align_up(T * rp.ldd * 4, 256);
+  out->dlen = reinterpret_cast<int32_t*>(w);
+  w += align_up(T * 4, 256);
+  out->flag = reinterpret_cast<int32_t*>(w);
+  w += align_up(T * 4, 256);
+  out->any_flag = reinterpret_cast<uint32_t*>(w);
+  out->ldd = rp.ldd;
+  p.any_flag = out->any_flag;
+
+  CUtensorMap tq, tk;
+  if (!make_tmap_bf16_2d(&tq, a->q_idx, (uint64_t)a->T, 128, 256, kRM, 64) ||
+      !make_tmap_bf16_2d(&tk, a->k_idx, (uint64_t)a->n, 128, 256, kRN, 64))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(prefill_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kRouteSmem);
+  if (e != cudaSuccess) return e;
+  prefill_route_kernel<<<rp.grid, kRThreads, kRouteSmem, s>>>(tq, tk, p);
+  launches_add(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prefill_densify_kernel<<<a->T, 256, 0, s>>>(p, out->dval, out->dtok, out->dlen, out->flag, rp.ldd);
+  launches_add(1);
+  return cudaGetLastError();
+}
+
+}  // namespace clsa

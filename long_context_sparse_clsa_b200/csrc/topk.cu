@@ -116,10 +116,13 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
                                                         const int32_t* __restrict__ seq_lens, int n_max,
                                                         int k, int C, int chunk, int32_t* __restrict__ idx,
                                                         int32_t* __restrict__ count, void* ws_header,
-                                                        uint32_t* __restrict__ row_ws_all, int causal_base) {
+                                                        uint32_t* __restrict__ row_ws_all, int causal_base,
+                                                        const int32_t* __restrict__ row_skip, int skip_val,
+                                                        const int32_t* __restrict__ idx_map, int ld_map) {
   __shared__ TopkSmem sm;
   const int b = blockIdx.y;
   const int c = blockIdx.x;
+  if (row_skip && row_skip[b] == skip_val) return;  // uniform for the row's CTAs
   const int len = max(0, min(causal_base >= 0 ? causal_base + b + 1 : seq_lens[b], n_max));
   const int keff = min(k, len);
   uint32_t* row_ws = row_ws_all + (size_t)b * kRowWords;
@@ -135,8 +138,9 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
   if (keff == 0) return;
   const int lo = c * chunk;
   const int hi = min(len, lo + chunk);
+  const int32_t* map = idx_map ? idx_map + (size_t)b * ld_map : nullptr;
   if (keff == len) {  // every token is selected
-    for (int j = lo + threadIdx.x; j < hi; j += kThreads) out[j] = j;
+    for (int j = lo + threadIdx.x; j < hi; j += kThreads) out[j] = map ? map[j] : j;
     return;
   }
 
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const float* __restrict_
     uint32_t tile_sel;
     const uint32_t pos = written + block_excl_scan(sel, sm.warp_tot, &tile_sel);
     if (sel) {
-      if (off + pos < (uint32_t)keff) out[off + pos] = j;
+      if (off + pos < (uint32_t)keff) out[off + pos] = map ? map[j] : j;
       else record_error(ws_header, CLSA_ERR_BAD_INDEX, ((long long)b << 32) | (off + pos));
     }
     ties_seen += tile_eq;
@@ -282,13 +286,15 @@ size_t topk_ws_bytes(int B, int n_max, int /*k*/) {
 
 cudaError_t launch_topk(const float* scores, const int32_t* seq_lens, int B, int n_max, int k,
                         int32_t* idx, int32_t* count, void* ws_header, void* topk_ws, cudaStream_t s,
-                        int causal_base) {
+                        int causal_base, const int32_t* row_skip, int skip_val, const int32_t* idx_map,
+                        int ld_map) {
   const TopkLaunchCfg cfg = topk_cfg(B, n_max);
   dim3 grid(cfg.C, B);
   int C = cfg.C, chunk = cfg.chunk;
   uint32_t* rw = static_cast<uint32_t*>(topk_ws);
   void* args[] = {(void*)&scores, (void*)&seq_lens, (void*)&n_max, (void*)&k, (void*)&C, (void*)&chunk,
-                  (void*)&idx, (void*)&count, (void*)&ws_header, (void*)&rw, (void*)&causal_base};
+                  (void*)&idx, (void*)&count, (void*)&ws_header, (void*)&rw, (void*)&causal_base,
+                  (void*)&row_skip, (void*)&skip_val, (void*)&idx_map, (void*)&ld_map};
   cudaError_t e;
   if (C > 1) e = cudaLaunchCooperativeKernel((const void*)topk_kernel, grid, dim3(kThreads), args, 0, s);
   else e = cudaLaunchKernel((const void*)topk_kernel, grid, dim3(kThreads), args, 0, s);
