@@ -15,14 +15,17 @@
 //            causal mask, then
 //              warm-up tiles: keep the row's 16 largest scores;
 //              threshold:     tau = the m-th largest of the warm-up sample, m chosen so
-//                             that ~1.4 k_eff tokens of the whole row score >= tau;
+//                             that ~2 k_eff tokens of the whole row score >= tau;
 //              every tile:    append (key, token) of scores >= tau to the row's slice
 //                             buffer, in token order.
 //   The warm-up tiles are spread over the slice and scored a second time in the main
 //   pass (about 4 extra tiles per ~100).
 // prefill_densify_kernel: per row, concatenate the slice buffers (token order) into a
-//   dense candidate row; a row whose slice buffer overflowed or whose candidates number
-//   fewer than k_eff is flagged for the exact fallback (score the whole row, select).
+//   dense candidate row.  The row is exact iff at least k_eff candidates score >= the
+//   largest tau any of its slices used: every dropped token then scores strictly below
+//   the k_eff-th candidate, so it cannot be selected (ties included).  A row failing
+//   that, or with an overflowed slice buffer, is flagged for the exact fallback (score
+//   the whole row, select).
 // The exact TopK over each dense candidate row is the radix-select kernel of topk.cu.
 #include <cmath>
 #include <cstdio>
@@ -63,8 +66,9 @@ constexpr int kRM = 128;        // rows per query block (TMEM lanes)
 constexpr int kRN = 128;        // keys per tile
 constexpr int kRStages = 4;     // K tile ring
 constexpr int kRThreads = 320;  // 10 warps
-constexpr int kWarm = 4;        // warm-up tiles per unit
-constexpr int kTrack = 16;      // largest warm-up scores kept per row
+constexpr int kWarm = 8;        // warm-up tiles per unit
+constexpr int kTrack = 32;      // largest warm-up scores kept per row
+constexpr int kMinSample = 8;   // fewer expected sample scores above the boundary: no bound
 constexpr uint32_t kABlock = kRM * 128 * 2;  // one query block, both 64-column atoms: 32 KiB
 constexpr uint32_t kBTile = kRN * 128 * 2;   // one key tile, both atoms: 32 KiB
 constexpr uint32_t kAtomA = kRM * 128;       // 16 KiB
@@ -75,6 +79,7 @@ struct RouteParams {
   uint32_t* cand_val;  // [T][S][cap] candidate scores (fp32 bits)
   int32_t* cand_tok;   // [T][S][cap]
   int32_t* cand_cnt;   // [T][S]  (> cap: overflow)
+  float* cand_tau;     // [T][S]  the bound the slice used (-inf: every token kept)
   uint32_t* any_flag;  // set by the densify step when some row needs the exact fallback
   void* ws_header;
 };
@@ -264,20 +269,24 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
         if (++buf == 2) { buf = 0; ph_tfull ^= 1u; }
         if (it + 1 == ut.nwarm && row_ok) {
-          // m-th largest warm-up score, m = expected count of the sample above the k_eff
-          // boundary, inflated 1.4x; no usable bound (tau = -inf, every token a candidate)
-          // when all tokens are selected or the sample is too small for m <= kTrack
-          const float m_f = 1.4f * (float)keff * (float)seen / (float)(t + 1);
+          // m-th largest warm-up score, m = twice the expected count of the sample above
+          // the k_eff boundary; no bound (tau = -inf, every token a candidate) when all
+          // tokens are selected or the sample is too small (m < kMinSample or > kTrack).
+          // The bound is a guess: the densify step verifies it row by row.
+          const float m_f = 2.0f * (float)keff * (float)seen / (float)(t + 1);
           const int m = (int)ceilf(m_f);
           tau = -INFINITY;
-          if (keff < t + 1 && m >= 1 && m <= kTrack && seen >= m) {
+          if (keff < t + 1 && m >= kMinSample && m <= kTrack && seen >= m) {
 #pragma unroll
             for (int y = 0; y < kTrack; ++y)
               if (y == m - 1) tau = top[y];
           }
         }
       }
-      if (row_ok) p.cand_cnt[(size_t)i * p.S + s] = cnt;
+      if (row_ok) {
+        p.cand_cnt[(size_t)i * p.S + s] = cnt;
+        p.cand_tau[(size_t)i * p.S + s] = ut.count() > 0 ? tau : -INFINITY;
+      }
     }
   }
   tc::fence_before_sync();
@@ -294,32 +303,47 @@ __global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams 
                                                               int32_t* __restrict__ flag, int ldd) {
   __shared__ int off[65];
   __shared__ int bad;
+  __shared__ float tmax;
+  __shared__ int above;
   const int i = blockIdx.x;
   const int t = p.n - p.T + i;
   const int keff = min(p.k, t + 1);
   if (threadIdx.x == 0) {
     int acc = 0, over = 0;
+    float tm = -INFINITY;
     for (int s2 = 0; s2 < p.S; ++s2) {
       const int c = p.cand_cnt[(size_t)i * p.S + s2];
       off[s2] = acc;
       over |= c > p.cap;
       acc += min(c, p.cap);
+      tm = fmaxf(tm, p.cand_tau[(size_t)i * p.S + s2]);
     }
     off[p.S] = acc;
     bad = over || acc < keff;
-    flag[i] = bad;
-    dlen[i] = bad ? 0 : acc;
-    if (bad) atomicOr(p.any_flag, 1u);
+    tmax = tm;
+    above = 0;
   }
   __syncthreads();
-  if (bad) return;
-  for (int s2 = 0; s2 < p.S; ++s2) {
-    const int o = off[s2], c = off[s2 + 1] - o;
-    const size_t src = ((size_t)i * p.S + s2) * p.cap;
-    for (int e = threadIdx.x; e < c; e += blockDim.x) {
-      dval[(size_t)i * ldd + o + e] = p.cand_val[src + e];
-      dtok[(size_t)i * ldd + o + e] = p.cand_tok[src + e];
+  if (!bad) {
+    int mine = 0;
+    for (int s2 = 0; s2 < p.S; ++s2) {
+      const int o = off[s2], c = off[s2 + 1] - o;
+      const size_t src = ((size_t)i * p.S + s2) * p.cap;
+      for (int e = threadIdx.x; e < c; e += blockDim.x) {
+        const uint32_t v = p.cand_val[src + e];
+        dval[(size_t)i * ldd + o + e] = v;
+        dtok[(size_t)i * ldd + o + e] = p.cand_tok[src + e];
+        mine += __uint_as_float(v) >= tmax;
+      }
     }
+    if (mine) atomicAdd(&above, mine);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!bad && above < keff) bad = 1;  // some slice's bound may have dropped a selected token
+    flag[i] = bad;
+    dlen[i] = bad ? 0 : off[p.S];
+    if (bad) atomicOr(p.any_flag, 1u);
   }
 }
 
@@ -334,7 +358,7 @@ RoutePlan route_plan(int n, int T, int k) {
   rp.S = std::max(1, std::min(64, sms / npairs));
   rp.nunits = npairs * rp.S;
   rp.grid = std::min(rp.nunits, sms);
-  const int expect = (int)std::ceil(1.4 * std::min(k, n) / rp.S);
+  const int expect = (int)std::ceil(2.0 * std::min(k, n) / rp.S);
   rp.cap = std::max(256, std::min(16384, (4 * expect + 63) / 64 * 64));
   rp.ldd = rp.S * rp.cap;
   return rp;
@@ -353,7 +377,7 @@ size_t prefill_route_ws_bytes(const clsa_prefill_args* a) {
   const size_t T = (size_t)a->T;
   size_t off = 0;
   off += 2 * align_up(T * rp.S * rp.cap * 4, 256);  // slice buffers (values, tokens)
-  off += align_up(T * rp.S * 4, 256);               // slice counts
+  off += 2 * align_up(T * rp.S * 4, 256);           // slice counts, slice bounds
   off += 2 * align_up(T * rp.ldd * 4, 256);         // dense candidate rows
   off += 2 * align_up(T * 4, 256);                  // dense lengths, fallback flags
   off += 256;                                       // any-flag word
@@ -378,6 +402,8 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
   p.cand_tok = reinterpret_cast<int32_t*>(w);
   w += align_up(T * rp.S * rp.cap * 4, 256);
   p.cand_cnt = reinterpret_cast<int32_t*>(w);
+  w += align_up(T * rp.S * 4, 256);
+  p.cand_tau = reinterpret_cast<float*>(w);
   w += align_up(T * rp.S * 4, 256);
   out->dval = reinterpret_cast<uint32_t*>(w);
   w += align_up(T * rp.ldd * 4, 256);
