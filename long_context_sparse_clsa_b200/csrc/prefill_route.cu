@@ -64,7 +64,7 @@ namespace {
 
 constexpr int kRM = 128;        // rows per query block (TMEM lanes)
 constexpr int kRN = 128;        // keys per tile
-constexpr int kRStages = 4;     // K tile ring
+constexpr int kRStages = 3;     // K tile ring
 constexpr int kRThreads = 320;  // 10 warps
 constexpr int kWarm = 8;        // warm-up tiles per unit
 constexpr int kTrack = 32;      // largest warm-up scores kept per row
@@ -85,6 +85,7 @@ struct RouteParams {
 };
 
 struct RouteSmem {
+  float top[kTrack][256];  // per epilogue thread (column): its row's largest warm-up scores, descending
   uint64_t full[kRStages], empty[kRStages];
   uint64_t tfull[2], tempty[2];
   uint64_t afull, aempty;
@@ -222,9 +223,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
       const bool row_ok = i < p.T;
       const int t = p.n - p.T + i;                    // its cache position
       const int keff = min(p.k, t + 1);
-      float top[kTrack];
-#pragma unroll
-      for (int x = 0; x < kTrack; ++x) top[x] = -INFINITY;
+      const int et = threadIdx.x - 64;  // epilogue thread 0..255: its column of sm.top
+      for (int y = 0; y < kTrack; ++y) sm.top[y][et] = -INFINITY;
       int seen = 0, cnt = 0;
       float tau = -INFINITY;
       const size_t slot = ((size_t)(row_ok ? i : 0) * p.S + s) * p.cap;
@@ -239,28 +239,34 @@ __global__ void __launch_bounds__(kRThreads, 1)
           tc::ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + h * kRN + cb), v);
           tc::ld_wait();
           if (!row_ok) continue;
+          const int nv = min(32, t - (j0 + cb) + 1);  // causally visible columns of this chunk
+          if (warm) {
+            float low = sm.top[kTrack - 1][et];
+            seen += max(0, nv);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int j = j0 + cb + c;
-            const float val = __uint_as_float(v[c]);
-            if (j > t) continue;
-            if (warm) {
-              ++seen;
-              if (val > top[kTrack - 1]) {  // insert into the descending list
-                float x = val;
-#pragma unroll
-                for (int y = 0; y < kTrack; ++y) {
-                  const float hi = fmaxf(top[y], x), lo = fminf(top[y], x);
-                  top[y] = hi;
-                  x = lo;
+            for (int c = 0; c < 32; ++c) {
+              const float val = __uint_as_float(v[c]);
+              if (c < nv && val > low) {
+                int y = kTrack - 1;  // insertion from the bottom of the descending list
+                while (y > 0 && sm.top[y - 1][et] < val) {
+                  sm.top[y][et] = sm.top[y - 1][et];
+                  --y;
                 }
+                sm.top[y][et] = val;
+                low = sm.top[kTrack - 1][et];
               }
-            } else if (val >= tau) {
-              if (cnt < p.cap) {
-                p.cand_val[slot + cnt] = __float_as_uint(val);
-                p.cand_tok[slot + cnt] = j;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float val = __uint_as_float(v[c]);
+              if (c < nv && val >= tau) {
+                if (cnt < p.cap) {
+                  p.cand_val[slot + cnt] = v[c];
+                  p.cand_tok[slot + cnt] = j0 + cb + c;
+                }
+                ++cnt;
               }
-              ++cnt;
             }
           }
         }
@@ -276,11 +282,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
           const float m_f = 2.0f * (float)keff * (float)seen / (float)(t + 1);
           const int m = (int)ceilf(m_f);
           tau = -INFINITY;
-          if (keff < t + 1 && m >= kMinSample && m <= kTrack && seen >= m) {
-#pragma unroll
-            for (int y = 0; y < kTrack; ++y)
-              if (y == m - 1) tau = top[y];
-          }
+          if (keff < t + 1 && m >= kMinSample && m <= kTrack && seen >= m) tau = sm.top[m - 1][et];
         }
       }
       if (row_ok) {
