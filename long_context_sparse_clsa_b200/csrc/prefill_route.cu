@@ -276,13 +276,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (++buf == 2) { buf = 0; ph_tfull ^= 1u; }
         if (it + 1 == ut.nwarm && row_ok) {
           // m-th largest warm-up score, m = twice the expected count of the sample above
-          // the k_eff boundary; no bound (tau = -inf, every token a candidate) when all
-          // tokens are selected or the sample is too small (m < kMinSample or > kTrack).
+          // the k_eff boundary (at most kTrack); no bound (tau = -inf, every token a
+          // candidate) when all tokens are selected or the sample is too small.
           // The bound is a guess: the densify step verifies it row by row.
           const float m_f = 2.0f * (float)keff * (float)seen / (float)(t + 1);
-          const int m = (int)ceilf(m_f);
+          const int m = min(kTrack, (int)ceilf(m_f));  // a shallower bound only raises the count
           tau = -INFINITY;
-          if (keff < t + 1 && m >= kMinSample && m <= kTrack && seen >= m) tau = sm.top[m - 1][et];
+          if (keff < t + 1 && m >= kMinSample && seen >= m) tau = sm.top[m - 1][et];
         }
       }
       if (row_ok) {
