@@ -76,8 +76,7 @@ constexpr uint32_t kAtomB = kRN * 128;
 
 struct RouteParams {
   int n, T, k, S, cap, nunits;
-  uint32_t* cand_val;  // [T][S][cap] candidate scores (fp32 bits)
-  int32_t* cand_tok;   // [T][S][cap]
+  uint2* cand;         // [T][S][cap] candidates: (score fp32 bits, token)
   int32_t* cand_cnt;   // [T][S]  (> cap: overflow)
   float* cand_tau;     // [T][S]  the bound the slice used (-inf: every token kept)
   uint32_t* any_flag;  // set by the densify step when some row needs the exact fallback
@@ -256,15 +255,24 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 low = sm.top[kTrack - 1][et];
               }
             }
-          } else {
+          } else if (nv >= 32 && cnt + 32 <= p.cap) {
+            // common case: all 32 columns visible, room for all: one compare and one
+            // predicated 8-byte store per score
+            uint2* dst = p.cand + slot;
+            const int jb = j0 + cb;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float val = __uint_as_float(v[c]);
-              if (c < nv && val >= tau) {
-                if (cnt < p.cap) {
-                  p.cand_val[slot + cnt] = v[c];
-                  p.cand_tok[slot + cnt] = j0 + cb + c;
-                }
+              if (__uint_as_float(v[c]) >= tau) {
+                dst[cnt] = make_uint2(v[c], (uint32_t)(jb + c));
+                ++cnt;
+              }
+            }
+          } else {
+            const int jb = j0 + cb;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (c < nv && __uint_as_float(v[c]) >= tau) {
+                if (cnt < p.cap) p.cand[slot + cnt] = make_uint2(v[c], (uint32_t)(jb + c));
                 ++cnt;
               }
             }
@@ -332,10 +340,10 @@ __global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams 
       const int o = off[s2], c = off[s2 + 1] - o;
       const size_t src = ((size_t)i * p.S + s2) * p.cap;
       for (int e = threadIdx.x; e < c; e += blockDim.x) {
-        const uint32_t v = p.cand_val[src + e];
-        dval[(size_t)i * ldd + o + e] = v;
-        dtok[(size_t)i * ldd + o + e] = p.cand_tok[src + e];
-        mine += __uint_as_float(v) >= tmax;
+        const uint2 cv = p.cand[src + e];
+        dval[(size_t)i * ldd + o + e] = cv.x;
+        dtok[(size_t)i * ldd + o + e] = (int32_t)cv.y;
+        mine += __uint_as_float(cv.x) >= tmax;
       }
     }
     if (mine) atomicAdd(&above, mine);
@@ -378,7 +386,7 @@ size_t prefill_route_ws_bytes(const clsa_prefill_args* a) {
   const RoutePlan rp = route_plan(a->n, a->T, a->k);
   const size_t T = (size_t)a->T;
   size_t off = 0;
-  off += 2 * align_up(T * rp.S * rp.cap * 4, 256);  // slice buffers (values, tokens)
+  off += align_up(T * rp.S * rp.cap * 8, 256);      // slice buffers (score, token)
   off += 2 * align_up(T * rp.S * 4, 256);           // slice counts, slice bounds
   off += 2 * align_up(T * rp.ldd * 4, 256);         // dense candidate rows
   off += 2 * align_up(T * 4, 256);                  // dense lengths, fallback flags
@@ -399,10 +407,8 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
   p.cap = rp.cap;
   p.nunits = rp.nunits;
   p.ws_header = ws_header;
-  p.cand_val = reinterpret_cast<uint32_t*>(w);
-  w += align_up(T * rp.S * rp.cap * 4, 256);
-  p.cand_tok = reinterpret_cast<int32_t*>(w);
-  w += align_up(T * rp.S * rp.cap * 4, 256);
+  p.cand = reinterpret_cast<uint2*>(w);
+  w += align_up(T * rp.S * rp.cap * 8, 256);
   p.cand_cnt = reinterpret_cast<int32_t*>(w);
   w += align_up(T * rp.S * 4, 256);
   p.cand_tau = reinterpret_cast<float*>(w);
