@@ -29,6 +29,7 @@
 // The exact TopK over each dense candidate row is the radix-select kernel of topk.cu.
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -80,6 +81,7 @@ struct RouteParams {
   int32_t* cand_cnt;   // [T][S]  (> cap: overflow)
   float* cand_tau;     // [T][S]  the bound the slice used (-inf: every token kept)
   uint32_t* any_flag;  // set by the densify step when some row needs the exact fallback
+  unsigned long long* trace;  // CTA 0 per-step stamps [3][512] (producer, MMA, epilogue) or null
   void* ws_header;
 };
 
@@ -166,6 +168,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         for (int it = 0; it < ut.count(); ++it) {
           if (!mbar_wait(&sm.empty[stage], ph_empty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 401); sm.abort_flag = 1; break; }
           const int j0 = ut.tile(it) * kRN;
+          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[it] = globaltimer_ns();
           mbar_arrive_expect_tx(&sm.full[stage], kBTile);
           for (int a = 0; a < 2; ++a) tma_load_2d(sB + stage * kBTile + a * kAtomB, &tk, a * 64, j0, &sm.full[stage]);
           if (++stage == kRStages) { stage = 0; ph_empty ^= 1u; }
@@ -203,6 +206,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
           }
           tc::mma_commit(&sm.empty[stage]);
           tc::mma_commit(&sm.tfull[buf]);
+          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[512 + it] = globaltimer_ns();
           if (++stage == kRStages) { stage = 0; ph_full ^= 1u; }
           if (++buf == 2) { buf = 0; ph_tempty ^= 1u; }
         }
@@ -281,6 +285,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+        if (p.trace && blockIdx.x == 0 && warp == 2 && lane == 0 && it < 512) p.trace[1024 + it] = globaltimer_ns();
         if (++buf == 2) { buf = 0; ph_tfull ^= 1u; }
         if (it + 1 == ut.nwarm && row_ok) {
           // m-th largest warm-up score, m = twice the expected count of the sample above
@@ -391,6 +396,7 @@ size_t prefill_route_ws_bytes(const clsa_prefill_args* a) {
   off += 2 * align_up(T * rp.ldd * 4, 256);         // dense candidate rows
   off += 2 * align_up(T * 4, 256);                  // dense lengths, fallback flags
   off += 256;                                       // any-flag word
+  off += 3 * 512 * 8;                               // step stamps (CLSA_TRACE=1)
   return off;
 }
 
@@ -422,6 +428,9 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
   out->flag = reinterpret_cast<int32_t*>(w);
   w += align_up(T * 4, 256);
   out->any_flag = reinterpret_cast<uint32_t*>(w);
+  w += 256;
+  const char* tr = std::getenv("CLSA_TRACE");
+  p.trace = (tr && tr[0] == '1') ? reinterpret_cast<unsigned long long*>(w) : nullptr;
   out->ldd = rp.ldd;
   p.any_flag = out->any_flag;
 
