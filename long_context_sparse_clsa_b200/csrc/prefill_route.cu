@@ -8,18 +8,22 @@
 //   unit     = two 128-row query blocks x one slice of the key range (so every CTA has
 //              work; the two blocks share each K_idx tile, halving its L2 traffic)
 //   warp 0   TMA producer: the unit's two Q_idx blocks once, then 128-key K_idx tiles
-//            into a 4-stage ring (128-byte swizzle, the UMMA K-major layout)
+//            into a 3-stage ring (128-byte swizzle, the UMMA K-major layout)
 //   warp 1   MMA issuer: per tile, 2 x 8 tcgen05.mma (M=128, N=128, K=16) into one of
 //            two TMEM buffers; commits free the ring stage and publish the buffer
-//   warps 2-9 epilogue, one query row per thread (TMEM lane): tcgen05.ld 128 scores,
-//            causal mask, then
-//              warm-up tiles: keep the row's 16 largest scores;
-//              threshold:     tau = the m-th largest of the warm-up sample, m chosen so
-//                             that ~2 k_eff tokens of the whole row score >= tau;
-//              every tile:    append (key, token) of scores >= tau to the row's slice
-//                             buffer, in token order.
+//   warps 2-9 epilogue, one query row per thread (TMEM lane): tcgen05.ld 32 scores at a
+//            time, causal mask, then
+//              warm-up tiles: a 32-bin histogram of the row's scores over
+//                             [mean, mean + 1.25 (max - mean)] of its first visible tile,
+//                             in a thread-private shared-memory column;
+//              threshold:     tau = the lower edge of the bin where the count from the
+//                             top reaches m, m chosen so that ~2 k_eff tokens of the
+//                             whole row score >= tau;
+//              every tile:    a bit mask of the 32 scores >= tau, the scores staged in a
+//                             private shared-memory row, and one (score, token) store per
+//                             set bit into the row's slice buffer, in token order.
 //   The warm-up tiles are spread over the slice and scored a second time in the main
-//   pass (about 4 extra tiles per ~100).
+//   pass (8 extra tiles per ~110).
 // prefill_densify_kernel: per row, concatenate the slice buffers (token order) into a
 //   dense candidate row.  The row is exact iff at least k_eff candidates score >= the
 //   largest tau any of its slices used: every dropped token then scores strictly below
@@ -68,7 +72,9 @@ constexpr int kRN = 128;        // keys per tile
 constexpr int kRStages = 3;     // K tile ring
 constexpr int kRThreads = 320;  // 10 warps
 constexpr int kWarm = 8;        // warm-up tiles per unit
-constexpr int kTrack = 32;      // largest warm-up scores kept per row
+constexpr int kBins = 32;       // warm-up histogram bins per row
+constexpr int kStagePitch = 36; // words per staged row
+constexpr int kTraceSlots = 12; // producer issue, MMA operands ready, MMA issued, 8 epilogue warps done
 constexpr int kMinSample = 8;   // fewer expected sample scores above the boundary: no bound
 constexpr uint32_t kABlock = kRM * 128 * 2;  // one query block, both 64-column atoms: 32 KiB
 constexpr uint32_t kBTile = kRN * 128 * 2;   // one key tile, both atoms: 32 KiB
@@ -81,12 +87,18 @@ struct RouteParams {
   int32_t* cand_cnt;   // [T][S]  (> cap: overflow)
   float* cand_tau;     // [T][S]  the bound the slice used (-inf: every token kept)
   uint32_t* any_flag;  // set by the densify step when some row needs the exact fallback
-  unsigned long long* trace;  // CTA 0 per-step stamps [3][512] (producer, MMA, epilogue) or null
+  unsigned long long* trace;  // CTA 0 per-step stamps [512][kTraceSlots] or null
   void* ws_header;
 };
 
 struct RouteSmem {
-  float top[kTrack][256];  // per epilogue thread (column): its row's largest warm-up scores, descending
+  // per epilogue thread, private: its row's warm-up histogram (column et of hist), then,
+  // in the main pass, its 32 staged scores (row et of stage, padded so that eight
+  // 16-byte stores of a quarter-warp hit distinct banks)
+  union {
+    uint32_t hist[kBins][256];
+    uint32_t stage[256][kStagePitch];
+  } u;
   uint64_t full[kRStages], empty[kRStages];
   uint64_t tfull[2], tempty[2];
   uint64_t afull, aempty;
@@ -94,6 +106,22 @@ struct RouteSmem {
   int abort_flag;
 };
 constexpr size_t kRouteSmem = 1024 /*align slack*/ + 2 * kABlock + kRStages * kBTile + sizeof(RouteSmem);
+
+// warm-up histogram bin of a score: round(sat(score * hs + hb) * (kBins - 1)), the
+// rounding done by adding 1.5 * 2^23 (the sum's low mantissa bits are the integer)
+__device__ __forceinline__ int hist_bin(uint32_t bits, float hs, float hb) {
+  const float x = __saturatef(fmaf(__uint_as_float(bits), hs, hb));
+  return __float_as_int(fmaf(x, (float)(kBins - 1), 12582912.f)) - 0x4B400000;
+}
+
+// predicated 8-byte global store (no branch)
+__device__ __forceinline__ void st_global_v2_if(uint2* p, uint32_t a, uint32_t b, bool pred) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %3, 0;\n @q st.global.v2.u32 [%0], {%1, %2};\n}" ::"l"(p), "r"(a),
+               "r"(b), "r"((uint32_t)pred));
+}
+
+// barrier among the eight epilogue warps only (named barrier 1)
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // the unit's tiles: main pass = [t_lo, t_hi); warm-up = kWarm tiles spread over it
 struct UnitTiles {
@@ -159,16 +187,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
       uint32_t ph_empty = 1, ph_aempty = 1;
       for (int u = blockIdx.x; u < p.nunits && !*(volatile int*)&sm.abort_flag; u += gridDim.x) {
         const UnitTiles ut = unit_tiles(p, u);
-        if (!mbar_wait(&sm.aempty, ph_aempty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 400); sm.abort_flag = 1; break; }
+        if (!mbar_wait_sleep(&sm.aempty, ph_aempty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 400); sm.abort_flag = 1; break; }
         ph_aempty ^= 1u;
         mbar_arrive_expect_tx(&sm.afull, 2 * kABlock);
         for (int h = 0; h < 2; ++h)
           for (int a = 0; a < 2; ++a)
             tma_load_2d(sA + h * kABlock + a * kAtomA, &tq, a * 64, ut.r0 + h * kRM, &sm.afull);
         for (int it = 0; it < ut.count(); ++it) {
-          if (!mbar_wait(&sm.empty[stage], ph_empty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 401); sm.abort_flag = 1; break; }
+          if (!mbar_wait_sleep(&sm.empty[stage], ph_empty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 401); sm.abort_flag = 1; break; }
           const int j0 = ut.tile(it) * kRN;
-          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[it] = globaltimer_ns();
+          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[it * kTraceSlots] = globaltimer_ns();
           mbar_arrive_expect_tx(&sm.full[stage], kBTile);
           for (int a = 0; a < 2; ++a) tma_load_2d(sB + stage * kBTile + a * kAtomB, &tk, a * 64, j0, &sm.full[stage]);
           if (++stage == kRStages) { stage = 0; ph_empty ^= 1u; }
@@ -183,10 +211,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
       uint32_t ph_full = 0, ph_tempty = 1, ph_afull = 0;
       for (int u = blockIdx.x; u < p.nunits && !*(volatile int*)&sm.abort_flag; u += gridDim.x) {
         const UnitTiles ut = unit_tiles(p, u);
-        if (!mbar_wait(&sm.afull, ph_afull)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 410); sm.abort_flag = 1; break; }
+        if (!mbar_wait_sleep(&sm.afull, ph_afull)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 410); sm.abort_flag = 1; break; }
         ph_afull ^= 1u;
         for (int it = 0; it < ut.count(); ++it) {
-          if (!mbar_wait(&sm.full[stage], ph_full) || !mbar_wait(&sm.tempty[buf], ph_tempty)) {
+          const bool got_full = mbar_wait_sleep(&sm.full[stage], ph_full);
+          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[it * kTraceSlots + 1] = globaltimer_ns();
+          if (!got_full || !mbar_wait_sleep(&sm.tempty[buf], ph_tempty)) {
             record_error(p.ws_header, CLSA_ERR_TIMEOUT, 411);
             sm.abort_flag = 1;
             break;
@@ -206,7 +236,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
           }
           tc::mma_commit(&sm.empty[stage]);
           tc::mma_commit(&sm.tfull[buf]);
-          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[512 + it] = globaltimer_ns();
+          if (p.trace && blockIdx.x == 0 && it < 512) p.trace[it * kTraceSlots + 2] = globaltimer_ns();
           if (++stage == kRStages) { stage = 0; ph_full ^= 1u; }
           if (++buf == 2) { buf = 0; ph_tempty ^= 1u; }
         }
@@ -217,67 +247,134 @@ __global__ void __launch_bounds__(kRThreads, 1)
     // ------------------------------------------------------------ epilogue (one row per thread)
     const int q = warp & 3;             // TMEM lane quarter this warp may read
     const int h = (warp - 2) >> 2;      // query block of this warpgroup
+    const int et = threadIdx.x - 64;    // epilogue thread 0..255: its private smem column / row
+    uint32_t* const stage = sm.u.stage[et];
     int buf = 0;
     uint32_t ph_tfull = 0;
-    for (int u = blockIdx.x; u < p.nunits && !*(volatile int*)&sm.abort_flag; u += gridDim.x) {
+    bool dead = false;
+    // Every epilogue warp runs the same units and steps, so the named barriers below
+    // match even after a timeout (a dead warp keeps stepping without touching TMEM).
+    for (int u = blockIdx.x; u < p.nunits; u += gridDim.x) {
+      epi_bar();  // the previous unit's staging rows are free for this unit's histograms
       const UnitTiles ut = unit_tiles(p, u);
       const int s = u % p.S;
       const int i = ut.r0 + h * kRM + q * 32 + lane;  // query row
       const bool row_ok = i < p.T;
       const int t = p.n - p.T + i;                    // its cache position
       const int keff = min(p.k, t + 1);
-      const int et = threadIdx.x - 64;  // epilogue thread 0..255: its column of sm.top
-      for (int y = 0; y < kTrack; ++y) sm.top[y][et] = -INFINITY;
+#pragma unroll
+      for (int y = 0; y < kBins; ++y) sm.u.hist[y][et] = 0u;
+      bool have = false;       // histogram range fixed
+      float hs = 0.f, hb = 0.f, lo = 0.f, span = 0.f;  // bin map: sat(score * hs + hb) * (kBins - 1)
       int seen = 0, cnt = 0;
       float tau = -INFINITY;
-      const size_t slot = ((size_t)(row_ok ? i : 0) * p.S + s) * p.cap;
+      uint2* const dst = p.cand + ((size_t)(row_ok ? i : 0) * p.S + s) * p.cap;
+      const int capm1 = p.cap - 1;
       for (int it = 0; it < ut.count(); ++it) {
-        if (!mbar_wait(&sm.tfull[buf], ph_tfull)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 420); sm.abort_flag = 1; break; }
+        if (!dead && !mbar_wait_sleep(&sm.tfull[buf], ph_tfull)) {
+          record_error(p.ws_header, CLSA_ERR_TIMEOUT, 420);
+          sm.abort_flag = 1;
+          dead = true;
+        }
+        dead = __any_sync(0xffffffffu, dead || *(volatile int*)&sm.abort_flag);
         tc::fence_after_sync();
         const int j0 = ut.tile(it) * kRN;
         const bool warm = it < ut.nwarm;
-#pragma unroll 1
-        for (int cb = 0; cb < kRN; cb += 32) {
-          uint32_t v[32];
-          tc::ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + h * kRN + cb), v);
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + h * kRN);
+        if (!dead) {
+          uint32_t v[kRN];
+          tc::ld_32x32b_x128(tbase, v);
           tc::ld_wait();
-          if (!row_ok) continue;
-          const int nv = min(32, t - (j0 + cb) + 1);  // causally visible columns of this chunk
+          const int nvis = row_ok ? max(0, min(kRN, t - j0 + 1)) : 0;  // causally visible columns
           if (warm) {
-            float low = sm.top[kTrack - 1][et];
-            seen += max(0, nv);
+            if (__any_sync(0xffffffffu, !have)) {
+              // histogram range from this tile's visible scores: [mean, mean + 1.25 (max -
+              // mean)]; larger scores count in the top bin, smaller ones in bin 0
+              float mx = -INFINITY, s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float val = __uint_as_float(v[c]);
-              if (c < nv && val > low) {
-                int y = kTrack - 1;  // insertion from the bottom of the descending list
-                while (y > 0 && sm.top[y - 1][et] < val) {
-                  sm.top[y][et] = sm.top[y - 1][et];
-                  --y;
+              for (int c = 0; c < kRN; c += 2) {
+                if (c < nvis) {
+                  mx = fmaxf(mx, __uint_as_float(v[c]));
+                  s0 += __uint_as_float(v[c]);
                 }
-                sm.top[y][et] = val;
-                low = sm.top[kTrack - 1][et];
+                if (c + 1 < nvis) {
+                  mx = fmaxf(mx, __uint_as_float(v[c + 1]));
+                  s1 += __uint_as_float(v[c + 1]);
+                }
+              }
+              if (!have && nvis > 0) {
+                lo = (s0 + s1) / (float)nvis;
+                span = 1.25f * (mx - lo);
+                if (span > 0.f && span < INFINITY) {
+                  hs = 1.f / span;
+                  hb = -lo * hs;
+                  have = true;
+                }
               }
             }
-          } else if (nv >= 32 && cnt + 32 <= p.cap) {
-            // common case: all 32 columns visible, room for all: one compare and one
-            // predicated 8-byte store per score
-            uint2* dst = p.cand + slot;
-            const int jb = j0 + cb;
+            if (have) {
+              seen += nvis;
+              if (nvis == kRN) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (__uint_as_float(v[c]) >= tau) {
-                dst[cnt] = make_uint2(v[c], (uint32_t)(jb + c));
-                ++cnt;
+                for (int c = 0; c < kRN; ++c) atomicAdd(&sm.u.hist[hist_bin(v[c], hs, hb)][et], 1u);
+              } else {
+#pragma unroll
+                for (int c = 0; c < kRN; ++c)
+                  if (c < nvis) atomicAdd(&sm.u.hist[hist_bin(v[c], hs, hb)][et], 1u);
               }
             }
           } else {
-            const int jb = j0 + cb;
+            // one compare per score into four 32-bit masks (independent chains)
+            uint32_t mk[4];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c < nv && __uint_as_float(v[c]) >= tau) {
-                if (cnt < p.cap) p.cand[slot + cnt] = make_uint2(v[c], (uint32_t)(jb + c));
-                ++cnt;
+            for (int k = 0; k < 4; ++k) {
+              uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                a0 |= __uint_as_float(v[32 * k + c]) >= tau ? 1u << c : 0u;
+                a1 |= __uint_as_float(v[32 * k + c + 8]) >= tau ? 1u << (c + 8) : 0u;
+                a2 |= __uint_as_float(v[32 * k + c + 16]) >= tau ? 1u << (c + 16) : 0u;
+                a3 |= __uint_as_float(v[32 * k + c + 24]) >= tau ? 1u << (c + 24) : 0u;
+              }
+              mk[k] = (a0 | a1) | (a2 | a3);
+            }
+            if (nvis < kRN) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int nv = nvis - 32 * k;
+                mk[k] &= nv >= 32 ? 0xffffffffu : nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
+              }
+            }
+            // per 32 columns: stage the scores in this thread's smem row, then one
+            // (score, token) store per set bit, in column order; the first four without
+            // branches, the rare rest in a loop.  Overflow past the buffer is counted
+            // (the row is flagged) and written to its last slot.
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              uint32_t mm = mk[k];
+              if (__any_sync(0xffffffffu, mm != 0u)) {
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                  reinterpret_cast<uint4*>(stage)[c4] = make_uint4(v[32 * k + 4 * c4], v[32 * k + 4 * c4 + 1],
+                                                                   v[32 * k + 4 * c4 + 2], v[32 * k + 4 * c4 + 3]);
+                const uint32_t jb = (uint32_t)(j0 + 32 * k);
+                const int pc = __popc(mm);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c = (__ffs(mm) - 1) & 31;
+                  st_global_v2_if(dst + min(cnt + e, capm1), stage[c], jb + (uint32_t)c, mm != 0u);
+                  mm &= mm - 1u;
+                }
+                if (__any_sync(0xffffffffu, mm != 0u)) {
+                  int e = 4;
+                  while (mm) {
+                    const int c = __ffs(mm) - 1;
+                    dst[min(cnt + e, capm1)] = make_uint2(stage[c], jb + (uint32_t)c);
+                    ++e;
+                    mm &= mm - 1u;
+                  }
+                }
+                cnt += pc;
               }
             }
           }
@@ -285,17 +382,28 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
-        if (p.trace && blockIdx.x == 0 && warp == 2 && lane == 0 && it < 512) p.trace[1024 + it] = globaltimer_ns();
+        if (p.trace && blockIdx.x == 0 && lane == 0 && it < 512) p.trace[it * kTraceSlots + 1 + warp] = globaltimer_ns();
         if (++buf == 2) { buf = 0; ph_tfull ^= 1u; }
-        if (it + 1 == ut.nwarm && row_ok) {
-          // m-th largest warm-up score, m = twice the expected count of the sample above
-          // the k_eff boundary (at most kTrack); no bound (tau = -inf, every token a
-          // candidate) when all tokens are selected or the sample is too small.
-          // The bound is a guess: the densify step verifies it row by row.
-          const float m_f = 2.0f * (float)keff * (float)seen / (float)(t + 1);
-          const int m = min(kTrack, (int)ceilf(m_f));  // a shallower bound only raises the count
+        if (it + 1 == ut.nwarm) {
+          // lower edge of the highest bin at which the sample count from the top reaches
+          // m = twice the expected count of the sample above the k_eff boundary; no bound
+          // (tau = -inf, every token a candidate) when all tokens are selected or the
+          // sample is too small.  The bound is a guess: the densify step verifies it.
           tau = -INFINITY;
-          if (keff < t + 1 && m >= kMinSample && seen >= m) tau = sm.top[m - 1][et];
+          if (have && keff < t + 1) {
+            const int m = (int)ceilf(2.0f * (float)keff * (float)seen / (float)(t + 1));
+            if (m >= kMinSample && seen >= m) {
+              int cum = 0;
+              for (int y = kBins - 1; y >= 1; --y) {  // bin 0 also holds every lower score
+                cum += (int)sm.u.hist[y][et];
+                if (cum >= m) {
+                  tau = lo + ((float)y - 0.5f) * span / (float)(kBins - 1);
+                  break;
+                }
+              }
+            }
+          }
+          epi_bar();  // every histogram is read: the staging rows may overwrite them
         }
       }
       if (row_ok) {
@@ -396,7 +504,7 @@ size_t prefill_route_ws_bytes(const clsa_prefill_args* a) {
   off += 2 * align_up(T * rp.ldd * 4, 256);         // dense candidate rows
   off += 2 * align_up(T * 4, 256);                  // dense lengths, fallback flags
   off += 256;                                       // any-flag word
-  off += 3 * 512 * 8;                               // step stamps (CLSA_TRACE=1)
+  off += 512 * kTraceSlots * 8;                     // step stamps (CLSA_TRACE=1)
   return off;
 }
 
