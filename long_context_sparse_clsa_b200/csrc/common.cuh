@@ -259,6 +259,32 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) 
   }
   return true;
 }
+// Non-suspending probe of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Warp-wide bounded wait: lane 0 polls without suspending, the others wait at the
+// warp barrier, then every lane observes the completed phase itself.  Call with the
+// whole warp converged; returns the same value in every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  uint32_t ok = 1;
+  if ((threadIdx.x & 31) == 0 && !mbar_test_wait(bar, parity)) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_test_wait(bar, parity)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        ok = 0;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) ok = mbar_test_wait(bar, parity) ? 1u : 0u;  // completed: true at once, with ordering
+  return __all_sync(0xffffffffu, ok != 0);
+}
 // global -> shared bulk copy completing on `bar` (dst, src 16-byte aligned, bytes % 16 == 0)
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

@@ -74,7 +74,7 @@ constexpr int kRThreads = 320;  // 10 warps
 constexpr int kWarm = 8;        // warm-up tiles per unit
 constexpr int kBins = 32;       // warm-up histogram bins per row
 constexpr int kStagePitch = 36; // words per staged row
-constexpr int kTraceSlots = 12; // producer issue, MMA operands ready, MMA issued, 8 epilogue warps done
+constexpr int kTraceSlots = 20; // producer issue, MMA operands ready, MMA issued, epilogue warps done, started
 constexpr int kMinSample = 8;   // fewer expected sample scores above the boundary: no bound
 constexpr uint32_t kABlock = kRM * 128 * 2;  // one query block, both 64-column atoms: 32 KiB
 constexpr uint32_t kBTile = kRN * 128 * 2;   // one key tile, both atoms: 32 KiB
@@ -112,6 +112,31 @@ constexpr size_t kRouteSmem = 1024 /*align slack*/ + 2 * kABlock + kRStages * kB
 __device__ __forceinline__ int hist_bin(uint32_t bits, float hs, float hb) {
   const float x = __saturatef(fmaf(__uint_as_float(bits), hs, hb));
   return __float_as_int(fmaf(x, (float)(kBins - 1), 12582912.f)) - 0x4B400000;
+}
+
+// shared-memory increment by shared-window address (a generic atomic is slower)
+__device__ __forceinline__ void red_shared_inc(uint32_t addr) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+}
+
+// 1 when score >= tau, else 0 (exactly; a difference below 2^-100 in magnitude also
+// gives 1, which only adds a candidate)
+__device__ __forceinline__ float ge01(uint32_t bits, float tau) {
+  return __saturatef(fmaf(__fsub_rn(__uint_as_float(bits), tau), 0x1p100f, 1.f));
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t x;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x) : "r"(addr) : "memory");
+  return x;
+}
+
+// 16-byte shared store, done only when `pred` is non-zero (no branch)
+__device__ __forceinline__ void st_shared_v4_if(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                                uint32_t pred) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %5, 0;\n @q st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n}" ::"r"(addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(pred)
+               : "memory");
 }
 
 // predicated 8-byte global store (no branch)
@@ -248,7 +273,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
     const int q = warp & 3;             // TMEM lane quarter this warp may read
     const int h = (warp - 2) >> 2;      // query block of this warpgroup
     const int et = threadIdx.x - 64;    // epilogue thread 0..255: its private smem column / row
-    uint32_t* const stage = sm.u.stage[et];
+    const uint32_t hist_col = smem_u32(&sm.u.hist[0][et]);  // bin b at + b * 1024 bytes
+    const uint32_t stage_addr = smem_u32(sm.u.stage[et] + 4);  // scores at words 4..35; word 3 is read for an empty mask
     int buf = 0;
     uint32_t ph_tfull = 0;
     bool dead = false;
@@ -269,112 +295,133 @@ __global__ void __launch_bounds__(kRThreads, 1)
       int seen = 0, cnt = 0;
       float tau = -INFINITY;
       uint2* const dst = p.cand + ((size_t)(row_ok ? i : 0) * p.S + s) * p.cap;
-      const int capm1 = p.cap - 1;
       for (int it = 0; it < ut.count(); ++it) {
-        if (!dead && !mbar_wait_sleep(&sm.tfull[buf], ph_tfull)) {
-          record_error(p.ws_header, CLSA_ERR_TIMEOUT, 420);
+        if (!dead && !mbar_wait_warp(&sm.tfull[buf], ph_tfull)) {
+          if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 420);
           sm.abort_flag = 1;
           dead = true;
         }
         dead = __any_sync(0xffffffffu, dead || *(volatile int*)&sm.abort_flag);
+        if (p.trace && blockIdx.x == 0 && lane == 0 && it < 512) p.trace[it * kTraceSlots + 8 + 1 + warp] = globaltimer_ns();
         tc::fence_after_sync();
         const int j0 = ut.tile(it) * kRN;
         const bool warm = it < ut.nwarm;
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + h * kRN);
-        if (!dead) {
-          uint32_t v[kRN];
-          tc::ld_32x32b_x128(tbase, v);
-          tc::ld_wait();
-          const int nvis = row_ok ? max(0, min(kRN, t - j0 + 1)) : 0;  // causally visible columns
-          if (warm) {
-            if (__any_sync(0xffffffffu, !have)) {
-              // histogram range from this tile's visible scores: [mean, mean + 1.25 (max -
-              // mean)]; larger scores count in the top bin, smaller ones in bin 0
-              float mx = -INFINITY, s0 = 0.f, s1 = 0.f;
+        const int nvis = row_ok ? max(0, min(kRN, t - j0 + 1)) : 0;  // causally visible columns
+        if (!dead && warm && __any_sync(0xffffffffu, !have)) {
+          // histogram range from this tile's visible scores: [mean, mean + 1.25 (max -
+          // mean)]; larger scores count in the top bin, smaller ones in bin 0
+          float mx = -INFINITY, s0 = 0.f, s1 = 0.f;
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t v[64];
+            tc::ld_32x32b_x64(tbase + (uint32_t)(64 * hf), v);
+            tc::ld_wait();
 #pragma unroll
-              for (int c = 0; c < kRN; c += 2) {
-                if (c < nvis) {
-                  mx = fmaxf(mx, __uint_as_float(v[c]));
-                  s0 += __uint_as_float(v[c]);
-                }
-                if (c + 1 < nvis) {
-                  mx = fmaxf(mx, __uint_as_float(v[c + 1]));
-                  s1 += __uint_as_float(v[c + 1]);
-                }
+            for (int c = 0; c < 64; c += 2) {
+              if (64 * hf + c < nvis) {
+                mx = fmaxf(mx, __uint_as_float(v[c]));
+                s0 += __uint_as_float(v[c]);
               }
-              if (!have && nvis > 0) {
-                lo = (s0 + s1) / (float)nvis;
-                span = 1.25f * (mx - lo);
-                if (span > 0.f && span < INFINITY) {
-                  hs = 1.f / span;
-                  hb = -lo * hs;
-                  have = true;
-                }
+              if (64 * hf + c + 1 < nvis) {
+                mx = fmaxf(mx, __uint_as_float(v[c + 1]));
+                s1 += __uint_as_float(v[c + 1]);
               }
             }
-            if (have) {
-              seen += nvis;
-              if (nvis == kRN) {
-#pragma unroll
-                for (int c = 0; c < kRN; ++c) atomicAdd(&sm.u.hist[hist_bin(v[c], hs, hb)][et], 1u);
-              } else {
-#pragma unroll
-                for (int c = 0; c < kRN; ++c)
-                  if (c < nvis) atomicAdd(&sm.u.hist[hist_bin(v[c], hs, hb)][et], 1u);
-              }
+          }
+          if (!have && nvis > 0) {
+            lo = (s0 + s1) / (float)nvis;
+            span = 1.25f * (mx - lo);
+            if (span > 0.f && span < INFINITY) {
+              hs = 1.f / span;
+              hb = -lo * hs;
+              have = true;
             }
-          } else {
-            // one compare per score into four 32-bit masks (independent chains)
-            uint32_t mk[4];
+          }
+        }
+        if (!dead && warm && have) seen += nvis;
+        if (!dead && !(warm && !__any_sync(0xffffffffu, have))) {
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t v[64];
+            tc::ld_32x32b_x64(tbase + (uint32_t)(64 * hf), v);
+            tc::ld_wait();
+            const int nvh = nvis - 64 * hf;  // visible columns of this half (may be <= 0 or > 64)
+            if (warm) {
+              if (have) {
+                if (nvh >= 64) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+                  for (int c = 0; c < 64; ++c) red_shared_inc(hist_col + (uint32_t)hist_bin(v[c], hs, hb) * 1024u);
+                } else {
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                a0 |= __uint_as_float(v[32 * k + c]) >= tau ? 1u << c : 0u;
-                a1 |= __uint_as_float(v[32 * k + c + 8]) >= tau ? 1u << (c + 8) : 0u;
-                a2 |= __uint_as_float(v[32 * k + c + 16]) >= tau ? 1u << (c + 16) : 0u;
-                a3 |= __uint_as_float(v[32 * k + c + 24]) >= tau ? 1u << (c + 24) : 0u;
-              }
-              mk[k] = (a0 | a1) | (a2 | a3);
-            }
-            if (nvis < kRN) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int nv = nvis - 32 * k;
-                mk[k] &= nv >= 32 ? 0xffffffffu : nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
-              }
-            }
-            // per 32 columns: stage the scores in this thread's smem row, then one
-            // (score, token) store per set bit, in column order; the first four without
-            // branches, the rare rest in a loop.  Overflow past the buffer is counted
-            // (the row is flagged) and written to its last slot.
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint32_t mm = mk[k];
-              if (__any_sync(0xffffffffu, mm != 0u)) {
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                  reinterpret_cast<uint4*>(stage)[c4] = make_uint4(v[32 * k + 4 * c4], v[32 * k + 4 * c4 + 1],
-                                                                   v[32 * k + 4 * c4 + 2], v[32 * k + 4 * c4 + 3]);
-                const uint32_t jb = (uint32_t)(j0 + 32 * k);
-                const int pc = __popc(mm);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int c = (__ffs(mm) - 1) & 31;
-                  st_global_v2_if(dst + min(cnt + e, capm1), stage[c], jb + (uint32_t)c, mm != 0u);
-                  mm &= mm - 1u;
+                  for (int c = 0; c < 64; ++c)
+                    if (c < nvh) red_shared_inc(hist_col + (uint32_t)hist_bin(v[c], hs, hb) * 1024u);
                 }
+              }
+            } else {
+              // one compare per score into two 32-bit masks, on the FMA pipe: ge01 is exactly
+              // 1 or 0, and the weighted sums of 16 of them are exact integers
+              uint32_t mk[2];
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                float l0 = 0.f, l1 = 0.f, u0 = 0.f, u1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {
+                  l0 = fmaf(ge01(v[32 * k + c], tau), (float)(1u << c), l0);
+                  l1 = fmaf(ge01(v[32 * k + c + 1], tau), (float)(1u << (c + 1)), l1);
+                  u0 = fmaf(ge01(v[32 * k + 16 + c], tau), (float)(1u << c), u0);
+                  u1 = fmaf(ge01(v[32 * k + 16 + c + 1], tau), (float)(1u << (c + 1)), u1);
+                }
+                // 2^23 + m (m < 2^16) is exact: the low 16 bits of its encoding are m
+                mk[k] = __byte_perm(__float_as_uint((l0 + l1) + 8388608.f), __float_as_uint((u0 + u1) + 8388608.f),
+                                    0x5410);
+                const int nv = nvh - 32 * k;
+                if (nv < 32) mk[k] &= nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
+              }
+              // per 32 columns: stage the scores of every 4-column group that holds a
+              // candidate of this row in its smem row, then one (score, token) store per set
+              // bit, in column order
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                uint32_t mm = mk[k];
                 if (__any_sync(0xffffffffu, mm != 0u)) {
-                  int e = 4;
-                  while (mm) {
-                    const int c = __ffs(mm) - 1;
-                    dst[min(cnt + e, capm1)] = make_uint2(stage[c], jb + (uint32_t)c);
-                    ++e;
-                    mm &= mm - 1u;
+#pragma unroll
+                  for (int g = 0; g < 8; ++g)
+                    st_shared_v4_if(stage_addr + 16u * g, v[32 * k + 4 * g], v[32 * k + 4 * g + 1],
+                                    v[32 * k + 4 * g + 2], v[32 * k + 4 * g + 3], (mm >> (4 * g)) & 0xfu);
+                  const uint32_t jb = (uint32_t)(j0 + 64 * hf + 32 * k);
+                  const int pc = __popc(mm);
+                  if (cnt + pc <= p.cap) {
+                    // common case: room for every candidate; the first four without
+                    // branches (immediate offsets from one pointer), the rare rest in a loop
+                    uint2* const out = dst + cnt;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                      const uint32_t lsb = mm & (0u - mm);
+                      const int c = 31 - __clz(lsb);  // -1 when mm == 0: reads the pad word, store off
+                      st_global_v2_if(out + e, ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c, mm != 0u);
+                      mm ^= lsb;
+                    }
+                    if (__any_sync(0xffffffffu, mm != 0u)) {
+                      int e = 4;
+                      while (mm) {
+                        const int c = __ffs(mm) - 1;
+                        out[e++] = make_uint2(ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c);
+                        mm &= mm - 1u;
+                      }
+                    }
+                  } else {
+                    // overflow: keep counting (the row is flagged), stop writing past the buffer
+                    int e = 0;
+                    while (mm) {
+                      const int c = __ffs(mm) - 1;
+                      if (cnt + e < p.cap) dst[cnt + e] = make_uint2(ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c);
+                      ++e;
+                      mm &= mm - 1u;
+                    }
                   }
+                  cnt += pc;
                 }
-                cnt += pc;
               }
             }
           }
