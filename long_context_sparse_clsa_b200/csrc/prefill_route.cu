@@ -119,10 +119,20 @@ __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
 
-// 1 when score >= tau, else 0 (exactly; a difference below 2^-100 in magnitude also
-// gives 1, which only adds a candidate)
-__device__ __forceinline__ float ge01(uint32_t bits, float tau) {
-  return __saturatef(fmaf(__fsub_rn(__uint_as_float(bits), tau), 0x1p100f, 1.f));
+// 1 when score >= tau, else 0, in one saturating FMA.  With tb = nextbelow(tau), a
+// power of two sc = 2^(100 - exponent of tau) and negt = -tb * sc (both exact),
+// score * sc + negt is (score - tb) * sc rounded once: >= 1 when score >= tau (the gap
+// tau - tb is 2^-23 |tau| or more, times sc >= 2^77), <= 0 when score <= tb; an
+// infinite product keeps its sign.  |tau| < 2^-20 is lowered to -2^-20 first (a lower
+// bound only adds candidates).  Keep-all rows (tau = -inf) do not use it.
+__device__ __forceinline__ float ge01(uint32_t bits, float sc, float negt) {
+  return __saturatef(fmaf(__uint_as_float(bits), sc, negt));
+}
+__device__ __forceinline__ void ge_setup(float tau, float& sc, float& negt) {
+  if (fabsf(tau) < 0x1p-20f) tau = -0x1p-20f;
+  const int e = ((__float_as_int(tau) >> 23) & 0xff) - 127;  // exponent (tau normal here)
+  sc = __int_as_float((127 + 100 - e) << 23);                 // 2^(100 - e), e in [-20, 127]
+  negt = -nextafterf(tau, -INFINITY) * sc;
 }
 
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
@@ -361,20 +371,23 @@ __global__ void __launch_bounds__(kRThreads, 1)
             } else {
               // one compare per score into two 32-bit masks, on the FMA pipe: ge01 is exactly
               // 1 or 0, and the weighted sums of 16 of them are exact integers
+              float sc = 1.f, negt = 0.f;
+              ge_setup(tau, sc, negt);
               uint32_t mk[2];
 #pragma unroll
               for (int k = 0; k < 2; ++k) {
                 float l0 = 0.f, l1 = 0.f, u0 = 0.f, u1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < 16; c += 2) {
-                  l0 = fmaf(ge01(v[32 * k + c], tau), (float)(1u << c), l0);
-                  l1 = fmaf(ge01(v[32 * k + c + 1], tau), (float)(1u << (c + 1)), l1);
-                  u0 = fmaf(ge01(v[32 * k + 16 + c], tau), (float)(1u << c), u0);
-                  u1 = fmaf(ge01(v[32 * k + 16 + c + 1], tau), (float)(1u << (c + 1)), u1);
+                  l0 = fmaf(ge01(v[32 * k + c], sc, negt), (float)(1u << c), l0);
+                  l1 = fmaf(ge01(v[32 * k + c + 1], sc, negt), (float)(1u << (c + 1)), l1);
+                  u0 = fmaf(ge01(v[32 * k + 16 + c], sc, negt), (float)(1u << c), u0);
+                  u1 = fmaf(ge01(v[32 * k + 16 + c + 1], sc, negt), (float)(1u << (c + 1)), u1);
                 }
                 // 2^23 + m (m < 2^16) is exact: the low 16 bits of its encoding are m
                 mk[k] = __byte_perm(__float_as_uint((l0 + l1) + 8388608.f), __float_as_uint((u0 + u1) + 8388608.f),
                                     0x5410);
+                if (tau == -INFINITY) mk[k] = 0xffffffffu;  // keep-all row
                 const int nv = nvh - 32 * k;
                 if (nv < 32) mk[k] &= nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
               }
