@@ -4,13 +4,16 @@ L-layer sparse GQA attention) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode128k]
                     [--impl {clsa,reference}] [--no-graph] [--no-cpu-baseline]
+                    [--l2 {rotate,flush}] [--sets R]
 
 One JSON line on rank 0.  A step is one decode token per sequence through the
 whole path; the default workload is the 128K-context decode (batch 1, n=131072,
 d_idx=128, k=2048, L=24, 32 query / 8 KV heads, d=128, bf16, 1% planted tokens).
 Device time is measured with CUDA events around each step on the stream the
-library launches on, with L2 flushed (a 512 MiB write and read-back) before every step
-outside the timed events.  With N > 1 every rank runs its own sequences (weak
+library launches on.  Between steps the inputs rotate through R sets whose K_idx
+copies together exceed twice the 126 MB L2 (``--l2 rotate``, the default: each step
+reads its K_idx and K/V rows from HBM, the kernel code stays cached), or L2 is
+flushed by a 512 MiB write and read-back outside the timed events (``--l2 flush``).  With N > 1 every rank runs its own sequences (weak
 scaling, no collective on the data path); the step time is the max over ranks.
 
 ``--impl reference`` times the CPU oracle (float64 numpy) on the host cores on a
@@ -46,6 +49,9 @@ def parse():
     ap.add_argument("--workload", default="decode128k")
     ap.add_argument("--impl", default="clsa", choices=["clsa", "reference"])
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
+                    help="between steps: rotate through input sets larger than L2 (default), or flush L2")
+    ap.add_argument("--sets", type=int, default=6, help="input sets rotated through (--l2 rotate)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-steps", type=int, default=2)
     return ap.parse_args()
@@ -228,8 +234,28 @@ def run_clsa(args):
     L, B, Hq, d, k = w.L, w.B, w.Hq, w.d, w.k
     out = {"O": torch.empty_like(dv["Q"]), "idx": torch.empty(B, k, dtype=torch.int32, device=dev),
            "count": torch.empty(B, dtype=torch.int32, device=dev)}
-    a = clsa.decode_args(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], k, out["O"],
-                         out["idx"], out["count"])
+    # Input sets: set 0 is the seeded workload; set r > 0 permutes the rows of every
+    # sequence's K_idx (the same scores, planted tokens included, at other positions, so
+    # each set selects and gathers other K/V rows).  With --l2 rotate, step i uses set
+    # i % R and the R K_idx copies together exceed L2, so every step streams its K_idx
+    # and K/V rows from HBM while the kernel code stays cached; with --l2 flush, one set
+    # and a 512 MiB write + read-back before every step.
+    kidx_bytes = dv["k_idx"].numel() * dv["k_idx"].element_size()
+    R = 1
+    if args.l2 == "rotate":  # at least two sets, and at least twice L2 in K_idx alone
+        R = max(2, min(max(1, args.sets), 16), int(np.ceil(2 * 126e6 / kidx_bytes)))
+    gen = torch.Generator(device="cpu").manual_seed(1234 + rank)
+    kidx_sets = [dv["k_idx"]]
+    for r in range(1, R):
+        kr = dv["k_idx"].clone()
+        for b in range(B):
+            nb = int(inp.seq_lens[b])
+            perm = torch.randperm(nb, generator=gen).to(dev)
+            kr[b, :nb] = dv["k_idx"][b, perm]
+        kidx_sets.append(kr)
+    args_sets = [clsa.decode_args(dv["q_idx"], kx, dv["K"], dv["V"], dv["Q"], dv["seq_lens"], k, out["O"],
+                                  out["idx"], out["count"]) for kx in kidx_sets]
+    a = args_sets[0]
     ws = clsa.Workspace(clsa.decode_workspace_size(a))
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     flush_view = flush.view(torch.int32)
@@ -240,13 +266,17 @@ def run_clsa(args):
         flush.fill_(1)
         flush_view.max()
 
-    def step():
-        clsa.decode_step_args(a, ws)
+    def between_steps():
+        if args.l2 == "flush":
+            flush_l2()
+
+    def step(r=0):
+        clsa.decode_step_args(args_sets[r], ws)
 
     step()
     torch.cuda.synchronize()
     launches_per_step = clsa.last_launch_count()
-    graph = None
+    graphs = None
     if not args.no_graph:
         try:
             s2 = torch.cuda.Stream()
@@ -255,23 +285,26 @@ def run_clsa(args):
                 step()
             stream.wait_stream(s2)
             torch.cuda.synchronize()
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                step()
+            graphs = []
+            for r in range(R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    step(r)
+                graphs.append(g)
             torch.cuda.synchronize()
         except Exception as ex:  # graph capture unsupported: time eager launches
-            graph = None
+            graphs = None
             print(f"# graph capture failed, timing eager launches: {ex}", file=sys.stderr)
 
-    def run_step():
-        if graph is not None:
-            graph.replay()
+    def run_step(i):
+        if graphs is not None:
+            graphs[i % R].replay()
         else:
-            step()
+            step(i % R)
 
-    for _ in range(max(args.warmup, 3)):
-        flush_l2()
-        run_step()
+    for i in range(max(args.warmup, 3, R)):
+        between_steps()
+        run_step(i)
     torch.cuda.synchronize()
 
     def barrier():
@@ -283,10 +316,10 @@ def run_clsa(args):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     with ClockSampler(local) as clk:
-        for e0, e1 in evs:
-            flush_l2()
+        for i, (e0, e1) in enumerate(evs):
+            between_steps()
             e0.record(stream)
-            run_step()
+            run_step(i)
             e1.record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -362,12 +395,12 @@ def run_clsa(args):
     e2e_steps = min(args.steps, 50)
     tot = 0.0
     for i in range(e2e_steps + 3):
-        flush_l2()
+        between_steps()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         dv["q_idx"].copy_(q_idx_h, non_blocking=True)
         dv["Q"].copy_(Q_h, non_blocking=True)
-        clsa.decode_step_args(a, ws)
+        clsa.decode_step_args(args_sets[i % R], ws)
         O_h.copy_(out["O"], non_blocking=True)
         idx_h.copy_(out["idx"], non_blocking=True)
         cnt_h.copy_(out["count"], non_blocking=True)
@@ -400,8 +433,11 @@ def run_clsa(args):
         "data": "synthetic (seeded N(0,1), 1% planted index keys)",
         "config": {"workload": w.name, "B": w.B, "n": w.n_max, "d_idx": w.d_idx, "k": w.k, "L": w.L,
                    "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every step (512 MiB write + read-back, outside the timed events)",
-                   "launch": "cuda graph" if graph is not None else "eager"},
+                   "l2": (f"inputs larger than L2: {R} rotating K_idx sets ({R * kidx_bytes / 2**20:.0f} MiB, row "
+                          f"permutations of the seeded cache), step i uses set i % {R}; no flush"
+                          if args.l2 == "rotate" else
+                          "flushed before every step (512 MiB write + read-back, outside the timed events)"),
+                   "launch": "cuda graph" if graphs is not None else "eager"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": dom_bytes, "us_per_launch": dom_us},

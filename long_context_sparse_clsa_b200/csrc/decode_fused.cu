@@ -13,19 +13,19 @@
 //     8 rows in flight per lane group, fp32 dot product, shuffle reduce.  (Measured
 //     on B200: deep plain loads stream a 32 MiB slice set faster than a 1-D bulk-copy
 //     ring with one CTA per SM.)  Scores stay on chip and go to global memory
-//     (L2-resident).  The first half of the slice feeds a 12-bit histogram that is
-//     added to the group's global histogram before the second half is read.
-//  2. Candidate bound.  After its slice, a CTA reads the group histogram as it
-//     stands: whatever subset of tokens it counts, its k-th largest bin is a lower
-//     bound on the true k-th largest score, so every token of the true TopK scores
-//     at least the bin's lower edge tau.  The CTA writes its tokens with
-//     key >= tau, in token order, to its own segment of the candidate list.
+//     (L2-resident), and feed a 12-bit key histogram of the slice.
+//  2. Candidates.  From its own histogram a CTA picks the bound E: the lowest bin edge
+//     with at most kWin of its tokens at or above it.  It writes those tokens, in token
+//     order, to its window of the candidate list, and E beside them.  No CTA waits
+//     for another before this point.
 //  3. One barrier for the group.  Every CTA then resolves the exact TopK from the
-//     candidate list by itself (12+12+8-bit radix select over the candidate keys,
-//     ties to the earlier list position = lower token index), ranks the selected
-//     tokens in ascending token order, writes its share of idx, and keeps the
-//     tokens of its attention unit.  If the candidates do not fit in shared
-//     memory, the same selection runs over the whole row of scores instead.
+//     candidate list by itself (a linear-key histogram and an exact rank count in the
+//     boundary bin; ties to the earlier list position = lower token index).  The
+//     result is the TopK of the row iff every CTA's bound E is at or below the k_eff-th
+//     candidate key (a token left out of a window scores below its E); otherwise, or
+//     with too few candidates, the same selection runs digit by digit over the whole
+//     row of scores.  The selected tokens are ranked in ascending token order; each
+//     CTA writes its share of idx and keeps the tokens of its attention unit.
 //  4. Attention.  A unit is (KV head g, split s of the selected ranks); its rows
 //     are all L*G (layer, query head) pairs of head g, so every selected K/V row is
 //     read once for all layers.  mma.sync m16n8k16 bf16 -> fp32, online softmax in
@@ -48,8 +48,9 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 4096;          // digit histograms of the selection
 constexpr int kTauBits = 12;          // key bits of the candidate-bound histogram
-constexpr int kCoarse = (1 << kTauBits) / 64;  // coarse bins of 64 fine bins
 constexpr int kTauBins = 1 << kTauBits;
+constexpr int kScanU = 4;             // rows per lane group per scan stage
+constexpr int kScanS = 3;             // scan stages in flight (ring after the histogram in `big`)
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
 constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
@@ -62,9 +63,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // per-row global state (u32 words)
-constexpr int kRowHist = 0;                       // [kTauBins] partial histogram (self-clearing)
-constexpr int kRowCoarse = kTauBins;              // [kCoarse] the same histogram, 64 fine bins per bin
-constexpr int kRowArrive = kTauBins + 256;        // CTAs that published their first half
+constexpr int kRowBound = 0;                      // [kMaxGroups] each CTA's candidate bound E (key)
 constexpr int kRowBar = kTauBins + 256 + 32;      // row-group barrier state [2]
 constexpr int kRowCnt = kTauBins + 256 + 64;      // [kMaxGroups] candidate count per CTA
 constexpr int kRowHeadBar = kRowCnt + kMaxGroups; // [Hkv][2] head-group barrier states (<= 64 heads)
@@ -95,7 +94,11 @@ struct FusedParams {
 
 constexpr int kTraceSlots = 32;
 __device__ __forceinline__ void stamp(const FusedParams& p, int phase) {
-  if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + phase] = globaltimer_ns();
+  if (p.trace && threadIdx.x == 0) {
+    p.trace[blockIdx.x * kTraceSlots + phase] = globaltimer_ns();
+    if (phase == 1) p.trace[blockIdx.x * kTraceSlots + 29] = clock64();  // SM clock calibration
+    if (phase == 9) p.trace[blockIdx.x * kTraceSlots + 30] = clock64();
+  }
 }
 
 struct Plan {
@@ -137,6 +140,7 @@ struct Smem {
 constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
 constexpr size_t kSmemBig = 128 * 1024;
 constexpr size_t smem_bytes() { return align_up(sizeof(Smem), 128) + kSmemQ + kSmemBig; }
+static_assert(kTauBins * 4 + kScanS * kScanU * kThreads * 16 <= (int)kSmemBig, "scan histogram + ring exceed big");
 
 // ---------------------------------------------------------------------------
 // small block-wide helpers (512 threads)
@@ -346,32 +350,41 @@ __device__ __forceinline__ float row_dot(const uint4 v, const float (&q)[8]) {
   return acc;
 }
 
-// Rows [j0, j1) of the slice; the loads of the next batch of U rows per group are in
-// flight while the current batch is reduced.
+// Rows [j0, j1) of the slice, streamed through a ring of S stages of U rows per lane
+// group in shared memory (16-byte cp.async, L2 only).  Every thread reads back only the
+// chunks it copied, so no barrier is needed: S - 1 stages stay in flight while one is
+// reduced.
 template <int DIDX>
-__device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32_t* th, const __nv_bfloat16* src,
-                                          float* sc, const float (&q)[8], int j0, int j1, int nrows, bool hist) {
-  constexpr int LPR = DIDX / 8;                 // lanes per row (16-byte loads)
+__device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32_t* th, uint4* ring,
+                                          const __nv_bfloat16* src, float* sc, const float (&q)[8], int j0, int j1,
+                                          int nrows, bool hist) {
+  constexpr int LPR = DIDX / 8;                 // lanes per row (16-byte chunks)
   constexpr int GROUPS = kThreads / LPR;        // row groups per CTA
-  constexpr int U = 8;                          // rows in flight per group
   const int grp = threadIdx.x / LPR, sub = threadIdx.x % LPR;
-  auto load = [&](uint4 (&v)[U], int base0) {
+  constexpr int ROWS = GROUPS * kScanU;         // rows per stage
+  auto issue = [&](int st, int base0) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < kScanU; ++u) {
       const int j = base0 + grp + u * GROUPS;
-      v[u] = j < j1 ? ld_stream_v4(src + (size_t)j * DIDX + sub * 8) : make_uint4(0, 0, 0, 0);
+      if (j < j1) cp_async_16(ring + (st * kScanU + u) * kThreads + threadIdx.x, src + (size_t)j * DIDX + sub * 8, 16);
     }
+    cp_async_commit();  // one group per stage, empty or not
   };
-  uint4 cur[U], nxt[U];
-  if (j0 < j1) load(cur, j0);
-  // the trip count is the same for every thread (the shuffles below need whole warps)
-  for (int base0 = j0; base0 < j1; base0 += GROUPS * U) {
-    const bool more = base0 + GROUPS * U < j1;
-    if (more) load(nxt, base0 + GROUPS * U);
+  const int nst = (j1 - j0 + ROWS - 1) / ROWS;  // the same for every thread (whole-warp shuffles below)
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+  for (int st = 0; st < kScanS; ++st) {
+    if (st < nst) issue(st, j0 + st * ROWS);
+    else cp_async_commit();
+  }
+  for (int it = 0; it < nst; ++it) {
+    cp_async_wait<kScanS - 1>();  // stage it has landed
+    const int st = it % kScanS;
+    const int base0 = j0 + it * ROWS;
+#pragma unroll
+    for (int u = 0; u < kScanU; ++u) {
       const int j = base0 + grp + u * GROUPS;
-      float acc = row_dot<DIDX>(cur[u], q);
+      const uint4 v = j < j1 ? ring[(st * kScanU + u) * kThreads + threadIdx.x] : make_uint4(0, 0, 0, 0);
+      float acc = row_dot<DIDX>(v, q);
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (sub == 0 && j < j1) {
@@ -380,15 +393,14 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
         if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
       }
     }
-    if (more) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) cur[u] = nxt[u];
-    }
+    if (it + kScanS < nst) issue(st, j0 + (it + kScanS) * ROWS);  // refill the slot just read
+    else cp_async_commit();
   }
+  cp_async_wait<0>();
 }
 
 template <int DIDX>
-__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool publish) {
+__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool hist) {
   const Plan& pl = sm.plan;
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
@@ -405,37 +417,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
   }
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
-  const int half = publish ? nrows / 2 : 0;
-  scan_rows<DIDX>(p, sm, th, src, sc, q, 0, half, nrows, true);
-  if (publish) {
-    // First-half histogram (fine bins, and coarse sums of 64) to the group.  The last four
-    // warps publish (named barrier 1 among them) while the other warps start the second
-    // half; the publishers join the scan afterwards.
-    __syncthreads();
-    constexpr int kPubThreads = 128;
-    const int pt = threadIdx.x - (kThreads - kPubThreads);
-    if (pt >= 0) {
-      uint32_t* gh = p.row_ws + (size_t)pl.b * kRowWords + kRowHist;
-      for (int v = pt; v < kTauBins / 4; v += kPubThreads) {  // consecutive threads, consecutive bins
-        const uint4 x = *reinterpret_cast<const uint4*>(th + v * 4);
-        if (x.x) atomicAdd(gh + v * 4, x.x);
-        if (x.y) atomicAdd(gh + v * 4 + 1, x.y);
-        if (x.z) atomicAdd(gh + v * 4 + 2, x.z);
-        if (x.w) atomicAdd(gh + v * 4 + 3, x.w);
-        // the 16 threads of a half-warp hold exactly the 64 fine bins of one coarse bin
-        uint32_t sum = x.x + x.y + x.z + x.w;
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if ((pt & 15) == 0 && sum) atomicAdd(gh + kRowCoarse + ((v * 4) >> 6), sum);
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(kPubThreads) : "memory");
-      if (pt == 0) {
-        __threadfence();
-        red_add_release_gpu(p.row_ws + (size_t)pl.b * kRowWords + kRowArrive, 1u);
-      }
-    }
-  }
-  scan_rows<DIDX>(p, sm, th, src, sc, q, half, nrows, nrows, false);
+  scan_rows<DIDX>(p, sm, th, reinterpret_cast<uint4*>(th + kTauBins), src, sc, q, 0, nrows, nrows, hist);
   __syncthreads();
   return true;
 }
@@ -446,73 +428,32 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool pu
 __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   const Plan& pl = sm.plan;
   uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
-  // wait briefly for a quarter of the group's first halves: the bound is scaled to the
-  // share it has counted, so a smaller sample only widens the candidate count's spread
-  if (threadIdx.x == 0) {
-    const unsigned long long t0 = globaltimer_ns();
-    const uint32_t want = (uint32_t)(pl.Cb + 3) / 4;
-    while (ld_acquire_gpu(rw + kRowArrive) < want && globaltimer_ns() - t0 < 5000ull) __nanosleep(32);
-  }
-  stamp(p, 13);
-  __syncthreads();
-  // The bound: the bin where the count from the top reaches 1.25 k_eff scaled to the share
-  // of the row counted so far (then the candidates hold about 1.25 k_eff tokens; too few is
-  // caught after the barrier).  Warp 0 finds the coarse bin, then the fine bin inside it.
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    constexpr int CPL = kCoarse / 32;  // coarse bins per lane, lane 0 holding the top ones
-    uint32_t cc[CPL];
+  // The local bound E: the lower edge of the lowest 12-bit key bin such that the slice
+  // holds at most kWin tokens at or above it (E = 0: every token).  Thread t sums the
+  // eight bins 4088 - 8t .. 4095 - 8t; one scan from the top finds the bin.
+  {
+    const int hi = kTauBins - 8 * threadIdx.x;  // this thread's bins: [hi - 8, hi)
+    uint32_t h[8], local = 0;
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) cc[i] = __ldcg(rw + kRowCoarse + kCoarse - CPL * (lane + 1) + i);
-    uint32_t local = 0;
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) local += cc[i];
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+    for (int i = 0; i < 8; ++i) {
+      h[i] = th[hi - 8 + i];
+      local += h[i];
     }
-    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-    const uint32_t need = max(1u, (uint32_t)(1.25f * (float)pl.keff * (float)total / (float)pl.len));
-    const uint32_t before = incl - local;
-    int tc = -1;
-    uint32_t above = 0;
-    if (before < need && need <= incl) {
+    uint32_t total;
+    const uint32_t before = block_scan(local, sm.warp_tot, &total);  // tokens in higher bins
+    if (threadIdx.x == 0 && total <= (uint32_t)kWin) sm.tau_key = 0u;
+    if (before <= (uint32_t)kWin && before + local > (uint32_t)kWin) {
       uint32_t acc = before;
-      for (int i = CPL - 1; i >= 0; --i) {  // bins from the top of this lane's run
-        if (acc + cc[i] >= need) {
-          tc = kCoarse - CPL * (lane + 1) + i;
-          above = acc;
+#pragma unroll
+      for (int i = 7; i >= 0; --i) {
+        if (acc + h[i] > (uint32_t)kWin) {  // bin hi - 8 + i would overflow: E is its upper edge
+          const int bin = hi - 8 + i;  // the top bin alone overflowing: publish nothing
+          sm.tau_key = bin + 1 < kTauBins ? ((uint32_t)(bin + 1)) << (32 - kTauBits) : 0xFFFFFFFFu;
           break;
         }
-        acc += cc[i];
+        acc += h[i];
       }
     }
-    const uint32_t hit = __ballot_sync(0xffffffffu, tc >= 0);
-    uint32_t tau = 0u;  // everything is a candidate when too few tokens were counted
-    if (hit) {
-      const int src_lane = __ffs(hit) - 1;
-      tc = __shfl_sync(0xffffffffu, tc, src_lane);
-      above = __shfl_sync(0xffffffffu, above, src_lane);
-      // the 64 fine bins of coarse bin tc, two per lane from the top
-      const uint2 f2 = __ldcg(reinterpret_cast<const uint2*>(rw + kRowHist + tc * 64 + 62 - 2 * lane));
-      const uint32_t fl = f2.x + f2.y;
-      uint32_t fi = fl;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, fi, o);
-        if (lane >= o) fi += y;
-      }
-      const uint32_t fb = above + fi - fl;
-      int tf = -1;
-      if (fb < need && need <= fb + fl) tf = (fb + f2.y >= need) ? 63 - 2 * lane : 62 - 2 * lane;
-      const uint32_t fh = __ballot_sync(0xffffffffu, tf >= 0);
-      if (fh) tf = __shfl_sync(0xffffffffu, tf, __ffs(fh) - 1);
-      else tf = 0;
-      tau = ((uint32_t)(tc * 64 + tf)) << (32 - kTauBits);
-    }
-    if (lane == 0) sm.tau_key = tau;
   }
   stamp(p, 14);
   stamp(p, 16);
@@ -542,7 +483,10 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
     written += tot;
   }
   for (int i = (int)written + threadIdx.x; i < kWin; i += kThreads) __stcg(ck + i, 0u);  // empty slots
-  if (threadIdx.x == 0) __stcg(rw + kRowCnt + pl.c, written);  // > kWin: overflow
+  if (threadIdx.x == 0) {
+    __stcg(rw + kRowCnt + pl.c, written);  // <= kWin by the choice of the bound
+    __stcg(rw + kRowBound + pl.c, tau);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -640,7 +584,7 @@ __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& 
 // (key, position) pair of the k_eff-th candidate.  False if the boundary bin holds
 // more than 1024 candidates (then the generic digit-by-digit path runs).
 // ---------------------------------------------------------------------------
-__device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_t keff) {
+__device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, int P, uint32_t keff) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll 8
@@ -669,6 +613,7 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
+  stamp(p, 19);
   int shift = 0;
   while (((kmax - kmin) >> shift) >= 2048u) ++shift;
 #pragma unroll 8
@@ -677,7 +622,9 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
     if (k != 0u) atomicAdd(&sm.hist[(k - kmin) >> shift], 1u);
   }
   __syncthreads();
+  stamp(p, 20);
   select_bin_wide(sm, sm.hist, 2048, keff);
+  stamp(p, 21);
   const int T = sm.sel_bin;
   if (T < 0) return false;
   const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
@@ -693,6 +640,7 @@ __device__ bool select_candidates(Smem& sm, const uint32_t* skey, int P, uint32_
     }
   }
   __syncthreads();
+  stamp(p, 22);
   for (int e = threadIdx.x; e < (int)m; e += kThreads) {
     const uint32_t ke = sm.list_key[e];
     const int pe = sm.list_pos[e];
@@ -1137,13 +1085,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
     stamp(p, 3);
-    // everyone has read the partial histogram: clear this CTA's share for the next call
-    {
-      const int per = (kTauBins + pl.Cb - 1) / pl.Cb;
-      for (int i = pl.c * per + threadIdx.x; i < min(kTauBins, (pl.c + 1) * per); i += kThreads) rw[kRowHist + i] = 0u;
-      if (pl.c == 0 && threadIdx.x < kCoarse) rw[kRowCoarse + threadIdx.x] = 0u;
-      if (pl.c == 0 && threadIdx.x == 0) rw[kRowArrive] = 0u;
-    }
     // candidate windows: every count (one load each), then every valid slot copied to a
     // dense list in window order (= token order), all copies in flight at once
     {
@@ -1155,7 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
       if (threadIdx.x == 0) {
         sm.seg_off[pl.Cb] = (int)total;
         sm.ctot = (int)total;
-        // too few candidates (the scaled bound overshot) or a full window: whole-row path
+        // too few candidates: whole-row path
         sm.fast = !over && total >= (uint32_t)pl.keff && total <= (uint32_t)kCandCap;
       }
       __syncthreads();
@@ -1180,16 +1121,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     stamp(p, 4);
     bool done = false;
     if (sm.fast) {
-      done = select_candidates(sm, skey, sm.ctot, (uint32_t)pl.keff);
+      done = select_candidates(p, sm, skey, sm.ctot, (uint32_t)pl.keff);
+      // exact iff every CTA's unpublished tokens (keys below its bound E) lie strictly
+      // below the k_eff-th candidate key
+      const uint32_t e = threadIdx.x < pl.Cb ? __ldcg(rw + kRowBound + threadIdx.x) : 0u;
+      done = !__syncthreads_or(!done || e > sm.theta_key);
       stamp(p, 5);
       if (done) compact_candidates(p, sm, skey, stok, sm.ctot);
     }
-    if (!done) {  // a window overflowed, or a boundary bin of heavy ties: digit-by-digit select
-      CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, sm.fast != 0};
-      const int P = sm.fast ? sm.ctot : pl.len;
-      resolve_theta(sm, src, P, (uint32_t)pl.keff, p.ws_header);
+    if (!done) {  // too few candidates, a bound above the boundary, or a boundary bin of
+                  // heavy ties: digit-by-digit select over the whole row
+      CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, false};
+      resolve_theta(sm, src, pl.len, (uint32_t)pl.keff, p.ws_header);
       stamp(p, 5);
-      compact_selected(p, sm, src, P);
+      compact_selected(p, sm, src, pl.len);
     }
     if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + 31] = (unsigned long long)sm.ctot | ((unsigned long long)sm.fast << 32);
   }
