@@ -15,7 +15,7 @@
 //     ring with one CTA per SM.)  Scores stay on chip and go to global memory
 //     (L2-resident), and feed a 12-bit key histogram of the slice.
 //  2. Candidates.  From its own histogram a CTA picks the bound E: the lowest bin edge
-//     with at most kWin of its tokens at or above it.  It writes those tokens, in token
+//     with at most win of its tokens at or above it.  It writes those tokens, in token
 //     order, to its window of the candidate list, and E beside them.  No CTA waits
 //     for another before this point.
 //  3. One barrier for the group.  Every CTA then resolves the exact TopK from the
@@ -57,13 +57,13 @@ constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
 constexpr int kTokBlk = 64;           // tokens per attention block
 constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096); also slice scores kept on chip
 constexpr int kCandCap = 16384;       // candidate slots kept in shared memory (key + index)
-constexpr int kWin = 64;              // candidate window per CTA (more: the group takes the whole-row path)
 constexpr int kMaxGroups = 256;       // CTAs per launch
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // per-row global state (u32 words)
 constexpr int kRowBound = 0;                      // [kMaxGroups] each CTA's candidate bound E (key)
+constexpr int kRowMax = kMaxGroups;               // [kMaxGroups] an upper bound on each CTA's largest key
 constexpr int kRowBar = kTauBins + 256 + 32;      // row-group barrier state [2]
 constexpr int kRowCnt = kTauBins + 256 + 64;      // [kMaxGroups] candidate count per CTA
 constexpr int kRowHeadBar = kRowCnt + kMaxGroups; // [Hkv][2] head-group barrier states (<= 64 heads)
@@ -82,8 +82,8 @@ struct FusedParams {
   float* lse;
   float* scores;       // [B][n_max]
   uint32_t* row_ws;    // [B][kRowWords]
-  uint32_t* cand_key;  // [B][kMaxGroups][kWin]  candidate keys per CTA window (0 = empty slot)
-  int32_t* cand_tok;   // [B][kMaxGroups][kWin]
+  uint32_t* cand_key;  // [B][kCandCap]  candidate keys, the group's windows back to back (0 = empty slot)
+  int32_t* cand_tok;   // [B][kCandCap]
   float* Op;           // [gridDim][rows][D]  split partials, one slot per CTA
   float* Ml;           // [gridDim][rows][2]
   void* ws_header;
@@ -108,6 +108,7 @@ struct Plan {
   int unit_g0, unit_step, nunits_here;  // heads this CTA attends: g0, g0+step, ... (count)
   int split;             // split index of this CTA's units
   int tok0, tok1;        // selected-rank range of the unit
+  int win;               // candidate window per CTA (slots, a multiple of 4)
 };
 
 struct Smem {
@@ -126,6 +127,7 @@ struct Smem {
   uint32_t red_min[kWarps], red_max[kWarps];
   uint32_t theta_key, theta_pos;
   int list_n;
+  uint32_t slice_max, emax, kmax;
   union {                          // slice scores until the candidates are out, then the
     float score[kMaxUnitTok];      // boundary-bin list of the selection, then unit tokens
     int unit_tok[kMaxUnitTok];
@@ -303,6 +305,12 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
       const int chunk = (len + Cb - 1) / Cb;
       pl.r0 = min(len, pl.c * chunk);
       pl.r1 = min(len, pl.r0 + chunk);
+      // window: the expected share e = k_eff / C_b of the TopK per CTA plus 6 sqrt(e) + 4
+      // (a CTA holding more TopK tokens than its window sends the group to the whole-row
+      // path); all windows of the group fit kCandCap
+      const float e = (float)pl.keff / (float)Cb;
+      const int wn = ((int)ceilf(e + 6.f * sqrtf(e) + 4.f) + 3) & ~3;
+      pl.win = max(4, min(wn, (kCandCap / Cb) & ~3));
       break;
     }
     start += Cb;
@@ -429,7 +437,7 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   const Plan& pl = sm.plan;
   uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
   // The local bound E: the lower edge of the lowest 12-bit key bin such that the slice
-  // holds at most kWin tokens at or above it (E = 0: every token).  Thread t sums the
+  // holds at most win tokens at or above it (E = 0: every token).  Thread t sums the
   // eight bins 4088 - 8t .. 4095 - 8t; one scan from the top finds the bin.
   {
     const int hi = kTauBins - 8 * threadIdx.x;  // this thread's bins: [hi - 8, hi)
@@ -439,14 +447,27 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
       h[i] = th[hi - 8 + i];
       local += h[i];
     }
+    uint32_t top = 0;  // 1 + the highest non-empty bin of this thread's run (0: none)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (h[i] != 0u) top = (uint32_t)(hi - 8 + i + 1);
+    top = __reduce_max_sync(0xffffffffu, top);
+    if ((threadIdx.x & 31) == 0) sm.red_max[threadIdx.x >> 5] = top;
     uint32_t total;
-    const uint32_t before = block_scan(local, sm.warp_tot, &total);  // tokens in higher bins
-    if (threadIdx.x == 0 && total <= (uint32_t)kWin) sm.tau_key = 0u;
-    if (before <= (uint32_t)kWin && before + local > (uint32_t)kWin) {
+    const uint32_t before = block_scan(local, sm.warp_tot, &total);  // tokens in higher bins (syncs)
+    if (threadIdx.x == 0) {
+      uint32_t t = 0;
+      for (int w2 = 0; w2 < kWarps; ++w2) t = max(t, sm.red_max[w2]);
+      // the upper edge of the highest non-empty bin bounds every key of the slice
+      sm.slice_max = t == 0 ? 0u : (t >= (uint32_t)kTauBins ? 0xFFFFFFFFu : (t << (32 - kTauBits)) - 1u);
+    }
+    const uint32_t win = (uint32_t)pl.win;
+    if (threadIdx.x == 0 && total <= win) sm.tau_key = 0u;
+    if (before <= win && before + local > win) {
       uint32_t acc = before;
 #pragma unroll
       for (int i = 7; i >= 0; --i) {
-        if (acc + h[i] > (uint32_t)kWin) {  // bin hi - 8 + i would overflow: E is its upper edge
+        if (acc + h[i] > win) {  // bin hi - 8 + i would overflow: E is its upper edge
           const int bin = hi - 8 + i;  // the top bin alone overflowing: publish nothing
           sm.tau_key = bin + 1 < kTauBins ? ((uint32_t)(bin + 1)) << (32 - kTauBits) : 0xFFFFFFFFu;
           break;
@@ -459,12 +480,12 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   stamp(p, 16);
   __syncthreads();
   const uint32_t tau = sm.tau_key;
-  // this CTA's tokens with key >= tau, in token order, to its window of kWin slots
+  // this CTA's tokens with key >= tau, in token order, to its window of win slots
   const float* gsc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
   const int n = pl.r1 - pl.r0;
   const bool on_chip = n <= kMaxUnitTok;
-  uint32_t* ck = p.cand_key + ((size_t)pl.b * kMaxGroups + pl.c) * kWin;
-  int32_t* ct = p.cand_tok + ((size_t)pl.b * kMaxGroups + pl.c) * kWin;
+  uint32_t* ck = p.cand_key + (size_t)pl.b * kCandCap + (size_t)pl.c * pl.win;
+  int32_t* ct = p.cand_tok + (size_t)pl.b * kCandCap + (size_t)pl.c * pl.win;
   uint32_t written = 0;
   for (int base = 0; base < n; base += kThreads) {
     const int j = base + threadIdx.x;
@@ -476,16 +497,17 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
     }
     uint32_t tot;
     const uint32_t pos = written + block_flag_scan(f, sm.warp_tot2, &tot);
-    if (f && pos < (uint32_t)kWin) {
+    if (f && pos < (uint32_t)pl.win) {
       __stcg(ck + pos, key);
       __stcg(ct + pos, pl.r0 + j);
     }
     written += tot;
   }
-  for (int i = (int)written + threadIdx.x; i < kWin; i += kThreads) __stcg(ck + i, 0u);  // empty slots
+  for (int i = (int)written + threadIdx.x; i < pl.win; i += kThreads) __stcg(ck + i, 0u);  // empty slots
   if (threadIdx.x == 0) {
-    __stcg(rw + kRowCnt + pl.c, written);  // <= kWin by the choice of the bound
+    __stcg(rw + kRowCnt + pl.c, written);  // <= win by the choice of the bound
     __stcg(rw + kRowBound + pl.c, tau);
+    __stcg(rw + kRowMax + pl.c, sm.slice_max);
   }
 }
 
@@ -584,56 +606,51 @@ __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& 
 // (key, position) pair of the k_eff-th candidate.  False if the boundary bin holds
 // more than 1024 candidates (then the generic digit-by-digit path runs).
 // ---------------------------------------------------------------------------
-__device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, int P, uint32_t keff) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-#pragma unroll 8
-  for (int i = threadIdx.x; i < P; i += kThreads) {
-    const uint32_t k = skey[i];
-    if (k == 0u) continue;  // empty window slot
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    sm.red_min[w] = kmin;
-    sm.red_max[w] = kmax;
-  }
-  for (int i = threadIdx.x; i < 2048; i += kThreads) sm.hist[i] = 0;
+__device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, int P, uint32_t keff,
+                                  uint32_t emax, uint32_t kmax) {
+  // Loops stay rolled: this runs once per call, so its code is fetched cold every time.
+  if (kmax < emax) return false;
+  for (int i = threadIdx.x; i < 4096; i += kThreads) sm.hist[i] = 0;
   if (threadIdx.x == 0) sm.list_n = 0;
   __syncthreads();
-  kmin = lane < kWarps ? sm.red_min[lane] : 0xFFFFFFFFu;
-  kmax = lane < kWarps ? sm.red_max[lane] : 0u;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  stamp(p, 19);
+  // stage A: 2048 linear bins over [E_max, kmax]; keys below E_max cannot be selected
   int shift = 0;
-  while (((kmax - kmin) >> shift) >= 2048u) ++shift;
-#pragma unroll 8
+  while (((kmax - emax) >> shift) >= 2048u) ++shift;
+#pragma unroll 1
   for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = skey[i];
-    if (k != 0u) atomicAdd(&sm.hist[(k - kmin) >> shift], 1u);
+    if (k >= emax && k != 0u) atomicAdd(&sm.hist[(k - emax) >> shift], 1u);
+  }
+  __syncthreads();
+  stamp(p, 19);
+  select_bin_wide(sm, sm.hist, 2048, keff);
+  const int T = sm.sel_bin;
+  if (T < 0) return false;                  // fewer than k_eff keys >= E_max: not exact
+  const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
+  // stage B: 2048 sub-bins of bin T
+  const uint32_t loT = emax + ((uint32_t)T << shift);
+  const uint32_t hiT = T == 2047 ? kmax : loT + (1u << shift) - 1u;  // bin T = [loT, hiT]
+  const int shift2 = max(0, shift - 11);
+  uint32_t* hist2 = sm.hist + 2048;
+#pragma unroll 1
+  for (int i = threadIdx.x; i < P; i += kThreads) {
+    const uint32_t k = skey[i];
+    if (k >= loT && k <= hiT && k != 0u) atomicAdd(&hist2[(k - loT) >> shift2], 1u);
   }
   __syncthreads();
   stamp(p, 20);
-  select_bin_wide(sm, sm.hist, 2048, keff);
+  select_bin_wide(sm, hist2, 2048, need);
+  const int T2 = sm.sel_bin;
+  const uint32_t need2 = need - sm.sel_above;  // rank inside sub-bin T2
+  const uint32_t m = hist2[T2];
+  if (m > 1024u) return false;  // heavy ties: the digit-by-digit path
   stamp(p, 21);
-  const int T = sm.sel_bin;
-  if (T < 0) return false;
-  const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
-  const uint32_t m = sm.hist[T];
-  if (m > 1024u) return false;
-#pragma unroll 8
+  // the keys of sub-bin T2 (few) with their list positions
+  const uint32_t lo2 = loT + ((uint32_t)T2 << shift2), hi2 = lo2 + (1u << shift2) - 1u;
+#pragma unroll 1
   for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = skey[i];
-    if (k != 0u && (int)((k - kmin) >> shift) == T) {
+    if (k >= lo2 && k <= hi2 && k <= hiT && k != 0u) {
       const int q = atomicAdd(&sm.list_n, 1);
       sm.list_key[q] = k;
       sm.list_pos[q] = i;
@@ -641,7 +658,7 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
   }
   __syncthreads();
   stamp(p, 22);
-  for (int e = threadIdx.x; e < (int)m; e += kThreads) {
+  for (int e = threadIdx.x; e < (int)m; e += kThreads) {  // rank inside the sub-bin
     const uint32_t ke = sm.list_key[e];
     const int pe = sm.list_pos[e];
     uint32_t r = 0;
@@ -649,7 +666,7 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
       const uint32_t kf = sm.list_key[f];
       r += kf > ke || (kf == ke && sm.list_pos[f] < pe);
     }
-    if (r == need - 1) {
+    if (r == need2 - 1) {
       sm.theta_key = ke;
       sm.theta_pos = (uint32_t)pe;
     }
@@ -1085,47 +1102,52 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
     stamp(p, 3);
-    // candidate windows: every count (one load each), then every valid slot copied to a
-    // dense list in window order (= token order), all copies in flight at once
-    {
-      const uint32_t v = threadIdx.x < pl.Cb ? __ldcg(rw + kRowCnt + threadIdx.x) : 0u;
-      const bool over = __syncthreads_or(v > (uint32_t)kWin);
-      uint32_t total;
-      const uint32_t before = block_scan(v, sm.warp_tot, &total);
-      if (threadIdx.x < pl.Cb) sm.seg_off[threadIdx.x] = (int)before;
-      if (threadIdx.x == 0) {
-        sm.seg_off[pl.Cb] = (int)total;
-        sm.ctot = (int)total;
-        // too few candidates: whole-row path
-        sm.fast = !over && total >= (uint32_t)pl.keff && total <= (uint32_t)kCandCap;
-      }
-      __syncthreads();
-    }
+    // the group's windows (back to back, token order, empty slots key 0) to shared
+    // memory in 16-byte copies, all in flight while the group totals are reduced
     uint32_t* skey = reinterpret_cast<uint32_t*>(big);
     int32_t* stok = reinterpret_cast<int32_t*>(big + kCandCap * 4);
-    if (sm.fast) {
-      const uint32_t* gk = p.cand_key + (size_t)pl.b * kMaxGroups * kWin;
-      const int32_t* gt = p.cand_tok + (size_t)pl.b * kMaxGroups * kWin;
-      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-      for (int c = warp; c < pl.Cb; c += kWarps) {  // one warp per window
-        const int o = sm.seg_off[c], n = sm.seg_off[c + 1] - o;
-        for (int i = lane; i < n; i += 32) {
-          cp_async_4(skey + o + i, gk + c * kWin + i);
-          cp_async_4(stok + o + i, gt + c * kWin + i);
-        }
+    const int nslot = pl.Cb * pl.win;  // a multiple of 4
+    {
+      const uint4* gk = reinterpret_cast<const uint4*>(p.cand_key + (size_t)pl.b * kCandCap);
+      const uint4* gt = reinterpret_cast<const uint4*>(p.cand_tok + (size_t)pl.b * kCandCap);
+      for (int i = threadIdx.x; i < nslot / 4; i += kThreads) {
+        cp_async_16(skey + 4 * i, gk + i, 16);
+        cp_async_16(stok + 4 * i, gt + i, 16);
       }
       cp_async_commit();
+      // candidate total, the largest bound E_max and the largest key bound over the group
+      const bool mine = threadIdx.x < pl.Cb;
+      const uint32_t v = mine ? __ldcg(rw + kRowCnt + threadIdx.x) : 0u;
+      const uint32_t e = mine ? __ldcg(rw + kRowBound + threadIdx.x) : 0u;
+      const uint32_t x = mine ? __ldcg(rw + kRowMax + threadIdx.x) : 0u;
+      const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+      const uint32_t vs = __reduce_add_sync(0xffffffffu, v), es = __reduce_max_sync(0xffffffffu, e),
+                     xs = __reduce_max_sync(0xffffffffu, x);
+      if (lane == 0) {
+        sm.warp_tot[w] = vs;
+        sm.red_min[w] = es;
+        sm.red_max[w] = xs;
+      }
       cp_async_wait<0>();
+      __syncthreads();
+      const uint32_t total = __reduce_add_sync(0xffffffffu, lane < kWarps ? sm.warp_tot[lane] : 0u);
+      const uint32_t emax = __reduce_max_sync(0xffffffffu, lane < kWarps ? sm.red_min[lane] : 0u);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, lane < kWarps ? sm.red_max[lane] : 0u);
+      if (threadIdx.x == 0) {
+        sm.ctot = nslot;
+        sm.fast = total >= (uint32_t)pl.keff;  // too few candidates: whole-row path
+        sm.emax = emax;
+        sm.kmax = kmax;
+      }
       __syncthreads();
     }
     stamp(p, 4);
     bool done = false;
     if (sm.fast) {
-      done = select_candidates(p, sm, skey, sm.ctot, (uint32_t)pl.keff);
       // exact iff every CTA's unpublished tokens (keys below its bound E) lie strictly
-      // below the k_eff-th candidate key
-      const uint32_t e = threadIdx.x < pl.Cb ? __ldcg(rw + kRowBound + threadIdx.x) : 0u;
-      done = !__syncthreads_or(!done || e > sm.theta_key);
+      // below the k_eff-th candidate key, i.e. iff at least k_eff candidates have keys
+      // >= E_max (checked inside)
+      done = select_candidates(p, sm, skey, sm.ctot, (uint32_t)pl.keff, sm.emax, sm.kmax);
       stamp(p, 5);
       if (done) compact_candidates(p, sm, skey, stok, sm.ctot);
     }
@@ -1195,7 +1217,7 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   off += (size_t)kMaxGroups * kTraceSlots * 8;                  // phase stamps (CLSA_TRACE=1)
   off += align_up((size_t)a->B * a->n_max * 4, 256);           // scores (when not an output)
   off += align_up((size_t)a->B * kRowWords * 4, 256);          // row state
-  off += 2 * align_up((size_t)a->B * kMaxGroups * kWin * 4, 256);  // candidate windows
+  off += 2 * align_up((size_t)a->B * kCandCap * 4, 256);  // candidate windows
   off += align_up((size_t)cfg.ncta * rows * kD * 4, 256);      // split partials
   off += align_up((size_t)cfg.ncta * rows * 2 * 4, 256);
   return off;
@@ -1236,9 +1258,9 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   p.row_ws = reinterpret_cast<uint32_t*>(w);
   w += align_up((size_t)a->B * kRowWords * 4, 256);
   p.cand_key = reinterpret_cast<uint32_t*>(w);
-  w += align_up((size_t)a->B * kMaxGroups * kWin * 4, 256);
+  w += align_up((size_t)a->B * kCandCap * 4, 256);
   p.cand_tok = reinterpret_cast<int32_t*>(w);
-  w += align_up((size_t)a->B * kMaxGroups * kWin * 4, 256);
+  w += align_up((size_t)a->B * kCandCap * 4, 256);
   p.Op = reinterpret_cast<float*>(w);
   w += align_up((size_t)cfg.ncta * p.rows * kD * 4, 256);
   p.Ml = reinterpret_cast<float*>(w);
