@@ -285,6 +285,10 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   if (ok) ok = mbar_test_wait(bar, parity) ? 1u : 0u;  // completed: true at once, with ordering
   return __all_sync(0xffffffffu, ok != 0);
 }
+// bulk prefetch of [src, src + bytes) into L2 (src 16-byte aligned, bytes % 16 == 0)
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // global -> shared bulk copy completing on `bar` (dst, src 16-byte aligned, bytes % 16 == 0)
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

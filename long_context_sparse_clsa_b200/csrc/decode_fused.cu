@@ -127,7 +127,7 @@ struct Smem {
   uint32_t red_min[kWarps], red_max[kWarps];
   uint32_t theta_key, theta_pos;
   int list_n;
-  uint32_t slice_max, emax, kmax;
+  uint32_t slice_max, emax, kmax, pf_key;
   union {                          // slice scores until the candidates are out, then the
     float score[kMaxUnitTok];      // boundary-bin list of the selection, then unit tokens
     int unit_tok[kMaxUnitTok];
@@ -137,6 +137,7 @@ struct Smem {
     };
   };
   float cm[512], cl[512];          // split-combine staging (m, l per row x split)
+  float rowM[kMaxRows], rowD[kMaxRows];  // split-combine: max and denominator per row
 };
 // dynamic shared memory: [Smem][sQ: kMaxRows x kSTR bf16][big: 128 KiB, reused by phase]
 constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
@@ -282,6 +283,7 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
   const int ncta = gridDim.x;
   long long total = 0;
   int nb = 0;
+#pragma unroll 1
   for (int b = 0; b < p.B; ++b) {
     const int len = max(0, min(p.seq_lens[b], p.n_max));
     total += len;
@@ -291,6 +293,7 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
   if (nb == 0) return;
   const int spare = ncta - nb;
   int start = 0;
+#pragma unroll 1
   for (int b = 0; b < p.B; ++b) {
     const int len = max(0, min(p.seq_lens[b], p.n_max));
     if (len == 0) continue;
@@ -475,11 +478,26 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
         acc += h[i];
       }
     }
+    // the prefetch bound: the same rule for ~1.5 e + 8 tokens (the likely selected ones)
+    const uint32_t w2 = min(win, (uint32_t)ceilf(1.5f * (float)pl.keff / (float)pl.Cb) + 8u);
+    if (threadIdx.x == 0 && total <= w2) sm.pf_key = 0u;
+    if (before <= w2 && before + local > w2) {
+      uint32_t acc = before;
+#pragma unroll
+      for (int i = 7; i >= 0; --i) {
+        if (acc + h[i] > w2) {
+          const int bin = hi - 8 + i;
+          sm.pf_key = bin + 1 < kTauBins ? ((uint32_t)(bin + 1)) << (32 - kTauBits) : 0xFFFFFFFFu;
+          break;
+        }
+        acc += h[i];
+      }
+    }
   }
   stamp(p, 14);
   stamp(p, 16);
   __syncthreads();
-  const uint32_t tau = sm.tau_key;
+  const uint32_t tau = sm.tau_key, pf = sm.pf_key;
   // this CTA's tokens with key >= tau, in token order, to its window of win slots
   const float* gsc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
   const int n = pl.r1 - pl.r0;
@@ -487,6 +505,7 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
   uint32_t* ck = p.cand_key + (size_t)pl.b * kCandCap + (size_t)pl.c * pl.win;
   int32_t* ct = p.cand_tok + (size_t)pl.b * kCandCap + (size_t)pl.c * pl.win;
   uint32_t written = 0;
+#pragma unroll 1
   for (int base = 0; base < n; base += kThreads) {
     const int j = base + threadIdx.x;
     uint32_t key = 0;
@@ -500,6 +519,11 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
     if (f && pos < (uint32_t)pl.win) {
       __stcg(ck + pos, key);
       __stcg(ct + pos, pl.r0 + j);
+      if (key >= pf) {  // a likely TopK token: its K and V rows (all heads) into L2 now
+        const size_t row = ((size_t)pl.b * p.n_max + pl.r0 + j) * p.Hkv * kD;
+        bulk_prefetch_l2(p.K + row, (uint32_t)(p.Hkv * kD * 2));
+        bulk_prefetch_l2(p.V + row, (uint32_t)(p.Hkv * kD * 2));
+      }
     }
     written += tot;
   }
@@ -717,6 +741,7 @@ __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, __nv_bfloat16* sQ, int mt_rows) {
   constexpr int VPR = kD * 2 / 16;
+#pragma unroll 1
   for (int v = threadIdx.x; v < mt_rows * VPR; v += kThreads) {
     const int r = v / VPR, c = v % VPR;
     __nv_bfloat16* dst = sQ + r * kSTR + c * 8;
@@ -733,6 +758,7 @@ __device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, 
 __device__ __forceinline__ void load_kv_block(const FusedParams& p, const Smem& sm, int b, int g, int blk0, int ntok,
                                               __nv_bfloat16* dk, __nv_bfloat16* dv) {
   constexpr int VPR = kD * 2 / 16;
+#pragma unroll 1
   for (int v = threadIdx.x; v < kTokBlk * VPR; v += kThreads) {
     const int r = v / VPR, c = v % VPR;
     const int i = blk0 + r;
@@ -957,8 +983,10 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
 
 // ---------------------------------------------------------------------------
 // phase 5: merge the nsplit partials of head g for rows r = split, split + nsplit, ...
-// Every (m, l) is staged first (one round trip), then each row's partial
-// vectors are fetched six at a time by up to kWarps / rows warps.
+// The partial vectors of those rows are staged in shared memory by 16-byte copies, all
+// in flight at once (one L2 round trip per batch of 128), while the (m, l) pairs give
+// each row M = max m and den = sum 2^(m - M) l; then one warp per row sums its splits
+// in split order (the same order every call: the result is deterministic).
 // ---------------------------------------------------------------------------
 __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan& pl, int g) {
   stamp(p, 18);
@@ -967,82 +995,86 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
   const int nr = (p.rows - pl.split + ns - 1) / ns;
   if (nr <= 0) return;
   const size_t cta0 = (size_t)pl.start + (size_t)g * ns;  // CTA holding split 0 of head g
-  for (int t = threadIdx.x; t < nr * ns; t += kThreads) {
+  const int npair = nr * ns;                              // pair t: row ri = t / ns, split t % ns
+  constexpr int kPB = 128;                                // pairs per batch: 64 KiB staged
+  float4* stg = reinterpret_cast<float4*>(big);           // [kPB][32]
+  float4* acc = stg + kPB * 32;                           // [nr][32] (nr <= kMaxRows: 64 KiB)
+  auto issue = [&](int t0) {
+    const int nb = min(kPB, npair - t0);
+    #pragma unroll 1
+    for (int x = threadIdx.x; x < nb * 32; x += kThreads) {
+      const int t = t0 + x / 32, ri = t / ns, s2 = t % ns;
+      cp_async_16(stg + x, p.Op + ((cta0 + s2) * p.rows + pl.split + ri * ns) * kD + (x % 32) * 4, 16);
+    }
+    cp_async_commit();
+  };
+  issue(0);
+  #pragma unroll 1
+  for (int t = threadIdx.x; t < npair; t += kThreads) {
     const int ri = t / ns, s2 = t % ns;
-    const float2 ml =
-        __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
     sm.cm[t] = ml.x;
     sm.cl[t] = ml.y;
   }
+  #pragma unroll 1
+  for (int i = threadIdx.x; i < nr * 32; i += kThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
   stamp(p, 17);
-  const int parts = nr >= kWarps ? 1 : kWarps / nr;
-  const int rows_per_pass = kWarps / parts;
-  float* stage = reinterpret_cast<float*>(big);  // [(parts-1) * rows_per_pass][kD]
-  const int part = warp % parts;
-  for (int rbase = 0; rbase < nr; rbase += rows_per_pass) {
-    const int slot = warp / parts;
-    const int ri = rbase + slot;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll 1
+  for (int ri = warp; ri < nr; ri += kWarps) {
     float M = -INFINITY, den = 0.f;
-    const bool live = ri < nr;
-    const int r = pl.split + ri * ns;
-    if (live) {
-      for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, sm.cm[ri * ns + s2]);
-      M = warp_max(M);
-      if (M != -INFINITY) {
-        for (int s2 = lane; s2 < ns; s2 += 32) den = fmaf(exp2f(sm.cm[ri * ns + s2] - M), sm.cl[ri * ns + s2], den);
-        den = warp_sum(den);
-        for (int s0 = part; s0 < ns; s0 += 6 * parts) {
-          float4 v[6];
-          float w[6];
-#pragma unroll
-          for (int u = 0; u < 6; ++u) {
-            const int s2 = s0 + u * parts;
-            if (s2 < ns) {
-              w[u] = exp2f(sm.cm[ri * ns + s2] - M);
-              v[u] = __ldcg(reinterpret_cast<const float4*>(p.Op + ((cta0 + s2) * p.rows + r) * kD) + lane);
-            } else {
-              w[u] = 0.f;
-              v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 6; ++u) {
-            acc[0] = fmaf(w[u], v[u].x, acc[0]);
-            acc[1] = fmaf(w[u], v[u].y, acc[1]);
-            acc[2] = fmaf(w[u], v[u].z, acc[2]);
-            acc[3] = fmaf(w[u], v[u].w, acc[3]);
-          }
-        }
+    #pragma unroll 1
+    for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, sm.cm[ri * ns + s2]);
+    M = warp_max(M);
+    if (M != -INFINITY)
+      #pragma unroll 1
+      for (int s2 = lane; s2 < ns; s2 += 32) den = fmaf(exp2f(sm.cm[ri * ns + s2] - M), sm.cl[ri * ns + s2], den);
+    den = warp_sum(den);
+    if (lane == 0) {
+      sm.rowM[ri] = M;
+      sm.rowD[ri] = den;
+    }
+  }
+  #pragma unroll 1
+  for (int t0 = 0; t0 < npair; t0 += kPB) {
+    if (t0 > 0) issue(t0);
+    cp_async_wait<0>();
+    __syncthreads();  // this batch (and, first time, every row's M) is visible
+    const int nb = min(kPB, npair - t0);
+    #pragma unroll 1
+    for (int ri = warp; ri < nr; ri += kWarps) {
+      const int s_lo = max(0, t0 - ri * ns), s_hi = min(ns, t0 + nb - ri * ns);
+      if (s_lo >= s_hi) continue;
+      const float M = sm.rowM[ri];
+      float4 a = acc[ri * 32 + lane];
+      #pragma unroll 1
+      for (int s2 = s_lo; s2 < s_hi; ++s2) {
+        const int t = ri * ns + s2;
+        const float w = M == -INFINITY ? 0.f : exp2f(sm.cm[t] - M);
+        const float4 v = stg[(t - t0) * 32 + lane];
+        a.x = fmaf(w, v.x, a.x);
+        a.y = fmaf(w, v.y, a.y);
+        a.z = fmaf(w, v.z, a.z);
+        a.w = fmaf(w, v.w, a.w);
       }
+      acc[ri * 32 + lane] = a;
     }
-    if (parts > 1) {
-      if (live && part > 0)
-        *reinterpret_cast<float4*>(stage + ((size_t)(part - 1) * rows_per_pass + slot) * kD + lane * 4) =
-            make_float4(acc[0], acc[1], acc[2], acc[3]);
-      __syncthreads();
-      if (live && part == 0)
-        for (int pp = 1; pp < parts; ++pp) {
-          const float4 o = *reinterpret_cast<const float4*>(stage + ((size_t)(pp - 1) * rows_per_pass + slot) * kD + lane * 4);
-          acc[0] += o.x;
-          acc[1] += o.y;
-          acc[2] += o.z;
-          acc[3] += o.w;
-        }
-    }
-    if (live && part == 0) {
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-      const int l = r / p.G, h = g * p.G + r % p.G;
-      __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
-      uint2 wv;
-      wv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-      wv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-      *reinterpret_cast<uint2*>(out) = wv;
-      if (p.lse && lane == 0)
-        p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
-    }
-    __syncthreads();
+    __syncthreads();  // before the next batch overwrites the stage
+  }
+  #pragma unroll 1
+  for (int ri = warp; ri < nr; ri += kWarps) {
+    const int r = pl.split + ri * ns;
+    const float den = sm.rowD[ri], M = sm.rowM[ri];
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const float4 a = acc[ri * 32 + lane];
+    const int l = r / p.G, h = g * p.G + r % p.G;
+    __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
+    uint2 wv;
+    wv.x = pack_bf16x2(a.x * inv, a.y * inv);
+    wv.y = pack_bf16x2(a.z * inv, a.w * inv);
+    *reinterpret_cast<uint2*>(out) = wv;
+    if (p.lse && lane == 0)
+      p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
   }
 }
 
@@ -1064,6 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   __syncthreads();
   const Plan pl = sm.plan;
   if (blockIdx.x == 0) {  // sequences with no tokens: count 0, idx -1, O = 0, lse = -inf
+#pragma unroll 1
     for (int b = 0; b < p.B; ++b) {
       if (max(0, min(p.seq_lens[b], p.n_max)) > 0) continue;
       for (int i = threadIdx.x; i < p.k; i += kThreads) p.idx[(size_t)b * p.k + i] = -1;
@@ -1204,6 +1237,10 @@ FusedCfg fused_cfg() {
 bool fused_decode_supported(const clsa_decode_args* a) {
   if (a->dtype != CLSA_BF16 || a->d != kD || (a->d_idx != 64 && a->d_idx != 128)) return false;
   if (a->K_S != nullptr) return false;
+  // 16-byte copies and L2 bulk prefetches of K_idx, K and V rows
+  if ((reinterpret_cast<uintptr_t>(a->k_idx) | reinterpret_cast<uintptr_t>(a->K) |
+       reinterpret_cast<uintptr_t>(a->V)) % 16 != 0)
+    return false;
   if (a->Hkv > 64 || a->L * (a->Hq / a->Hkv) > kMaxRows || a->k > kMaxUnitTok) return false;
   const FusedCfg cfg = fused_cfg();
   if (!cfg.ok || a->B > cfg.ncta / 2) return false;
