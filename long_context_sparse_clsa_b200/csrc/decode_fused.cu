@@ -399,9 +399,12 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (sub == 0 && j < j1) {
-        __stcg(sc + j, acc);
-        if (nrows <= kMaxUnitTok) sm.score[j] = acc;
-        if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
+        if (nrows <= kMaxUnitTok) {
+          sm.score[j] = acc;  // global copy and histogram after the stream (off its critical path)
+        } else {
+          __stcg(sc + j, acc);
+          if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
+        }
       }
     }
     if (it + kScanS < nst) issue(st, j0 + (it + kScanS) * ROWS);  // refill the slot just read
@@ -429,6 +432,15 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool hi
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
   scan_rows<DIDX>(p, sm, th, reinterpret_cast<uint4*>(th + kTauBins), src, sc, q, 0, nrows, nrows, hist);
+  if (nrows <= kMaxUnitTok) {
+    __syncthreads();
+#pragma unroll 1
+    for (int j = threadIdx.x; j < nrows; j += kThreads) {
+      const float x = sm.score[j];
+      __stcg(sc + j, x);
+      if (hist) atomicAdd(&th[float_key(x) >> (32 - kTauBits)], 1u);
+    }
+  }
   __syncthreads();
   return true;
 }
