@@ -9,8 +9,8 @@ L-layer sparse GQA attention) on B200.
 One JSON line on rank 0.  A step is one decode token per sequence through the
 whole path; the default workload is the 128K-context decode (batch 1, n=131072,
 d_idx=128, k=2048, L=24, 32 query / 8 KV heads, d=128, bf16, 1% planted tokens).
-Device time is measured with CUDA events around each step on the stream the
-library launches on.  Between steps the inputs rotate through R sets whose K_idx
+Device time is measured with CUDA events on the stream the library launches on: one
+pair around the K back-to-back steps (``--l2 rotate``), or one pair per step.  Between steps the inputs rotate through R sets whose K_idx
 copies together exceed twice the 126 MB L2 (``--l2 rotate``, the default: each step
 reads its K_idx and K/V rows from HBM, the kernel code stays cached), or L2 is
 flushed by a 512 MiB write and read-back outside the timed events (``--l2 flush``).  With N > 1 every rank runs its own sequences (weak
@@ -313,21 +313,32 @@ def run_clsa(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # The timed region: K steps back to back on the stream, one event pair around them (with
+    # --l2 flush, one pair per step so that the flushes stay outside the timed events).
     barrier()
     with ClockSampler(local) as clk:
-        for i, (e0, e1) in enumerate(evs):
-            between_steps()
+        if args.l2 == "rotate":
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            run_step(i)
+            for i in range(args.steps):
+                run_step(i)
             e1.record(stream)
-        torch.cuda.synchronize()
+            torch.cuda.synchronize()
+            total_ms = e0.elapsed_time(e1)
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for i, (a0, a1) in enumerate(evs):
+                between_steps()
+                a0.record(stream)
+                run_step(i)
+                a1.record(stream)
+            torch.cuda.synchronize()
+            total_ms = sum(a0.elapsed_time(a1) for a0, a1 in evs)
     barrier()
     st = ws.status()
     if st[0] != "CLSA_OK":
         raise RuntimeError(f"device error during timing: {st}")
-    times = [e0.elapsed_time(e1) for e0, e1 in evs]  # ms
-    total_ms = sum(times)
     if world > 1:
         import torch.distributed as dist
         t = torch.tensor([total_ms], device=dev)
