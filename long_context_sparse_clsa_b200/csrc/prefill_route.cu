@@ -67,24 +67,28 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 
 namespace {
 
-constexpr int kRM = 128;        // rows per query block (TMEM lanes)
-constexpr int kRN = 128;        // keys per tile
-constexpr int kRStages = 3;     // K tile ring
-constexpr int kRThreads = 320;  // 10 warps
-constexpr int kWarm = 8;        // warm-up tiles per unit
-constexpr int kBins = 32;       // warm-up histogram bins per row
-constexpr int kStagePitch = 36; // words per staged row
-constexpr int kTraceSlots = 20; // producer issue, MMA operands ready, MMA issued, epilogue warps done, started
-constexpr int kMinSample = 8;   // fewer expected sample scores above the boundary: no bound
+constexpr int kRM = 128;         // rows per query block (TMEM lanes)
+constexpr int kRN = 128;         // keys per tile: two 64-key halves
+constexpr int kRH = 64;          // keys per half
+constexpr int kRStages = 2;      // K tile ring
+constexpr int kEpiWarps = 16;    // 4 lane quarters x 2 query blocks x 2 key halves
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kRThreads = 64 + kEpiThreads;  // + producer warp + MMA warp
+constexpr int kWarm = 8;         // warm-up tiles per unit
+constexpr int kBins = 32;        // warm-up histogram bins per row
+constexpr int kStagePitch = 36;  // words per staged row
+constexpr int kTraceSlots = 40;  // producer issue, MMA operands ready, MMA issued, epilogue warps done, started
+constexpr int kMinSample = 8;    // fewer expected sample scores above the boundary: no bound
 constexpr uint32_t kABlock = kRM * 128 * 2;  // one query block, both 64-column atoms: 32 KiB
 constexpr uint32_t kBTile = kRN * 128 * 2;   // one key tile, both atoms: 32 KiB
 constexpr uint32_t kAtomA = kRM * 128;       // 16 KiB
 constexpr uint32_t kAtomB = kRN * 128;
+constexpr uint32_t kHalfB = kRH * 128;       // one half of one atom of the key tile: 8 KiB
 
 struct RouteParams {
   int n, T, k, S, cap, nunits;
-  uint2* cand;         // [T][S][cap] candidates: (score fp32 bits, token)
-  int32_t* cand_cnt;   // [T][S]  (> cap: overflow)
+  uint2* cand;         // [T][S][2][cap/2] candidates: (score fp32 bits, token), per key half
+  int32_t* cand_cnt;   // [T][S][2]  (> cap/2: overflow)
   float* cand_tau;     // [T][S]  the bound the slice used (-inf: every token kept)
   uint32_t* any_flag;  // set by the densify step when some row needs the exact fallback
   unsigned long long* trace;  // CTA 0 per-step stamps [512][kTraceSlots] or null
@@ -92,13 +96,15 @@ struct RouteParams {
 };
 
 struct RouteSmem {
-  // per epilogue thread, private: its row's warm-up histogram (column et of hist), then,
-  // in the main pass, its 32 staged scores (row et of stage, padded so that eight
-  // 16-byte stores of a quarter-warp hit distinct banks)
+  // per epilogue thread, private: its warm-up histogram (column et of hist), then, in the
+  // main pass, its 32 staged scores (row et of stage, padded so that eight 16-byte
+  // stores of a quarter-warp hit distinct banks)
   union {
-    uint32_t hist[kBins][256];
-    uint32_t stage[256][kStagePitch];
+    uint32_t hist[kBins][kEpiThreads];
+    uint32_t stage[kEpiThreads][kStagePitch];
   } u;
+  float xmax[kEpiThreads], xsum[kEpiThreads];  // range exchange between the two halves of a row
+  int xcnt[kEpiThreads], xseen[kEpiThreads];
   uint64_t full[kRStages], empty[kRStages];
   uint64_t tfull[2], tempty[2];
   uint64_t afull, aempty;
@@ -106,6 +112,7 @@ struct RouteSmem {
   int abort_flag;
 };
 constexpr size_t kRouteSmem = 1024 /*align slack*/ + 2 * kABlock + kRStages * kBTile + sizeof(RouteSmem);
+static_assert(kRouteSmem <= 227 * 1024, "shared memory");
 
 // warm-up histogram bin of a score: round(sat(score * hs + hb) * (kBins - 1)), the
 // rounding done by adding 1.5 * 2^23 (the sum's low mantissa bits are the integer)
@@ -155,17 +162,22 @@ __device__ __forceinline__ void st_global_v2_if(uint2* p, uint32_t a, uint32_t b
                "r"(b), "r"((uint32_t)pred));
 }
 
-// barrier among the eight epilogue warps only (named barrier 1)
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// barrier among the epilogue warps only (named barrier 1)
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
-// the unit's tiles: main pass = [t_lo, t_hi); warm-up = kWarm tiles spread over it
+// A unit's key slice, in 64-key blocks [b_lo, b_hi), is cut into two contiguous halves
+// [b_lo, b_mid) and [b_mid, b_hi); step tau loads block b_lo + tau of the first half and
+// b_mid + tau of the second (absent past b_hi).  Main pass: tau = 0 .. L-1; warm-up:
+// nwarm steps spread over the same range.
 struct UnitTiles {
-  int r0, t_lo, t_hi, nwarm;
-  __device__ int count() const { return nwarm + (t_hi - t_lo); }
-  __device__ int tile(int it) const {  // tile index of step it
-    if (it < nwarm) return t_lo + (int)(((long long)it * (t_hi - t_lo)) / nwarm);
-    return t_lo + (it - nwarm);
+  int r0, b_lo, b_mid, b_hi, L, nwarm;
+  __device__ int count() const { return nwarm + L; }
+  __device__ int tau(int it) const {
+    if (it < nwarm) return (int)(((long long)it * L) / nwarm);
+    return it - nwarm;
   }
+  __device__ int block(int it, int half) const { return (half ? b_mid : b_lo) + tau(it); }
+  __device__ bool valid(int it, int half) const { return block(it, half) < (half ? b_hi : b_mid); }
 };
 
 __device__ __forceinline__ UnitTiles unit_tiles(const RouteParams& p, int u) {
@@ -173,10 +185,12 @@ __device__ __forceinline__ UnitTiles unit_tiles(const RouteParams& p, int u) {
   const int pair = u / p.S, s = u % p.S;
   ut.r0 = pair * 2 * kRM;
   const int tmax = p.n - p.T + min(ut.r0 + 2 * kRM, p.T) - 1;  // largest position of the pair
-  const int ntile = tmax / kRN + 1;
-  ut.t_lo = (int)(((long long)s * ntile) / p.S);
-  ut.t_hi = (int)(((long long)(s + 1) * ntile) / p.S);
-  ut.nwarm = min(kWarm, ut.t_hi - ut.t_lo);
+  const int nblk = tmax / kRH + 1;
+  ut.b_lo = (int)(((long long)s * nblk) / p.S);
+  ut.b_hi = (int)(((long long)(s + 1) * nblk) / p.S);
+  ut.L = (ut.b_hi - ut.b_lo + 1) / 2;
+  ut.b_mid = ut.b_lo + ut.L;
+  ut.nwarm = min(kWarm, ut.L);
   return ut;
 }
 
@@ -187,7 +201,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~uintptr_t(1023));
   unsigned char* sA = smem;                    // [2 blocks][2 atoms][128 rows][128 B]
-  unsigned char* sB = smem + 2 * kABlock;      // [stage][2 atoms][128 keys][128 B]
+  unsigned char* sB = smem + 2 * kABlock;      // [stage][2 atoms][2 halves x 64 keys][128 B]
   RouteSmem& sm = *reinterpret_cast<RouteSmem*>(sB + kRStages * kBTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -198,7 +212,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.tfull[i], 1);
-      mbar_init(&sm.tempty[i], 8);
+      mbar_init(&sm.tempty[i], kEpiWarps);
     }
     mbar_init(&sm.afull, 1);
     mbar_init(&sm.aempty, 1);
@@ -230,10 +244,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
             tma_load_2d(sA + h * kABlock + a * kAtomA, &tq, a * 64, ut.r0 + h * kRM, &sm.afull);
         for (int it = 0; it < ut.count(); ++it) {
           if (!mbar_wait_sleep(&sm.empty[stage], ph_empty)) { record_error(p.ws_header, CLSA_ERR_TIMEOUT, 401); sm.abort_flag = 1; break; }
-          const int j0 = ut.tile(it) * kRN;
           if (p.trace && blockIdx.x == 0 && it < 512) p.trace[it * kTraceSlots] = globaltimer_ns();
           mbar_arrive_expect_tx(&sm.full[stage], kBTile);
-          for (int a = 0; a < 2; ++a) tma_load_2d(sB + stage * kBTile + a * kAtomB, &tk, a * 64, j0, &sm.full[stage]);
+          // key rows 0..63 of the tile: block of the first half; 64..127: of the second
+          // (past the slice, or past n: loaded, masked by the epilogue / zero-filled)
+          for (int hf = 0; hf < 2; ++hf)
+            for (int a = 0; a < 2; ++a)
+              tma_load_2d(sB + stage * kBTile + a * kAtomB + hf * kHalfB, &tk, a * 64, ut.block(it, hf) * kRH,
+                          &sm.full[stage]);
           if (++stage == kRStages) { stage = 0; ph_empty ^= 1u; }
         }
       }
@@ -279,12 +297,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (one row per thread)
-    const int q = warp & 3;             // TMEM lane quarter this warp may read
-    const int h = (warp - 2) >> 2;      // query block of this warpgroup
-    const int et = threadIdx.x - 64;    // epilogue thread 0..255: its private smem column / row
-    const uint32_t hist_col = smem_u32(&sm.u.hist[0][et]);  // bin b at + b * 1024 bytes
+    // ------------------------------------------------------------ epilogue (one row half per thread)
+    const int w = warp - 2;
+    const int q = warp & 3;                    // TMEM lane quarter this warp may read
+    const int g4 = w >> 2;
+    const int blk = g4 & 1, hc = g4 >> 1;      // query block, key half
+    const int et = w * 32 + lane;              // epilogue thread 0..511: its private smem column / row
+    const int pt = et ^ (kEpiThreads / 2);     // the thread holding the other half of the same row
+    const uint32_t hist_col = smem_u32(&sm.u.hist[0][et]);  // bin b at + b * 4 * kEpiThreads bytes
     const uint32_t stage_addr = smem_u32(sm.u.stage[et] + 4);  // scores at words 4..35; word 3 is read for an empty mask
+    const int caph = p.cap / 2;
     int buf = 0;
     uint32_t ph_tfull = 0;
     bool dead = false;
@@ -294,17 +316,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
       epi_bar();  // the previous unit's staging rows are free for this unit's histograms
       const UnitTiles ut = unit_tiles(p, u);
       const int s = u % p.S;
-      const int i = ut.r0 + h * kRM + q * 32 + lane;  // query row
+      const int i = ut.r0 + blk * kRM + q * 32 + lane;  // query row
       const bool row_ok = i < p.T;
-      const int t = p.n - p.T + i;                    // its cache position
+      const int t = p.n - p.T + i;                      // its cache position
       const int keff = min(p.k, t + 1);
 #pragma unroll
       for (int y = 0; y < kBins; ++y) sm.u.hist[y][et] = 0u;
-      bool have = false;       // histogram range fixed
+      bool have = false;  // histogram range fixed
       float hs = 0.f, hb = 0.f, lo = 0.f, span = 0.f;  // bin map: sat(score * hs + hb) * (kBins - 1)
       int seen = 0, cnt = 0;
       float tau = -INFINITY;
-      uint2* const dst = p.cand + ((size_t)(row_ok ? i : 0) * p.S + s) * p.cap;
+      uint2* const dst = p.cand + ((size_t)((row_ok ? i : 0) * p.S + s) * 2 + hc) * caph;
       for (int it = 0; it < ut.count(); ++it) {
         if (!dead && !mbar_wait_warp(&sm.tfull[buf], ph_tfull)) {
           if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 420);
@@ -312,129 +334,128 @@ __global__ void __launch_bounds__(kRThreads, 1)
           dead = true;
         }
         dead = __any_sync(0xffffffffu, dead || *(volatile int*)&sm.abort_flag);
-        if (p.trace && blockIdx.x == 0 && lane == 0 && it < 512) p.trace[it * kTraceSlots + 8 + 1 + warp] = globaltimer_ns();
+        if (p.trace && blockIdx.x == 0 && lane == 0 && it < 512) p.trace[it * kTraceSlots + 3 + kEpiWarps + w] = globaltimer_ns();
         tc::fence_after_sync();
-        const int j0 = ut.tile(it) * kRN;
         const bool warm = it < ut.nwarm;
-        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + h * kRN);
-        const int nvis = row_ok ? max(0, min(kRN, t - j0 + 1)) : 0;  // causally visible columns
-        if (!dead && warm && __any_sync(0xffffffffu, !have)) {
-          // histogram range from this tile's visible scores: [mean, mean + 1.25 (max -
-          // mean)]; larger scores count in the top bin, smaller ones in bin 0
+        const int j0 = ut.block(it, hc) * kRH;
+        const int nvis = (row_ok && ut.valid(it, hc)) ? max(0, min(kRH, t - j0 + 1)) : 0;  // visible keys
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256 + blk * kRN + hc * kRH);
+        if (warm && it == 0) {
+          // histogram range of the row from this first tile, both halves:
+          // [mean, mean + 1.25 (max - mean)]; larger scores count in the top bin
           float mx = -INFINITY, s0 = 0.f, s1 = 0.f;
+          if (!dead) {
 #pragma unroll 1
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t v[64];
-            tc::ld_32x32b_x64(tbase + (uint32_t)(64 * hf), v);
-            tc::ld_wait();
+            for (int ch = 0; ch < 2; ++ch) {
+              uint32_t v[32];
+              tc::ld_32x32b_x32(tbase + (uint32_t)(32 * ch), v);
+              tc::ld_wait();
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              if (64 * hf + c < nvis) {
-                mx = fmaxf(mx, __uint_as_float(v[c]));
-                s0 += __uint_as_float(v[c]);
-              }
-              if (64 * hf + c + 1 < nvis) {
-                mx = fmaxf(mx, __uint_as_float(v[c + 1]));
-                s1 += __uint_as_float(v[c + 1]);
+              for (int c = 0; c < 32; c += 2) {
+                if (32 * ch + c < nvis) {
+                  mx = fmaxf(mx, __uint_as_float(v[c]));
+                  s0 += __uint_as_float(v[c]);
+                }
+                if (32 * ch + c + 1 < nvis) {
+                  mx = fmaxf(mx, __uint_as_float(v[c + 1]));
+                  s1 += __uint_as_float(v[c + 1]);
+                }
               }
             }
           }
-          if (!have && nvis > 0) {
-            lo = (s0 + s1) / (float)nvis;
-            span = 1.25f * (mx - lo);
+          sm.xmax[et] = mx;
+          sm.xsum[et] = s0 + s1;
+          sm.xcnt[et] = nvis;
+          epi_bar();
+          const float mx2 = fmaxf(mx, sm.xmax[pt]), sum2 = s0 + s1 + sm.xsum[pt];
+          const int c2 = nvis + sm.xcnt[pt];
+          if (row_ok && c2 > 0) {
+            // the pair sums in the same order on both threads: the same range
+            lo = (hc == 0 ? (s0 + s1) + sm.xsum[pt] : sm.xsum[pt] + (s0 + s1)) / (float)c2;
+            span = 1.25f * (mx2 - lo);
             if (span > 0.f && span < INFINITY) {
               hs = 1.f / span;
               hb = -lo * hs;
               have = true;
             }
           }
+          (void)sum2;
         }
-        if (!dead && warm && have) seen += nvis;
-        if (!dead && !(warm && !__any_sync(0xffffffffu, have))) {
+        if (!dead && (!warm || __any_sync(0xffffffffu, have))) {
+          float sc = 1.f, negt = 0.f;
+          if (!warm) ge_setup(tau, sc, negt);
+          if (warm && have) seen += nvis;
 #pragma unroll 1
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t v[64];
-            tc::ld_32x32b_x64(tbase + (uint32_t)(64 * hf), v);
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t v[32];
+            tc::ld_32x32b_x32(tbase + (uint32_t)(32 * ch), v);
             tc::ld_wait();
-            const int nvh = nvis - 64 * hf;  // visible columns of this half (may be <= 0 or > 64)
+            const int nv = nvis - 32 * ch;  // visible columns of this chunk (may be <= 0 or > 32)
             if (warm) {
               if (have) {
-                if (nvh >= 64) {
+                if (nv >= 32) {
 #pragma unroll
-                  for (int c = 0; c < 64; ++c) red_shared_inc(hist_col + (uint32_t)hist_bin(v[c], hs, hb) * 1024u);
+                  for (int c = 0; c < 32; ++c)
+                    red_shared_inc(hist_col + (uint32_t)hist_bin(v[c], hs, hb) * (4u * kEpiThreads));
                 } else {
 #pragma unroll
-                  for (int c = 0; c < 64; ++c)
-                    if (c < nvh) red_shared_inc(hist_col + (uint32_t)hist_bin(v[c], hs, hb) * 1024u);
+                  for (int c = 0; c < 32; ++c)
+                    if (c < nv) red_shared_inc(hist_col + (uint32_t)hist_bin(v[c], hs, hb) * (4u * kEpiThreads));
                 }
               }
             } else {
-              // one compare per score into two 32-bit masks, on the FMA pipe: ge01 is exactly
+              // one compare per score into a 32-bit mask, on the FMA pipe: ge01 is exactly
               // 1 or 0, and the weighted sums of 16 of them are exact integers
-              float sc = 1.f, negt = 0.f;
-              ge_setup(tau, sc, negt);
-              uint32_t mk[2];
+              float l0 = 0.f, l1 = 0.f, u0 = 0.f, u1 = 0.f;
 #pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                float l0 = 0.f, l1 = 0.f, u0 = 0.f, u1 = 0.f;
-#pragma unroll
-                for (int c = 0; c < 16; c += 2) {
-                  l0 = fmaf(ge01(v[32 * k + c], sc, negt), (float)(1u << c), l0);
-                  l1 = fmaf(ge01(v[32 * k + c + 1], sc, negt), (float)(1u << (c + 1)), l1);
-                  u0 = fmaf(ge01(v[32 * k + 16 + c], sc, negt), (float)(1u << c), u0);
-                  u1 = fmaf(ge01(v[32 * k + 16 + c + 1], sc, negt), (float)(1u << (c + 1)), u1);
-                }
-                // 2^23 + m (m < 2^16) is exact: the low 16 bits of its encoding are m
-                mk[k] = __byte_perm(__float_as_uint((l0 + l1) + 8388608.f), __float_as_uint((u0 + u1) + 8388608.f),
-                                    0x5410);
-                if (tau == -INFINITY) mk[k] = 0xffffffffu;  // keep-all row
-                const int nv = nvh - 32 * k;
-                if (nv < 32) mk[k] &= nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
+              for (int c = 0; c < 16; c += 2) {
+                l0 = fmaf(ge01(v[c], sc, negt), (float)(1u << c), l0);
+                l1 = fmaf(ge01(v[c + 1], sc, negt), (float)(1u << (c + 1)), l1);
+                u0 = fmaf(ge01(v[16 + c], sc, negt), (float)(1u << c), u0);
+                u1 = fmaf(ge01(v[16 + c + 1], sc, negt), (float)(1u << (c + 1)), u1);
               }
-              // per 32 columns: stage the scores of every 4-column group that holds a
-              // candidate of this row in its smem row, then one (score, token) store per set
-              // bit, in column order
+              // 2^23 + m (m < 2^16) is exact: the low 16 bits of its encoding are m
+              uint32_t mm = __byte_perm(__float_as_uint((l0 + l1) + 8388608.f),
+                                        __float_as_uint((u0 + u1) + 8388608.f), 0x5410);
+              if (tau == -INFINITY) mm = 0xffffffffu;  // keep-all row
+              if (nv < 32) mm &= nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
+              // stage the scores of every 4-column group that holds a candidate in this
+              // thread's smem row, then one (score, token) store per set bit, in column order
+              if (__any_sync(0xffffffffu, mm != 0u)) {
 #pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                uint32_t mm = mk[k];
-                if (__any_sync(0xffffffffu, mm != 0u)) {
+                for (int g = 0; g < 8; ++g)
+                  st_shared_v4_if(stage_addr + 16u * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3],
+                                  (mm >> (4 * g)) & 0xfu);
+                const uint32_t jb = (uint32_t)(j0 + 32 * ch);
+                const int pc = __popc(mm);
+                if (cnt + pc <= caph) {
+                  uint2* const out = dst + cnt;
 #pragma unroll
-                  for (int g = 0; g < 8; ++g)
-                    st_shared_v4_if(stage_addr + 16u * g, v[32 * k + 4 * g], v[32 * k + 4 * g + 1],
-                                    v[32 * k + 4 * g + 2], v[32 * k + 4 * g + 3], (mm >> (4 * g)) & 0xfu);
-                  const uint32_t jb = (uint32_t)(j0 + 64 * hf + 32 * k);
-                  const int pc = __popc(mm);
-                  if (cnt + pc <= p.cap) {
-                    // common case: room for every candidate; the first four without
-                    // branches (immediate offsets from one pointer), the rare rest in a loop
-                    uint2* const out = dst + cnt;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                      const uint32_t lsb = mm & (0u - mm);
-                      const int c = 31 - __clz(lsb);  // -1 when mm == 0: reads the pad word, store off
-                      st_global_v2_if(out + e, ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c, mm != 0u);
-                      mm ^= lsb;
-                    }
-                    if (__any_sync(0xffffffffu, mm != 0u)) {
-                      int e = 4;
-                      while (mm) {
-                        const int c = __ffs(mm) - 1;
-                        out[e++] = make_uint2(ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c);
-                        mm &= mm - 1u;
-                      }
-                    }
-                  } else {
-                    // overflow: keep counting (the row is flagged), stop writing past the buffer
-                    int e = 0;
+                  for (int e = 0; e < 4; ++e) {
+                    const uint32_t lsb = mm & (0u - mm);
+                    const int c = 31 - __clz(lsb);  // -1 when mm == 0: reads the pad word, store off
+                    st_global_v2_if(out + e, ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c, mm != 0u);
+                    mm ^= lsb;
+                  }
+                  if (__any_sync(0xffffffffu, mm != 0u)) {
+                    int e = 4;
                     while (mm) {
                       const int c = __ffs(mm) - 1;
-                      if (cnt + e < p.cap) dst[cnt + e] = make_uint2(ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c);
-                      ++e;
+                      out[e++] = make_uint2(ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c);
                       mm &= mm - 1u;
                     }
                   }
-                  cnt += pc;
+                } else {
+                  // overflow: keep counting (the row is flagged), stop writing past the buffer
+                  int e = 0;
+                  while (mm) {
+                    const int c = __ffs(mm) - 1;
+                    if (cnt + e < caph) dst[cnt + e] = make_uint2(ld_shared_u32(stage_addr + 4 * c), jb + (uint32_t)c);
+                    ++e;
+                    mm &= mm - 1u;
+                  }
                 }
+                cnt += pc;
               }
             }
           }
@@ -442,20 +463,24 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
-        if (p.trace && blockIdx.x == 0 && lane == 0 && it < 512) p.trace[it * kTraceSlots + 1 + warp] = globaltimer_ns();
+        if (p.trace && blockIdx.x == 0 && lane == 0 && it < 512) p.trace[it * kTraceSlots + 3 + w] = globaltimer_ns();
         if (++buf == 2) { buf = 0; ph_tfull ^= 1u; }
         if (it + 1 == ut.nwarm) {
-          // lower edge of the highest bin at which the sample count from the top reaches
-          // m = twice the expected count of the sample above the k_eff boundary; no bound
-          // (tau = -inf, every token a candidate) when all tokens are selected or the
-          // sample is too small.  The bound is a guess: the densify step verifies it.
+          // lower edge of the highest bin at which the sample count (both halves) from the
+          // top reaches m = twice the expected count of the sample above the k_eff
+          // boundary; no bound (tau = -inf, every token a candidate) when all tokens are
+          // selected or the sample is too small.  The bound is a guess: the densify step
+          // verifies it.  Both threads of a row compute the same tau.
+          sm.xseen[et] = seen;
+          epi_bar();  // both halves' histograms are complete
+          const int seen2 = seen + sm.xseen[pt];
           tau = -INFINITY;
           if (have && keff < t + 1) {
-            const int m = (int)ceilf(2.0f * (float)keff * (float)seen / (float)(t + 1));
-            if (m >= kMinSample && seen >= m) {
+            const int m = (int)ceilf(2.0f * (float)keff * (float)seen2 / (float)(t + 1));
+            if (m >= kMinSample && seen2 >= m) {
               int cum = 0;
               for (int y = kBins - 1; y >= 1; --y) {  // bin 0 also holds every lower score
-                cum += (int)sm.u.hist[y][et];
+                cum += (int)(sm.u.hist[y][et] + sm.u.hist[y][pt]);
                 if (cum >= m) {
                   tau = lo + ((float)y - 0.5f) * span / (float)(kBins - 1);
                   break;
@@ -467,8 +492,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
       }
       if (row_ok) {
-        p.cand_cnt[(size_t)i * p.S + s] = cnt;
-        p.cand_tau[(size_t)i * p.S + s] = ut.count() > 0 ? tau : -INFINITY;
+        p.cand_cnt[((size_t)i * p.S + s) * 2 + hc] = cnt;
+        if (hc == 0) p.cand_tau[(size_t)i * p.S + s] = ut.count() > 0 ? tau : -INFINITY;
       }
     }
   }
@@ -477,14 +502,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
   if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
-// One CTA per row: concatenate the row's slice buffers (slices in key order, tokens
-// ascending inside a slice) into a dense candidate row, or flag the row for the exact
-// fallback when a slice overflowed or the candidates number fewer than k_eff.
+// One CTA per row: concatenate the row's buffers (slices in key order, each slice's two
+// halves in key order, tokens ascending inside a buffer) into a dense candidate row, or
+// flag the row for the exact fallback when a buffer overflowed or the candidates number
+// fewer than k_eff.
 __global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams p, uint32_t* __restrict__ dval,
                                                               int32_t* __restrict__ dtok,
                                                               int32_t* __restrict__ dlen,
                                                               int32_t* __restrict__ flag, int ldd) {
-  __shared__ int off[65];
+  __shared__ int off[2 * 64 + 1];
   __shared__ int bad;
   __shared__ float tmax;
   __shared__ int above;
@@ -492,16 +518,17 @@ __global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams 
   const int t = p.n - p.T + i;
   const int keff = min(p.k, t + 1);
   if (threadIdx.x == 0) {
+    const int caph = p.cap / 2;
     int acc = 0, over = 0;
     float tm = -INFINITY;
-    for (int s2 = 0; s2 < p.S; ++s2) {
-      const int c = p.cand_cnt[(size_t)i * p.S + s2];
-      off[s2] = acc;
-      over |= c > p.cap;
-      acc += min(c, p.cap);
-      tm = fmaxf(tm, p.cand_tau[(size_t)i * p.S + s2]);
+    for (int b2 = 0; b2 < 2 * p.S; ++b2) {
+      const int c = p.cand_cnt[(size_t)i * p.S * 2 + b2];
+      off[b2] = acc;
+      over |= c > caph;
+      acc += min(c, caph);
     }
-    off[p.S] = acc;
+    for (int s2 = 0; s2 < p.S; ++s2) tm = fmaxf(tm, p.cand_tau[(size_t)i * p.S + s2]);
+    off[2 * p.S] = acc;
     bad = over || acc < keff;
     tmax = tm;
     above = 0;
@@ -509,9 +536,9 @@ __global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams 
   __syncthreads();
   if (!bad) {
     int mine = 0;
-    for (int s2 = 0; s2 < p.S; ++s2) {
-      const int o = off[s2], c = off[s2 + 1] - o;
-      const size_t src = ((size_t)i * p.S + s2) * p.cap;
+    for (int b2 = 0; b2 < 2 * p.S; ++b2) {
+      const int o = off[b2], c = off[b2 + 1] - o;
+      const size_t src = ((size_t)i * p.S * 2 + b2) * (p.cap / 2);
       for (int e = threadIdx.x; e < c; e += blockDim.x) {
         const uint2 cv = p.cand[src + e];
         dval[(size_t)i * ldd + o + e] = cv.x;
@@ -525,7 +552,7 @@ __global__ void __launch_bounds__(256) prefill_densify_kernel(const RouteParams 
   if (threadIdx.x == 0) {
     if (!bad && above < keff) bad = 1;  // some slice's bound may have dropped a selected token
     flag[i] = bad;
-    dlen[i] = bad ? 0 : off[p.S];
+    dlen[i] = bad ? 0 : off[2 * p.S];
     if (bad) atomicOr(p.any_flag, 1u);
   }
 }
@@ -560,7 +587,8 @@ size_t prefill_route_ws_bytes(const clsa_prefill_args* a) {
   const size_t T = (size_t)a->T;
   size_t off = 0;
   off += align_up(T * rp.S * rp.cap * 8, 256);      // slice buffers (score, token)
-  off += 2 * align_up(T * rp.S * 4, 256);           // slice counts, slice bounds
+  off += align_up(T * rp.S * 2 * 4, 256);           // buffer counts (slice x half)
+  off += align_up(T * rp.S * 4, 256);               // slice bounds
   off += 2 * align_up(T * rp.ldd * 4, 256);         // dense candidate rows
   off += 2 * align_up(T * 4, 256);                  // dense lengths, fallback flags
   off += 256;                                       // any-flag word
@@ -584,7 +612,7 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
   p.cand = reinterpret_cast<uint2*>(w);
   w += align_up(T * rp.S * rp.cap * 8, 256);
   p.cand_cnt = reinterpret_cast<int32_t*>(w);
-  w += align_up(T * rp.S * 4, 256);
+  w += align_up(T * rp.S * 2 * 4, 256);
   p.cand_tau = reinterpret_cast<float*>(w);
   w += align_up(T * rp.S * 4, 256);
   out->dval = reinterpret_cast<uint32_t*>(w);
@@ -604,7 +632,7 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
 
   CUtensorMap tq, tk;
   if (!make_tmap_bf16_2d(&tq, a->q_idx, (uint64_t)a->T, 128, 256, kRM, 64) ||
-      !make_tmap_bf16_2d(&tk, a->k_idx, (uint64_t)a->n, 128, 256, kRN, 64))
+      !make_tmap_bf16_2d(&tk, a->k_idx, (uint64_t)a->n, 128, 256, kRH, 64))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(prefill_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kRouteSmem);
