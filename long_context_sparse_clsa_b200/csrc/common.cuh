@@ -267,14 +267,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// Warp-wide bounded wait: lane 0 polls without suspending, the others wait at the
-// warp barrier, then every lane observes the completed phase itself.  Call with the
+// Warp-wide bounded wait: lane 0 polls (try_wait, which may suspend it), the others wait
+// at the warp barrier, then every lane observes the completed phase itself.  Call with the
 // whole warp converged; returns the same value in every lane.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   uint32_t ok = 1;
-  if ((threadIdx.x & 31) == 0 && !mbar_test_wait(bar, parity)) {
+  if ((threadIdx.x & 31) == 0 && !mbar_try_wait(bar, parity)) {  // try_wait may suspend: no busy spin
     const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_test_wait(bar, parity)) {
+    while (!mbar_try_wait(bar, parity)) {
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         ok = 0;
         break;

@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       float hs = 0.f, hb = 0.f, lo = 0.f, span = 0.f;  // bin map: sat(score * hs + hb) * (kBins - 1)
       int seen = 0, cnt = 0;
       float tau = -INFINITY;
+      float sc = 1.f, negt = 0.f;  // the compare of the main pass (set with tau)
       uint2* const dst = p.cand + ((size_t)((row_ok ? i : 0) * p.S + s) * 2 + hc) * caph;
       for (int it = 0; it < ut.count(); ++it) {
         if (!dead && !mbar_wait_warp(&sm.tfull[buf], ph_tfull)) {
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
           sm.xsum[et] = s0 + s1;
           sm.xcnt[et] = nvis;
           epi_bar();
-          const float mx2 = fmaxf(mx, sm.xmax[pt]), sum2 = s0 + s1 + sm.xsum[pt];
+          const float mx2 = fmaxf(mx, sm.xmax[pt]);
           const int c2 = nvis + sm.xcnt[pt];
           if (row_ok && c2 > 0) {
             // the pair sums in the same order on both threads: the same range
@@ -379,11 +380,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
               have = true;
             }
           }
-          (void)sum2;
         }
         if (!dead && (!warm || __any_sync(0xffffffffu, have))) {
-          float sc = 1.f, negt = 0.f;
-          if (!warm) ge_setup(tau, sc, negt);
           if (warm && have) seen += nvis;
 #pragma unroll 1
           for (int ch = 0; ch < 2; ++ch) {
@@ -488,6 +486,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
               }
             }
           }
+          ge_setup(tau, sc, negt);
           epi_bar();  // every histogram is read: the staging rows may overwrite them
         }
       }
