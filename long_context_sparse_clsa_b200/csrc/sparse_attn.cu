@@ -14,7 +14,8 @@
 // Selector's gather into the attention.
 //
 // bf16: mma.sync m16n8k16 (fp32 accumulate), one warp per 16 rows, operands via
-// ldmatrix from padded shared tiles.  fp32: FFMA, one lane per token for the
+// ldmatrix from padded shared tiles; a ring of kStages token blocks keeps the gathered
+// rows of the next blocks in flight while one is reduced.  fp32: FFMA, one lane per token for the
 // scores and one lane per column for the output.
 #include <cmath>
 
@@ -28,6 +29,7 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kBlk = 64;  // tokens per shared-memory block (bf16 path)
+constexpr int kStages = 4;  // K/V blocks in flight (bf16 path): gathered rows have HBM latency
 
 struct AttnParams {
   const void* Q;
@@ -64,6 +66,18 @@ __device__ __forceinline__ const T* kv_row(const AttnParams& p, const T* base, i
   }
 }
 
+// token t's head-g row of the [B][kv][Hkv][D] cache (t already read from the index list)
+template <typename T, int D>
+__device__ __forceinline__ const T* kv_row_tok(const AttnParams& p, const T* base, int b, int g, int i, int t,
+                                               bool& ok) {
+  ok = (unsigned)t < (unsigned)p.n_max;
+  if (!ok) {
+    record_error(p.ws_header, CLSA_ERR_BAD_INDEX, ((long long)b << 32) | (unsigned)i);
+    return base;
+  }
+  return base + (((size_t)b * p.kv_bstride + t) * p.Hkv + g) * D;
+}
+
 // (layer, head) of CTA-local row r in layer group lgrp; false if r is padding
 __device__ __forceinline__ bool row_coords(const AttnParams& p, int lgrp, int g, int r, int& l, int& h) {
   if (r >= p.rows) return false;
@@ -81,8 +95,9 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   const int NW = blockDim.x >> 5;
-  __nv_bfloat16* sK = sQ + NW * 16 * STR;      // [2][kBlk][STR]
-  __nv_bfloat16* sV = sK + 2 * kBlk * STR;     // [2][kBlk][STR]
+  __nv_bfloat16* sK = sQ + NW * 16 * STR;            // [kStages][kBlk][STR]
+  __nv_bfloat16* sV = sK + kStages * kBlk * STR;     // [kStages][kBlk][STR]
+  int* sIdx = reinterpret_cast<int*>(sV + kStages * kBlk * STR);  // [chunk] this split's token indices
 
   const int split = blockIdx.x, g = blockIdx.y;
   const int b = blockIdx.z / p.nlg, lgrp = blockIdx.z % p.nlg;
@@ -95,6 +110,10 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
   const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(p.Q);
   const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(p.K);
   const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(p.V);
+  // the split's token indices, read once (coalesced): the gathers below then depend only on
+  // shared memory, not on a global load per row
+  if constexpr (GATHER)
+    for (int j = threadIdx.x; j < t1 - t0; j += blockDim.x) sIdx[j] = __ldg(p.idx + (size_t)b * p.k + t0 + j);
 
   // ---- Q tile -> shared (zero rows for padding)
   {
@@ -121,8 +140,14 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
       int bytes = 0;
       if (i < t1) {
         bool ok;
-        srck = kv_row<__nv_bfloat16, D, GATHER>(p, Kg, b, g, i, ok);
-        srcv = kv_row<__nv_bfloat16, D, GATHER>(p, Vg, b, g, i, ok);
+        if constexpr (GATHER) {
+          const int tk = sIdx[i - t0];
+          srck = kv_row_tok<__nv_bfloat16, D>(p, Kg, b, g, i, tk, ok);
+          srcv = kv_row_tok<__nv_bfloat16, D>(p, Vg, b, g, i, tk, ok);
+        } else {
+          srck = kv_row<__nv_bfloat16, D, GATHER>(p, Kg, b, g, i, ok);
+          srcv = kv_row<__nv_bfloat16, D, GATHER>(p, Vg, b, g, i, ok);
+        }
         if (ok) {
           srck += c * 8;
           srcv += c * 8;
@@ -139,7 +164,11 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
   };
 
   const int nblk = t1 > t0 ? (t1 - t0 + kBlk - 1) / kBlk : 0;
-  if (nblk > 0) load_block(0, t0);
+  if constexpr (GATHER) __syncthreads();  // sIdx is visible to every thread
+  for (int j = 0; j < kStages - 1; ++j) {  // blocks 0 .. kStages-2 in flight (one group each)
+    if (j < nblk) load_block(j, t0 + j * kBlk);
+    else cp_async_commit();
+  }
   __syncthreads();
 
   uint32_t qa[D / 16][4];
@@ -157,14 +186,14 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
   for (int bi = 0; bi < nblk; ++bi) {
-    const int stage = bi & 1;
+    const int stage = bi % kStages;
     const int blk0 = t0 + bi * kBlk;
-    if (bi + 1 < nblk) {
-      load_block(stage ^ 1, blk0 + kBlk);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+    {  // block bi + kStages - 1 into the stage block bi - 1 used (released by its trailing sync)
+      const int nb = bi + kStages - 1;
+      if (nb < nblk) load_block(nb % kStages, t0 + nb * kBlk);
+      else cp_async_commit();
     }
+    cp_async_wait<kStages - 1>();  // block bi has landed
     __syncthreads();
     const __nv_bfloat16* tk = sK + stage * kBlk * STR;
     const __nv_bfloat16* tv = sV + stage * kBlk * STR;
@@ -505,7 +534,7 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
   cudaError_t e = cudaSuccess;
   if (sh.dt == CLSA_BF16) {
     const int NW = (pl.rows + 15) / 16;
-    auto smem = [&](int D) { return (NW * 16 + 4 * kBlk) * (D + 8) * 2; };
+    auto smem = [&](int D) { return (NW * 16 + 2 * kStages * kBlk) * (D + 8) * 2 + pl.chunk * 4; };
 #define CLSA_ATTN_BF16(D, GA)                                                  \
   do {                                                                         \
     auto kern = attn_bf16_kernel<D, GA>;                                       \

@@ -1,7 +1,7 @@
 """Run one stage of the CLSA path on a named workload, for profilers.
 
     python -m long_context_sparse_clsa_b200.profile_cases --stage decode_step \
-        [--workload decode128k] [--reps 3] [--batch B]
+        [--workload decode128k] [--reps 3] [--batch B] [--rows T]
 
 Stages: index_scores, topk, gather_kv, sparse_attn, decode_step, prefill_chunk.
 Inputs are the seeded synthetic workloads of ``inputs.py``; ``--batch`` replaces
@@ -25,10 +25,13 @@ def main():
     ap.add_argument("--workload", default="decode128k")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--rows", type=int, default=0, help="prefill rows T (default: the workload's)")
     a = ap.parse_args()
     w = WORKLOADS[a.workload]
     if a.batch:
         w = replace(w, B=a.batch)
+    if a.rows:
+        w = replace(w, T=a.rows)
     inp = make_inputs(w)
     dv = clsa.to_device(inp)
     if w.mode == "prefill":
