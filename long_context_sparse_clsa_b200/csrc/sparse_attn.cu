@@ -89,15 +89,19 @@ __device__ __forceinline__ bool row_coords(const AttnParams& p, int lgrp, int g,
 // ---------------------------------------------------------------------------
 // bf16 tensor-core path
 // ---------------------------------------------------------------------------
-template <int D, bool GATHER>
-__global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
+// MINB = 1: up to 8 warps, kStages-deep ring, Q fragments held in registers.
+// MINB = 2: up to 6 warps and two CTAs per SM (their loads overlap each other's math):
+// a 2-deep ring per CTA and Q fragments re-read from shared memory at each k-step.
+template <int D, bool GATHER, int MINB>
+__global__ void __launch_bounds__(MINB == 2 ? 192 : 256, MINB) attn_bf16_kernel(const AttnParams p) {
+  constexpr int NST = MINB == 2 ? 2 : kStages;
   constexpr int STR = D + 8;  // padded row (elements): 16-byte aligned, ldmatrix conflict-free
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   const int NW = blockDim.x >> 5;
   __nv_bfloat16* sK = sQ + NW * 16 * STR;            // [kStages][kBlk][STR]
-  __nv_bfloat16* sV = sK + kStages * kBlk * STR;     // [kStages][kBlk][STR]
-  int* sIdx = reinterpret_cast<int*>(sV + kStages * kBlk * STR);  // [chunk] this split's token indices
+  __nv_bfloat16* sV = sK + NST * kBlk * STR;     // [kStages][kBlk][STR]
+  int* sIdx = reinterpret_cast<int*>(sV + NST * kBlk * STR);  // [chunk] this split's token indices
 
   const int split = blockIdx.x, g = blockIdx.y;
   const int b = blockIdx.z / p.nlg, lgrp = blockIdx.z % p.nlg;
@@ -165,19 +169,23 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
 
   const int nblk = t1 > t0 ? (t1 - t0 + kBlk - 1) / kBlk : 0;
   if constexpr (GATHER) __syncthreads();  // sIdx is visible to every thread
-  for (int j = 0; j < kStages - 1; ++j) {  // blocks 0 .. kStages-2 in flight (one group each)
+  for (int j = 0; j < NST - 1; ++j) {  // blocks 0 .. NST-2 in flight (one group each)
     if (j < nblk) load_block(j, t0 + j * kBlk);
     else cp_async_commit();
   }
   __syncthreads();
 
-  uint32_t qa[D / 16][4];
-#pragma unroll
-  for (int ks = 0; ks < D / 16; ++ks) {
+  constexpr int QR = MINB == 2 ? 1 : D / 16;  // Q fragments kept in registers
+  uint32_t qa[QR][4];
+  auto load_qa = [&](int ks, uint32_t (&f)[4]) {
     const int mi = lane >> 3;
     const int row = warp * 16 + (lane & 7) + 8 * (mi & 1);
     const int col = ks * 16 + 8 * (mi >> 1);
-    ldmatrix_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], sQ + row * STR + col);
+    ldmatrix_x4(f[0], f[1], f[2], f[3], sQ + row * STR + col);
+  };
+  if constexpr (MINB == 1) {
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) load_qa(ks, qa[ks]);
   }
 
   float o[D / 8][4];
@@ -186,14 +194,14 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
   for (int bi = 0; bi < nblk; ++bi) {
-    const int stage = bi % kStages;
+    const int stage = bi % NST;
     const int blk0 = t0 + bi * kBlk;
-    {  // block bi + kStages - 1 into the stage block bi - 1 used (released by its trailing sync)
-      const int nb = bi + kStages - 1;
-      if (nb < nblk) load_block(nb % kStages, t0 + nb * kBlk);
+    {  // block bi + NST - 1 into the stage block bi - 1 used (released by its trailing sync)
+      const int nb = bi + NST - 1;
+      if (nb < nblk) load_block(nb % NST, t0 + nb * kBlk);
       else cp_async_commit();
     }
-    cp_async_wait<kStages - 1>();  // block bi has landed
+    cp_async_wait<NST - 1>();  // block bi has landed
     __syncthreads();
     const __nv_bfloat16* tk = sK + stage * kBlk * STR;
     const __nv_bfloat16* tv = sV + stage * kBlk * STR;
@@ -204,6 +212,9 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
     for (int i = 0; i < kBlk / 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t qf[4];
+      if constexpr (MINB == 2) load_qa(ks, qf);
+      const uint32_t(&qk)[4] = MINB == 2 ? qf : qa[MINB == 2 ? 0 : ks];
 #pragma unroll
       for (int nt2 = 0; nt2 < kBlk / 16; ++nt2) {
         const int mi = lane >> 3;
@@ -211,8 +222,8 @@ __global__ void __launch_bounds__(256) attn_bf16_kernel(const AttnParams p) {
         const int col = ks * 16 + 8 * (mi & 1);
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4(r0, r1, r2, r3, tk + tok * STR + col);
-        mma_bf16_16816(s[2 * nt2], qa[ks], r0, r1);
-        mma_bf16_16816(s[2 * nt2 + 1], qa[ks], r2, r3);
+        mma_bf16_16816(s[2 * nt2], qk, r0, r1);
+        mma_bf16_16816(s[2 * nt2 + 1], qk, r2, r3);
       }
     }
     // scale, mask, row max
@@ -534,12 +545,19 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
   cudaError_t e = cudaSuccess;
   if (sh.dt == CLSA_BF16) {
     const int NW = (pl.rows + 15) / 16;
-    auto smem = [&](int D) { return (NW * 16 + 2 * kStages * kBlk) * (D + 8) * 2 + pl.chunk * 4; };
-#define CLSA_ATTN_BF16(D, GA)                                                  \
-  do {                                                                         \
-    auto kern = attn_bf16_kernel<D, GA>;                                       \
-    e = set_smem(kern, smem(D));                                               \
-    if (e == cudaSuccess) kern<<<grid, NW * 32, smem(D), s>>>(p);              \
+    const bool two = NW <= 6;  // two CTAs per SM fit
+    auto smem = [&](int D, int nst) { return (NW * 16 + 2 * nst * kBlk) * (D + 8) * 2 + pl.chunk * 4; };
+#define CLSA_ATTN_BF16(D, GA)                                                           \
+  do {                                                                                  \
+    if (two) {                                                                          \
+      auto kern = attn_bf16_kernel<D, GA, 2>;                                           \
+      e = set_smem(kern, smem(D, 2));                                                   \
+      if (e == cudaSuccess) kern<<<grid, NW * 32, smem(D, 2), s>>>(p);                 \
+    } else {                                                                            \
+      auto kern = attn_bf16_kernel<D, GA, 1>;                                           \
+      e = set_smem(kern, smem(D, kStages));                                             \
+      if (e == cudaSuccess) kern<<<grid, NW * 32, smem(D, kStages), s>>>(p);           \
+    }                                                                                   \
   } while (0)
     if (sh.d == 128) {
       if (sh.gather) CLSA_ATTN_BF16(128, true);
