@@ -50,7 +50,7 @@ constexpr int kBins = 4096;          // digit histograms of the selection
 constexpr int kTauBits = 12;          // key bits of the candidate-bound histogram
 constexpr int kTauBins = 1 << kTauBits;
 constexpr int kScanU = 4;             // rows per lane group per scan stage
-constexpr int kScanS = 3;             // scan stages in flight (ring after the histogram in `big`)
+constexpr int kScanS = 4;             // scan stages in flight (the whole of `big`)
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
 constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
@@ -143,7 +143,8 @@ struct Smem {
 constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
 constexpr size_t kSmemBig = 128 * 1024;
 constexpr size_t smem_bytes() { return align_up(sizeof(Smem), 128) + kSmemQ + kSmemBig; }
-static_assert(kTauBins * 4 + kScanS * kScanU * kThreads * 16 <= (int)kSmemBig, "scan histogram + ring exceed big");
+static_assert(kScanS * kScanU * kThreads * 16 <= (int)kSmemBig, "scan ring exceeds big");
+static_assert(kTauBins <= kBins, "the slice histogram lives in Smem::hist");
 
 // ---------------------------------------------------------------------------
 // small block-wide helpers (512 threads)
@@ -414,7 +415,7 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
 }
 
 template <int DIDX>
-__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool hist) {
+__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigned char* ring, bool hist) {
   const Plan& pl = sm.plan;
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
@@ -431,7 +432,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, bool hi
   }
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
-  scan_rows<DIDX>(p, sm, th, reinterpret_cast<uint4*>(th + kTauBins), src, sc, q, 0, nrows, nrows, hist);
+  scan_rows<DIDX>(p, sm, th, reinterpret_cast<uint4*>(ring), src, sc, q, 0, nrows, nrows, hist);
   if (nrows <= kMaxUnitTok) {
     __syncthreads();
 #pragma unroll 1
@@ -1133,7 +1134,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQ, MT * 16);  // lands during the scan
 
   const bool all_sel = pl.keff == pl.len;
-  if (!scan_slice<DIDX>(p, sm, reinterpret_cast<uint32_t*>(big), !all_sel)) return;
+  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel)) return;
   stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
@@ -1142,7 +1143,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     for (int i = threadIdx.x; i < pl.tok1 - pl.tok0; i += kThreads) sm.unit_tok[i] = pl.tok0 + i;
     __syncthreads();
   } else {
-    write_candidates(p, sm, reinterpret_cast<uint32_t*>(big));
+    write_candidates(p, sm, sm.hist);
     stamp(p, 2);
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
