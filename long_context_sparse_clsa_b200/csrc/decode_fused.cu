@@ -663,31 +663,36 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
   select_bin_wide(sm, sm.hist, 2048, keff);
   const int T = sm.sel_bin;
   if (T < 0) return false;                  // fewer than k_eff keys >= E_max: not exact
-  const uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
-  // stage B: 2048 sub-bins of bin T
+  uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
   const uint32_t loT = emax + ((uint32_t)T << shift);
   const uint32_t hiT = T == 2047 ? kmax : loT + (1u << shift) - 1u;  // bin T = [loT, hiT]
-  const int shift2 = max(0, shift - 11);
-  uint32_t* hist2 = sm.hist + 2048;
+  uint32_t lo2 = loT, hi2 = hiT;  // the keys ranked exactly: bin T, or its stage-B sub-bin
+  uint32_t m = sm.hist[T];
+  if (m > 64u) {
+    // stage B (a crowded bin only): 2048 sub-bins of bin T
+    const int shift2 = max(0, shift - 11);
+    uint32_t* hist2 = sm.hist + 2048;
 #pragma unroll 1
-  for (int i = threadIdx.x; i < P; i += kThreads) {
-    const uint32_t k = skey[i];
-    if (k >= loT && k <= hiT && k != 0u) atomicAdd(&hist2[(k - loT) >> shift2], 1u);
+    for (int i = threadIdx.x; i < P; i += kThreads) {
+      const uint32_t k = skey[i];
+      if (k >= loT && k <= hiT && k != 0u) atomicAdd(&hist2[(k - loT) >> shift2], 1u);
+    }
+    __syncthreads();
+    select_bin_wide(sm, hist2, 2048, need);
+    const int T2 = sm.sel_bin;
+    need -= sm.sel_above;  // rank inside sub-bin T2
+    m = hist2[T2];
+    lo2 = loT + ((uint32_t)T2 << shift2);
+    hi2 = min(hiT, lo2 + (1u << shift2) - 1u);
   }
-  __syncthreads();
-  stamp(p, 20);
-  select_bin_wide(sm, hist2, 2048, need);
-  const int T2 = sm.sel_bin;
-  const uint32_t need2 = need - sm.sel_above;  // rank inside sub-bin T2
-  const uint32_t m = hist2[T2];
   if (m > 1024u) return false;  // heavy ties: the digit-by-digit path
+  stamp(p, 20);
   stamp(p, 21);
-  // the keys of sub-bin T2 (few) with their list positions
-  const uint32_t lo2 = loT + ((uint32_t)T2 << shift2), hi2 = lo2 + (1u << shift2) - 1u;
+  // the keys of that bin (few) with their list positions
 #pragma unroll 1
   for (int i = threadIdx.x; i < P; i += kThreads) {
     const uint32_t k = skey[i];
-    if (k >= lo2 && k <= hi2 && k <= hiT && k != 0u) {
+    if (k >= lo2 && k <= hi2 && k != 0u) {
       const int q = atomicAdd(&sm.list_n, 1);
       sm.list_key[q] = k;
       sm.list_pos[q] = i;
@@ -703,7 +708,7 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
       const uint32_t kf = sm.list_key[f];
       r += kf > ke || (kf == ke && sm.list_pos[f] < pe);
     }
-    if (r == need2 - 1) {
+    if (r == need - 1) {
       sm.theta_key = ke;
       sm.theta_pos = (uint32_t)pe;
     }
