@@ -416,7 +416,7 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
 
 template <int DIDX>
 __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigned char* ring, bool hist) {
-  const Plan& pl = sm.plan;
+  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
   float* sc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
@@ -450,7 +450,7 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigne
 // phase 2: candidate bound tau from the group histogram, candidate segment
 // ---------------------------------------------------------------------------
 __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
-  const Plan& pl = sm.plan;
+  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
   // The local bound E: the lower edge of the lowest 12-bit key bin such that the slice
   // holds at most win tokens at or above it (E = 0: every token).  Thread t sums the
@@ -611,7 +611,7 @@ __device__ void resolve_theta(Smem& sm, const CandSrc& src, int P, uint32_t keff
 
 // rank the selected positions in order; keep the unit's tokens, write this CTA's share of idx
 __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& src, int P) {
-  const Plan& pl = sm.plan;
+  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const uint32_t theta = sm.theta, ties = sm.ties_needed;
   int32_t* out = p.idx + (size_t)pl.b * p.k;
   uint32_t eq_seen = 0, sel_seen = 0;
@@ -723,7 +723,7 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
 // one block scan visits only the selected ones.
 __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, const int32_t* stok,
                                    int P) {
-  const Plan& pl = sm.plan;
+  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const uint32_t tk = sm.theta_key, tp = sm.theta_pos;
   int run = (P + kThreads - 1) / kThreads;
   run += (run & 1) ^ 1;
