@@ -776,6 +776,7 @@ __device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, 
 __device__ __forceinline__ void load_kv_block(const FusedParams& p, const Smem& sm, int b, int g, int blk0, int ntok,
                                               __nv_bfloat16* dk, __nv_bfloat16* dv) {
   constexpr int VPR = kD * 2 / 16;
+  const int len = sm.plan.len;  // read once: the copies below clobber memory
 #pragma unroll 1
   for (int v = threadIdx.x; v < kTokBlk * VPR; v += kThreads) {
     const int r = v / VPR, c = v % VPR;
@@ -785,7 +786,7 @@ __device__ __forceinline__ void load_kv_block(const FusedParams& p, const Smem& 
     int bytes = 0;
     if (i < ntok) {
       const int t = sm.unit_tok[i];
-      if ((unsigned)t < (unsigned)sm.plan.len) {
+      if ((unsigned)t < (unsigned)len) {
         const size_t off = (((size_t)b * p.n_max + t) * p.Hkv + g) * kD + c * 8;
         sk += off;
         sv += off;
@@ -1006,7 +1007,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
 // each row M = max m and den = sum 2^(m - M) l; then one warp per row sums its splits
 // in split order (the same order every call: the result is deterministic).
 // ---------------------------------------------------------------------------
-__device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan& pl, int g) {
+__device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan pl, int g) {
   stamp(p, 18);
   const int ns = pl.nsplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
