@@ -92,18 +92,18 @@ __device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Count-up barrier among `n` co-resident CTAs: state[0] counts arrivals (a
-// fire-and-forget release add), every CTA polls it until it reaches n, then
-// counts itself in state[1]; the last CTA to pass returns both words to zero, off
-// the critical path, so the state is clean for the next use.  Bounded wait:
-// false (and CLSA_ERR_TIMEOUT with `site`) if it runs out.
+// Count-up barrier among `n` co-resident CTAs: `state` counts arrivals (a
+// fire-and-forget release add after the CTA's bar.sync, which orders every thread's
+// earlier writes before it) and every CTA polls it until it reaches n: one L2 round
+// trip after the last arrival.  The word is used once per launch; the caller returns it
+// to zero once no CTA polls it any more.  Bounded wait: false (and CLSA_ERR_TIMEOUT
+// with `site`) if it runs out.
 __device__ __forceinline__ bool count_barrier(uint32_t* state, uint32_t n, void* ws, int site) {
   __shared__ int s_ok2;
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
     if (n > 1) {
-      __threadfence();
       red_add_release_gpu(state, 1u);
       if (ld_acquire_gpu(state) < n) {
         const unsigned long long t0 = globaltimer_ns();
@@ -114,10 +114,6 @@ __device__ __forceinline__ bool count_barrier(uint32_t* state, uint32_t n, void*
             break;
           }
         }
-      }
-      if (ok && atomicAdd(state + 1, 1u) == n - 1) {  // everyone has seen n: reset
-        state[0] = 0u;
-        state[1] = 0u;
       }
     }
     s_ok2 = ok;

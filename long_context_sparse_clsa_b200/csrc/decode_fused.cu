@@ -82,6 +82,7 @@ struct FusedParams {
   float* lse;
   float* scores;       // [B][n_max]
   uint32_t* row_ws;    // [B][kRowWords]
+  uint32_t* leave;     // CTAs of this launch past their last count barrier
   uint32_t* cand_key;  // [B][kCandCap]  candidate keys, the group's windows back to back (0 = empty slot)
   int32_t* cand_tok;   // [B][kCandCap]
   float* Op;           // [gridDim][rows][D]  split partials, one slot per CTA
@@ -342,6 +343,26 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
 __device__ __forceinline__ void abort_cta(Smem& sm, const FusedParams& p, int site) {
   record_error(p.ws_header, CLSA_ERR_TIMEOUT, site);
   sm.abort_flag = 1;
+}
+
+// The count-barrier words are zeroed by the last CTA to leave them: every CTA counts
+// itself in p.leave right after its last count barrier (leave_issue) and reads the
+// old count only at its end (leave_finish), so no barrier waits on that atomic.  The
+// CTA that saw gridDim.x - 1 runs after every CTA has stopped polling, and the next
+// launch starts from zeroed words.
+__device__ __forceinline__ uint32_t leave_issue(const FusedParams& p) {
+  return threadIdx.x == 0 ? atomicAdd(p.leave, 1u) : 0u;
+}
+__device__ __forceinline__ void leave_finish(const FusedParams& p, uint32_t old) {
+  if (threadIdx.x != 0 || old != gridDim.x - 1) return;
+#pragma unroll 1
+  for (int b = 0; b < p.B; ++b) {
+    uint32_t* rw = p.row_ws + (size_t)b * kRowWords;
+    rw[kRowBar] = 0u;
+#pragma unroll 1
+    for (int g = 0; g < p.Hkv; ++g) rw[kRowHeadBar + 2 * g] = 0u;
+  }
+  *p.leave = 0u;
 }
 
 template <int DIDX>
@@ -970,6 +991,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, u
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    stamp(p, 13);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int r = mt * 16 + gid + 8 * half;
@@ -1129,7 +1151,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
           p.lse[((size_t)(i / p.Hq) * p.B + b) * p.Hq + i % p.Hq] = -INFINITY;
     }
   }
-  if (pl.b < 0) return;
+  if (pl.b < 0) {
+    leave_finish(p, leave_issue(p));
+    return;
+  }
+  const bool head_bar = pl.nsplit > 1 && pl.nunits_here > 0;  // the split combine waits on the head's splits
+  uint32_t left = 0;
   const int MT = (p.rows + 15) / 16;
   if (pl.c == 0) {
     for (int i = pl.keff + threadIdx.x; i < p.k; i += kThreads) p.idx[(size_t)pl.b * p.k + i] = -1;
@@ -1144,6 +1171,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
+    if (!head_bar) left = leave_issue(p);
     int32_t* out = p.idx + (size_t)pl.b * p.k;
     for (int j = pl.r0 + threadIdx.x; j < pl.r1; j += kThreads) out[j] = j;
     for (int i = threadIdx.x; i < pl.tok1 - pl.tok0; i += kThreads) sm.unit_tok[i] = pl.tok0 + i;
@@ -1153,6 +1181,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     stamp(p, 2);
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
+    if (!head_bar) left = leave_issue(p);
     stamp(p, 3);
     // the group's windows (back to back, token order, empty slots key 0) to shared
     // memory in 16-byte copies, all in flight while the group totals are reduced
@@ -1223,12 +1252,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     else attend_unit<4>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
   }
   stamp(p, 7);
-  if (pl.nsplit > 1 && pl.nunits_here > 0) {
+  if (head_bar) {
     uint32_t* hb = p.row_ws + (size_t)pl.b * kRowWords + kRowHeadBar + 2 * pl.unit_g0;
     if (!count_barrier(hb, pl.nsplit, p.ws_header, 2)) return;
+    left = leave_issue(p);
     stamp(p, 8);
     combine_head(p, sm, big, pl, pl.unit_g0);
   }
+  leave_finish(p, left);
   stamp(p, 9);
 }
 
@@ -1272,7 +1303,7 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   size_t off = 0;
   off += (size_t)kMaxGroups * kTraceSlots * 8;                  // phase stamps (CLSA_TRACE=1)
   off += align_up((size_t)a->B * a->n_max * 4, 256);           // scores (when not an output)
-  off += align_up((size_t)a->B * kRowWords * 4, 256);          // row state
+  off += align_up(((size_t)a->B * kRowWords + 1) * 4, 256);    // row state, leave count
   off += 2 * align_up((size_t)a->B * kCandCap * 4, 256);  // candidate windows
   off += align_up((size_t)cfg.ncta * rows * kD * 4, 256);      // split partials
   off += align_up((size_t)cfg.ncta * rows * 2 * 4, 256);
@@ -1312,7 +1343,8 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   w += align_up((size_t)a->B * a->n_max * 4, 256);
   p.scores = a->scores ? a->scores : ws_scores;
   p.row_ws = reinterpret_cast<uint32_t*>(w);
-  w += align_up((size_t)a->B * kRowWords * 4, 256);
+  p.leave = p.row_ws + (size_t)a->B * kRowWords;
+  w += align_up(((size_t)a->B * kRowWords + 1) * 4, 256);
   p.cand_key = reinterpret_cast<uint32_t*>(w);
   w += align_up((size_t)a->B * kCandCap * 4, 256);
   p.cand_tok = reinterpret_cast<int32_t*>(w);
