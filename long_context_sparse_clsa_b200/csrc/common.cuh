@@ -281,6 +281,23 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
   if (ok) ok = mbar_test_wait(bar, parity) ? 1u : 0u;  // completed: true at once, with ordering
   return __all_sync(0xffffffffu, ok != 0);
 }
+// As mbar_wait_warp, but lane 0 spins on test_wait (never suspends): for short waits
+// (an MMA of a few hundred cycles) where a suspended poller would wake late.
+__device__ __forceinline__ bool mbar_spin_warp(uint64_t* bar, uint32_t parity) {
+  uint32_t ok = 1;
+  if ((threadIdx.x & 31) == 0 && !mbar_test_wait(bar, parity)) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_test_wait(bar, parity)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        ok = 0;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) ok = mbar_test_wait(bar, parity) ? 1u : 0u;
+  return __all_sync(0xffffffffu, ok != 0);
+}
 // bulk prefetch of [src, src + bytes) into L2 (src 16-byte aligned, bytes % 16 == 0)
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");

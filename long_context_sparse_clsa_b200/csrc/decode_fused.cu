@@ -28,9 +28,9 @@
 //     CTA writes its share of idx and keeps the tokens of its attention unit.
 //  4. Attention.  A unit is (KV head g, split s of the selected ranks); its rows
 //     are all L*G (layer, query head) pairs of head g, so every selected K/V row is
-//     read once for all layers.  mma.sync m16n8k16 bf16 -> fp32, online softmax in
-//     exp2, two warp sets per 16-row tile over alternating 64-token blocks,
-//     merged in shared memory.
+//     read once for all layers.  tcgen05.mma bf16 -> fp32 in TMEM over 64-token
+//     chunks (S = Q K^T, then P V with V as an MN-major operand), online softmax in
+//     exp2 with the output accumulated in registers.
 //  5. Splits of one head meet at a barrier and merge with the log-sum-exp rule.
 //
 // Every wait is bounded (kWaitLimitNs); running out records CLSA_ERR_TIMEOUT.
@@ -39,6 +39,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace clsa {
 
@@ -54,7 +55,6 @@ constexpr int kScanS = 4;             // scan stages in flight (the whole of `bi
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
 constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
-constexpr int kTokBlk = 64;           // tokens per attention block
 constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096); also slice scores kept on chip
 constexpr int kCandCap = 16384;       // candidate slots kept in shared memory (key + index)
 constexpr int kMaxGroups = 256;       // CTAs per launch
@@ -114,6 +114,8 @@ struct Plan {
 
 struct Smem {
   Plan plan;
+  uint64_t bar_s, bar_o;  // attention: S and O_c MMAs complete
+  uint32_t tmem_base;
   int abort_flag;
   uint32_t tau_key;
   int all_selected;
@@ -338,11 +340,6 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
   const int per = (pl.keff + pl.nsplit - 1) / pl.nsplit;
   pl.tok0 = min(pl.keff, pl.split * per);
   pl.tok1 = min(pl.keff, pl.tok0 + per);
-}
-
-__device__ __forceinline__ void abort_cta(Smem& sm, const FusedParams& p, int site) {
-  record_error(p.ws_header, CLSA_ERR_TIMEOUT, site);
-  sm.abort_flag = 1;
 }
 
 // The count-barrier words are zeroed by the last CTA to leave them: every CTA counts
@@ -776,14 +773,45 @@ __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_
 }
 
 // ---------------------------------------------------------------------------
-// phase 4: attention of one unit (head g, tokens sm.unit_tok[0..ntok))
+// phase 4: attention of one unit (head g, tokens sm.unit_tok[0..ntok)), on the 5th
+// generation tensor cores.  The unit's M = 128 rows (the L*G (layer, query head) rows of
+// head g, zero above p.rows) stay in shared memory as the A operand; the tokens go in
+// chunks of 64:
+//   S = Q K_c^T        tcgen05.mma M128 N64 (K = d, 8 steps) -> TMEM columns [0, 64)
+//   softmax            every warp: one row (its TMEM lane), 16 of the 64 columns; the
+//                      chunk's row max is exchanged through shared memory, so the four
+//                      warps of a row share one running max m
+//   O_c = P_c V_c      P_c (bf16) in shared memory (A, K-major), V_c as the MN-major B
+//                      operand straight from its row-major [token][d] tile;
+//                      M128 N128 (K = 64 tokens, 4 steps) -> TMEM columns [128, 256)
+//   o = o 2^(m_old - m) + O_c   in registers, 32 of the d columns per thread
+// K/V chunks are gathered by 16-byte async copies into the 128-byte-swizzle layout, two
+// chunks ahead in a 3-stage ring.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, __nv_bfloat16* sQ, int mt_rows) {
-  constexpr int VPR = kD * 2 / 16;
+constexpr int kAttnTok = 64;                         // tokens per chunk
+constexpr int kAttnStages = 3;                       // K/V chunk ring
+constexpr uint32_t kKVAtom = kAttnTok * 128;         // 64 rows x 128 bytes: 8 KiB
+constexpr uint32_t kKVTile = 2 * kKVAtom;            // K or V chunk, both 64-column atoms
+constexpr uint32_t kQAtom = kMaxRows * 128;          // 16 KiB
+constexpr uint32_t kPTile = kMaxRows * 128;          // P chunk: 128 rows x 64 tokens bf16
+constexpr uint32_t kTmemCols = 256;                  // S at [0, 64), O_c at [128, 256)
+constexpr int kOPitch = kD + 4;                      // staged partial row, floats
+constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(kMaxRows, kAttnTok);
+constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kMaxRows, kD) | (1u << 16);  // B (V) MN-major
+static_assert(kAttnStages * 2 * kKVTile + kPTile + 1024 <= kSmemBig, "attention tiles exceed big");
+static_assert(2 * kQAtom + 1024 <= kSmemQ, "Q tile exceeds its region");
+static_assert(kMaxRows * kOPitch * 4 + 1024 <= kSmemBig, "partial staging exceeds big");
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* q) {
+  return q + ((1024u - (smem_u32(q) & 1023u)) & 1023u);
+}
+
+// Q rows of head g in the 128-byte-swizzle K-major layout (two 64-column atoms)
+__device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, unsigned char* sQa) {
 #pragma unroll 1
-  for (int v = threadIdx.x; v < mt_rows * VPR; v += kThreads) {
-    const int r = v / VPR, c = v % VPR;
-    __nv_bfloat16* dst = sQ + r * kSTR + c * 8;
+  for (int v = threadIdx.x; v < kMaxRows * 16; v += kThreads) {
+    const int r = v >> 4, c = v & 15;
+    unsigned char* dst = sQa + (c >> 3) * kQAtom + tc::sw128_offset(r, c & 7);
     if (r < p.rows) {
       const int l = r / p.G, h = g * p.G + r % p.G;
       cp_async_16(dst, p.Q + (((size_t)l * p.B + b) * p.Hq + h) * kD + c * 8, 16);
@@ -794,232 +822,195 @@ __device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, 
   cp_async_commit();
 }
 
-__device__ __forceinline__ void load_kv_block(const FusedParams& p, const Smem& sm, int b, int g, int blk0, int ntok,
-                                              __nv_bfloat16* dk, __nv_bfloat16* dv) {
-  constexpr int VPR = kD * 2 / 16;
-  const int len = sm.plan.len;  // read once: the copies below clobber memory
+// K and V rows of tokens [64 c, 64 c + 64) of the unit, same layout (rows past ntok: zero)
+__device__ __forceinline__ void load_kv_chunk(const FusedParams& p, const Smem& sm, int b, int g, int len, int c,
+                                              int ntok, unsigned char* dk, unsigned char* dv) {
 #pragma unroll 1
-  for (int v = threadIdx.x; v < kTokBlk * VPR; v += kThreads) {
-    const int r = v / VPR, c = v % VPR;
-    const int i = blk0 + r;
+  for (int v = threadIdx.x; v < kAttnTok * 16; v += kThreads) {
+    const int r = v >> 4, j = v & 15;
+    const int i = c * kAttnTok + r;
     const __nv_bfloat16* sk = p.K;
     const __nv_bfloat16* sv = p.V;
     int bytes = 0;
     if (i < ntok) {
       const int t = sm.unit_tok[i];
       if ((unsigned)t < (unsigned)len) {
-        const size_t off = (((size_t)b * p.n_max + t) * p.Hkv + g) * kD + c * 8;
+        const size_t off = (((size_t)b * p.n_max + t) * p.Hkv + g) * kD + j * 8;
         sk += off;
         sv += off;
         bytes = 16;
-      } else if (c == 0) {
+      } else if (j == 0) {
         record_error(p.ws_header, CLSA_ERR_BAD_INDEX, ((long long)b << 32) | (unsigned)i);
       }
     }
-    cp_async_16(dk + r * kSTR + c * 8, sk, bytes);
-    cp_async_16(dv + r * kSTR + c * 8, sv, bytes);
+    const uint32_t o = (uint32_t)(j >> 3) * kKVAtom + tc::sw128_offset(r, j & 7);
+    cp_async_16(dk + o, sk, bytes);
+    cp_async_16(dv + o, sv, bytes);
   }
-  cp_async_commit();
 }
 
-// NT = n-tiles (8 tokens each) one warp set handles per 64-token block; NS = 64 / (8 NT) sets
-template <int NT>
-__device__ void attend_unit(const FusedParams& p, Smem& sm, __nv_bfloat16* sQ, unsigned char* big, int g,
-                            int ntok, bool q_loaded, int unit_split) {
-  constexpr int NS = kTokBlk / (8 * NT);
-  const Plan& pl = sm.plan;
+// `it` counts the chunks this CTA has run (the phase of both MMA barriers)
+__device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, unsigned char* kv, int g, int ntok,
+                            bool q_loaded, uint32_t tmem, uint32_t& it) {
+  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const int b = pl.b;
-  const int MT = (p.rows + 15) / 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const bool active = warp < MT * NS;
-  const int mt = warp % MT, set = warp / MT;
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(big);  // [2][kTokBlk][kSTR]
-  __nv_bfloat16* sV = sK + 2 * kTokBlk * kSTR;
-  if (!q_loaded) load_q_tile(p, b, g, sQ, MT * 16);
-  const int nblk = (ntok + kTokBlk - 1) / kTokBlk;
-  if (nblk > 0) {
-    load_kv_block(p, sm, b, g, 0, ntok, sK, sV);
-    cp_async_wait<1>();  // the Q tile (older group) has landed
-  } else {
-    cp_async_wait<0>();
+  const int q4 = warp & 3, cg = warp >> 2;  // TMEM lane quarter; column group
+  const int row = q4 * 32 + lane;
+  unsigned char* sP = kv + kAttnStages * 2 * kKVTile;
+  if (!q_loaded) load_q_tile(p, b, g, sQa);
+  const int nch = (ntok + kAttnTok - 1) / kAttnTok;
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    if (c < nch) load_kv_chunk(p, sm, b, g, pl.len, c, ntok, kv + c * 2 * kKVTile, kv + c * 2 * kKVTile + kKVTile);
+    cp_async_commit();
   }
-  __syncthreads();
-
-  // Q fragments are re-read from shared memory per k-step (keeps the register budget of 512 threads)
-  const __nv_bfloat16* qrow = sQ + (mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * kSTR + 8 * (lane >> 4);
-  float o[kD / 8][4];
+  const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+  float o[32];
 #pragma unroll
-  for (int i = 0; i < kD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  for (int j = 0; j < 32; ++j) o[j] = 0.f;
+  float m = -INFINITY, lp = 0.f;
+  bool dead = false;
 
-  for (int bi = 0; bi < nblk; ++bi) {
-    const int stage = bi & 1;
-    const int blk0 = bi * kTokBlk;
-    if (bi + 1 < nblk) {
-      load_kv_block(p, sm, b, g, blk0 + kTokBlk, ntok, sK + (stage ^ 1) * kTokBlk * kSTR,
-                    sV + (stage ^ 1) * kTokBlk * kSTR);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+#pragma unroll 1
+  for (int c = 0; c < nch; ++c) {
+    const int st = c % kAttnStages;
+    unsigned char* sK = kv + st * 2 * kKVTile;
+    unsigned char* sV = sK + kKVTile;
+    cp_async_wait<1>();  // chunk c (and the Q tile) landed; chunk c + 1 may be in flight
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
     __syncthreads();
-    if (bi == 0) stamp(p, 10);
-    if (active) {
-      const __nv_bfloat16* tk = sK + stage * kTokBlk * kSTR + set * NT * 8 * kSTR;
-      const __nv_bfloat16* tv = sV + stage * kTokBlk * kSTR + set * NT * 8 * kSTR;
-      const int tbase = blk0 + set * NT * 8;
-      float s[NT][4];
+    if (c == 0) stamp(p, 10);
+    if (threadIdx.x == 0) {
+      tc::fence_after_sync();
 #pragma unroll
-      for (int i = 0; i < NT; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < kD / 16; ++ks) {
-        uint32_t qa[4];
-        ldmatrix_x4(qa[0], qa[1], qa[2], qa[3], qrow + ks * 16);
-#pragma unroll
-        for (int nt2 = 0; nt2 < NT / 2; ++nt2) {
-          const int mi = lane >> 3;
-          const int tok = nt2 * 16 + 8 * (mi >> 1) + (lane & 7);
-          const int col = ks * 16 + 8 * (mi & 1);
-          uint32_t r0, r1, r2, r3;
-          ldmatrix_x4(r0, r1, r2, r3, tk + tok * kSTR + col);
-          mma_bf16_16816(s[2 * nt2], qa, r0, r1);
-          mma_bf16_16816(s[2 * nt2 + 1], qa, r2, r3);
-        }
-      }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int tok = tbase + nt * 8 + 2 * tig + (e & 1);
-          s[nt][e] = tok < ntok ? s[nt][e] * p.scale_log2 : -INFINITY;
-        }
-        mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
-        mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
-      }
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
-      const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float c0 = exp2f(m0 - ref0), c1 = exp2f(m1 - ref1);
-      m0 = mn0;
-      m1 = mn1;
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        s[nt][0] = exp2f(s[nt][0] - ref0);
-        s[nt][1] = exp2f(s[nt][1] - ref0);
-        s[nt][2] = exp2f(s[nt][2] - ref1);
-        s[nt][3] = exp2f(s[nt][3] - ref1);
-        rs0 += s[nt][0] + s[nt][1];
-        rs1 += s[nt][2] + s[nt][3];
-      }
-      l0 = l0 * c0 + rs0;
-      l1 = l1 * c1 + rs1;
-#pragma unroll
-      for (int nd = 0; nd < kD / 8; ++nd) {
-        o[nd][0] *= c0;
-        o[nd][1] *= c0;
-        o[nd][2] *= c1;
-        o[nd][3] *= c1;
-      }
-#pragma unroll
-      for (int kk = 0; kk < NT / 2; ++kk) {
-        uint32_t pa[4];
-        pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-        pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-        pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-        for (int nd2 = 0; nd2 < kD / 16; ++nd2) {
-          const int mi = lane >> 3;
-          const int tok = kk * 16 + 8 * (mi & 1) + (lane & 7);
-          const int col = nd2 * 16 + 8 * (mi >> 1);
-          uint32_t r0, r1, r2, r3;
-          ldmatrix_x4_trans(r0, r1, r2, r3, tv + tok * kSTR + col);
-          mma_bf16_16816(o[2 * nd2], pa, r0, r1);
-          mma_bf16_16816(o[2 * nd2 + 1], pa, r2, r3);
-        }
-      }
+      for (int ks = 0; ks < kD / 16; ++ks)
+        tc::mma_bf16(tmem, tc::sw128_desc(smem_u32(sQa) + (ks >> 2) * kQAtom + (ks & 3) * 32),
+                     tc::sw128_desc(smem_u32(sK) + (ks >> 2) * kKVAtom + (ks & 3) * 32), kIdescQK, ks > 0);
+      tc::mma_commit(&sm.bar_s);
     }
-    __syncthreads();
-  }
+    // chunk c + 2 into the stage of chunk c - 1, whose MMAs have completed
+    if (c + 2 < nch) {
+      unsigned char* nk = kv + ((c + 2) % kAttnStages) * 2 * kKVTile;
+      load_kv_chunk(p, sm, b, g, pl.len, c + 2, ntok, nk, nk + kKVTile);
+    }
+    cp_async_commit();
 
-  stamp(p, 11);
-  // ---- merge the NS token sets of each m-tile (thread-private slots in shared memory)
-  float* xo = reinterpret_cast<float*>(big);                  // [NS-1][MT][64][32]
-  float* xm = xo + (size_t)(NS - 1) * MT * 64 * 32;           // [NS-1][MT][4][32]
-  if (active && set > 0) {
-    float* d = xo + ((size_t)(set - 1) * MT + mt) * 64 * 32;
-#pragma unroll
-    for (int nd = 0; nd < kD / 8; ++nd)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) d[(nd * 4 + e) * 32 + lane] = o[nd][e];
-    float* dm = xm + ((size_t)(set - 1) * MT + mt) * 4 * 32;
-    dm[0 * 32 + lane] = m0;
-    dm[1 * 32 + lane] = m1;
-    dm[2 * 32 + lane] = l0;
-    dm[3 * 32 + lane] = l1;
-  }
-  __syncthreads();
-  if (active && set == 0) {
-    for (int s2 = 1; s2 < NS; ++s2) {
-      const float* d = xo + ((size_t)(s2 - 1) * MT + mt) * 64 * 32;
-      const float* dm = xm + ((size_t)(s2 - 1) * MT + mt) * 4 * 32;
-      const float om0 = dm[lane], om1 = dm[32 + lane], ol0 = dm[64 + lane], ol1 = dm[96 + lane];
-      const float nm0 = fmaxf(m0, om0), nm1 = fmaxf(m1, om1);
-      const float r0 = nm0 == -INFINITY ? 0.f : nm0, r1 = nm1 == -INFINITY ? 0.f : nm1;
-      const float a0 = exp2f(m0 - r0), b0 = exp2f(om0 - r0);
-      const float a1 = exp2f(m1 - r1), b1 = exp2f(om1 - r1);
-#pragma unroll
-      for (int nd = 0; nd < kD / 8; ++nd) {
-        o[nd][0] = o[nd][0] * a0 + d[(nd * 4 + 0) * 32 + lane] * b0;
-        o[nd][1] = o[nd][1] * a0 + d[(nd * 4 + 1) * 32 + lane] * b0;
-        o[nd][2] = o[nd][2] * a1 + d[(nd * 4 + 2) * 32 + lane] * b1;
-        o[nd][3] = o[nd][3] * a1 + d[(nd * 4 + 3) * 32 + lane] * b1;
-      }
-      l0 = l0 * a0 + ol0 * b0;
-      l1 = l1 * a1 + ol1 * b1;
-      m0 = nm0;
-      m1 = nm1;
+    if (!dead && !mbar_spin_warp(&sm.bar_s, it & 1u)) {
+      if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 30);
+      dead = true;
     }
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    stamp(p, 13);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = mt * 16 + gid + 8 * half;
-      if (r >= p.rows) continue;
-      const int l = r / p.G, h = g * p.G + r % p.G;
-      const float m = half ? m1 : m0;
-      const float ls = half ? l1 : l0;
-      if (pl.nsplit == 1) {
-        const float inv = ls > 0.f ? 1.f / ls : 0.f;
-        __nv_bfloat16* out = p.O + (((size_t)l * p.B + b) * p.Hq + h) * kD;
-#pragma unroll
-        for (int nd = 0; nd < kD / 8; ++nd)
-          *reinterpret_cast<uint32_t*>(out + nd * 8 + 2 * tig) =
-              pack_bf16x2(o[nd][2 * half] * inv, o[nd][2 * half + 1] * inv);
-        if (p.lse && tig == 0)
-          p.lse[((size_t)l * p.B + b) * p.Hq + h] = ls > 0.f ? (m + log2f(ls)) * kLn2 : -INFINITY;
+    if (c == 0) stamp(p, 15);
+    tc::fence_after_sync();
+    float s[16];
+    float cmx = -INFINITY;
+    {
+      uint32_t v[16];
+      if (!dead) {
+        tc::ld_32x32b_x16(tl + (uint32_t)(16 * cg), v);
+        tc::ld_wait();
       } else {
-        const size_t pi = (size_t)blockIdx.x * p.rows + r;  // partial slot of this CTA
-        float* op = p.Op + pi * kD;
 #pragma unroll
-        for (int nd = 0; nd < kD / 8; ++nd)
-          __stcg(reinterpret_cast<float2*>(op + nd * 8 + 2 * tig), make_float2(o[nd][2 * half], o[nd][2 * half + 1]));
-        if (tig == 0) __stcg(reinterpret_cast<float2*>(p.Ml + pi * 2), make_float2(m, ls));
+        for (int j = 0; j < 16; ++j) v[j] = 0u;
+      }
+      const int t0 = c * kAttnTok + 16 * cg;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        s[j] = t0 + j < ntok ? __uint_as_float(v[j]) * p.scale_log2 : -INFINITY;
+        cmx = fmaxf(cmx, s[j]);
       }
     }
+    sm.cm[cg * kMaxRows + row] = cmx;
+    __syncthreads();
+    if (c == 0) stamp(p, 23);
+    const float mn = fmaxf(fmaxf(m, fmaxf(sm.cm[row], sm.cm[kMaxRows + row])),
+                           fmaxf(sm.cm[2 * kMaxRows + row], sm.cm[3 * kMaxRows + row]));
+    const float alpha = exp2f(m - mn);  // m = -inf on the first chunk: 0
+    m = mn;
+    {
+      uint32_t pw[8];
+      float rs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float a = exp2f(s[2 * j] - mn), e = exp2f(s[2 * j + 1] - mn);
+        rs += a + e;
+        pw[j] = pack_bf16x2(a, e);
+      }
+      lp = lp * alpha + rs;
+      *reinterpret_cast<uint4*>(sP + tc::sw128_offset(row, 2 * cg)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      *reinterpret_cast<uint4*>(sP + tc::sw128_offset(row, 2 * cg + 1)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < kAttnTok / 16; ++ks)
+        tc::mma_bf16(tmem + 128u, tc::sw128_desc(smem_u32(sP) + ks * 32),
+                     tc::sw128_desc_mn(smem_u32(sV) + ks * 16 * 128, kKVAtom), kIdescPV, ks > 0);
+      tc::mma_commit(&sm.bar_o);
+    }
+    if (c == 0) stamp(p, 24);
+    if (!dead && !mbar_spin_warp(&sm.bar_o, it & 1u)) {
+      if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 31);
+      dead = true;
+    }
+    if (c == 0) stamp(p, 25);
+    tc::fence_after_sync();
+    if (!dead) {
+      uint32_t v[32];
+      tc::ld_32x32b_x32(tl + 128u + (uint32_t)(32 * cg), v);
+      tc::ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) o[j] = fmaf(o[j], alpha, __uint_as_float(v[j]));
+    }
+    if (c == 0) stamp(p, 26);
+    ++it;
+  }
+  cp_async_wait<0>();  // no copy of this unit outlives it (the trailing groups are empty)
+  stamp(p, 11);
+
+  // row sum over the four column groups, in a fixed order
+  sm.cl[cg * kMaxRows + row] = lp;
+  tc::fence_before_sync();
+  __syncthreads();
+  const float ls = (sm.cl[row] + sm.cl[kMaxRows + row]) + (sm.cl[2 * kMaxRows + row] + sm.cl[3 * kMaxRows + row]);
+  stamp(p, 13);
+  if (row < p.rows) {
+    const int l = row / p.G, h = g * p.G + row % p.G;
+    if (pl.nsplit == 1) {
+      const float inv = ls > 0.f ? 1.f / ls : 0.f;
+      uint4* out = reinterpret_cast<uint4*>(p.O + (((size_t)l * p.B + b) * p.Hq + h) * kD + 32 * cg);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        out[j] = make_uint4(pack_bf16x2(o[8 * j] * inv, o[8 * j + 1] * inv),
+                            pack_bf16x2(o[8 * j + 2] * inv, o[8 * j + 3] * inv),
+                            pack_bf16x2(o[8 * j + 4] * inv, o[8 * j + 5] * inv),
+                            pack_bf16x2(o[8 * j + 6] * inv, o[8 * j + 7] * inv));
+      if (p.lse && cg == 0)
+        p.lse[((size_t)l * p.B + b) * p.Hq + h] = ls > 0.f ? (m + log2f(ls)) * kLn2 : -INFINITY;
+    }
+  }
+  if (pl.nsplit > 1) {
+    // this CTA's partial rows are one contiguous block of p.Op: stage them in shared
+    // memory (row pitch kOPitch floats: conflict-free 16-byte stores down a column),
+    // then write the block with whole-line stores
+    float* stg = reinterpret_cast<float*>(kv);
+    float4* srow = reinterpret_cast<float4*>(stg + row * kOPitch + 32 * cg);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) srow[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+    if (cg == 0 && row < p.rows)
+      __stcg(reinterpret_cast<float2*>(p.Ml + ((size_t)blockIdx.x * p.rows + row) * 2), make_float2(m, ls));
+    __syncthreads();
+    float4* op = reinterpret_cast<float4*>(p.Op + (size_t)blockIdx.x * p.rows * kD);
+#pragma unroll 1
+    for (int i = threadIdx.x; i < p.rows * (kD / 4); i += kThreads)
+      __stcg(op + i, *reinterpret_cast<const float4*>(stg + (i / (kD / 4)) * kOPitch + 4 * (i % (kD / 4))));
   }
   stamp(p, 12);
-  __syncthreads();
+  __syncthreads();  // cm / cl and the tiles are free for the next unit
 }
 
 // ---------------------------------------------------------------------------
@@ -1157,14 +1148,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   }
   const bool head_bar = pl.nsplit > 1 && pl.nunits_here > 0;  // the split combine waits on the head's splits
   uint32_t left = 0;
-  const int MT = (p.rows + 15) / 16;
   if (pl.c == 0) {
     for (int i = pl.keff + threadIdx.x; i < p.k; i += kThreads) p.idx[(size_t)pl.b * p.k + i] = -1;
     if (threadIdx.x == 0) p.count[pl.b] = pl.keff;
   }
   if (pl.c == pl.Cb - 1)  // score tail beyond the sequence
     for (int j = pl.len + threadIdx.x; j < p.n_max; j += kThreads) p.scores[(size_t)pl.b * p.n_max + j] = -INFINITY;
-  if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQ, MT * 16);  // lands during the scan
+  unsigned char* sQa = align1024(reinterpret_cast<unsigned char*>(sQ));
+  if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQa);  // lands during the scan
 
   const bool all_sel = pl.keff == pl.len;
   if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel)) return;
@@ -1243,13 +1234,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   }
   stamp(p, 6);
 
-  // ---- attention units
-  const int ntok = pl.tok1 - pl.tok0;
-  const int NS = min(4, kWarps / MT) >= 4 ? 4 : 2;
-  for (int u = 0; u < pl.nunits_here; ++u) {
-    const int g = pl.unit_g0 + u * pl.unit_step;
-    if (NS == 4) attend_unit<2>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
-    else attend_unit<4>(p, sm, sQ, big, g, ntok, u == 0, pl.split);
+  // ---- attention units (TMEM held only for this phase: no return path in between)
+  if (pl.nunits_here > 0) {
+    const int ntok = pl.tok1 - pl.tok0;
+    if (threadIdx.x < 32) {
+      tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+      tc::tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+      mbar_init(&sm.bar_s, 1);
+      mbar_init(&sm.bar_o, 1);
+      fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_base;
+    unsigned char* kv = align1024(big);
+    uint32_t it = 0;
+    for (int u = 0; u < pl.nunits_here; ++u)
+      attend_unit(p, sm, sQa, kv, pl.unit_g0 + u * pl.unit_step, ntok, u == 0, tmem, it);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tc::tmem_dealloc(tmem, kTmemCols);
   }
   stamp(p, 7);
   if (head_bar) {
@@ -1287,9 +1294,11 @@ FusedCfg fused_cfg() {
 bool fused_decode_supported(const clsa_decode_args* a) {
   if (a->dtype != CLSA_BF16 || a->d != kD || (a->d_idx != 64 && a->d_idx != 128)) return false;
   if (a->K_S != nullptr) return false;
-  // 16-byte copies and L2 bulk prefetches of K_idx, K and V rows
+  // 16-byte copies and L2 bulk prefetches of K_idx, K and V rows; 16-byte Q copies and O stores
   if ((reinterpret_cast<uintptr_t>(a->k_idx) | reinterpret_cast<uintptr_t>(a->K) |
-       reinterpret_cast<uintptr_t>(a->V)) % 16 != 0)
+       reinterpret_cast<uintptr_t>(a->V) | reinterpret_cast<uintptr_t>(a->Q) | reinterpret_cast<uintptr_t>(a->O)) %
+          16 !=
+      0)
     return false;
   if (a->Hkv > 64 || a->L * (a->Hq / a->Hkv) > kMaxRows || a->k > kMaxUnitTok) return false;
   const FusedCfg cfg = fused_cfg();
