@@ -525,8 +525,6 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
       }
     }
   }
-  stamp(p, 14);
-  stamp(p, 16);
   __syncthreads();
   const uint32_t tau = sm.tau_key, pf = sm.pf_key;
   // this CTA's tokens with key >= tau, in token order, to its window of win slots
@@ -776,31 +774,38 @@ __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_
 // phase 4: attention of one unit (head g, tokens sm.unit_tok[0..ntok)), on the 5th
 // generation tensor cores.  The unit's M = 128 rows (the L*G (layer, query head) rows of
 // head g, zero above p.rows) stay in shared memory as the A operand; the tokens go in
-// chunks of 64:
-//   S = Q K_c^T        tcgen05.mma M128 N64 (K = d, 8 steps) -> TMEM columns [0, 64)
-//   softmax            every warp: one row (its TMEM lane), 16 of the 64 columns; the
-//                      chunk's row max is exchanged through shared memory, so the four
+// chunks of TOK (128 when the unit fits one chunk, else 64 in a 3-stage ring):
+//   S = Q K_c^T        tcgen05.mma M128 N=TOK (K = d, 8 steps) -> TMEM
+//   softmax            every warp: one row (its TMEM lane), TOK/4 of the chunk's columns;
+//                      the chunk's row max is exchanged through shared memory, so the four
 //                      warps of a row share one running max m
 //   O_c = P_c V_c      P_c (bf16) in shared memory (A, K-major), V_c as the MN-major B
 //                      operand straight from its row-major [token][d] tile;
-//                      M128 N128 (K = 64 tokens, 4 steps) -> TMEM columns [128, 256)
+//                      M128 N128 (K = TOK tokens) -> TMEM columns [128, 256)
 //   o = o 2^(m_old - m) + O_c   in registers, 32 of the d columns per thread
-// K/V chunks are gathered by 16-byte async copies into the 128-byte-swizzle layout, two
-// chunks ahead in a 3-stage ring.
+// The S MMAs of chunk c + 1 are issued right behind the P V MMAs of chunk c (S is
+// double-buffered in TMEM).  K/V chunks are gathered by 16-byte async copies into the
+// 128-byte-swizzle layout, two chunks ahead.  Each tcgen05.mma costs tens of cycles to
+// issue whatever its N, so the wide chunk halves the instruction count of a short unit.
 // ---------------------------------------------------------------------------
-constexpr int kAttnTok = 64;                         // tokens per chunk
-constexpr int kAttnStages = 3;                       // K/V chunk ring
-constexpr uint32_t kKVAtom = kAttnTok * 128;         // 64 rows x 128 bytes: 8 KiB
-constexpr uint32_t kKVTile = 2 * kKVAtom;            // K or V chunk, both 64-column atoms
 constexpr uint32_t kQAtom = kMaxRows * 128;          // 16 KiB
-constexpr uint32_t kPTile = kMaxRows * 128;          // P chunk: 128 rows x 64 tokens bf16
-constexpr uint32_t kTmemCols = 256;                  // S at [0, 64), O_c at [128, 256)
+constexpr uint32_t kTmemCols = 256;                  // S at [0, 128), O_c at [128, 256)
 constexpr int kOPitch = kD + 4;                      // staged partial row, floats
-constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(kMaxRows, kAttnTok);
 constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kMaxRows, kD) | (1u << 16);  // B (V) MN-major
-static_assert(kAttnStages * 2 * kKVTile + kPTile + 1024 <= kSmemBig, "attention tiles exceed big");
 static_assert(2 * kQAtom + 1024 <= kSmemQ, "Q tile exceeds its region");
 static_assert(kMaxRows * kOPitch * 4 + 1024 <= kSmemBig, "partial staging exceeds big");
+
+template <int TOK>
+struct AttnShape {
+  static constexpr int kStages = TOK == 64 ? 3 : 1;         // the wide chunk runs alone
+  static constexpr uint32_t kKVAtom = TOK * 128;            // TOK rows x 128 bytes
+  static constexpr uint32_t kKVTile = 2 * kKVAtom;          // K or V chunk, both 64-column atoms
+  static constexpr uint32_t kPAtom = kMaxRows * 128;        // 64 tokens of P
+  static constexpr int kPerThread = TOK / 4;                // S columns per thread
+  static constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(kMaxRows, TOK);
+  static_assert(kStages * 2 * kKVTile + (TOK / 64) * kPAtom + 1024 <= kSmemBig, "attention tiles exceed big");
+  static_assert(TOK * (TOK == 64 ? 2 : 1) <= 128, "S buffers overlap O");
+};
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* q) {
   return q + ((1024u - (smem_u32(q) & 1023u)) & 1023u);
@@ -822,13 +827,14 @@ __device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, 
   cp_async_commit();
 }
 
-// K and V rows of tokens [64 c, 64 c + 64) of the unit, same layout (rows past ntok: zero)
+// K and V rows of tokens [TOK c, TOK c + TOK) of the unit, same layout (rows past ntok: zero)
+template <int TOK>
 __device__ __forceinline__ void load_kv_chunk(const FusedParams& p, const Smem& sm, int b, int g, int len, int c,
                                               int ntok, unsigned char* dk, unsigned char* dv) {
 #pragma unroll 1
-  for (int v = threadIdx.x; v < kAttnTok * 16; v += kThreads) {
+  for (int v = threadIdx.x; v < TOK * 16; v += kThreads) {
     const int r = v >> 4, j = v & 15;
-    const int i = c * kAttnTok + r;
+    const int i = c * TOK + r;
     const __nv_bfloat16* sk = p.K;
     const __nv_bfloat16* sv = p.V;
     int bytes = 0;
@@ -843,57 +849,75 @@ __device__ __forceinline__ void load_kv_chunk(const FusedParams& p, const Smem& 
         record_error(p.ws_header, CLSA_ERR_BAD_INDEX, ((long long)b << 32) | (unsigned)i);
       }
     }
-    const uint32_t o = (uint32_t)(j >> 3) * kKVAtom + tc::sw128_offset(r, j & 7);
+    const uint32_t o = (uint32_t)(j >> 3) * AttnShape<TOK>::kKVAtom + tc::sw128_offset(r, j & 7);
     cp_async_16(dk + o, sk, bytes);
     cp_async_16(dv + o, sv, bytes);
   }
 }
 
-// `it` counts the chunks this CTA has run (the phase of both MMA barriers)
+template <int N>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&v)[N]) {
+  if constexpr (N == 16) tc::ld_32x32b_x16(taddr, v);
+  else tc::ld_32x32b_x32(taddr, v);
+}
+
+// `it` counts the chunks this CTA has run (the phase of both MMA barriers).  TOK = 128
+// only for a unit of at most 128 tokens (one chunk).
+template <int TOK>
 __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, unsigned char* kv, int g, int ntok,
                             bool q_loaded, uint32_t tmem, uint32_t& it) {
+  using SH = AttnShape<TOK>;
+  constexpr int NPT = SH::kPerThread;
   const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const int b = pl.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3, cg = warp >> 2;  // TMEM lane quarter; column group
   const int row = q4 * 32 + lane;
-  unsigned char* sP = kv + kAttnStages * 2 * kKVTile;
+  unsigned char* sP = kv + SH::kStages * 2 * SH::kKVTile;
   if (!q_loaded) load_q_tile(p, b, g, sQa);
-  const int nch = (ntok + kAttnTok - 1) / kAttnTok;
+  const int nch = (ntok + TOK - 1) / TOK;
 #pragma unroll 1
   for (int c = 0; c < 2; ++c) {
-    if (c < nch) load_kv_chunk(p, sm, b, g, pl.len, c, ntok, kv + c * 2 * kKVTile, kv + c * 2 * kKVTile + kKVTile);
+    if (c < nch && c < SH::kStages)
+      load_kv_chunk<TOK>(p, sm, b, g, pl.len, c, ntok, kv + c * 2 * SH::kKVTile, kv + c * 2 * SH::kKVTile + SH::kKVTile);
     cp_async_commit();
   }
   const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+  const bool live = q4 * 32 < p.rows;  // warp-uniform: rows of this lane quarter exist
   float o[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) o[j] = 0.f;
   float m = -INFINITY, lp = 0.f;
   bool dead = false;
-
-#pragma unroll 1
-  for (int c = 0; c < nch; ++c) {
-    const int st = c % kAttnStages;
-    unsigned char* sK = kv + st * 2 * kKVTile;
-    unsigned char* sV = sK + kKVTile;
-    cp_async_wait<1>();  // chunk c (and the Q tile) landed; chunk c + 1 may be in flight
+  // S = Q K_c^T into TMEM columns [TOK (c & 1), +TOK); issued by thread 0
+  auto issue_qk = [&](int c) {
+    const uint32_t kb = smem_u32(kv + (c % SH::kStages) * 2 * SH::kKVTile);
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks)
+      tc::mma_bf16(tmem + (uint32_t)(TOK * (c & 1)),
+                   tc::sw128_desc(smem_u32(sQa) + (ks >> 2) * kQAtom + (ks & 3) * 32),
+                   tc::sw128_desc(kb + (ks >> 2) * SH::kKVAtom + (ks & 3) * 32), SH::kIdescQK, ks > 0);
+    tc::mma_commit(&sm.bar_s);
+  };
+  if (nch > 0) {
+    cp_async_wait<1>();  // chunk 0 (and the Q tile) landed
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    if (c == 0) stamp(p, 10);
+    stamp(p, 10);
     if (threadIdx.x == 0) {
       tc::fence_after_sync();
-#pragma unroll
-      for (int ks = 0; ks < kD / 16; ++ks)
-        tc::mma_bf16(tmem, tc::sw128_desc(smem_u32(sQa) + (ks >> 2) * kQAtom + (ks & 3) * 32),
-                     tc::sw128_desc(smem_u32(sK) + (ks >> 2) * kKVAtom + (ks & 3) * 32), kIdescQK, ks > 0);
-      tc::mma_commit(&sm.bar_s);
+      issue_qk(0);
     }
+  }
+
+#pragma unroll 1
+  for (int c = 0; c < nch; ++c) {
+    unsigned char* sV = kv + (c % SH::kStages) * 2 * SH::kKVTile + SH::kKVTile;
     // chunk c + 2 into the stage of chunk c - 1, whose MMAs have completed
-    if (c + 2 < nch) {
-      unsigned char* nk = kv + ((c + 2) % kAttnStages) * 2 * kKVTile;
-      load_kv_chunk(p, sm, b, g, pl.len, c + 2, ntok, nk, nk + kKVTile);
+    if (SH::kStages == 3 && c + 2 < nch) {
+      unsigned char* nk = kv + ((c + 2) % SH::kStages) * 2 * SH::kKVTile;
+      load_kv_chunk<TOK>(p, sm, b, g, pl.len, c + 2, ntok, nk, nk + SH::kKVTile);
     }
     cp_async_commit();
 
@@ -901,72 +925,84 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
       if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 30);
       dead = true;
     }
-    if (c == 0) stamp(p, 15);
     tc::fence_after_sync();
-    float s[16];
-    float cmx = -INFINITY;
-    {
-      uint32_t v[16];
+    // the scores are read from TMEM twice (for the row max, then for P) rather than held
+    // across the exchange: registers stay within budget for 32 columns
+    const uint32_t ts = tl + (uint32_t)(TOK * (c & 1) + NPT * cg);
+    const int t0 = c * TOK + NPT * cg;
+    const int nv = ntok - t0;  // valid columns of this thread (may be <= 0 or > NPT)
+    if (live) {
+      uint32_t v[NPT];
+      float cmx = -INFINITY;
       if (!dead) {
-        tc::ld_32x32b_x16(tl + (uint32_t)(16 * cg), v);
+        tmem_ld_row<NPT>(ts, v);
+        tc::ld_wait();
+#pragma unroll
+        for (int j = 0; j < NPT; ++j)
+          if (j < nv) cmx = fmaxf(cmx, __uint_as_float(v[j]));
+      }
+      sm.cm[cg * kMaxRows + row] = cmx * p.scale_log2;  // scale > 0: the max commutes
+    }
+    __syncthreads();
+    float alpha = 1.f;
+    if (live) {
+      const float mn = fmaxf(fmaxf(m, fmaxf(sm.cm[row], sm.cm[kMaxRows + row])),
+                             fmaxf(sm.cm[2 * kMaxRows + row], sm.cm[3 * kMaxRows + row]));
+      alpha = fast_exp2(m - mn);  // m = -inf on the first chunk: 0
+      m = mn;
+      uint32_t v[NPT];
+      if (!dead) {
+        tmem_ld_row<NPT>(ts, v);
         tc::ld_wait();
       } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0u;
+        for (int j = 0; j < NPT; ++j) v[j] = 0xff800000u;  // -inf: P = 0
       }
-      const int t0 = c * kAttnTok + 16 * cg;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        s[j] = t0 + j < ntok ? __uint_as_float(v[j]) * p.scale_log2 : -INFINITY;
-        cmx = fmaxf(cmx, s[j]);
-      }
-    }
-    sm.cm[cg * kMaxRows + row] = cmx;
-    __syncthreads();
-    if (c == 0) stamp(p, 23);
-    const float mn = fmaxf(fmaxf(m, fmaxf(sm.cm[row], sm.cm[kMaxRows + row])),
-                           fmaxf(sm.cm[2 * kMaxRows + row], sm.cm[3 * kMaxRows + row]));
-    const float alpha = exp2f(m - mn);  // m = -inf on the first chunk: 0
-    m = mn;
-    {
-      uint32_t pw[8];
       float rs = 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float a = exp2f(s[2 * j] - mn), e = exp2f(s[2 * j + 1] - mn);
-        rs += a + e;
-        pw[j] = pack_bf16x2(a, e);
+      for (int q = 0; q < NPT / 8; ++q) {  // 8 tokens = one 16-byte chunk of the P row
+        uint32_t pw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int j0 = 8 * q + 2 * j;
+          const float a = j0 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -mn)) : 0.f;
+          const float e = j0 + 1 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -mn)) : 0.f;
+          rs += a + e;
+          pw[j] = pack_bf16x2(a, e);
+        }
+        const int ch = (NPT * cg) / 8 + q;  // 16-byte chunk of the row: atom ch / 8, chunk ch % 8
+        *reinterpret_cast<uint4*>(sP + (ch >> 3) * SH::kPAtom + tc::sw128_offset(row, ch & 7)) =
+            make_uint4(pw[0], pw[1], pw[2], pw[3]);
       }
       lp = lp * alpha + rs;
-      *reinterpret_cast<uint4*>(sP + tc::sw128_offset(row, 2 * cg)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-      *reinterpret_cast<uint4*>(sP + tc::sw128_offset(row, 2 * cg + 1)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
     }
+    if (SH::kStages == 3 && c + 1 < nch) cp_async_wait<1>();  // chunk c + 1 landed (c + 2 may be in flight)
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     if (threadIdx.x == 0) {
+      // O_c = P_c V_c, then S of the next chunk into the other S buffer
       tc::fence_after_sync();
 #pragma unroll
-      for (int ks = 0; ks < kAttnTok / 16; ++ks)
-        tc::mma_bf16(tmem + 128u, tc::sw128_desc(smem_u32(sP) + ks * 32),
-                     tc::sw128_desc_mn(smem_u32(sV) + ks * 16 * 128, kKVAtom), kIdescPV, ks > 0);
+      for (int ks = 0; ks < TOK / 16; ++ks)
+        tc::mma_bf16(tmem + 128u, tc::sw128_desc(smem_u32(sP) + (ks >> 2) * SH::kPAtom + (ks & 3) * 32),
+                     tc::sw128_desc_mn(smem_u32(sV) + ks * 16 * 128, SH::kKVAtom), kIdescPV, ks > 0);
       tc::mma_commit(&sm.bar_o);
+      if (c + 1 < nch) issue_qk(c + 1);
     }
-    if (c == 0) stamp(p, 24);
     if (!dead && !mbar_spin_warp(&sm.bar_o, it & 1u)) {
       if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 31);
       dead = true;
     }
-    if (c == 0) stamp(p, 25);
     tc::fence_after_sync();
-    if (!dead) {
+    if (live && !dead) {
       uint32_t v[32];
       tc::ld_32x32b_x32(tl + 128u + (uint32_t)(32 * cg), v);
       tc::ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; ++j) o[j] = fmaf(o[j], alpha, __uint_as_float(v[j]));
     }
-    if (c == 0) stamp(p, 26);
+    tc::fence_before_sync();  // O_c is read before the next chunk's P barrier lets P V overwrite it
     ++it;
   }
   cp_async_wait<0>();  // no copy of this unit outlives it (the trailing groups are empty)
@@ -974,7 +1010,6 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
 
   // row sum over the four column groups, in a fixed order
   sm.cl[cg * kMaxRows + row] = lp;
-  tc::fence_before_sync();
   __syncthreads();
   const float ls = (sm.cl[row] + sm.cl[kMaxRows + row]) + (sm.cl[2 * kMaxRows + row] + sm.cl[3 * kMaxRows + row]);
   stamp(p, 13);
@@ -1252,8 +1287,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     const uint32_t tmem = sm.tmem_base;
     unsigned char* kv = align1024(big);
     uint32_t it = 0;
-    for (int u = 0; u < pl.nunits_here; ++u)
-      attend_unit(p, sm, sQa, kv, pl.unit_g0 + u * pl.unit_step, ntok, u == 0, tmem, it);
+    for (int u = 0; u < pl.nunits_here; ++u) {
+      const int g = pl.unit_g0 + u * pl.unit_step;
+      if (ntok <= 128) attend_unit<128>(p, sm, sQa, kv, g, ntok, u == 0, tmem, it);
+      else attend_unit<64>(p, sm, sQa, kv, g, ntok, u == 0, tmem, it);
+    }
     tc::fence_before_sync();
     __syncthreads();
     if (threadIdx.x < 32) tc::tmem_dealloc(tmem, kTmemCols);
