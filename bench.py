@@ -386,7 +386,8 @@ def run_clsa(args):
         dom, dom_us, dom_bytes = "decode_fused_kernel", ms_per_step * 1e3, by["total"]
         traffic = profile_traffic("decode_fused_kernel", w.name,
                                   ["long_context_sparse_clsa_b200/csrc/decode_fused.cu",
-                                   "long_context_sparse_clsa_b200/csrc/common.cuh"])
+                                   "long_context_sparse_clsa_b200/csrc/common.cuh",
+                                   "long_context_sparse_clsa_b200/csrc/tcgen05.cuh"])
     else:
         dom, dom_us = "index_scores", kern["index_scores"]
         dom_bytes = by["kidx"] + by["qidx"] + 4 * sum(int(n) for n in inp.seq_lens)
