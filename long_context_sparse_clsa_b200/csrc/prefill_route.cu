@@ -126,20 +126,22 @@ __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
 }
 
-// 1 when score >= tau, else 0, in one saturating FMA.  With tb = nextbelow(tau), a
-// power of two sc = 2^(100 - exponent of tau) and negt = -tb * sc (both exact),
-// score * sc + negt is (score - tb) * sc rounded once: >= 1 when score >= tau (the gap
-// tau - tb is 2^-23 |tau| or more, times sc >= 2^77), <= 0 when score <= tb; an
-// infinite product keeps its sign.  |tau| < 2^-20 is lowered to -2^-20 first (a lower
-// bound only adds candidates).  Keep-all rows (tau = -inf) do not use it.
-__device__ __forceinline__ float ge01(uint32_t bits, float sc, float negt) {
-  return __saturatef(fmaf(__uint_as_float(bits), sc, negt));
+// The main-pass test of a pair of scores against the row bound tau, in two instructions:
+// both scores rounded toward zero to bf16 in one conversion, then one packed compare with
+// rz(tau), 0xffff in each half that passes.  Rounding toward zero is monotone, so every
+// score >= tau passes (a superset test); a score that passes below tau lies within one
+// bf16 step of it and is only an extra candidate: exactness is decided later on the fp32
+// scores (ties and all), and a dropped score has rz(score) < rz(tau), hence score < tau.
+// tau = -inf (every token kept) passes every finite score.
+__device__ __forceinline__ uint32_t rz_bf16x2(float hi, float lo) {
+  uint32_t d;
+  asm("cvt.rz.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
 }
-__device__ __forceinline__ void ge_setup(float tau, float& sc, float& negt) {
-  if (fabsf(tau) < 0x1p-20f) tau = -0x1p-20f;
-  const int e = ((__float_as_int(tau) >> 23) & 0xff) - 127;  // exponent (tau normal here)
-  sc = __int_as_float((127 + 100 - e) << 23);                 // 2^(100 - e), e in [-20, 127]
-  negt = -nextafterf(tau, -INFINITY) * sc;
+__device__ __forceinline__ uint32_t ge_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       float hs = 0.f, hb = 0.f, lo = 0.f, span = 0.f;  // bin map: sat(score * hs + hb) * (kBins - 1)
       int seen = 0, cnt = 0;
       float tau = -INFINITY;
-      float sc = 1.f, negt = 0.f;  // the compare of the main pass (set with tau)
+      uint32_t tau2 = rz_bf16x2(-INFINITY, -INFINITY);  // rz(tau) in both halves (set with tau)
       uint2* const dst = p.cand + ((size_t)((row_ok ? i : 0) * p.S + s) * 2 + hc) * caph;
       for (int it = 0; it < ut.count(); ++it) {
         if (!dead && !mbar_wait_warp(&sm.tfull[buf], ph_tfull)) {
@@ -402,20 +404,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 }
               }
             } else {
-              // one compare per score into a 32-bit mask, on the FMA pipe: ge01 is exactly
-              // 1 or 0, and the weighted sums of 16 of them are exact integers
-              float l0 = 0.f, l1 = 0.f, u0 = 0.f, u1 = 0.f;
+              // bit c of the mask: column c passes (columns c and c + 16 share one
+              // conversion and one packed compare; two accumulators halve the OR chain)
+              uint32_t ma = 0u, mb = 0u;
 #pragma unroll
               for (int c = 0; c < 16; c += 2) {
-                l0 = fmaf(ge01(v[c], sc, negt), (float)(1u << c), l0);
-                l1 = fmaf(ge01(v[c + 1], sc, negt), (float)(1u << (c + 1)), l1);
-                u0 = fmaf(ge01(v[16 + c], sc, negt), (float)(1u << c), u0);
-                u1 = fmaf(ge01(v[16 + c + 1], sc, negt), (float)(1u << (c + 1)), u1);
+                ma |= ge_bf16x2(rz_bf16x2(__uint_as_float(v[16 + c]), __uint_as_float(v[c])), tau2) & (0x10001u << c);
+                mb |= ge_bf16x2(rz_bf16x2(__uint_as_float(v[17 + c]), __uint_as_float(v[c + 1])), tau2) &
+                      (0x20002u << c);
               }
-              // 2^23 + m (m < 2^16) is exact: the low 16 bits of its encoding are m
-              uint32_t mm = __byte_perm(__float_as_uint((l0 + l1) + 8388608.f),
-                                        __float_as_uint((u0 + u1) + 8388608.f), 0x5410);
-              if (tau == -INFINITY) mm = 0xffffffffu;  // keep-all row
+              uint32_t mm = ma | mb;
               if (nv < 32) mm &= nv <= 0 ? 0u : (0xffffffffu >> (32 - nv));
               // stage the scores of every 4-column group that holds a candidate in this
               // thread's smem row, then one (score, token) store per set bit, in column order
@@ -423,7 +421,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
                 for (int g = 0; g < 8; ++g)
                   st_shared_v4_if(stage_addr + 16u * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3],
-                                  (mm >> (4 * g)) & 0xfu);
+                                  mm & (0xfu << (4 * g)));
                 const uint32_t jb = (uint32_t)(j0 + 32 * ch);
                 const int pc = __popc(mm);
                 if (cnt + pc <= caph) {
@@ -486,7 +484,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
               }
             }
           }
-          ge_setup(tau, sc, negt);
+          tau2 = rz_bf16x2(tau, tau);
           epi_bar();  // every histogram is read: the staging rows may overwrite them
         }
       }
