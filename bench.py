@@ -5,6 +5,7 @@ L-layer sparse GQA attention) on B200.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode128k]
                     [--impl {clsa,reference}] [--no-graph] [--no-cpu-baseline]
                     [--l2 {rotate,flush}] [--sets R]
+                    [--variant {clsa,per_layer_routing,yoco_dense,standard}]
 
 One JSON line on rank 0.  A step is one decode token per sequence through the
 whole path; the default workload is the 128K-context decode (batch 1, n=131072,
@@ -52,6 +53,9 @@ def parse():
     ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
                     help="between steps: rotate through input sets larger than L2 (default), or flush L2")
     ap.add_argument("--sets", type=int, default=6, help="input sets rotated through (--l2 rotate)")
+    ap.add_argument("--variant", default="clsa",
+                    choices=["clsa", "per_layer_routing", "yoco_dense", "standard"],
+                    help="a comparison system built from the library's calls (one GPU; not the default line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-steps", type=int, default=2)
     return ap.parse_args()
@@ -465,10 +469,112 @@ def run_clsa(args):
     print(json.dumps(line), flush=True)
 
 
+def run_variant(args):
+    """Time a comparison system of the pages' ablation (per-layer routing, YOCO only,
+    standard attention) on the same workload, built from the library's own calls."""
+    import torch
+    from long_context_sparse_clsa_b200 import clsa
+    from long_context_sparse_clsa_b200 import baselines
+    from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs
+    if args.gpus != 1:
+        raise SystemExit("--variant runs on one GPU")
+    torch.cuda.set_device(0)
+    clsa.load_library()
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    dev = dv["K"].device
+    stream = torch.cuda.current_stream()
+    L, B, Hq, Hkv, d, k, n = w.L, w.B, w.Hq, w.Hkv, w.d, w.k, w.n_max
+    eb = 2 if w.dtype == "bf16" else 4
+    Ob = torch.empty_like(dv["Q"])
+    lens = [int(x) for x in inp.seq_lens]
+    gen = torch.Generator(device="cpu").manual_seed(4321)
+
+    def permuted(x):
+        """x [B][n_max][...] with every sequence's valid rows in a seeded random order"""
+        y = x.clone()
+        for b in range(B):
+            perm = torch.randperm(lens[b], generator=gen).to(dev)
+            y[b, :lens[b]] = x[b, perm]
+        return y
+
+    # every layer's extra inputs are row permutations of the seeded ones (layer 0: the seeded
+    # tensors): the same value distribution, other rows selected / read
+    qo_bytes = 2 * L * B * Hq * d * eb
+    if args.variant == "per_layer_routing":
+        kx = [dv["k_idx"]] + [permuted(dv["k_idx"]) for _ in range(L - 1)]
+        qx = [dv["q_idx"]] * L
+        idx = torch.empty(L, B, k, dtype=torch.int32, device=dev)
+        cnt = torch.empty(L, B, dtype=torch.int32, device=dev)
+        sysm = baselines.PerLayerRouting(qx, kx, dv["K"], dv["V"], dv["Q"], dv["seq_lens"], k, Ob, idx, cnt)
+        sel = sum(min(k, x) for x in lens)
+        step_bytes_ = L * (sum(lens) * w.d_idx * eb + B * w.d_idx * eb + 2 * sel * Hkv * d * eb) + qo_bytes
+        note = "every layer: its own indexer scan over the shared cache, its own TopK, attention (L fused steps)"
+    elif args.variant == "yoco_dense":
+        sysm = baselines.YocoDense(dv["K"], dv["V"], dv["Q"], dv["seq_lens"], Ob)
+        step_bytes_ = 2 * sum(lens) * Hkv * d * eb + qo_bytes
+        note = "every layer dense over the one shared cache (one call, the L*G rows of a head read each row once)"
+    else:
+        Ks = [dv["K"]] + [permuted(dv["K"]) for _ in range(L - 1)]
+        Vs = [dv["V"]] + [permuted(dv["V"]) for _ in range(L - 1)]
+        sysm = baselines.StandardAttention(Ks, Vs, dv["Q"], dv["seq_lens"], Ob)
+        step_bytes_ = L * 2 * sum(lens) * Hkv * d * eb + qo_bytes
+        note = "every layer dense over its own cache (L calls)"
+    launches = sysm.step()
+    torch.cuda.synchronize()
+    graph = None
+    if not args.no_graph:
+        s2 = torch.cuda.Stream()
+        s2.wait_stream(stream)
+        with torch.cuda.stream(s2):
+            sysm.step()
+        stream.wait_stream(s2)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            sysm.step()
+        torch.cuda.synchronize()
+    run = graph.replay if graph is not None else sysm.step
+    for _ in range(max(args.warmup, 3)):
+        run()
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    st = sysm.ws.status()
+    if st[0] != "CLSA_OK":
+        raise RuntimeError(f"device error during timing: {st}")
+    ms = e0.elapsed_time(e1) / args.steps
+    hbm, _, peak_kind = peaks()
+    gbs = step_bytes_ / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "variant": args.variant, "value": B / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "us_per_step": ms * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1); extra layers' inputs are seeded row permutations)",
+        "config": {"workload": w.name, "B": B, "n": n, "d_idx": w.d_idx, "k": k, "L": L, "Hq": Hq, "Hkv": Hkv,
+                   "d": d, "system": note, "l2": "every step reads more than L2 (no flush)",
+                   "launch": "cuda graph" if graph is not None else "eager"},
+        "roofline": {"bound": "hbm", "kernel": "whole step", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "traffic": None, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_step": step_bytes_},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.variant != "clsa":
+        run_variant(args)
     else:
         run_clsa(args)
 

@@ -24,7 +24,8 @@
  *              outputs O are written in the same dtype (bf16 rounded to nearest
  *              even from fp32); scores and lse are always fp32.  All scoring,
  *              softmax and accumulation are fp32.
- * Shapes.      d, d_idx in {64, 128}; Hq % Hkv == 0; 1 <= k <= 4096;
+ * Shapes.      d, d_idx in {64, 128}; Hq % Hkv == 0; 1 <= k <= 4096
+ *              (clsa_sparse_attn: 1 <= k <= 2^24, the rows are read directly);
  *              B >= 1; 0 <= seq_lens[b] <= n_max (seq_lens is device int32).
  *              Other shapes return CLSA_ERR_UNSUPPORTED before any launch.
  * scale.       Attention scale; a value <= 0 selects 1/sqrt(d).
@@ -133,7 +134,9 @@ CLSA_API clsa_status clsa_gather_kv(const void* K, const void* V, const int32_t*
  * is the per-layer call a model makes layer by layer).  K_S, V_S [B][k][Hkv][d]
  * compact rows, count [B] valid rows per sequence.  O [L][B][Hq][d] out;
  * lse [L][B][Hq] fp32 out (natural-log sum of exp of the scaled scores), may
- * be NULL.  A sequence with count 0 gets O = 0 and lse = -inf.
+ * be NULL.  A sequence with count 0 gets O = 0 and lse = -inf.  k may exceed
+ * the selection limit (up to 2^24): passing the whole cache as K_S/V_S with
+ * count = seq_lens is dense attention over it.
  * Split-k flash decoding with an online softmax; fp32 accumulation. */
 CLSA_API size_t clsa_sparse_attn_workspace_size(int B, int k, int L, int Hq, int Hkv, int d);
 CLSA_API clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void* V_S, const int32_t* count,

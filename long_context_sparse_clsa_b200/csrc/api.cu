@@ -40,10 +40,14 @@ struct CallScope {
 };
 
 // attention shape checks shared by clsa_sparse_attn and clsa_decode_step
-clsa_status check_attn(int B, int k, int L, int Hq, int Hkv, int d, clsa_dtype dt) {
+// kmax: 4096 for the selection paths; clsa_sparse_attn reads K_S/V_S rows directly and
+// takes any k up to kMaxDirectK (a whole cache: dense attention)
+constexpr int kMaxSelectK = 4096;
+constexpr int kMaxDirectK = 1 << 24;
+clsa_status check_attn(int B, int k, int L, int Hq, int Hkv, int d, clsa_dtype dt, int kmax = kMaxSelectK) {
   if (B < 1 || k < 1 || L < 1 || Hq < 1 || Hkv < 1) return CLSA_ERR_INVALID_ARG;
   if (!dtype_ok(dt)) return CLSA_ERR_INVALID_ARG;
-  if (!dims_ok(d) || Hq % Hkv != 0 || k > 4096) return CLSA_ERR_UNSUPPORTED;
+  if (!dims_ok(d) || Hq % Hkv != 0 || k > kmax) return CLSA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if (G > (dt == CLSA_BF16 ? 128 : 32)) return CLSA_ERR_UNSUPPORTED;
   return CLSA_OK;
@@ -200,7 +204,7 @@ clsa_status clsa_gather_kv(const void* K, const void* V, const int32_t* idx, con
 }
 
 size_t clsa_sparse_attn_workspace_size(int B, int k, int L, int Hq, int Hkv, int d) {
-  if (check_attn(B, k, L, Hq, Hkv, d, CLSA_BF16) != CLSA_OK) return 0;
+  if (check_attn(B, k, L, Hq, Hkv, d, CLSA_BF16, kMaxDirectK) != CLSA_OK) return 0;
   // the larger of the bf16 and fp32 plans, so one size serves both dtypes
   AttnShape a{B, k, L, Hq, Hkv, d, CLSA_BF16, false, 0, 0};
   AttnShape f{B, k, L, Hq, Hkv, d, CLSA_F32, false, 0, 0};
@@ -211,7 +215,7 @@ clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void* V_S, co
                              int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, void* O, float* lse,
                              void* ws, size_t ws_bytes, void* stream) {
   CallScope scope;
-  clsa_status st = check_attn(B, k, L, Hq, Hkv, d, dt);
+  clsa_status st = check_attn(B, k, L, Hq, Hkv, d, dt, kMaxDirectK);
   if (st != CLSA_OK) return st;
   if (!Q || !K_S || !V_S || !count || !O) return CLSA_ERR_INVALID_ARG;
   for (const void* p : {Q, K_S, V_S, (const void*)O})

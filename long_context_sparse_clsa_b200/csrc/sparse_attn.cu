@@ -546,7 +546,8 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
   if (sh.dt == CLSA_BF16) {
     const int NW = (pl.rows + 15) / 16;
     const bool two = NW <= 6;  // two CTAs per SM fit
-    auto smem = [&](int D, int nst) { return (NW * 16 + 2 * nst * kBlk) * (D + 8) * 2 + pl.chunk * 4; };
+    // the split's token list lives in shared memory only when gathering by index
+    auto smem = [&](int D, int nst) { return (NW * 16 + 2 * nst * kBlk) * (D + 8) * 2 + (sh.gather ? pl.chunk * 4 : 0); };
 #define CLSA_ATTN_BF16(D, GA)                                                           \
   do {                                                                                  \
     if (two) {                                                                          \

@@ -1,0 +1,90 @@
+"""GPU parity of the comparison systems built from the library's calls (per-layer
+routing, dense attention over one shared cache, standard attention with per-layer
+caches) against the CPU oracle, at sizes that span several attention splits and a
+cache longer than the selection limit.  Tolerances as in test_gpu_parity.py."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import clsa_oracle as O
+from long_context_sparse_clsa_b200 import clsa
+from long_context_sparse_clsa_b200.baselines import PerLayerRouting, StandardAttention, YocoDense
+from long_context_sparse_clsa_b200.inputs import make_inputs, scaled
+from parity_util import check_near_tie_sets, max_abs, tensor_f64
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_sparse_clsa_b200.build import build
+    build()
+    clsa.load_library()
+
+
+def _dense_oracle(inp_Q, inp_K, inp_V, lens):
+    """Dense attention = sparse attention over every valid row (idx = 0..len-1)."""
+    B = len(lens)
+    n_max = inp_K.shape[1]
+    idx = np.tile(np.arange(n_max, dtype=np.int64), (B, 1))
+    return O.sparse_attention(inp_Q, inp_K, inp_V, idx, np.asarray(lens))[0]
+
+
+def test_per_layer_routing():
+    base = scaled("decode32k", n_max=5000 + 13, k=400, L=3)
+    layers = [make_inputs(base, seed=21 + l) for l in range(base.L)]
+    kv = layers[0]  # the shared cache and the queries
+    dvs = [clsa.to_device(x) for x in layers]
+    Q, K, V, lens = dvs[0]["Q"], dvs[0]["K"], dvs[0]["V"], dvs[0]["seq_lens"]
+    Ob = torch.empty_like(Q)
+    idx = torch.empty(base.L, base.B, base.k, dtype=torch.int32, device=Q.device)
+    cnt = torch.empty(base.L, base.B, dtype=torch.int32, device=Q.device)
+    sysm = PerLayerRouting([d["q_idx"] for d in dvs], [d["k_idx"] for d in dvs], K, V, Q, lens, base.k, Ob, idx, cnt)
+    sysm.step()
+    torch.cuda.synchronize()
+    assert sysm.ws.status()[0] == "CLSA_OK"
+    got = tensor_f64(Ob)
+    for l, x in enumerate(layers):
+        i_np, c_np = idx[l].cpu().numpy(), cnt[l].cpu().numpy()
+        check_near_tie_sets(i_np, c_np, O.index_scores(x.q_idx, x.k_idx, x.seq_lens), x.seq_lens, base.k)
+        want, _ = O.sparse_attention(kv.Q[l:l + 1], kv.K, kv.V, i_np, c_np)
+        assert max_abs(got[l:l + 1], want) <= TOL[base.dtype]
+    # the layers' selections differ: the routing really ran per layer
+    assert not torch.equal(idx[0], idx[1])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_yoco_dense_longer_than_selection_limit(dtype):
+    """Dense attention over a shared cache of 6000+ rows (above the 4096 selection
+    limit), ragged lengths, several splits."""
+    w = scaled("ragged16", B=3, n_max=6000 + 37, lens=(4097, 6037), k=16, L=2, Hq=8, Hkv=2, d=64, d_idx=64,
+               dtype=dtype, plant=0.0, seed=9)
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    Ob = torch.empty_like(dv["Q"])
+    sysm = YocoDense(dv["K"], dv["V"], dv["Q"], dv["seq_lens"], Ob)
+    sysm.step()
+    torch.cuda.synchronize()
+    assert sysm.ws.status()[0] == "CLSA_OK"
+    want = _dense_oracle(inp.Q, inp.K, inp.V, inp.seq_lens)
+    assert max_abs(tensor_f64(Ob), want) <= TOL[dtype]
+
+
+def test_standard_attention_per_layer_caches():
+    w = scaled("decode32k", n_max=4500, k=16, L=2, plant=0.0)
+    caches = [make_inputs(w, seed=40 + l) for l in range(w.L)]
+    dvs = [clsa.to_device(x) for x in caches]
+    Q = dvs[0]["Q"]
+    Ob = torch.empty_like(Q)
+    sysm = StandardAttention([d["K"] for d in dvs], [d["V"] for d in dvs], Q, dvs[0]["seq_lens"], Ob)
+    sysm.step()
+    torch.cuda.synchronize()
+    assert sysm.ws.status()[0] == "CLSA_OK"
+    got = tensor_f64(Ob)
+    for l, x in enumerate(caches):
+        want = _dense_oracle(caches[0].Q[l:l + 1], x.K, x.V, x.seq_lens)
+        assert max_abs(got[l:l + 1], want) <= TOL[w.dtype]
