@@ -83,6 +83,9 @@ int prefill_route_ldd(const clsa_prefill_args* a);  // dense candidate row lengt
 size_t prefill_route_ws_bytes(const clsa_prefill_args* a);
 cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, void* ws, cudaStream_t s,
                                  PrefillRouteBufs* out);
+// per-row sparse attention of a prefill chunk on tcgen05 (bf16, d = 128); else the split-k kernel
+bool prefill_attn_tc_supported(const clsa_prefill_args* a);
+cudaError_t launch_prefill_attn_tc(const clsa_prefill_args* a, float scale, void* ws_header, cudaStream_t s);
 size_t prefill_ws_bytes(const clsa_prefill_args* a);
 clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_body, cudaStream_t s);
 

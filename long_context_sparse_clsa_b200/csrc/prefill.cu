@@ -204,8 +204,12 @@ clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_bo
     if (e != cudaSuccess) return CLSA_ERR_CUDA;
   }
   const float scale = a->scale > 0.f ? a->scale : 1.0f / sqrtf((float)a->d);
-  AttnShape sh{a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype, true, a->n, 0};
-  e = launch_sparse_attn(sh, a->Q, a->K, a->V, a->idx, a->count, scale, a->O, a->lse, ws_header, w + lay.attn, s);
+  if (prefill_attn_tc_supported(a)) {
+    e = launch_prefill_attn_tc(a, scale, ws_header, s);
+  } else {
+    AttnShape sh{a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype, true, a->n, 0};
+    e = launch_sparse_attn(sh, a->Q, a->K, a->V, a->idx, a->count, scale, a->O, a->lse, ws_header, w + lay.attn, s);
+  }
   return e == cudaSuccess ? CLSA_OK : CLSA_ERR_CUDA;
 }
 
