@@ -49,6 +49,8 @@ constexpr uint32_t kTmemCols = 256;                 // S at [0, 128) (two buffer
 constexpr uint32_t kIdescQK = tc::idesc_bf16_f32(kM, kTok);
 constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kM, kD) | (1u << 16);  // B (V) MN-major
 
+static_assert(kThreadsPA == 256 && kTok == 64, "the gather maps 256 threads onto 64 rows x 16 columns");
+
 struct PAParams {
   const __nv_bfloat16* Q;   // [L][T][Hq][d]
   const __nv_bfloat16* K;   // [n][Hkv][d]
@@ -142,28 +144,23 @@ __global__ void __launch_bounds__(kThreadsPA, 2) prefill_attn_tc_kernel(const PA
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
+  // the gather: thread x copies 16-byte column j = x % 16 of chunk rows x / 16 + 16 i
+  // (i = 0..3); the swizzled destinations of those rows are 2 KiB apart
+  const int gj = threadIdx.x & 15, gr0 = threadIdx.x >> 4;
+  const uint32_t go0 = (uint32_t)(gj >> 3) * kKVAtom + tc::sw128_offset(gr0, gj & 7);
+  const size_t gcol = (size_t)g * kD + gj * 8;
+  const size_t gstride = (size_t)p.Hkv * kD;
   auto load_chunk = [&](int c) {  // chunk c into stage c % 2
-    unsigned char* dk = kv + (c & 1) * kStageBytes;
+    unsigned char* dk = kv + (c & 1) * kStageBytes + go0;
     unsigned char* dv = dk + kKVTile;
-#pragma unroll 1
-    for (int v = threadIdx.x; v < kTok * 16; v += kThreadsPA) {
-      const int r = v >> 4, j = v & 15;
-      const int i = c * kTok + r;
-      const __nv_bfloat16* sk = p.K;
-      const __nv_bfloat16* sv = p.V;
-      int bytes = 0;
-      if (i < cnt) {
-        const int tk = stok[i];
-        if ((unsigned)tk < (unsigned)p.n) {
-          const size_t off = ((size_t)tk * p.Hkv + g) * kD + j * 8;
-          sk += off;
-          sv += off;
-          bytes = 16;
-        }
-      }
-      const uint32_t o = (uint32_t)(j >> 3) * kKVAtom + tc::sw128_offset(r, j & 7);
-      cp_async_16(dk + o, sk, bytes);
-      cp_async_16(dv + o, sv, bytes);
+#pragma unroll
+    for (int it = 0; it < kTok / 16; ++it) {
+      const int i = c * kTok + gr0 + 16 * it;
+      const int tk = i < cnt ? stok[i] : -1;
+      const bool ok = (unsigned)tk < (unsigned)p.n;
+      const size_t off = ok ? gcol + (size_t)tk * gstride : 0;
+      cp_async_16(dk + 2048 * it, p.K + off, ok ? 16 : 0);
+      cp_async_16(dv + 2048 * it, p.V + off, ok ? 16 : 0);
     }
   };
   auto issue_qk = [&](int c) {  // S of chunk c into TMEM columns [64 (c & 1), +64)
@@ -208,15 +205,21 @@ __global__ void __launch_bounds__(kThreadsPA, 2) prefill_attn_tc_kernel(const PA
     tc::fence_after_sync();
     const uint32_t ts = tl + (uint32_t)(kTok * (c & 1) + kNpt * cg);
     const int nv = cnt - (c * kTok + kNpt * cg);  // valid columns of this thread
+    const bool full = nv >= kNpt;  // warp-uniform: every column of this thread is a token
     if (live) {
       float cmx = -INFINITY;
       if (!dead) {
         uint32_t v[kNpt];
         tc::ld_32x32b_x32(ts, v);
         tc::ld_wait();
+        if (full) {
 #pragma unroll
-        for (int j = 0; j < kNpt; ++j)
-          if (j < nv) cmx = fmaxf(cmx, __uint_as_float(v[j]));
+          for (int j = 0; j < kNpt; j += 2) cmx = fmaxf(cmx, fmaxf(__uint_as_float(v[j]), __uint_as_float(v[j + 1])));
+        } else {
+#pragma unroll
+          for (int j = 0; j < kNpt; ++j)
+            if (j < nv) cmx = fmaxf(cmx, __uint_as_float(v[j]));
+        }
       }
       cm[cg * kM + row] = cmx * p.scale_log2;  // scale > 0: the max commutes
     }
@@ -235,14 +238,19 @@ __global__ void __launch_bounds__(kThreadsPA, 2) prefill_attn_tc_kernel(const PA
         for (int j = 0; j < kNpt; ++j) v[j] = 0xff800000u;
       }
       float rs = 0.f;
+      const int lim = full ? kNpt : nv;  // columns at or past lim are not tokens: P = 0
 #pragma unroll
       for (int q = 0; q < kNpt / 8; ++q) {
         uint32_t pw[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int j0 = 8 * q + 2 * j;
-          const float a = j0 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -mn)) : 0.f;
-          const float e = j0 + 1 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -mn)) : 0.f;
+          float a = fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -mn));
+          float e = fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -mn));
+          if (!full) {
+            a = j0 < lim ? a : 0.f;
+            e = j0 + 1 < lim ? e : 0.f;
+          }
           rs += a + e;
           pw[j] = pack_bf16x2(a, e);
         }
