@@ -50,7 +50,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 4096;          // digit histograms of the selection
 constexpr int kTauBits = 12;          // key bits of the candidate-bound histogram
 constexpr int kTauBins = 1 << kTauBits;
-constexpr int kScanU = 4;             // rows per lane group per scan stage
+constexpr int kScanU = 4;             // rows per lane group per scan stage (the reduction assumes 4)
 constexpr int kScanS = 4;             // scan stages in flight (the whole of `big`)
 constexpr int kMaxRows = 128;         // L*G rows per unit (8 m-tiles x 2 token sets = 16 warps)
 constexpr int kD = 128;               // head dim of the fused path
@@ -147,6 +147,7 @@ constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
 constexpr size_t kSmemBig = 128 * 1024;
 constexpr size_t smem_bytes() { return align_up(sizeof(Smem), 128) + kSmemQ + kSmemBig; }
 static_assert(kScanS * kScanU * kThreads * 16 <= (int)kSmemBig, "scan ring exceeds big");
+static_assert(kScanU == 4, "the scan reduction handles 4 rows per lane group");
 static_assert(kTauBins <= kBins, "the slice histogram lives in Smem::hist");
 
 // ---------------------------------------------------------------------------
@@ -410,19 +411,33 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
     cp_async_wait<kScanS - 1>();  // stage it has landed
     const int st = it % kScanS;
     const int base0 = j0 + it * ROWS;
+    // the stage's 4 rows per lane group: 4 independent partial dot products per lane, then
+    // one transposed reduction over the group's LPR lanes (each level sends the half of
+    // the rows the partner keeps): 2 + 1 + log2(LPR / 4) shuffles for all 4 rows
+    float acc[kScanU];
 #pragma unroll
     for (int u = 0; u < kScanU; ++u) {
       const int j = base0 + grp + u * GROUPS;
       const uint4 v = j < j1 ? ring[(st * kScanU + u) * kThreads + threadIdx.x] : make_uint4(0, 0, 0, 0);
-      float acc = row_dot<DIDX>(v, q);
+      acc[u] = row_dot<DIDX>(v, q);
+    }
+    const bool hi_a = (sub & (LPR / 2)) != 0, hi_b = (sub & (LPR / 4)) != 0;
+    float k0 = hi_a ? acc[2] : acc[0], k1 = hi_a ? acc[3] : acc[1];
+    k0 += __shfl_xor_sync(0xffffffffu, hi_a ? acc[0] : acc[2], LPR / 2);
+    k1 += __shfl_xor_sync(0xffffffffu, hi_a ? acc[1] : acc[3], LPR / 2);
+    float tot = hi_b ? k1 : k0;
+    tot += __shfl_xor_sync(0xffffffffu, hi_b ? k0 : k1, LPR / 4);
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (sub == 0 && j < j1) {
+    for (int o = LPR / 8; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    {
+      const int u = (hi_a ? 2 : 0) + (hi_b ? 1 : 0);  // the row this lane now holds in full
+      const int j = base0 + grp + u * GROUPS;
+      if ((sub & (LPR / 4 - 1)) == 0 && j < j1) {
         if (nrows <= kMaxUnitTok) {
-          sm.score[j] = acc;  // global copy and histogram after the stream (off its critical path)
+          sm.score[j] = tot;  // global copy and histogram after the stream (off its critical path)
         } else {
-          __stcg(sc + j, acc);
-          if (hist) atomicAdd(&th[float_key(acc) >> (32 - kTauBits)], 1u);
+          __stcg(sc + j, tot);
+          if (hist) atomicAdd(&th[float_key(tot) >> (32 - kTauBits)], 1u);
         }
       }
     }
@@ -450,7 +465,9 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigne
   }
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
+  stamp(p, 14);
   scan_rows<DIDX>(p, sm, th, reinterpret_cast<uint4*>(ring), src, sc, q, 0, nrows, nrows, hist);
+  stamp(p, 16);
   if (nrows <= kMaxUnitTok) {
     __syncthreads();
 #pragma unroll 1
