@@ -385,6 +385,32 @@ __device__ __forceinline__ float row_dot(const uint4 v, const float (&q)[8]) {
 // group in shared memory (16-byte cp.async, L2 only).  Every thread reads back only the
 // chunks it copied, so no barrier is needed: S - 1 stages stay in flight while one is
 // reduced.
+// stage st of the ring: rows base0 + grp + u * GROUPS (u < kScanU) of [.., j1)
+template <int DIDX>
+__device__ __forceinline__ void scan_issue(uint4* ring, const __nv_bfloat16* src, int st, int base0, int j1) {
+  constexpr int LPR = DIDX / 8;
+  constexpr int GROUPS = kThreads / LPR;
+  const int grp = threadIdx.x / LPR, sub = threadIdx.x % LPR;
+#pragma unroll
+  for (int u = 0; u < kScanU; ++u) {
+    const int j = base0 + grp + u * GROUPS;
+    if (j < j1) cp_async_16(ring + (st * kScanU + u) * kThreads + threadIdx.x, src + (size_t)j * DIDX + sub * 8, 16);
+  }
+  cp_async_commit();  // one group per stage, empty or not
+}
+// the ring's first kScanS stages: the stream starts as soon as the slice is known
+template <int DIDX>
+__device__ __forceinline__ void scan_start(uint4* ring, const __nv_bfloat16* src, int j0, int j1) {
+  constexpr int ROWS = kThreads / (DIDX / 8) * kScanU;
+  const int nst = (j1 - j0 + ROWS - 1) / ROWS;
+#pragma unroll
+  for (int st = 0; st < kScanS; ++st) {
+    if (st < nst) scan_issue<DIDX>(ring, src, st, j0 + st * ROWS, j1);
+    else cp_async_commit();
+  }
+}
+// reduce the stream begun by scan_start (no other async copy committed since), refilling
+// each stage as it is read
 template <int DIDX>
 __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32_t* th, uint4* ring,
                                           const __nv_bfloat16* src, float* sc, const float (&q)[8], int j0, int j1,
@@ -393,20 +419,8 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
   constexpr int GROUPS = kThreads / LPR;        // row groups per CTA
   const int grp = threadIdx.x / LPR, sub = threadIdx.x % LPR;
   constexpr int ROWS = GROUPS * kScanU;         // rows per stage
-  auto issue = [&](int st, int base0) {
-#pragma unroll
-    for (int u = 0; u < kScanU; ++u) {
-      const int j = base0 + grp + u * GROUPS;
-      if (j < j1) cp_async_16(ring + (st * kScanU + u) * kThreads + threadIdx.x, src + (size_t)j * DIDX + sub * 8, 16);
-    }
-    cp_async_commit();  // one group per stage, empty or not
-  };
+  auto issue = [&](int st, int base0) { scan_issue<DIDX>(ring, src, st, base0, j1); };
   const int nst = (j1 - j0 + ROWS - 1) / ROWS;  // the same for every thread (whole-warp shuffles below)
-#pragma unroll
-  for (int st = 0; st < kScanS; ++st) {
-    if (st < nst) issue(st, j0 + st * ROWS);
-    else cp_async_commit();
-  }
   for (int it = 0; it < nst; ++it) {
     cp_async_wait<kScanS - 1>();  // stage it has landed
     const int st = it % kScanS;
@@ -448,7 +462,8 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
 }
 
 template <int DIDX>
-__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigned char* ring, bool hist) {
+__device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigned char* ring, bool hist,
+                           bool started) {
   const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
@@ -463,6 +478,8 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigne
     unpack_bf16x2(qv.z, q[4], q[5]);
     unpack_bf16x2(qv.w, q[6], q[7]);
   }
+  if (!started) scan_start<DIDX>(reinterpret_cast<uint4*>(ring), src, 0, nrows);
+  stamp(p, 24);
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
   stamp(p, 14);
@@ -1173,11 +1190,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   unsigned char* big = smem + align_up(sizeof(Smem), 128) + kSmemQ;
 
   stamp(p, 0);
+  // One sequence: CTA c's slice is [c chunk, c chunk + chunk) with chunk = ceil(len /
+  // gridDim.x) (what make_plan gives for B = 1), so every thread starts the K_idx stream
+  // before the plan exists; the plan is checked against it below.
+  int pre_r0 = 0, pre_r1 = 0;
+  bool pre = false;
+  if (p.B == 1) {
+    const int len = max(0, min(p.seq_lens[0], p.n_max));
+    if (len > 0) {
+      const int chunk = (len + (int)gridDim.x - 1) / (int)gridDim.x;
+      pre_r0 = min(len, (int)blockIdx.x * chunk);
+      pre_r1 = min(len, pre_r0 + chunk);
+      scan_start<DIDX>(reinterpret_cast<uint4*>(big), p.k_idx + (size_t)pre_r0 * DIDX, 0, pre_r1 - pre_r0);
+      pre = true;
+    }
+  }
   if (threadIdx.x == 0) {
     make_plan(p, sm.plan);
     sm.abort_flag = 0;
   }
   __syncthreads();
+  stamp(p, 15);
   const Plan pl = sm.plan;
   if (blockIdx.x == 0) {  // sequences with no tokens: count 0, idx -1, O = 0, lse = -inf
 #pragma unroll 1
@@ -1207,10 +1240,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   if (pl.c == pl.Cb - 1)  // score tail beyond the sequence
     for (int j = pl.len + threadIdx.x; j < p.n_max; j += kThreads) p.scores[(size_t)pl.b * p.n_max + j] = -INFINITY;
   unsigned char* sQa = align1024(reinterpret_cast<unsigned char*>(sQ));
-  if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQa);  // lands during the scan
+  if (pre && (pl.b != 0 || pl.r0 != pre_r0 || pl.r1 != pre_r1)) {  // cannot happen: the plan's own slice
+    record_error(p.ws_header, CLSA_ERR_INVALID_ARG, 50);
+    cp_async_wait<0>();
+    pre = false;
+  }
 
   const bool all_sel = pl.keff == pl.len;
-  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel)) return;
+  stamp(p, 23);
+  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel, pre)) return;
+  if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQa);  // lands during the selection
   stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
