@@ -446,13 +446,10 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
     {
       const int u = (hi_a ? 2 : 0) + (hi_b ? 1 : 0);  // the row this lane now holds in full
       const int j = base0 + grp + u * GROUPS;
-      if ((sub & (LPR / 4 - 1)) == 0 && j < j1) {
-        if (nrows <= kMaxUnitTok) {
-          sm.score[j] = tot;  // global copy and histogram after the stream (off its critical path)
-        } else {
-          __stcg(sc + j, tot);
-          if (hist) atomicAdd(&th[float_key(tot) >> (32 - kTauBits)], 1u);
-        }
+      if ((sub & (LPR / 4 - 1)) == 0 && j < j1) {  // the stream is HBM-bound: store here
+        if (nrows <= kMaxUnitTok) sm.score[j] = tot;
+        __stcg(sc + j, tot);
+        if (hist) atomicAdd(&th[float_key(tot) >> (32 - kTauBits)], 1u);
       }
     }
     if (it + kScanS < nst) issue(st, j0 + (it + kScanS) * ROWS);  // refill the slot just read
@@ -485,15 +482,6 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigne
   stamp(p, 14);
   scan_rows<DIDX>(p, sm, th, reinterpret_cast<uint4*>(ring), src, sc, q, 0, nrows, nrows, hist);
   stamp(p, 16);
-  if (nrows <= kMaxUnitTok) {
-    __syncthreads();
-#pragma unroll 1
-    for (int j = threadIdx.x; j < nrows; j += kThreads) {
-      const float x = sm.score[j];
-      __stcg(sc + j, x);
-      if (hist) atomicAdd(&th[float_key(x) >> (32 - kTauBits)], 1u);
-    }
-  }
   __syncthreads();
   return true;
 }
