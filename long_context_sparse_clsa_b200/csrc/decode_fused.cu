@@ -683,7 +683,6 @@ __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& 
 // ---------------------------------------------------------------------------
 __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, int P, uint32_t keff,
                                   uint32_t emax, uint32_t kmax) {
-  // Loops stay rolled: this runs once per call, so its code is fetched cold every time.
   if (kmax < emax) return false;
   for (int i = threadIdx.x; i < 4096; i += kThreads) sm.hist[i] = 0;
   if (threadIdx.x == 0) sm.list_n = 0;
@@ -692,9 +691,13 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
   int shift = 0;
   while (((kmax - emax) >> shift) >= 2048u) ++shift;
 #pragma unroll 1
-  for (int i = threadIdx.x; i < P; i += kThreads) {
-    const uint32_t k = skey[i];
-    if (k >= emax && k != 0u) atomicAdd(&sm.hist[(k - emax) >> shift], 1u);
+  for (int i0 = threadIdx.x; i0 < P; i0 += 8 * kThreads) {  // 8 keys loaded before any atomic
+    uint32_t k[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) k[u] = i0 + u * kThreads < P ? skey[i0 + u * kThreads] : 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (k[u] >= emax && k[u] != 0u) atomicAdd(&sm.hist[(k[u] - emax) >> shift], 1u);
   }
   __syncthreads();
   stamp(p, 19);
@@ -711,9 +714,13 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
     const int shift2 = max(0, shift - 11);
     uint32_t* hist2 = sm.hist + 2048;
 #pragma unroll 1
-    for (int i = threadIdx.x; i < P; i += kThreads) {
-      const uint32_t k = skey[i];
-      if (k >= loT && k <= hiT && k != 0u) atomicAdd(&hist2[(k - loT) >> shift2], 1u);
+    for (int i0 = threadIdx.x; i0 < P; i0 += 8 * kThreads) {
+      uint32_t k[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) k[u] = i0 + u * kThreads < P ? skey[i0 + u * kThreads] : 0u;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (k[u] >= loT && k[u] <= hiT && k[u] != 0u) atomicAdd(&hist2[(k[u] - loT) >> shift2], 1u);
     }
     __syncthreads();
     select_bin_wide(sm, hist2, 2048, need);
@@ -728,12 +735,17 @@ __device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t
   stamp(p, 21);
   // the keys of that bin (few) with their list positions
 #pragma unroll 1
-  for (int i = threadIdx.x; i < P; i += kThreads) {
-    const uint32_t k = skey[i];
-    if (k >= lo2 && k <= hi2 && k != 0u) {
-      const int q = atomicAdd(&sm.list_n, 1);
-      sm.list_key[q] = k;
-      sm.list_pos[q] = i;
+  for (int i0 = threadIdx.x; i0 < P; i0 += 8 * kThreads) {
+    uint32_t k[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) k[u] = i0 + u * kThreads < P ? skey[i0 + u * kThreads] : 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (k[u] >= lo2 && k[u] <= hi2 && k[u] != 0u) {
+        const int q = atomicAdd(&sm.list_n, 1);
+        sm.list_key[q] = k[u];
+        sm.list_pos[q] = i0 + u * kThreads;
+      }
     }
   }
   __syncthreads();
@@ -781,13 +793,24 @@ __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_
   uint32_t tot;
   uint32_t rank = block_scan((uint32_t)__popcll(sel), sm.warp_tot, &tot);
   int32_t* out = p.idx + (size_t)pl.b * p.k;
-  while (sel) {
-    const int bit = __ffsll((long long)sel) - 1;
-    sel &= sel - 1;
-    const int t = stok[a + bit];
-    if ((int)rank >= pl.tok0 && (int)rank < pl.tok1) sm.unit_tok[rank - pl.tok0] = t;
-    if (t >= pl.r0 && t < pl.r1 && (int)rank < pl.keff) out[rank] = t;
-    ++rank;
+  // 8 slots at a time: their tokens loaded together, each selected slot's rank from a
+  // popcount of the selected slots before it (no serial chain through the slots)
+#pragma unroll 1
+  for (int c0 = 0; c0 < run; c0 += 8) {
+    const uint32_t m8 = (uint32_t)(sel >> c0) & 0xffu;
+    if (m8 == 0u) continue;
+    int32_t t[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) t[u] = (m8 >> u) & 1u ? stok[a + c0 + u] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if ((m8 >> u) & 1u) {
+        const int r = (int)rank + __popc(m8 & ((1u << u) - 1u));
+        if (r >= pl.tok0 && r < pl.tok1) sm.unit_tok[r - pl.tok0] = t[u];
+        if (t[u] >= pl.r0 && t[u] < pl.r1 && r < pl.keff) out[r] = t[u];
+      }
+    }
+    rank += (uint32_t)__popc(m8);
   }
   __syncthreads();
 }
