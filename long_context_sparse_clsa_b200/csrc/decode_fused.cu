@@ -790,8 +790,10 @@ __device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_
     for (int u = 0; u < 8; ++u)
       if (k[u] > tk || (k[u] == tk && (uint32_t)(a + c0 + u) <= tp)) sel |= 1ull << (c0 + u);
   }
+  stamp(p, 25);
   uint32_t tot;
   uint32_t rank = block_scan((uint32_t)__popcll(sel), sm.warp_tot, &tot);
+  stamp(p, 26);
   int32_t* out = p.idx + (size_t)pl.b * p.k;
   // 8 slots at a time: their tokens loaded together, each selected slot's rank from a
   // popcount of the selected slots before it (no serial chain through the slots)
@@ -1132,15 +1134,19 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
   for (int i = threadIdx.x; i < nr * 32; i += kThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   __syncthreads();
   stamp(p, 17);
+  // per row: M, den, and each split's weight 2^(m - M) in place of its m
   #pragma unroll 1
   for (int ri = warp; ri < nr; ri += kWarps) {
     float M = -INFINITY, den = 0.f;
     #pragma unroll 1
     for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, sm.cm[ri * ns + s2]);
     M = warp_max(M);
-    if (M != -INFINITY)
-      #pragma unroll 1
-      for (int s2 = lane; s2 < ns; s2 += 32) den = fmaf(exp2f(sm.cm[ri * ns + s2] - M), sm.cl[ri * ns + s2], den);
+    #pragma unroll 1
+    for (int s2 = lane; s2 < ns; s2 += 32) {
+      const float wgt = M == -INFINITY ? 0.f : exp2f(sm.cm[ri * ns + s2] - M);
+      den = fmaf(wgt, sm.cl[ri * ns + s2], den);
+      sm.cm[ri * ns + s2] = wgt;
+    }
     den = warp_sum(den);
     if (lane == 0) {
       sm.rowM[ri] = M;
@@ -1157,12 +1163,13 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
     for (int ri = warp; ri < nr; ri += kWarps) {
       const int s_lo = max(0, t0 - ri * ns), s_hi = min(ns, t0 + nb - ri * ns);
       if (s_lo >= s_hi) continue;
-      const float M = sm.rowM[ri];
       float4 a = acc[ri * 32 + lane];
-      #pragma unroll 1
+      // the splits in order (a fixed summation order: deterministic); unrolled so the
+      // staged loads overlap
+      #pragma unroll 6
       for (int s2 = s_lo; s2 < s_hi; ++s2) {
         const int t = ri * ns + s2;
-        const float w = M == -INFINITY ? 0.f : exp2f(sm.cm[t] - M);
+        const float w = sm.cm[t];
         const float4 v = stg[(t - t0) * 32 + lane];
         a.x = fmaf(w, v.x, a.x);
         a.y = fmaf(w, v.y, a.y);
