@@ -252,11 +252,27 @@ def _prefill_check(w, rows):
     want, want_lse = O.prefill_attention(inp.Q, inp.K, inp.V, i_np[rows], c_np[rows], rows)
     got = tensor_f64(r["O"])[:, rows]
     assert max_abs(got, want) <= TOL[w.dtype]
+    got_lse = tensor_f64(r["lse"])[:, rows]
+    assert max_abs(got_lse, want_lse) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse).max())
 
 
 def test_prefill_small():
     w = scaled("prefill4k", n_max=3000, T=300, k=256, L=2)
     _prefill_check(w, list(range(300)))
+
+
+def test_prefill_all_rows_new():
+    """n = T: row i selects among i + 1 tokens (k_eff = 1, 2, ..., k): partial and single-token
+    chunks of the per-row attention; 20 (layer, head) rows per KV head (not a multiple of 32)."""
+    w = scaled("prefill4k", n_max=700, T=700, k=300, L=5)
+    _prefill_check(w, [0, 1, 2, 62, 63, 64, 65, 127, 128, 299, 300, 511, 699])
+
+
+def test_prefill_layer_groups():
+    """L*G = 180 > 128 rows per KV head: the attention runs in two layer groups of 23 layers
+    (92 rows; the second group's last layer slot is past L)."""
+    w = scaled("prefill4k", n_max=1500, T=200, k=160, L=45, Hq=16, Hkv=4)
+    _prefill_check(w, list(range(0, 200, 7)) + [199])
 
 
 def test_prefill_full_size_sampled():
