@@ -18,6 +18,11 @@ are:
 
 Each is argument marshalling around the C ABI: every step runs in the library's
 kernels, and the calls of one step go out back to back on one stream.
+
+``attention_mass`` is the pages' sparsity diagnostic (picx.dev CLSA summary, Attention
+Sparsity Analysis): the share of each (layer, query head)'s dense softmax mass that the
+shared selection S captures, sum_{j in S} softmax_j = exp(lse_S - lse_all), from the lse
+of the sparse attention over S and of the dense attention over the whole cache.
 """
 from __future__ import annotations
 
@@ -85,3 +90,20 @@ class StandardAttention:
                              O=self.O[l:l + 1], want_lse=False)
             n += clsa.last_launch_count()
         return n
+
+
+def attention_mass(Q, K, V, seq_lens, lse_sparse, scale: float = 0.0, ws=None):
+    """Share of the dense softmax mass on the selected rows, per (layer, sequence, head).
+
+    lse_sparse [L][B][Hq]: the lse the decode step returned (softmax over S); the dense
+    lse over every cached row comes from one clsa_sparse_attn call with the cache as
+    K_S/V_S.  Returns (mass [L][B][Hq] fp32, lse_all).  The pages' figure (~80 % at 2048 of
+    32K tokens) needs trained weights; on synthetic N(0, 1) inputs the indexer keys are
+    independent of K, so the share is close to |S| / n.
+    """
+    import torch
+    L, B, Hq, d = Q.shape
+    O = torch.empty_like(Q)
+    lse_all = torch.empty(L, B, Hq, dtype=torch.float32, device=Q.device)
+    clsa.sparse_attn(Q, K, V, seq_lens, scale, ws=ws, O=O, lse=lse_all)
+    return torch.exp(lse_sparse - lse_all), lse_all

@@ -8,7 +8,7 @@ import torch
 
 from oracle import clsa_oracle as O
 from long_context_sparse_clsa_b200 import clsa
-from long_context_sparse_clsa_b200.baselines import PerLayerRouting, StandardAttention, YocoDense
+from long_context_sparse_clsa_b200.baselines import PerLayerRouting, StandardAttention, YocoDense, attention_mass
 from long_context_sparse_clsa_b200.inputs import make_inputs, scaled
 from parity_util import check_near_tie_sets, max_abs, tensor_f64
 
@@ -88,3 +88,25 @@ def test_standard_attention_per_layer_caches():
     for l, x in enumerate(caches):
         want = _dense_oracle(caches[0].Q[l:l + 1], x.K, x.V, x.seq_lens)
         assert max_abs(got[l:l + 1], want) <= TOL[w.dtype]
+
+
+def test_attention_mass():
+    """The share of dense softmax mass on the selection, against the oracle's full softmax
+    summed over the GPU's selected rows (the pages' sparsity diagnostic)."""
+    w = scaled("decode32k", n_max=6000, k=500, L=2, plant=0.0)
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    r = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], w.k)
+    mass, _ = attention_mass(dv["Q"], dv["K"], dv["V"], dv["seq_lens"], r["lse"])
+    torch.cuda.synchronize()
+    got = mass.cpu().double().numpy()
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    Kf, Qf = inp.f32("K").astype(np.float64), inp.f32("Q").astype(np.float64)
+    n = int(inp.seq_lens[0])
+    for l in range(w.L):
+        for h in range(w.Hq):
+            g = h // (w.Hq // w.Hkv)
+            wts, _ = O.attention_weights(Qf[l, 0, h], Kf[0, :n, g])
+            want = wts[i_np[0, :c_np[0]]].sum()
+            assert abs(got[l, 0, h] - want) <= 1e-3 * max(1.0, want) + 2e-3
+    assert np.all((got > 0) & (got <= 1 + 1e-3))
