@@ -18,6 +18,9 @@ Once: Cross-Layer Sparse Attention with Shared Routing" (CLSA):
   Limits": ``Attn(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V`` (fixes the scale).
 * zhichai.net post, "CLSA: Sharing the Index Across Layers": the "Selector"
   gathers K/V rows by the shared index.
+* picx.dev summary, "Methodology > Architecture Overview", multi-layer
+  distillation: ``Abar = 1/(L H) sum_{l,h} softmax(Q^(l,h) K^(h)^T)`` and the
+  per-query term ``KL(sg[Abar_t] || softmax(I_t))`` (forward only).
 
 All floating arithmetic is float64 on inputs upcast from their storage values.
 Readings where the pages are silent (each also listed in the design doc):
@@ -32,6 +35,10 @@ Readings where the pages are silent (each also listed in the design doc):
   position t sees tokens j <= t (causal);
 * one S_t per query token, shared by every layer and every head;
 * GQA maps query head h to KV head h // (Hq / Hkv).
+* the distillation target averages the distributions the layers attend with, so
+  its softmax takes the attention scale 1/sqrt(d) (the printed formula omits any
+  scale); softmax(I_t) takes none (the routing equation has none); a decode query
+  sees all len_b cached tokens; 0 log 0 = 0.
 
 Pins (tests/test_oracle_pins.py) tie every function here to something other than
 itself: brute-force rank counting for TopK, torch's scaled_dot_product_attention
@@ -48,6 +55,7 @@ import numpy as np
 __all__ = [
     "index_scores", "topk_select", "gather_kv", "sparse_attention", "attention_weights",
     "decode_step", "prefill_scores", "prefill_topk", "prefill_attention", "prefill_chunk",
+    "distill_target",
 ]
 
 
@@ -248,3 +256,42 @@ def prefill_chunk(q_idx, k_idx, K, V, Q, n: int, k: int,
     idx, count = prefill_topk(q_idx, k_idx, n, k, rows)
     O, lse = prefill_attention(Q, K, V, idx, count, rows, scale)
     return {"idx": idx, "count": count, "O": O, "lse": lse}
+
+
+# --------------------------------------------------------------------------
+# distillation target of the shared indexer (forward only)
+# --------------------------------------------------------------------------
+
+def distill_target(Q, K, I, seq_lens, scale: Optional[float] = None):
+    """Per decode query b: Abar_b = mean over every (layer, query head) of that head's
+    softmax over the len_b cached tokens (query head h reads KV head h // (Hq / Hkv)),
+    and kl[b] = KL(Abar_b || softmax(I_b[:len_b])).
+
+    Q [L][B][Hq][d]; K [B][n_max][Hkv][d]; I [B][n_max] indexer scores.  Returns float64
+    (Abar [B][n_max] with zeros past len_b, kl [B]; a sequence with no tokens gets kl 0).
+    """
+    Qf, Kf = _f64(Q), _f64(K)
+    If = np.asarray(I, dtype=np.float64)
+    L, B, Hq, d = Qf.shape
+    Hkv = Kf.shape[2]
+    G = Hq // Hkv
+    n_max = Kf.shape[1]
+    Abar = np.zeros((B, n_max))
+    kl = np.zeros(B)
+    for b in range(B):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        acc = np.zeros(n)
+        for l in range(L):
+            for h in range(Hq):
+                w, _ = attention_weights(Qf[l, b, h], Kf[b, :n, h // G], scale)
+                acc += w
+        a = acc / (L * Hq)
+        Abar[b, :n] = a
+        z = If[b, :n]
+        log_p = z - (z.max() + math.log(np.exp(z - z.max()).sum()))  # log softmax(I_b)
+        nz = a > 0
+        kl[b] = float(np.sum(a[nz] * (np.log(a[nz]) - log_p[nz])))
+    return Abar, kl
+

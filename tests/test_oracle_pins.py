@@ -368,3 +368,62 @@ def test_inputs_are_deterministic_and_shaped():
         assert (r.K[bb, r.seq_lens[bb]:] == 0).all()
     v = a.f32("K").ravel()
     assert abs(v.mean()) < 0.01 and abs(v.std() - 1.0) < 0.01
+
+
+# ----------------------------------------------------------------------- distillation target
+
+def _softmax_t(x):
+    return torch.softmax(torch.as_tensor(x, dtype=torch.float64), dim=-1).numpy()
+
+
+def test_distill_single_head_is_that_heads_softmax():
+    """L = 1, one head: Abar is that head's attention distribution (torch's softmax of the
+    scaled scores over the valid rows), zero past len."""
+    rng = np.random.default_rng(11)
+    d, n_max, n = 16, 30, 23
+    Q = rng.normal(size=(1, 1, 1, d))
+    K = rng.normal(size=(1, n_max, 1, d))
+    I = rng.normal(size=(1, n_max))
+    A, _ = O.distill_target(Q, K, I, [n])
+    want = _softmax_t((K[0, :n, 0] @ Q[0, 0, 0]) / np.sqrt(d))
+    assert np.allclose(A[0, :n], want, rtol=1e-12, atol=1e-15)
+    assert np.all(A[0, n:] == 0.0)
+
+
+def test_distill_head_mapping_with_a_zero_kv_head():
+    """Hq = 4, Hkv = 2: query heads 2, 3 read KV head 1.  With KV head 1 all zeros their
+    distributions are uniform, so Abar = (softmax_h0 + softmax_h1 + 2 / n) / 4 with h0, h1
+    on KV head 0 (a mapping h % Hkv would put heads 1 and 3 on the zero head instead)."""
+    rng = np.random.default_rng(12)
+    d, n = 8, 17
+    Q = rng.normal(size=(1, 1, 4, d))
+    K = rng.normal(size=(1, n, 2, d))
+    K[:, :, 1] = 0.0
+    A, _ = O.distill_target(Q, K, rng.normal(size=(1, n)), [n])
+    s0 = _softmax_t((K[0, :, 0] @ Q[0, 0, 0]) / np.sqrt(d))
+    s1 = _softmax_t((K[0, :, 0] @ Q[0, 0, 1]) / np.sqrt(d))
+    assert np.allclose(A[0], (s0 + s1 + 2.0 / n) / 4.0, rtol=1e-12, atol=1e-15)
+
+
+def test_distill_kl_against_scipy_and_closed_forms():
+    """kl = KL(Abar || softmax(I)) equals scipy's entropy(Abar, softmax(I)); it is >= 0, and
+    0 when I = log Abar + c; Abar sums to 1 over each sequence's rows."""
+    from scipy.stats import entropy
+    rng = np.random.default_rng(13)
+    L, B, Hq, Hkv, d, n_max = 3, 3, 4, 2, 8, 40
+    Q = rng.normal(size=(L, B, Hq, d))
+    K = rng.normal(size=(B, n_max, Hkv, d))
+    I = 3.0 * rng.normal(size=(B, n_max))
+    lens = [40, 7, 0]
+    A, kl = O.distill_target(Q, K, I, lens)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert kl[b] == 0.0 and np.all(A[b] == 0.0)
+            continue
+        assert abs(A[b, :n].sum() - 1.0) < 1e-12 and np.all(A[b, n:] == 0.0)
+        assert kl[b] >= 0.0
+        assert abs(kl[b] - entropy(A[b, :n], _softmax_t(I[b, :n]))) < 1e-12
+    I2 = I.copy()
+    I2[0, :40] = np.log(A[0, :40]) + 5.0
+    _, kl2 = O.distill_target(Q, K, I2, lens)
+    assert abs(kl2[0]) < 1e-12
