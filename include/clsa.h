@@ -145,6 +145,25 @@ CLSA_API clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void
                              void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Distillation target of the shared indexer (forward only)                   */
+/* ------------------------------------------------------------------------ */
+/* picx.dev CLSA summary, Methodology > Architecture Overview, multi-layer
+ * distillation: for each decode query b,
+ *   Abar_b = 1/(L Hq) sum_{l,h} softmax(Q^(l)[b,h] K[b]^T * scale)  over its len_b rows
+ *   kl[b]  = KL(Abar_b || softmax(I_b)),   I = the indexer scores (no scale)
+ * Query head h reads KV head h / (Hq / Hkv); scale <= 0 selects 1/sqrt(d).
+ * Q [L][B][Hq][d] and K [B][n_max][Hkv][d] in dt; scores [B][n_max] fp32 (e.g. from
+ * clsa_index_scores); seq_lens [B] device int32.  abar [B][n_max] fp32 out (0 past
+ * len_b), may be NULL; kl [B] fp32 out (0 for an empty sequence).  1 <= n_max <= 2^24.
+ * fp32 arithmetic; the result is deterministic (fixed reduction orders).
+ * Caller-owned workspace of clsa_distill_workspace_size bytes; errors as above. */
+CLSA_API size_t clsa_distill_workspace_size(int B, int n_max, int L, int Hq, int Hkv, int d);
+CLSA_API clsa_status clsa_distill_target(const void* Q, const void* K, const float* scores,
+                             const int32_t* seq_lens, int B, int n_max, int L, int Hq, int Hkv,
+                             int d, float scale, clsa_dtype dt, float* abar, float* kl, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* One decode step: score once, select once, gather once, attend in L layers */
 /* ------------------------------------------------------------------------ */
 typedef struct clsa_decode_args {

@@ -26,6 +26,7 @@ EXPORTS = [
     "clsa_index_scores", "clsa_topk_workspace_size", "clsa_topk", "clsa_topk_noalloc",
     "clsa_gather_kv_workspace_size",
     "clsa_gather_kv", "clsa_sparse_attn_workspace_size", "clsa_sparse_attn",
+    "clsa_distill_workspace_size", "clsa_distill_target",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
     "clsa_prefill_chunk", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
     "clsa_version", "clsa_last_launch_count",
@@ -80,6 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_sparse_attn_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
         "clsa_sparse_attn": (S, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp,
                                  _sz, _vp]),
+        "clsa_distill_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+        "clsa_distill_target": (S, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
         "clsa_decode_workspace_size": (_sz, [ctypes.POINTER(DecodeArgs)]),
         "clsa_decode_step": (S, [ctypes.POINTER(DecodeArgs), _vp, _sz, _vp]),
         "clsa_prefill_workspace_size": (_sz, [ctypes.POINTER(PrefillArgs)]),
@@ -232,6 +235,21 @@ def decode_args(q_idx, k_idx, K, V, Q, seq_lens, k, O, idx, count, scores=None, 
 
 def decode_workspace_size(args: DecodeArgs) -> int:
     return load_library().clsa_decode_workspace_size(ctypes.byref(args))
+
+
+def distill_target(Q, K, scores, seq_lens, scale: float = 0.0, ws: Optional[Workspace] = None,
+                   want_abar: bool = True):
+    """Distillation target (forward): Abar [B][n_max] (or None) and kl [B] (see clsa.h)."""
+    lib = load_library()
+    L, B, Hq, d = Q.shape
+    _, n_max, Hkv, _ = K.shape
+    need = lib.clsa_distill_workspace_size(B, n_max, L, Hq, Hkv, d)
+    ws = (ws or Workspace(need)).ensure(need)
+    abar = torch.empty(B, n_max, dtype=torch.float32, device=Q.device) if want_abar else None
+    kl = torch.empty(B, dtype=torch.float32, device=Q.device)
+    _check(lib.clsa_distill_target(_p(Q), _p(K), _p(scores), _p(seq_lens), B, n_max, L, Hq, Hkv, d, scale, _dt(Q),
+                                   _p(abar), _p(kl), ws.ptr, ws.nbytes, _stream()), "clsa_distill_target")
+    return abar, kl, ws
 
 
 def decode_step_args(args: DecodeArgs, ws: Workspace, stream=None):

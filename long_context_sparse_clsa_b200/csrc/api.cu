@@ -1,6 +1,7 @@
 // C ABI of libclsa.so: argument validation, workspace layout and launch order.
 // The operations are defined in include/clsa.h; every step of the path runs in
 // the kernels of this directory.
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -227,6 +228,29 @@ clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void* V_S, co
   char* w = static_cast<char*>(ws);
   return from_cuda(launch_sparse_attn(sh, Q, K_S, V_S, nullptr, count, resolve_scale(scale, d), O, lse, w,
                                       w + kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
+size_t clsa_distill_workspace_size(int B, int n_max, int L, int Hq, int Hkv, int d) {
+  if (check_attn(B, n_max, L, Hq, Hkv, d, CLSA_BF16, kMaxDirectK) != CLSA_OK) return 0;
+  return kWsHeader + std::max(distill_ws_bytes(B, n_max, L, Hq, Hkv, d, CLSA_BF16),
+                              distill_ws_bytes(B, n_max, L, Hq, Hkv, d, CLSA_F32));
+}
+
+clsa_status clsa_distill_target(const void* Q, const void* K, const float* scores, const int32_t* seq_lens, int B,
+                                int n_max, int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* abar,
+                                float* kl, void* ws, size_t ws_bytes, void* stream) {
+  CallScope scope;
+  clsa_status st = check_attn(B, n_max, L, Hq, Hkv, d, dt, kMaxDirectK);
+  if (st != CLSA_OK) return st;
+  if (!Q || !K || !scores || !seq_lens || !kl) return CLSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned4(scores) || !aligned4(seq_lens) || !aligned4(kl) ||
+      (abar && !aligned4(abar)))
+    return CLSA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < clsa_distill_workspace_size(B, n_max, L, Hq, Hkv, d) || !aligned16(ws))
+    return CLSA_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  return from_cuda(launch_distill(Q, K, scores, seq_lens, B, n_max, L, Hq, Hkv, d, resolve_scale(scale, d), dt, abar,
+                                  kl, w, w + kWsHeader, static_cast<cudaStream_t>(stream)));
 }
 
 size_t clsa_decode_workspace_size(const clsa_decode_args* a) {

@@ -63,6 +63,12 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
                                const int32_t* idx, const int32_t* count, float scale, void* O, float* lse,
                                void* ws_header, void* attn_ws, cudaStream_t s);
 
+// ----- distillation target (forward): Abar and KL(Abar || softmax(I)) ----------------
+size_t distill_ws_bytes(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dtype dt);
+cudaError_t launch_distill(const void* Q, const void* K, const float* scores, const int32_t* lens, int B, int n_max,
+                           int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* abar, float* kl,
+                           void* ws_header, void* ws, cudaStream_t s);
+
 // ----- fused decode step (one cooperative launch) -------------------------------
 bool fused_decode_supported(const clsa_decode_args* a);
 size_t fused_decode_ws_bytes(const clsa_decode_args* a);

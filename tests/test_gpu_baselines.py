@@ -110,3 +110,35 @@ def test_attention_mass():
             want = wts[i_np[0, :c_np[0]]].sum()
             assert abs(got[l, 0, h] - want) <= 1e-3 * max(1.0, want) + 2e-3
     assert np.all((got > 0) & (got <= 1 + 1e-3))
+
+
+@pytest.mark.parametrize("case", ["bf16_d128", "f32_d64_ragged"])
+def test_distill_target(case):
+    """Abar (the layer/head-averaged attention over the cache) and KL(Abar || softmax(I))
+    against the oracle, on the GPU's own indexer scores."""
+    if case == "bf16_d128":
+        w = scaled("decode32k", n_max=3000 + 17, k=16, L=2, plant=0.0)
+    else:
+        w = scaled("ragged16", B=3, n_max=1500, lens=(0, 1500), k=16, L=3, Hq=8, Hkv=2, d=64, d_idx=64,
+                   dtype="f32", plant=0.0, seed=4)
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    if w.B > 1:  # one empty sequence
+        inp.seq_lens[1] = 0
+        dv["seq_lens"][1] = 0
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    abar, kl, ws = clsa.distill_target(dv["Q"], dv["K"], sc, dv["seq_lens"])
+    torch.cuda.synchronize()
+    assert ws.status()[0] == "CLSA_OK"
+    I = tensor_f64(sc)
+    want_a, want_kl = O.distill_target(inp.Q, inp.K, I, inp.seq_lens)
+    got_a, got_kl = tensor_f64(abar), tensor_f64(kl)
+    for b, n in enumerate(inp.seq_lens):
+        n = int(n)
+        assert np.all(got_a[b, n:] == 0.0)
+        if n == 0:
+            assert got_kl[b] == 0.0
+            continue
+        assert np.max(np.abs(got_a[b, :n] - want_a[b, :n])) <= 1e-4 * np.max(want_a[b, :n])
+        assert abs(got_a[b, :n].sum() - 1.0) < 1e-4
+        assert abs(got_kl[b] - want_kl[b]) <= 1e-4 * max(1.0, abs(want_kl[b]))
