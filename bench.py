@@ -5,7 +5,7 @@ L-layer sparse GQA attention) on B200.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode128k]
                     [--impl {clsa,reference}] [--no-graph] [--no-cpu-baseline]
                     [--l2 {rotate,flush}] [--sets R]
-                    [--variant {clsa,per_layer_routing,yoco_dense,standard}]
+                    [--variant {clsa,per_layer_routing,yoco_dense,standard,distill_target}]
 
 One JSON line on rank 0.  A step is one decode token per sequence through the
 whole path; the default workload is the 128K-context decode (batch 1, n=131072,
@@ -54,7 +54,7 @@ def parse():
                     help="between steps: rotate through input sets larger than L2 (default), or flush L2")
     ap.add_argument("--sets", type=int, default=6, help="input sets rotated through (--l2 rotate)")
     ap.add_argument("--variant", default="clsa",
-                    choices=["clsa", "per_layer_routing", "yoco_dense", "standard"],
+                    choices=["clsa", "per_layer_routing", "yoco_dense", "standard", "distill_target"],
                     help="a comparison system built from the library's calls (one GPU; not the default line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-steps", type=int, default=2)
@@ -483,6 +483,24 @@ def run_clsa(args):
     print(json.dumps(line), flush=True)
 
 
+class _DistillStep:
+    """The distillation target as one timed step (preallocated outputs and workspace)."""
+
+    def __init__(self, Q, K, scores, seq_lens):
+        from long_context_sparse_clsa_b200 import clsa
+        import torch
+        self.args = (Q, K, scores, seq_lens)
+        L, B, Hq, d = Q.shape
+        self.ws = clsa.Workspace(clsa.load_library().clsa_distill_workspace_size(B, K.shape[1], L, Hq, K.shape[2], d))
+        self.abar = torch.empty(B, K.shape[1], dtype=torch.float32, device=Q.device)
+        self.kl = torch.empty(B, dtype=torch.float32, device=Q.device)
+
+    def step(self) -> int:
+        from long_context_sparse_clsa_b200 import clsa
+        clsa.distill_target(*self.args, ws=self.ws, abar=self.abar, kl=self.kl)
+        return clsa.last_launch_count()
+
+
 def run_variant(args):
     """Time a comparison system of the pages' ablation (per-layer routing, YOCO only,
     standard attention) on the same workload, built from the library's own calls."""
@@ -529,6 +547,12 @@ def run_variant(args):
         sysm = baselines.YocoDense(dv["K"], dv["V"], dv["Q"], dv["seq_lens"], Ob)
         step_bytes_ = 2 * sum(lens) * Hkv * d * eb + qo_bytes
         note = "every layer dense over the one shared cache (one call, the L*G rows of a head read each row once)"
+    elif args.variant == "distill_target":
+        sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+        sysm = _DistillStep(dv["Q"], dv["K"], sc, dv["seq_lens"])
+        # the two passes each stream the cache (K) once; I read and Abar written once
+        step_bytes_ = 2 * sum(lens) * Hkv * d * eb + 2 * sum(lens) * 4 + qo_bytes // 2
+        note = "Abar and KL(Abar || softmax(I)) over the whole cache: row lse pass + Abar pass (K read twice)"
     else:
         Ks = [dv["K"]] + [permuted(dv["K"]) for _ in range(L - 1)]
         Vs = [dv["V"]] + [permuted(dv["V"]) for _ in range(L - 1)]

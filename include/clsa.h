@@ -155,7 +155,9 @@ CLSA_API clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void
  * Q [L][B][Hq][d] and K [B][n_max][Hkv][d] in dt; scores [B][n_max] fp32 (e.g. from
  * clsa_index_scores); seq_lens [B] device int32.  abar [B][n_max] fp32 out (0 past
  * len_b), may be NULL; kl [B] fp32 out (0 for an empty sequence).  1 <= n_max <= 2^24.
- * fp32 arithmetic; the result is deterministic (fixed reduction orders).
+ * fp32 arithmetic; the result is deterministic (fixed reduction orders).  bf16 with
+ * d = 128 runs on the tensor cores (bf16 products, fp32 sums): two streaming passes over
+ * K (row lse, then Abar), 4 launches; other shapes run on CUDA cores.
  * Caller-owned workspace of clsa_distill_workspace_size bytes; errors as above. */
 CLSA_API size_t clsa_distill_workspace_size(int B, int n_max, int L, int Hq, int Hkv, int d);
 CLSA_API clsa_status clsa_distill_target(const void* Q, const void* K, const float* scores,

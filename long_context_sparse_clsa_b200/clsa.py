@@ -238,15 +238,18 @@ def decode_workspace_size(args: DecodeArgs) -> int:
 
 
 def distill_target(Q, K, scores, seq_lens, scale: float = 0.0, ws: Optional[Workspace] = None,
-                   want_abar: bool = True):
-    """Distillation target (forward): Abar [B][n_max] (or None) and kl [B] (see clsa.h)."""
+                   want_abar: bool = True, abar=None, kl=None):
+    """Distillation target (forward): Abar [B][n_max] (or None) and kl [B] (see clsa.h).
+    abar / kl: optional preallocated outputs (fp32 [B][n_max] / [B])."""
     lib = load_library()
     L, B, Hq, d = Q.shape
     _, n_max, Hkv, _ = K.shape
     need = lib.clsa_distill_workspace_size(B, n_max, L, Hq, Hkv, d)
     ws = (ws or Workspace(need)).ensure(need)
-    abar = torch.empty(B, n_max, dtype=torch.float32, device=Q.device) if want_abar else None
-    kl = torch.empty(B, dtype=torch.float32, device=Q.device)
+    if abar is None and want_abar:
+        abar = torch.empty(B, n_max, dtype=torch.float32, device=Q.device)
+    if kl is None:
+        kl = torch.empty(B, dtype=torch.float32, device=Q.device)
     _check(lib.clsa_distill_target(_p(Q), _p(K), _p(scores), _p(seq_lens), B, n_max, L, Hq, Hkv, d, scale, _dt(Q),
                                    _p(abar), _p(kl), ws.ptr, ws.nbytes, _stream()), "clsa_distill_target")
     return abar, kl, ws

@@ -1,5 +1,6 @@
 // Distillation target of the shared indexer, forward only (picx.dev CLSA summary,
-// Methodology > Architecture Overview, multi-layer distillation):
+// Methodology > Architecture Overview, multi-layer distillation).  bf16 with d = 128 runs
+// the tcgen05 path of distill_tc.cu; this file is the path for the other shapes:
 //   Abar_b = 1/(L Hq) sum_{l,h} softmax(Q^(l)[b,h] K[b]^T * scale)   over the len_b rows
 //   kl[b]  = KL(Abar_b || softmax(I_b))
 // with query head h reading KV head h / G, the attention scale of the layers, and no scale
@@ -15,6 +16,7 @@
 //    for the tile and its KL terms Abar (log Abar - (I - lse_I)) are summed into one
 //    partial per tile.
 // 4. kl_kernel: each sequence's tile partials in tile order (deterministic).
+#include <algorithm>
 #include <cmath>
 
 #include "common.cuh"
@@ -191,12 +193,15 @@ size_t distill_ws_bytes(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dt
   off += align_up((size_t)B * 4, 256);                                       // lse of I
   off += align_up((size_t)B * ntiles * 4, 256);                              // tile partials
   off += attn_ws_bytes(sh);
+  if (distill_tc_supported(B, n_max, L, Hq, Hkv, d, dt)) off = std::max(off, distill_tc_ws_bytes(B, n_max, L, Hq, Hkv));
   return off;
 }
 
 cudaError_t launch_distill(const void* Q, const void* K, const float* scores, const int32_t* lens, int B, int n_max,
                            int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* abar, float* kl,
                            void* ws_header, void* ws, cudaStream_t s) {
+  if (distill_tc_supported(B, n_max, L, Hq, Hkv, d, dt))
+    return launch_distill_tc(Q, K, scores, lens, B, n_max, L, Hq, Hkv, scale, abar, kl, ws_header, ws, s);
   const int ntiles = (n_max + kTileTok - 1) / kTileTok;
   char* w = static_cast<char*>(ws);
   void* O = w;

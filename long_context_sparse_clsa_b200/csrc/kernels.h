@@ -68,6 +68,12 @@ size_t distill_ws_bytes(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dt
 cudaError_t launch_distill(const void* Q, const void* K, const float* scores, const int32_t* lens, int B, int n_max,
                            int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* abar, float* kl,
                            void* ws_header, void* ws, cudaStream_t s);
+// tcgen05 path (bf16, d = 128, G <= 128): two streaming passes over the cache
+bool distill_tc_supported(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dtype dt);
+size_t distill_tc_ws_bytes(int B, int n_max, int L, int Hq, int Hkv);
+cudaError_t launch_distill_tc(const void* Q, const void* K, const float* scores, const int32_t* lens, int B, int n_max,
+                              int L, int Hq, int Hkv, float scale, float* abar, float* kl, void* ws_header, void* ws,
+                              cudaStream_t s);
 
 // ----- fused decode step (one cooperative launch) -------------------------------
 bool fused_decode_supported(const clsa_decode_args* a);

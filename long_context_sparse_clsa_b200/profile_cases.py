@@ -3,7 +3,7 @@
     python -m long_context_sparse_clsa_b200.profile_cases --stage decode_step \
         [--workload decode128k] [--reps 3] [--batch B] [--rows T]
 
-Stages: index_scores, topk, gather_kv, sparse_attn, decode_step, prefill_chunk.
+Stages: index_scores, topk, gather_kv, sparse_attn, decode_step, prefill_chunk, distill_target.
 Inputs are the seeded synthetic workloads of ``inputs.py``; ``--batch`` replaces
 the workload's batch (decode only).  Each stage runs once untimed and then
 ``--reps`` times, with a synchronize at the end and nothing else on the GPU.
@@ -21,7 +21,7 @@ from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs, replace
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--stage", required=True, choices=["index_scores", "topk", "gather_kv", "sparse_attn",
-                                                       "decode_step", "prefill_chunk"])
+                                                       "decode_step", "prefill_chunk", "distill_target"])
     ap.add_argument("--workload", default="decode128k")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=0)
@@ -40,6 +40,7 @@ def main():
         sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
         idx, cnt = clsa.topk(sc, dv["seq_lens"], w.k)
         KS, VS = clsa.gather_kv(dv["K"], dv["V"], idx, cnt)
+        dws = clsa.Workspace(clsa.load_library().clsa_distill_workspace_size(w.B, w.n_max, w.L, w.Hq, w.Hkv, w.d))
         fns = {
             "index_scores": lambda: clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"], sc),
             "topk": lambda: clsa.topk(sc, dv["seq_lens"], w.k, idx=idx, count=cnt),
@@ -47,6 +48,7 @@ def main():
             "sparse_attn": lambda: clsa.sparse_attn(dv["Q"], KS, VS, cnt),
             "decode_step": lambda: clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"],
                                                     dv["seq_lens"], w.k),
+            "distill_target": lambda: clsa.distill_target(dv["Q"], dv["K"], sc, dv["seq_lens"], ws=dws),
         }
         fn = fns[a.stage]
     fn()

@@ -112,20 +112,35 @@ def test_attention_mass():
     assert np.all((got > 0) & (got <= 1 + 1e-3))
 
 
-@pytest.mark.parametrize("case", ["bf16_d128", "f32_d64_ragged"])
+DISTILL_CASES = {
+    # (workload, explicit seq_lens or None)
+    "bf16_d128": (scaled("decode32k", n_max=3000 + 17, k=16, L=2, plant=0.0), None),
+    # rows = L G = 12 per KV head: the MMA's N rounds up to 16 (the 16-column tail)
+    "bf16_rows12": (scaled("ragged16", B=2, n_max=2000, lens=(1999, 2000), k=16, L=3, Hq=8, Hkv=2, d=128,
+                           d_idx=128, plant=0.0, seed=6), (1999, 2000)),
+    # G = 32, L = 5: two layer groups (128 and 32 rows); an empty sequence; ragged tails
+    "bf16_groups_ragged": (scaled("ragged16", B=3, n_max=9000, lens=(4097, 9000), k=16, L=5, Hq=32, Hkv=1,
+                                  d=128, d_idx=128, plant=0.0, seed=8), (9000, 0, 4097)),
+    "f32_d64_ragged": (scaled("ragged16", B=3, n_max=1500, lens=(0, 1500), k=16, L=3, Hq=8, Hkv=2, d=64, d_idx=64,
+                              dtype="f32", plant=0.0, seed=4), (None, 0, None)),
+    # the full decode workload (131072 cached rows, 24 layers x 32 heads)
+    "bf16_decode128k": (scaled("decode128k"), None),
+}
+
+
+@pytest.mark.parametrize("case", list(DISTILL_CASES))
 def test_distill_target(case):
     """Abar (the layer/head-averaged attention over the cache) and KL(Abar || softmax(I))
-    against the oracle, on the GPU's own indexer scores."""
-    if case == "bf16_d128":
-        w = scaled("decode32k", n_max=3000 + 17, k=16, L=2, plant=0.0)
-    else:
-        w = scaled("ragged16", B=3, n_max=1500, lens=(0, 1500), k=16, L=3, Hq=8, Hkv=2, d=64, d_idx=64,
-                   dtype="f32", plant=0.0, seed=4)
+    against the oracle, on the GPU's own indexer scores.  bf16 with d = 128 runs the
+    tensor-core passes, fp32 the CUDA-core path."""
+    w, lens = DISTILL_CASES[case]
     inp = make_inputs(w)
     dv = clsa.to_device(inp)
-    if w.B > 1:  # one empty sequence
-        inp.seq_lens[1] = 0
-        dv["seq_lens"][1] = 0
+    if lens is not None:
+        for b, n in enumerate(lens):
+            if n is not None:
+                inp.seq_lens[b] = n
+                dv["seq_lens"][b] = n
     sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
     abar, kl, ws = clsa.distill_target(dv["Q"], dv["K"], sc, dv["seq_lens"])
     torch.cuda.synchronize()
