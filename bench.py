@@ -299,7 +299,7 @@ def run_clsa(args):
     step()
     torch.cuda.synchronize()
     launches_per_step = clsa.last_launch_count()
-    graphs = None
+    graphs = round_graph = None
     if not args.no_graph:
         try:
             s2 = torch.cuda.Stream()
@@ -314,9 +314,15 @@ def run_clsa(args):
                 with torch.cuda.graph(g):
                     step(r)
                 graphs.append(g)
+            # the R steps of one rotation in one graph: consecutive steps keep the launch's
+            # programmatic serialization (the next step's launch overlaps this one's run)
+            round_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(round_graph):
+                for r in range(R):
+                    step(r)
             torch.cuda.synchronize()
         except Exception as ex:  # graph capture unsupported: time eager launches
-            graphs = None
+            graphs = round_graph = None
             print(f"# graph capture failed, timing eager launches: {ex}", file=sys.stderr)
 
     def run_step(i):
@@ -325,9 +331,22 @@ def run_clsa(args):
         else:
             step(i % R)
 
+    def run_steps(n):
+        """n steps, set i % R for step i: whole rotations from the R-step graph"""
+        i = 0
+        if graphs is not None:
+            while n - i >= R:
+                round_graph.replay()
+                i += R
+        while i < n:
+            run_step(i)
+            i += 1
+
     for i in range(max(args.warmup, 3, R)):
         between_steps()
         run_step(i)
+    if round_graph is not None and args.l2 == "rotate":
+        round_graph.replay()  # the first replay uploads the graph
     torch.cuda.synchronize()
 
     def barrier():
@@ -343,8 +362,7 @@ def run_clsa(args):
         if args.l2 == "rotate":
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for i in range(args.steps):
-                run_step(i)
+            run_steps(args.steps)
             e1.record(stream)
             torch.cuda.synchronize()
             total_ms = e0.elapsed_time(e1)
@@ -467,7 +485,8 @@ def run_clsa(args):
                           f"permutations of the seeded cache), step i uses set i % {R}; no flush"
                           if args.l2 == "rotate" else
                           "flushed before every step (512 MiB write + read-back, outside the timed events)"),
-                   "launch": "cuda graph" if graphs is not None else "eager"},
+                   "launch": (f"cuda graph ({R} steps per graph, one per input set)" if graphs is not None and
+                              args.l2 == "rotate" else "cuda graph" if graphs is not None else "eager")},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": dom_bytes, "us_per_launch": dom_us},

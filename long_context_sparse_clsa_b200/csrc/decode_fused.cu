@@ -1207,6 +1207,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + align_up(sizeof(Smem), 128));
   unsigned char* big = smem + align_up(sizeof(Smem), 128) + kSmemQ;
 
+  // launched with programmatic stream serialization: wait until the previous grid on the
+  // stream has completed and its memory is visible (a no-op otherwise), then let the next
+  // one be scheduled
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   stamp(p, 0);
   // One sequence: CTA c's slice is [c chunk, c chunk + chunk) with chunk = ceil(len /
   // gridDim.x) (what make_plan gives for B = 1), so every thread starts the K_idx stream
@@ -1431,6 +1436,37 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   return off;
 }
 
+// Cooperative launch with programmatic stream serialization: the launch of the next step
+// may be processed while this one runs (its CTAs wait at griddepcontrol.wait before any
+// work), which hides the launch latency between back-to-back steps.  Falls back to the
+// plain cooperative launch where the runtime refuses the pair of attributes.
+template <int DIDX>
+cudaError_t launch_fused(const FusedParams& p, int ncta, size_t smem, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<DIDX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  static bool pdl_ok = true;
+  if (pdl_ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ncta);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<DIDX>, p);
+    if (e != cudaErrorNotSupported && e != cudaErrorInvalidValue) return e;
+    (void)cudaGetLastError();
+    pdl_ok = false;
+  }
+  void* args[] = {(void*)&p};
+  return cudaLaunchCooperativeKernel((const void*)decode_fused_kernel<DIDX>, dim3(ncta), dim3(kThreads), args, smem, s);
+}
+
 cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws_header, void* ws_body,
                                 cudaStream_t s) {
   const FusedCfg cfg = fused_cfg();
@@ -1474,19 +1510,7 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   w += align_up((size_t)cfg.ncta * p.rows * kD * 4, 256);
   p.Ml = reinterpret_cast<float*>(w);
   const size_t smem = smem_bytes();
-  void* args[] = {(void*)&p};
-  cudaError_t e;
-  if (a->d_idx == 128) {
-    e = cudaFuncSetAttribute(decode_fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaLaunchCooperativeKernel((const void*)decode_fused_kernel<128>, dim3(cfg.ncta), dim3(kThreads), args,
-                                      smem, s);
-  } else {
-    e = cudaFuncSetAttribute(decode_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaLaunchCooperativeKernel((const void*)decode_fused_kernel<64>, dim3(cfg.ncta), dim3(kThreads), args,
-                                      smem, s);
-  }
+  const cudaError_t e = a->d_idx == 128 ? launch_fused<128>(p, cfg.ncta, smem, s) : launch_fused<64>(p, cfg.ncta, smem, s);
   launches_add(1);
   return e;
 }
