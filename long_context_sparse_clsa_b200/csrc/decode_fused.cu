@@ -1210,8 +1210,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   // launched with programmatic stream serialization: wait until the previous grid on the
   // stream has completed and its memory is visible (a no-op otherwise), then let the next
   // one be scheduled
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_enter();
   stamp(p, 0);
   // One sequence: CTA c's slice is [c chunk, c chunk + chunk) with chunk = ceil(len /
   // gridDim.x) (what make_plan gives for B = 1), so every thread starts the K_idx stream

@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kDThreads, 2)
   unsigned char* sK = base + kTileB;            // [kRing][2 atoms][128 tokens][128 B]
   DTSmem& sm = *reinterpret_cast<DTSmem*>(sK + kRing * kTileB);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_enter();
 
   // unit -> (b, g, layer group, split)
   int u = blockIdx.x;
@@ -337,6 +338,7 @@ __global__ void __launch_bounds__(kFinalT) distill_final_kernel(const float* __r
                                                                 float* __restrict__ tpart, int nt) {
   __shared__ float red[3][kFinalT / 32];
   __shared__ float smax;
+  pdl_enter();
   const int b = blockIdx.y, t = blockIdx.x;
   const int j = t * kFinalT + threadIdx.x;
   const int n = max(0, min(lens[b], n_max));
@@ -391,6 +393,7 @@ constexpr int kKlT = 256;
 __global__ void __launch_bounds__(kKlT) distill_kl_kernel(const float* __restrict__ tpart, int nt,
                                                          float* __restrict__ kl) {
   __shared__ float red[4][kKlT / 32];
+  pdl_enter();
   const int b = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float X = 0.f, S = 0.f, m = -INFINITY, e = 0.f;
   for (int t = threadIdx.x; t < nt; t += kKlT) {
@@ -490,11 +493,14 @@ cudaError_t launch_distill_tc(const void* Q, const void* K, const float* scores,
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(distill_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDTSmemBytes);
   if (e != cudaSuccess) return e;
-  distill_tc_kernel<1><<<pl.units, kDThreads, kDTSmemBytes, s>>>(tk, p);
-  distill_tc_kernel<2><<<pl.units, kDThreads, kDTSmemBytes, s>>>(tk, p);
-  distill_final_kernel<<<dim3(pl.nt, B), kFinalT, 0, s>>>(tokpart, scores, lens, n_max, pl.HG,
-                                                          1.f / (float)(L * Hq), abar, tpart, pl.nt);
-  distill_kl_kernel<<<B, kKlT, 0, s>>>(tpart, pl.nt, kl);
+  // each kernel waits at entry for the one before it (pdl_enter): launches overlap, work does not
+  e = launch_pdl(distill_tc_kernel<1>, dim3(pl.units), dim3(kDThreads), kDTSmemBytes, s, tk, p);
+  if (e == cudaSuccess) e = launch_pdl(distill_tc_kernel<2>, dim3(pl.units), dim3(kDThreads), kDTSmemBytes, s, tk, p);
+  if (e == cudaSuccess)
+    e = launch_pdl(distill_final_kernel, dim3(pl.nt, B), dim3(kFinalT), 0, s, (const float*)tokpart, scores, lens,
+                   n_max, pl.HG, 1.f / (float)(L * Hq), abar, tpart, pl.nt);
+  if (e == cudaSuccess) e = launch_pdl(distill_kl_kernel, dim3(B), dim3(kKlT), 0, s, (const float*)tpart, pl.nt, kl);
+  if (e != cudaSuccess) return e;
   launches_add(4);
   return cudaGetLastError();
 }
