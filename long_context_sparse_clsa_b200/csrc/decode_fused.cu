@@ -458,18 +458,24 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
   cp_async_wait<0>();
 }
 
+// this thread's 16-byte chunk of q_idx[b] (the chunk its scan lane multiplies)
+template <int DIDX>
+__device__ __forceinline__ uint4 load_q_chunk(const FusedParams& p, int b) {
+  return *reinterpret_cast<const uint4*>(p.q_idx + (size_t)b * DIDX + (threadIdx.x % (DIDX / 8)) * 8);
+}
+
+// started: the stream was begun by scan_start at entry, and qv holds load_q_chunk of the
+// sequence (both issued before the plan, so their latency overlaps it)
 template <int DIDX>
 __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigned char* ring, bool hist,
-                           bool started) {
+                           bool started, uint4 qv) {
   const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
   float* sc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
-  constexpr int LPR = DIDX / 8;
-  const int sub = threadIdx.x % LPR;
   float q[8];
   {
-    const uint4 qv = *reinterpret_cast<const uint4*>(p.q_idx + (size_t)pl.b * DIDX + sub * 8);
+    if (!started) qv = load_q_chunk<DIDX>(p, pl.b);
     unpack_bf16x2(qv.x, q[0], q[1]);
     unpack_bf16x2(qv.y, q[2], q[3]);
     unpack_bf16x2(qv.z, q[4], q[5]);
@@ -1217,12 +1223,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   // before the plan exists; the plan is checked against it below.
   int pre_r0 = 0, pre_r1 = 0;
   bool pre = false;
+  uint4 pre_q = make_uint4(0, 0, 0, 0);
   if (p.B == 1) {
     const int len = max(0, min(p.seq_lens[0], p.n_max));
     if (len > 0) {
       const int chunk = (len + (int)gridDim.x - 1) / (int)gridDim.x;
       pre_r0 = min(len, (int)blockIdx.x * chunk);
       pre_r1 = min(len, pre_r0 + chunk);
+      pre_q = load_q_chunk<DIDX>(p, 0);  // ahead of the K_idx stream (it would queue behind it)
       scan_start<DIDX>(reinterpret_cast<uint4*>(big), p.k_idx + (size_t)pre_r0 * DIDX, 0, pre_r1 - pre_r0);
       pre = true;
     }
@@ -1270,7 +1278,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
 
   const bool all_sel = pl.keff == pl.len;
   stamp(p, 23);
-  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel, pre)) return;
+  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel, pre, pre_q)) return;
   if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQa);  // lands during the selection
   stamp(p, 1);
 
