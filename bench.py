@@ -187,20 +187,10 @@ def time_oracle(inp, w, steps: int):
 
 # ------------------------------------------------------------------ main paths
 
-def dist_init(n_gpus):
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    return rank, world, local
-
-
 def run_reference(args):
-    rank, world, _ = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
-    if rank != 0:
+    from long_context_sparse_clsa_b200 import replicas
+    rank, world, _ = replicas.env_ranks()
+    if rank != 0:  # rank 0 alone times the oracle; the other ranks exit without work
         return
     from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs
     w = WORKLOADS[args.workload]
@@ -222,14 +212,13 @@ def run_reference(args):
 
 def run_clsa(args):
     import torch
-    rank, world, local = dist_init(args.gpus)
+    from long_context_sparse_clsa_b200 import replicas
+    rank, world, local = replicas.init("nccl")
     torch.cuda.set_device(local)
     from long_context_sparse_clsa_b200 import clsa
-    from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs, replace
+    from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs
     clsa.load_library()
-    w = WORKLOADS[args.workload]
-    if world > 1:  # each rank its own sequences: a different seed per rank
-        w = replace(w, seed=w.seed + rank)
+    w = replicas.rank_workload(WORKLOADS[args.workload], rank, world)  # each rank its own sequences
     inp = make_inputs(w)
     dv = clsa.to_device(inp)
     dev = torch.device("cuda", local)
@@ -350,9 +339,7 @@ def run_clsa(args):
     torch.cuda.synchronize()
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+        replicas.barrier(world)
         torch.cuda.synchronize()
 
     # The timed region: K steps back to back on the stream, one event pair around them (with
@@ -380,13 +367,9 @@ def run_clsa(args):
     st = ws.status()
     if st[0] != "CLSA_OK":
         raise RuntimeError(f"device error during timing: {st}")
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = replicas.max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * B / (ms_per_step / 1e3)
+    value = replicas.job_rate(world, B, ms_per_step)
 
     # ---- per-kernel timing (each C-ABI stage alone, same stream, L2 flushed) -----------
     sc = torch.empty(B, w.n_max, dtype=torch.float32, device=dev)
@@ -457,21 +440,14 @@ def run_clsa(args):
         if i >= 3:
             tot += e0.elapsed_time(e1)
     e2e_ms = tot / e2e_steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = replicas.max_over_ranks(e2e_ms, world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, threads, note = time_oracle(inp, w, args.cpu_sample_steps)
         cpu = {"value": w.B / dt, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note}
 
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finish(world)
     if rank != 0:
         return
     line = {
@@ -493,7 +469,7 @@ def run_clsa(args):
         "step_roofline": {"algorithmic_bytes": by["total"], "achieved_gbs": step_gbs, "peak": hbm,
                           "frac": step_gbs / hbm, "peak_kind": peak_kind},
         "kernels_us": kern,
-        "e2e": {"value": world * B / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": replicas.job_rate(world, B, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
