@@ -23,7 +23,7 @@ Once: Cross-Layer Sparse Attention with Shared Routing" (CLSA):
   per-query term ``KL(sg[Abar_t] || softmax(I_t))`` (forward only).
 
 All floating arithmetic is float64 on inputs upcast from their storage values.
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * the indexer has no scale, bias or activation (the routing equation is a bare
   product, single head);
