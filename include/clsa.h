@@ -222,6 +222,16 @@ CLSA_API clsa_status clsa_workspace_init(void* ws, size_t bytes, void* stream);
  * kernel-specific code (the offending index, or the wait site). */
 CLSA_API clsa_status clsa_read_device_status(void* ws, void* stream, int64_t* detail);
 CLSA_API const char* clsa_status_string(clsa_status s);
+/* Failure-detection self-test.  Launches one CTA on `stream` whose wait nothing will
+ * satisfy -- which = 0: the inter-CTA count barrier, for two CTAs with one launched;
+ * which = 1: an mbarrier phase that expects one arrival and gets none.  The wait runs
+ * out after the library's limit (200 ms of GPU time), records CLSA_ERR_TIMEOUT with
+ * detail 900 + which in `ws`, and the kernel returns: clsa_read_device_status then
+ * reports it, and the stream and context stay usable.  Returns CLSA_OK once launched;
+ * CLSA_ERR_INVALID_ARG for another `which`; CLSA_ERR_WORKSPACE if `ws` is NULL, not
+ * 16-byte aligned or under 512 bytes.  Uses the first 4 bytes after the 256-byte
+ * header as its barrier word (zeroed on `stream` first). */
+CLSA_API clsa_status clsa_selftest_timeout(int which, void* ws, size_t ws_bytes, void* stream);
 /* Library version as major*10000 + minor*100 + patch. */
 CLSA_API int clsa_version(void);
 /* Number of kernel launches the last call made on this host thread. */

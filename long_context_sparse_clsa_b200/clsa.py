@@ -29,7 +29,7 @@ EXPORTS = [
     "clsa_distill_workspace_size", "clsa_distill_target",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
     "clsa_prefill_chunk", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
-    "clsa_version", "clsa_last_launch_count",
+    "clsa_selftest_timeout", "clsa_version", "clsa_last_launch_count",
 ]
 
 
@@ -90,6 +90,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_workspace_init": (S, [_vp, _sz, _vp]),
         "clsa_read_device_status": (S, [_vp, _vp, ctypes.POINTER(ctypes.c_int64)]),
         "clsa_status_string": (ctypes.c_char_p, [S]),
+        "clsa_selftest_timeout": (S, [_i, _vp, _sz, _vp]),
         "clsa_version": (_i, []),
         "clsa_last_launch_count": (_i, []),
     }
@@ -253,6 +254,14 @@ def distill_target(Q, K, scores, seq_lens, scale: float = 0.0, ws: Optional[Work
     _check(lib.clsa_distill_target(_p(Q), _p(K), _p(scores), _p(seq_lens), B, n_max, L, Hq, Hkv, d, scale, _dt(Q),
                                    _p(abar), _p(kl), ws.ptr, ws.nbytes, _stream()), "clsa_distill_target")
     return abar, kl, ws
+
+
+def selftest_timeout(which: int, ws: Optional[Workspace] = None):
+    """Launch the failure-detection self-test (see clsa.h); returns its workspace, whose
+    status() then reads CLSA_ERR_TIMEOUT with detail 900 + which."""
+    ws = ws or Workspace(512)
+    _check(load_library().clsa_selftest_timeout(which, ws.ptr, ws.nbytes, _stream()), "clsa_selftest_timeout")
+    return ws
 
 
 def decode_step_args(args: DecodeArgs, ws: Workspace, stream=None):

@@ -140,6 +140,14 @@ clsa_status clsa_workspace_init(void* ws, size_t bytes, void* stream) {
   return from_cuda(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));
 }
 
+clsa_status clsa_selftest_timeout(int which, void* ws, size_t ws_bytes, void* stream) {
+  CallScope scope;
+  if (which != 0 && which != 1) return CLSA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kWsHeader + 256 || !aligned16(ws)) return CLSA_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  return from_cuda(launch_selftest_timeout(which, w, w + kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
 clsa_status clsa_read_device_status(void* ws, void* stream, int64_t* detail) {
   if (!ws) return CLSA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -75,6 +75,9 @@ cudaError_t launch_distill_tc(const void* Q, const void* K, const float* scores,
                               int L, int Hq, int Hkv, float scale, float* abar, float* kl, void* ws_header, void* ws,
                               cudaStream_t s);
 
+// ----- failure-detection self-test (a wait that runs out and reports) ------------
+cudaError_t launch_selftest_timeout(int which, void* ws_header, void* ws_body, cudaStream_t s);
+
 // ----- fused decode step (one cooperative launch) -------------------------------
 bool fused_decode_supported(const clsa_decode_args* a);
 size_t fused_decode_ws_bytes(const clsa_decode_args* a);

@@ -101,3 +101,12 @@ def test_oracle_is_not_imported_by_the_product():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle|clsa_oracle|#include.*oracle",
                                      text, re.M), f
+
+
+def test_selftest_rejects_bad_args(lib):
+    ws = ctypes.create_string_buffer(1024 + 16)
+    base = (ctypes.addressof(ws) + 15) & ~15
+    assert lib.clsa_selftest_timeout(2, base, 1024, None) == 1      # CLSA_ERR_INVALID_ARG
+    assert lib.clsa_selftest_timeout(0, None, 1024, None) == 3      # CLSA_ERR_WORKSPACE
+    assert lib.clsa_selftest_timeout(1, base, 300, None) == 3       # under 512 bytes
+    assert lib.clsa_selftest_timeout(0, base + 4, 1000, None) == 3  # not 16-byte aligned
