@@ -215,6 +215,13 @@ CLSA_API clsa_status clsa_prefill_chunk(const clsa_prefill_args* a, void* ws, si
 /* ------------------------------------------------------------------------ */
 /* Helpers                                                                    */
 /* ------------------------------------------------------------------------ */
+/* Workspace bytes of an operation, given its argument struct: op CLSA_OP_DECODE_STEP
+ * (args: const clsa_decode_args*) or CLSA_OP_PREFILL_CHUNK (args: const clsa_prefill_args*).
+ * The same value as clsa_decode_workspace_size / clsa_prefill_workspace_size; 0 for an
+ * unknown op, a NULL args, or arguments that call would reject.  The stage calls have their
+ * own size functions above. */
+typedef enum { CLSA_OP_DECODE_STEP = 0, CLSA_OP_PREFILL_CHUNK = 1 } clsa_op;
+CLSA_API size_t clsa_workspace_size(int op, const void* args);
 /* Zero `bytes` of workspace on `stream` (asynchronous). */
 CLSA_API clsa_status clsa_workspace_init(void* ws, size_t bytes, void* stream);
 /* Synchronise `stream`, return the first device-detected error recorded in

@@ -28,7 +28,7 @@ EXPORTS = [
     "clsa_gather_kv", "clsa_sparse_attn_workspace_size", "clsa_sparse_attn",
     "clsa_distill_workspace_size", "clsa_distill_target",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
-    "clsa_prefill_chunk", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
+    "clsa_prefill_chunk", "clsa_workspace_size", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
     "clsa_selftest_timeout", "clsa_version", "clsa_last_launch_count",
 ]
 
@@ -87,6 +87,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_decode_step": (S, [ctypes.POINTER(DecodeArgs), _vp, _sz, _vp]),
         "clsa_prefill_workspace_size": (_sz, [ctypes.POINTER(PrefillArgs)]),
         "clsa_prefill_chunk": (S, [ctypes.POINTER(PrefillArgs), _vp, _sz, _vp]),
+        "clsa_workspace_size": (_sz, [_i, _vp]),
         "clsa_workspace_init": (S, [_vp, _sz, _vp]),
         "clsa_read_device_status": (S, [_vp, _vp, ctypes.POINTER(ctypes.c_int64)]),
         "clsa_status_string": (ctypes.c_char_p, [S]),

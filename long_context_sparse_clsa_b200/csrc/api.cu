@@ -135,6 +135,15 @@ const char* clsa_status_string(clsa_status s) {
   return "CLSA_ERR_UNKNOWN";
 }
 
+size_t clsa_workspace_size(int op, const void* args) {
+  if (!args) return 0;
+  switch (op) {
+    case CLSA_OP_DECODE_STEP: return clsa_decode_workspace_size(static_cast<const clsa_decode_args*>(args));
+    case CLSA_OP_PREFILL_CHUNK: return clsa_prefill_workspace_size(static_cast<const clsa_prefill_args*>(args));
+    default: return 0;
+  }
+}
+
 clsa_status clsa_workspace_init(void* ws, size_t bytes, void* stream) {
   if (!ws || bytes < kWsHeader) return CLSA_ERR_INVALID_ARG;
   return from_cuda(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));

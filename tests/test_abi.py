@@ -110,3 +110,20 @@ def test_selftest_rejects_bad_args(lib):
     assert lib.clsa_selftest_timeout(0, None, 1024, None) == 3      # CLSA_ERR_WORKSPACE
     assert lib.clsa_selftest_timeout(1, base, 300, None) == 3       # under 512 bytes
     assert lib.clsa_selftest_timeout(0, base + 4, 1000, None) == 3  # not 16-byte aligned
+
+
+def test_generic_workspace_size_dispatches_by_op(lib):
+    a = clsa.DecodeArgs(dtype=1, B=1, n_max=4096, d_idx=128, k=256, L=2, Hq=8, Hkv=2, d=128)
+    for i, f in enumerate(["q_idx", "k_idx", "K", "V", "Q", "seq_lens", "O", "idx", "count"]):
+        setattr(a, f, 0x100000 * (i + 1))  # aligned placeholders: the size calls never dereference
+    p = clsa.PrefillArgs(dtype=1, n=4096, T=64, d_idx=128, k=256, L=2, Hq=8, Hkv=2, d=128)
+    for i, f in enumerate(["q_idx", "k_idx", "K", "V", "Q", "O", "idx", "count"]):
+        setattr(p, f, 0x100000 * (i + 1))
+    dec, pre = lib.clsa_decode_workspace_size(ctypes.byref(a)), lib.clsa_prefill_workspace_size(ctypes.byref(p))
+    assert dec > 0 and pre > 0
+    assert lib.clsa_workspace_size(0, ctypes.byref(a)) == dec  # CLSA_OP_DECODE_STEP
+    assert lib.clsa_workspace_size(1, ctypes.byref(p)) == pre  # CLSA_OP_PREFILL_CHUNK
+    assert lib.clsa_workspace_size(2, ctypes.byref(p)) == 0
+    assert lib.clsa_workspace_size(0, None) == 0
+    a.k = 0  # rejected arguments: size 0, as from the op's own call
+    assert lib.clsa_workspace_size(0, ctypes.byref(a)) == 0 == lib.clsa_decode_workspace_size(ctypes.byref(a))
