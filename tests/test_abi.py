@@ -127,3 +127,35 @@ def test_generic_workspace_size_dispatches_by_op(lib):
     assert lib.clsa_workspace_size(0, None) == 0
     a.k = 0  # rejected arguments: size 0, as from the op's own call
     assert lib.clsa_workspace_size(0, ctypes.byref(a)) == 0 == lib.clsa_decode_workspace_size(ctypes.byref(a))
+
+
+def test_header_is_c99_and_a_c_program_links_and_calls(lib, tmp_path):
+    """The boundary is a C ABI: clsa.h compiles as strict C99 and a C program links
+    libclsa.so and calls it (here only calls that need no GPU)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_clsa.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "clsa.h"
+int main(void) {
+  static char ws[1024];
+  clsa_decode_args a = {0};
+  if (clsa_version() < 100) return 1;
+  printf("%s\n", clsa_status_string(CLSA_ERR_TIMEOUT));
+  /* argument errors are returned before any device work */
+  if (clsa_selftest_timeout(7, ws, sizeof ws, NULL) != CLSA_ERR_INVALID_ARG) return 2;
+  if (clsa_workspace_size(CLSA_OP_PREFILL_CHUNK, NULL) != 0) return 3;
+  if (clsa_decode_step(&a, NULL, 0, NULL) == CLSA_OK) return 4;
+  return 0;
+}
+""")
+    exe = tmp_path / "use_clsa"
+    libdir = os.path.dirname(clsa.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(exe), "-L", libdir, "-l:libclsa.so", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == "CLSA_ERR_TIMEOUT"
