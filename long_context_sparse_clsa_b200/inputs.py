@@ -66,6 +66,9 @@ class Workload:
     plant     fraction of cache tokens whose index key is boosted toward the
               query (salient tokens), 0 for none
     T         prefill rows (the last T positions of the n-token cache)
+    q_corr    prefill only: correlation rho of consecutive rows' index queries, an AR(1)
+              sequence q_t = rho q_{t-1} + sqrt(1 - rho^2) z_t over the N(0, 1) draws
+              z_t (each row stays N(0, 1)); 0 leaves the draws independent
     """
 
     name: str
@@ -83,6 +86,7 @@ class Workload:
     plant: float = 0.0
     T: int = 0
     seed: int = 0
+    q_corr: float = 0.0
 
     @property
     def G(self) -> int:
@@ -108,6 +112,10 @@ WORKLOADS: Dict[str, Workload] = {
     # 4096 new rows appended to a 126976-token cache (n = 131072), causal
     "prefill4k": Workload("prefill4k", mode="prefill", n_max=131072, d_idx=128, k=2048,
                           L=24, Hq=32, Hkv=8, d=128, dtype="bf16", T=4096),
+    # the same with consecutive rows' index queries correlated (rho = 0.95): neighbouring
+    # rows select overlapping token sets, as consecutive tokens of real text tend to
+    "prefill4k_corr": Workload("prefill4k_corr", mode="prefill", n_max=131072, d_idx=128, k=2048,
+                               L=24, Hq=32, Hkv=8, d=128, dtype="bf16", T=4096, q_corr=0.95),
 }
 
 # stream ids, in the order the tensors are described
@@ -292,7 +300,14 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
         n, T = w.n_max, w.T
         if not (1 <= T <= n):
             raise ValueError("prefill needs 1 <= T <= n")
-        q = _store(counter_normal(seed, _S_QIDX, 0, T * w.d_idx).reshape(T, w.d_idx), w.dtype)
+        qz = counter_normal(seed, _S_QIDX, 0, T * w.d_idx).reshape(T, w.d_idx)
+        if w.q_corr:
+            if not 0.0 < w.q_corr < 1.0:
+                raise ValueError("q_corr must lie in [0, 1)")
+            rho, tail = np.float32(w.q_corr), np.float32(math.sqrt(1.0 - w.q_corr ** 2))
+            for t in range(1, T):  # in float32, row by row
+                qz[t] = rho * qz[t - 1] + tail * qz[t]
+        q = _store(qz, w.dtype)
         kidx = _store(counter_normal(seed, _S_KIDX, 0, n * w.d_idx).reshape(n, w.d_idx), w.dtype)
         lens = np.array([n], dtype=np.int32)
         K = _fill_rows(seed, _S_K, (1, n, w.Hkv, w.d), lens, w.dtype)[0]

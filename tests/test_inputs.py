@@ -85,3 +85,25 @@ def test_planted_rows_move_scores_by_three_norms():
     rest = np.setdiff1d(np.arange(n), js)
     assert abs(s[rest].std() / qn - 1.0) < 0.05
     assert abs((s[js].mean() - s[rest].mean()) / qn - 3.0) < 0.6
+
+
+def test_correlated_prefill_queries():
+    """q_corr: an AR(1) sequence of index queries over the prefill rows.  rho = 0 gives the
+    independent draws bit for bit; rho = 0.95 keeps each row N(0, 1), correlates neighbours
+    at ~rho, and makes neighbouring rows' TopK sets (the oracle's) overlap heavily, where
+    independent rows share few tokens."""
+    from oracle import clsa_oracle as O
+    base = scaled("prefill4k", n_max=2048, T=256, L=1, k=64)
+    np.testing.assert_array_equal(make_inputs(base).q_idx, make_inputs(scaled("prefill4k", n_max=2048, T=256, L=1,
+                                                                               k=64, q_corr=0.0)).q_idx)
+    overlap = {}
+    for rho in (0.0, 0.95):
+        inp = make_inputs(scaled("prefill4k", n_max=2048, T=256, L=1, k=64, q_corr=rho))
+        q = bf16_bits_to_f32(inp.q_idx).astype(np.float64)
+        if rho:
+            assert abs(q.std() - 1.0) < 0.05
+            assert abs(np.corrcoef(q[1:].ravel(), q[:-1].ravel())[0, 1] - rho) < 0.02
+        idx, cnt = O.prefill_topk(inp.q_idx, inp.k_idx, 2048, 64)
+        shared = [len(set(idx[t, :cnt[t]]) & set(idx[t + 1, :cnt[t + 1]])) / cnt[t] for t in range(255)]
+        overlap[rho] = float(np.mean(shared))
+    assert overlap[0.0] < 0.1 and overlap[0.95] > 0.5, overlap
