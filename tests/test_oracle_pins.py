@@ -427,3 +427,30 @@ def test_distill_kl_against_scipy_and_closed_forms():
     I2[0, :40] = np.log(A[0, :40]) + 5.0
     _, kl2 = O.distill_target(Q, K, I2, lens)
     assert abs(kl2[0]) < 1e-12
+
+
+def test_distill_invariances():
+    """Properties the definition fixes: softmax(I) is shift invariant, so kl ignores a constant
+    added to I (a missing lse of I would not); permuting the cached tokens (K rows with their
+    I) permutes Abar the same way and keeps kl; permuting the layers, or the query heads inside
+    one KV group, leaves the average Abar unchanged."""
+    rng = np.random.default_rng(14)
+    L, B, Hq, Hkv, d, n = 3, 2, 4, 2, 8, 33
+    Q = rng.normal(size=(L, B, Hq, d))
+    K = rng.normal(size=(B, n, Hkv, d))
+    I = 2.0 * rng.normal(size=(B, n))
+    lens = [n, 20]
+    A, kl = O.distill_target(Q, K, I, lens)
+    _, kl_shift = O.distill_target(Q, K, I + 7.5, lens)
+    np.testing.assert_allclose(kl_shift, kl, rtol=1e-10, atol=1e-12)
+    perm = rng.permutation(n)
+    K2, I2 = K[:, perm].copy(), I[:, perm].copy()
+    lens2 = [n, n]  # every row valid, so the permutation stays inside the valid range
+    A_full, kl_full = O.distill_target(Q, K, I, lens2)
+    A2, kl2 = O.distill_target(Q, K2, I2, lens2)
+    np.testing.assert_allclose(A2, A_full[:, perm], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(kl2, kl_full, rtol=1e-10)
+    Q3 = Q[rng.permutation(L)][:, :, [1, 0, 3, 2]]  # layers shuffled; heads swapped within each KV group
+    A3, kl3 = O.distill_target(Q3, K, I, lens)
+    np.testing.assert_allclose(A3, A, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(kl3, kl, rtol=1e-10)
