@@ -24,6 +24,7 @@ bounded sample of the same workload and prints the same line with
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -421,26 +422,94 @@ def run_clsa(args):
     step_gbs = by["total"] / (ms_per_step * 1e-3) / 1e9
 
     # ---- end to end through the public API with host buffers --------------------------
-    # pinned host images of the packed buffers: one H2D (q_idx, Q) and one D2H (O, idx, count)
-    in_h = in_buf.cpu().pin_memory()
-    out_h = torch.empty(out_buf.shape, dtype=torch.uint8).pin_memory()
-    h2d = in_h.numel()
-    d2h = out_h.numel()
-    e2e_steps = min(args.steps, 50)
-    tot = 0.0
-    for i in range(e2e_steps + 3):
-        between_steps()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        in_buf.copy_(in_h, non_blocking=True)
-        clsa.decode_step_args(args_sets[i % R], ws)
-        out_h.copy_(out_buf, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if i >= 3:
-            tot += e0.elapsed_time(e1)
-    e2e_ms = tot / e2e_steps
+    # Every step copies its inputs (q_idx, Q: one packed pinned host buffer) to the device,
+    # runs clsa_decode_step and copies its outputs (O, idx, count: one packed buffer) back
+    # to pinned host memory.  As in a serving loop the copies are pipelined with the compute:
+    # two device buffer pairs alternate, the H2D of step i + 1 and the D2H of step i run on
+    # copy streams ordered by events (step i waits for its H2D; step i + 2 waits for the D2H
+    # of step i before it overwrites that output buffer).  M steps are captured in one CUDA
+    # graph (copies included) and the timed region replays it; the pipeline drains at each
+    # replay's end.
+    in_h = [in_buf.cpu().pin_memory() for _ in range(2)]
+    out_h = [torch.empty(out_buf.shape, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    h2d = in_h[0].numel()
+    d2h = out_h[0].numel()
+    in_b = [in_buf, torch.empty_like(in_buf)]
+    out_b = [out_buf, torch.empty_like(out_buf)]
+
+    def rebase(t, old_buf, new_buf):
+        off = t.data_ptr() - old_buf.data_ptr()
+        return new_buf[off:off + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+
+    e2e_args = [[clsa.decode_args(rebase(dv["q_idx"], in_buf, in_b[p_]), kidx_sets[r], dv["K"], dv["V"],
+                                  rebase(dv["Q"], in_buf, in_b[p_]), dv["seq_lens"], k,
+                                  rebase(out["O"], out_buf, out_b[p_]), rebase(out["idx"], out_buf, out_b[p_]),
+                                  rebase(out["count"], out_buf, out_b[p_]))
+                 for p_ in range(2)] for r in range(R)]
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    M = 2 * R
+
+    def e2e_steps_on(cs, n):
+        """n pipelined steps issued from stream cs (capturable); returns nothing"""
+        ev = lambda: torch.cuda.Event()
+        c_done, d_done = [None] * n, [None] * n
+        s_h2d.wait_stream(cs)
+        s_d2h.wait_stream(cs)
+        for i in range(n):
+            p_ = i % 2
+            if i >= 2:
+                s_h2d.wait_event(c_done[i - 2])          # step i - 2 has read in_b[p_]
+            with torch.cuda.stream(s_h2d):
+                in_b[p_].copy_(in_h[p_], non_blocking=True)
+                h_ev = ev()
+                h_ev.record(s_h2d)
+            cs.wait_event(h_ev)
+            if i >= 2:
+                cs.wait_event(d_done[i - 2])              # the D2H of out_b[p_] is done
+            clsa.decode_step_args(e2e_args[i % R][p_], ws, stream=cs)
+            c_done[i] = ev()
+            c_done[i].record(cs)
+            s_d2h.wait_event(c_done[i])
+            with torch.cuda.stream(s_d2h):
+                out_h[p_].copy_(out_b[p_], non_blocking=True)
+                d_done[i] = ev()
+                d_done[i].record(s_d2h)
+        cs.wait_stream(s_h2d)
+        cs.wait_stream(s_d2h)
+
+    e2e_graph = None
+    if not args.no_graph:
+        try:
+            cap = torch.cuda.Stream()
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap):
+                e2e_steps_on(cap, 4)  # warm the streams and events outside capture
+            stream.wait_stream(cap)
+            torch.cuda.synchronize()
+            e2e_graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(e2e_graph):
+                e2e_steps_on(torch.cuda.current_stream(), M)
+            torch.cuda.synchronize()
+        except Exception as ex:
+            e2e_graph = None
+            print(f"# e2e graph capture failed, eager pipeline: {ex}", file=sys.stderr)
+    reps = max(1, min(args.steps, 400) // M)
+    for _ in range(2):  # warm-up (the first replay uploads the graph)
+        e2e_graph.replay() if e2e_graph is not None else e2e_steps_on(stream, M)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        e2e_graph.replay() if e2e_graph is not None else e2e_steps_on(stream, M)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / (reps * M)
     e2e_ms = replicas.max_over_ranks(e2e_ms, world, dev)
+    e2e_launch = (f"{M} pipelined steps per CUDA graph (H2D, step, D2H on three streams)"
+                  if e2e_graph is not None else f"{M} pipelined steps, eager")
+    st = ws.status()
+    if st[0] != "CLSA_OK":
+        raise RuntimeError(f"device error during the end-to-end timing: {st}")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -470,7 +539,7 @@ def run_clsa(args):
                           "frac": step_gbs / hbm, "peak_kind": peak_kind},
         "kernels_us": kern,
         "e2e": {"value": replicas.job_rate(world, B, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "launch": e2e_launch},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
@@ -602,10 +671,92 @@ def run_variant(args):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args):
+    """One prefill chunk per step (clsa_prefill_chunk: causal indexer GEMM with the candidate
+    filter, exact per-row TopK, per-row sparse attention over L layers).  Reports chunk
+    rows/s and the indexer kernel's useful-FLOP rate against the bf16 tensor peak."""
+    import torch
+    from long_context_sparse_clsa_b200 import clsa
+    from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs
+    if args.gpus != 1:
+        raise SystemExit("the prefill line runs on one GPU")
+    torch.cuda.set_device(0)
+    clsa.load_library()
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    stream = torch.cuda.current_stream()
+    T, n, k, L, Hq, d = w.T, w.n_max, w.k, w.L, w.Hq, w.d
+    out = {"O": torch.empty_like(dv["Q"]), "idx": torch.empty(T, k, dtype=torch.int32, device="cuda"),
+           "count": torch.empty(T, dtype=torch.int32, device="cuda")}
+    a = clsa.prefill_args(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], k, out["O"], out["idx"],
+                          out["count"])
+    ws = clsa.Workspace(clsa.prefill_workspace_size(a))
+    lib = clsa.load_library()
+
+    def chunk():
+        clsa._check(lib.clsa_prefill_chunk(ctypes.byref(a), ws.ptr, ws.nbytes, clsa._stream()), "clsa_prefill_chunk")
+
+    for _ in range(max(args.warmup, 3)):
+        chunk()
+    torch.cuda.synchronize()
+    launches = clsa.last_launch_count()
+    steps = max(1, min(args.steps, 50))
+    timer = clsa.LaunchTimer(16)
+    per_launch = []
+    with ClockSampler(0) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            chunk()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        for _ in range(min(steps, 10)):  # per-launch times of whole chunks (the attention of each
+            timer.arm()                  # chunk streams > 500 MB, so every route launch starts cold)
+            chunk()
+            torch.cuda.synchronize()
+            per_launch.append(timer.times_ms())
+    st = ws.status()
+    if st[0] != "CLSA_OK":
+        raise RuntimeError(f"device error during timing: {st}")
+    ms = e0.elapsed_time(e1) / steps
+    route_ms = statistics.median(pl_[0] for pl_ in per_launch)
+    attn_ms = statistics.median(pl_[-1] for pl_ in per_launch)
+    hbm, bf16, peak_kind = peaks()
+    sustained = None
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        sustained = json.load(open(pk)).get("bf16_tflops_sustained")
+    t0 = n - T
+    useful = 2 * w.d_idx * sum(t0 + i + 1 for i in range(T))   # causal rectangle of the indexer
+    tfs = useful / (route_ms * 1e-3) / 1e12
+    attn_flops = T * L * Hq * k * d * 4
+    line = {
+        "metric": METRIC, "variant": "prefill_chunk", "value": T / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": w.name, "T": T, "n": n, "d_idx": w.d_idx, "k": k, "L": L, "Hq": Hq, "Hkv": w.Hkv,
+                   "d": d, "l2": "each chunk's attention streams > 500 MB: every route launch starts cold",
+                   "launch": "eager (one clsa_prefill_chunk per step)"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_route_kernel", "achieved": tfs, "peak": bf16,
+                     "unit": "TFLOP/s", "frac": tfs / bf16, "traffic": None, "peak_kind": f"{peak_kind} burst",
+                     "frac_of_sustained": (tfs / sustained) if sustained else None,
+                     "useful_flops_per_launch": useful, "us_per_launch": route_ms * 1e3},
+        "launch_ms_median": [statistics.median(x) for x in zip(*per_launch)],
+        "attention": {"kernel": "last launch of the chunk", "ms": attn_ms,
+                      "useful_tflops": attn_flops / (attn_ms * 1e-3) / 1e12},
+        "gpu_launches": launches * steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload.startswith("prefill"):
+        run_prefill(args)
     elif args.variant != "clsa":
         run_variant(args)
     else:

@@ -107,8 +107,11 @@ CLSA_API clsa_status clsa_topk(const float* scores, const int32_t* seq_lens, int
  *   - Each call clears the part of the array it uses on `stream` before the
  *     kernel runs.  Calls that overlap on the GPU (other streams, other host
  *     threads) share the array and race: serialise them.
- *   - Sizes whose scratch would exceed 2 MiB (many rows that each need several
- *     CTAs, about B > 55 at n_max = 128K) return CLSA_ERR_UNSUPPORTED.
+ *   - A size is refused with CLSA_ERR_UNSUPPORTED exactly when
+ *     clsa_topk_workspace_size(B, n_max, k) exceeds 2 MiB (at n_max = 128K that
+ *     is a middle range of B, where each row still gets several CTAs).
+ *   - The array's address belongs to the device's primary context: after
+ *     cudaDeviceReset on a device, do not call this entry point there again.
  *   - Errors the kernel records on the device are not reported (there is no
  *     caller workspace to hold them); argument errors are returned as usual.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
@@ -243,6 +246,17 @@ CLSA_API clsa_status clsa_selftest_timeout(int which, void* ws, size_t ws_bytes,
 CLSA_API int clsa_version(void);
 /* Number of kernel launches the last call made on this host thread. */
 CLSA_API int clsa_last_launch_count(void);
+/* Launch timing (instrumentation; no counterpart on the pages).  Arms the next
+ * library call made on this host thread: on that call's stream it records
+ * events[0] before its first kernel launch and events[i] right after its i-th
+ * launch (a group of launches made together counts once), up to max_events
+ * events in all.  events are cudaEvent_t handles the caller created (timing
+ * enabled) and keeps alive until they complete; cudaEventElapsedTime of
+ * consecutive events then gives each launch's device time.  max_events = 0
+ * disarms.  Only the next call is armed.  clsa_timed_event_count() returns how
+ * many events the last armed call recorded. */
+CLSA_API clsa_status clsa_time_next_call(void* const* events, int max_events);
+CLSA_API int clsa_timed_event_count(void);
 
 #ifdef __cplusplus
 }

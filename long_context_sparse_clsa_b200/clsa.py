@@ -29,7 +29,8 @@ EXPORTS = [
     "clsa_distill_workspace_size", "clsa_distill_target",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
     "clsa_prefill_chunk", "clsa_workspace_size", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
-    "clsa_selftest_timeout", "clsa_version", "clsa_last_launch_count",
+    "clsa_selftest_timeout", "clsa_version", "clsa_last_launch_count", "clsa_time_next_call",
+    "clsa_timed_event_count",
 ]
 
 
@@ -94,6 +95,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_selftest_timeout": (S, [_i, _vp, _sz, _vp]),
         "clsa_version": (_i, []),
         "clsa_last_launch_count": (_i, []),
+        "clsa_time_next_call": (S, [ctypes.POINTER(ctypes.c_void_p), _i]),
+        "clsa_timed_event_count": (_i, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -134,6 +137,26 @@ def _check(code: int, where: str):
 def last_launch_count() -> int:
     """Kernel launches made by the most recent library call on this thread."""
     return load_library().clsa_last_launch_count()
+
+
+class LaunchTimer:
+    """Per-launch device times of one library call: arm() before the call; after the
+    stream has synchronized, times_ms() gives each launch's duration (events the library
+    records before its first launch and after each launch, on the call's stream)."""
+
+    def __init__(self, max_launches: int = 16):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(max_launches + 1)]
+        for e in self.events:  # torch creates the CUDA event on its first record
+            e.record()
+        torch.cuda.synchronize()
+        self._handles = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+
+    def arm(self):
+        _check(load_library().clsa_time_next_call(self._handles, len(self.events)), "clsa_time_next_call")
+
+    def times_ms(self):
+        n = load_library().clsa_timed_event_count()
+        return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(n - 1)]
 
 
 class Workspace:

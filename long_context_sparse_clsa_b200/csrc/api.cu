@@ -27,6 +27,11 @@ const DeviceInfo& device_info() {
 namespace {
 thread_local int g_launches = 0;
 thread_local int g_last_launches = 0;
+// launch timing: events armed for the next call (pending), and those of the running call
+thread_local cudaEvent_t const* g_ev_pending = nullptr;
+thread_local int g_ev_pending_max = 0;
+thread_local cudaEvent_t const* g_ev = nullptr;
+thread_local int g_ev_max = 0, g_ev_n = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -34,11 +39,6 @@ bool dims_ok(int d) { return d == 64 || d == 128; }
 bool dtype_ok(clsa_dtype dt) { return dt == CLSA_F32 || dt == CLSA_BF16; }
 
 clsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CLSA_OK : CLSA_ERR_CUDA; }
-
-struct CallScope {
-  CallScope() { g_launches = 0; }
-  ~CallScope() { g_last_launches = g_launches; }
-};
 
 // attention shape checks shared by clsa_sparse_attn and clsa_decode_step
 // kmax: 4096 for the selection paths; clsa_sparse_attn reads K_S/V_S rows directly and
@@ -108,8 +108,41 @@ float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / st
 
 }  // namespace
 
+CallScope::CallScope(void* stream) {
+  g_launches = 0;
+  g_ev = nullptr;
+  if (g_ev_pending) {  // an armed call: event 0 before its first launch
+    g_ev = g_ev_pending;
+    g_ev_max = g_ev_pending_max;
+    g_ev_pending = nullptr;
+    g_ev_n = 0;
+    if (g_ev_max > 0) {
+      if (cudaEventRecord(g_ev[0], static_cast<cudaStream_t>(stream)) == cudaSuccess) {
+        g_ev_n = 1;
+      } else {  // not a valid event: record nothing, and leave no error behind for the launches
+        (void)cudaGetLastError();
+        g_ev = nullptr;
+      }
+    }
+  }
+}
+CallScope::~CallScope() {
+  g_last_launches = g_launches;
+  g_ev = nullptr;
+}
+
 void launches_reset() { g_launches = 0; }
-void launches_add(int n) { g_launches += n; }
+void launches_add(int n, cudaStream_t s) {
+  g_launches += n;
+  if (g_ev && g_ev_n < g_ev_max) {
+    if (cudaEventRecord(g_ev[g_ev_n], s) == cudaSuccess) {
+      ++g_ev_n;
+    } else {
+      (void)cudaGetLastError();
+      g_ev = nullptr;
+    }
+  }
+}
 int launches_get() { return g_launches; }
 
 }  // namespace clsa
@@ -121,6 +154,15 @@ extern "C" {
 int clsa_version(void) { return 100; }  // 0.1.0
 
 int clsa_last_launch_count(void) { return clsa::g_last_launches; }
+
+clsa_status clsa_time_next_call(void* const* events, int max_events) {
+  if (max_events < 0 || (max_events > 0 && !events)) return CLSA_ERR_INVALID_ARG;
+  clsa::g_ev_pending = max_events > 0 ? reinterpret_cast<cudaEvent_t const*>(events) : nullptr;
+  clsa::g_ev_pending_max = max_events;
+  return CLSA_OK;
+}
+
+int clsa_timed_event_count(void) { return clsa::g_ev_n; }
 
 const char* clsa_status_string(clsa_status s) {
   switch (s) {
@@ -150,7 +192,7 @@ clsa_status clsa_workspace_init(void* ws, size_t bytes, void* stream) {
 }
 
 clsa_status clsa_selftest_timeout(int which, void* ws, size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   if (which != 0 && which != 1) return CLSA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < kWsHeader + 256 || !aligned16(ws)) return CLSA_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
@@ -176,7 +218,7 @@ clsa_status clsa_read_device_status(void* ws, void* stream, int64_t* detail) {
 
 clsa_status clsa_index_scores(const void* q_idx, const void* k_idx, const int32_t* seq_lens, int B, int n_max,
                               int d_idx, clsa_dtype dt, float* scores, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   if (!q_idx || !k_idx || !seq_lens || !scores || B < 1 || n_max < 1 || !dtype_ok(dt))
     return CLSA_ERR_INVALID_ARG;
   if (!dims_ok(d_idx)) return CLSA_ERR_UNSUPPORTED;
@@ -193,7 +235,7 @@ size_t clsa_topk_workspace_size(int B, int n_max, int k) {
 
 clsa_status clsa_topk(const float* scores, const int32_t* seq_lens, int B, int n_max, int k, int32_t* idx,
                       int32_t* count, void* ws, size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   if (!scores || !seq_lens || !idx || !count || B < 1 || n_max < 1 || k < 1) return CLSA_ERR_INVALID_ARG;
   if (k > 4096) return CLSA_ERR_UNSUPPORTED;
   for (const void* p : {(const void*)scores, (const void*)seq_lens, (const void*)idx, (const void*)count})
@@ -209,7 +251,7 @@ size_t clsa_gather_kv_workspace_size(void) { return kWsHeader; }
 clsa_status clsa_gather_kv(const void* K, const void* V, const int32_t* idx, const int32_t* count, int B,
                            int n_max, int k, int Hkv, int d, clsa_dtype dt, void* K_S, void* V_S, void* ws,
                            size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   if (!K || !V || !idx || !count || !K_S || !V_S || B < 1 || n_max < 1 || k < 1 || Hkv < 1 || !dtype_ok(dt))
     return CLSA_ERR_INVALID_ARG;
   if (!dims_ok(d) || k > 4096) return CLSA_ERR_UNSUPPORTED;
@@ -232,7 +274,7 @@ size_t clsa_sparse_attn_workspace_size(int B, int k, int L, int Hq, int Hkv, int
 clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void* V_S, const int32_t* count, int B, int k,
                              int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, void* O, float* lse,
                              void* ws, size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   clsa_status st = check_attn(B, k, L, Hq, Hkv, d, dt, kMaxDirectK);
   if (st != CLSA_OK) return st;
   if (!Q || !K_S || !V_S || !count || !O) return CLSA_ERR_INVALID_ARG;
@@ -256,7 +298,7 @@ size_t clsa_distill_workspace_size(int B, int n_max, int L, int Hq, int Hkv, int
 clsa_status clsa_distill_target(const void* Q, const void* K, const float* scores, const int32_t* seq_lens, int B,
                                 int n_max, int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* abar,
                                 float* kl, void* ws, size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   clsa_status st = check_attn(B, n_max, L, Hq, Hkv, d, dt, kMaxDirectK);
   if (st != CLSA_OK) return st;
   if (!Q || !K || !scores || !seq_lens || !kl) return CLSA_ERR_INVALID_ARG;
@@ -276,7 +318,7 @@ size_t clsa_decode_workspace_size(const clsa_decode_args* a) {
 }
 
 clsa_status clsa_decode_step(const clsa_decode_args* a, void* ws, size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   clsa_status st = check_decode(a);
   if (st != CLSA_OK) return st;
   const DecodeLayout lay = decode_layout(a);
@@ -311,7 +353,7 @@ size_t clsa_prefill_workspace_size(const clsa_prefill_args* a) {
 }
 
 clsa_status clsa_prefill_chunk(const clsa_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {
-  CallScope scope;
+  CallScope scope(stream);
   if (!a) return CLSA_ERR_INVALID_ARG;
   clsa_status st = check_attn(a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype);
   if (st != CLSA_OK) return st;

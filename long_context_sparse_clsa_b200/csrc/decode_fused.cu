@@ -34,6 +34,7 @@
 //  5. Splits of one head meet at a barrier and merge with the log-sum-exp rule.
 //
 // Every wait is bounded (kWaitLimitNs); running out records CLSA_ERR_TIMEOUT.
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 
@@ -58,6 +59,7 @@ constexpr int kSTR = kD + 8;          // padded bf16 row in shared memory
 constexpr int kMaxUnitTok = 4096;     // tokens one unit can hold (k <= 4096); also slice scores kept on chip
 constexpr int kCandCap = 16384;       // candidate slots kept in shared memory (key + index)
 constexpr int kMaxGroups = 256;       // CTAs per launch
+constexpr int kMaxDevices = 64;       // host-side per-device state
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -1399,16 +1401,14 @@ struct FusedCfg {
   bool ok = false;
 };
 
+// computed from the current device's attributes on every call (device_info() caches
+// them per host thread and device), so mixed devices and host threads get their own
 FusedCfg fused_cfg() {
-  static FusedCfg cfg;
-  static bool done = false;
-  if (!done) {
-    done = true;
-    const DeviceInfo& di = device_info();
-    if (di.sm_count > 0 && (size_t)di.max_smem_optin >= smem_bytes()) {
-      cfg.ncta = std::min(di.sm_count, kMaxGroups);
-      cfg.ok = true;
-    }
+  FusedCfg cfg;
+  const DeviceInfo& di = device_info();
+  if (di.sm_count > 0 && (size_t)di.max_smem_optin >= smem_bytes()) {
+    cfg.ncta = std::min(di.sm_count, kMaxGroups);
+    cfg.ok = true;
   }
   return cfg;
 }
@@ -1451,8 +1451,11 @@ template <int DIDX>
 cudaError_t launch_fused(const FusedParams& p, int ncta, size_t smem, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<DIDX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  static bool pdl_ok = true;
-  if (pdl_ok) {
+  // per device: whether the runtime took the pair of launch attributes there
+  static std::atomic<int> pdl_refused[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  if (pdl_refused[dev].load(std::memory_order_relaxed) == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ncta);
     cfg.blockDim = dim3(kThreads);
@@ -1468,7 +1471,7 @@ cudaError_t launch_fused(const FusedParams& p, int ncta, size_t smem, cudaStream
     e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<DIDX>, p);
     if (e != cudaErrorNotSupported && e != cudaErrorInvalidValue) return e;
     (void)cudaGetLastError();
-    pdl_ok = false;
+    pdl_refused[dev].store(1, std::memory_order_relaxed);
   }
   void* args[] = {(void*)&p};
   return cudaLaunchCooperativeKernel((const void*)decode_fused_kernel<DIDX>, dim3(ncta), dim3(kThreads), args, smem, s);
@@ -1518,7 +1521,7 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   p.Ml = reinterpret_cast<float*>(w);
   const size_t smem = smem_bytes();
   const cudaError_t e = a->d_idx == 128 ? launch_fused<128>(p, cfg.ncta, smem, s) : launch_fused<64>(p, cfg.ncta, smem, s);
-  launches_add(1);
+  launches_add(1, s);
   return e;
 }
 

@@ -218,7 +218,7 @@ cudaError_t launch_distill(const void* Q, const void* K, const float* scores, co
   if (e != cudaSuccess) return e;
   // 2. lse of the scores
   lse_kernel<<<B, 256, 0, s>>>(scores, lens, n_max, lse_I);
-  launches_add(1);
+  launches_add(1, s);
   // 3. Abar and the tile partials of the KL
   DistillParams p{Q, K, scores, lens, lse_row, lse_I, abar, partial, B, n_max, L, Hq, Hkv, Hq / Hkv, ntiles, scale};
   const dim3 grid(ntiles, B);
@@ -236,11 +236,11 @@ cudaError_t launch_distill(const void* Q, const void* K, const float* scores, co
     else CLSA_DISTILL(float, 64);
   }
 #undef CLSA_DISTILL
-  launches_add(1);
+  launches_add(1, s);
   if (e != cudaSuccess) return e;
   // 4. per-sequence KL
   kl_kernel<<<B, 32, 0, s>>>(partial, ntiles, kl);
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

@@ -501,7 +501,7 @@ cudaError_t launch_distill_tc(const void* Q, const void* K, const float* scores,
                    n_max, pl.HG, 1.f / (float)(L * Hq), abar, tpart, pl.nt);
   if (e == cudaSuccess) e = launch_pdl(distill_kl_kernel, dim3(B), dim3(kKlT), 0, s, (const float*)tpart, pl.nt, kl);
   if (e != cudaSuccess) return e;
-  launches_add(4);
+  launches_add(4, s);
   return cudaGetLastError();
 }
 

@@ -54,7 +54,7 @@ cudaError_t launch_gather_kv(const void* K, const void* V, const int32_t* idx, c
   gather_kv_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(K), static_cast<const uint4*>(V), idx, count,
                                         n_max, k, row_vec, static_cast<uint4*>(K_S), static_cast<uint4*>(V_S),
                                         ws_header);
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

@@ -107,7 +107,7 @@ cudaError_t launch_t(const void* q, const void* kx, const int32_t* lens, int B, 
   dim3 grid(gx, B);
   index_scores_kernel<T, DIDX, UNROLL><<<grid, 256, 0, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(kx), lens, n_max, scores);
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

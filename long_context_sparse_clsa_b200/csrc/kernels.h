@@ -15,9 +15,16 @@ struct DeviceInfo {
 };
 const DeviceInfo& device_info();
 
-// per-host-thread count of kernel launches in the current API call
+// per-host-thread count of kernel launches in the current API call; an entry point
+// holds a CallScope (with its stream) for its duration, so clsa_last_launch_count()
+// reports its launches, and a call armed by clsa_time_next_call records its events
+struct CallScope {
+  explicit CallScope(void* stream = nullptr);
+  ~CallScope();
+};
 void launches_reset();
-void launches_add(int n);
+// after each kernel launch (or group of n launches) on stream s
+void launches_add(int n, cudaStream_t s);
 int launches_get();
 
 // ----- indexer scan (routing equation, scores) ------------------------------

@@ -10,6 +10,8 @@
 //   2. per-row exact radix TopK (the decode top-k kernel with causal lengths)
 //   3. per-row sparse attention of every layer (the decode attention kernel in
 //      gather mode, each row its own sequence over the one shared cache)
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
@@ -171,7 +173,10 @@ clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_bo
   const int nsm = std::max(1, device_info().sm_count);
   const auto* q = static_cast<const __nv_bfloat16*>(a->q_idx);
   const auto* kx = static_cast<const __nv_bfloat16*>(a->k_idx);
-  const int smem = (a->d_idx / 64) * (kTcM + kTcN) * 128;
+  // Each CTA holds 256 TMEM columns of the SM's 512, so at most two may share an SM: the
+  // d_idx = 64 tiles (49 KB) are padded to 80 KB of shared memory, which lets no third
+  // CTA in (a third would wait in tcgen05.alloc until one of the two finished).
+  const int smem = std::max((a->d_idx / 64) * (kTcM + kTcN) * 128, 80 * 1024);
   auto scores_kernel = [&](const int32_t* only_rows, const uint32_t* any_flag) {
     if (a->d_idx == 128) {
       cudaFuncSetAttribute(prefill_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -182,7 +187,7 @@ clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_bo
       prefill_scores_tc_kernel<64><<<2 * nsm, 128, smem, s>>>(q, kx, a->n, a->T, scores, ws_header, only_rows,
                                                                 any_flag);
     }
-    launches_add(1);
+    launches_add(1, s);
     return cudaGetLastError();
   };
   cudaError_t e;

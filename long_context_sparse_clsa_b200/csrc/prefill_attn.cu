@@ -360,7 +360,7 @@ cudaError_t launch_prefill_attn_tc(const clsa_prefill_args* a, float scale, void
   if (e != cudaSuccess) return e;
   const long long units = (long long)a->Hkv * p.nlg * a->T;
   prefill_attn_tc_kernel<<<(unsigned)units, kThreadsPA, smem, s>>>(p);
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

@@ -635,10 +635,10 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
                                        (int)kRouteSmem);
   if (e != cudaSuccess) return e;
   prefill_route_kernel<<<rp.grid, kRThreads, kRouteSmem, s>>>(tq, tk, p);
-  launches_add(1);
+  launches_add(1, s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prefill_densify_kernel<<<a->T, 256, 0, s>>>(p, out->dval, out->dtok, out->dlen, out->flag, rp.ldd);
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

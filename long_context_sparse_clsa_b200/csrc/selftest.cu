@@ -36,7 +36,7 @@ cudaError_t launch_selftest_timeout(int which, void* ws_header, void* ws_body, c
   cudaError_t e = cudaMemsetAsync(word, 0, sizeof(uint32_t), s);  // a fresh barrier word
   if (e != cudaSuccess) return e;
   selftest_timeout_kernel<<<1, 32, 0, s>>>(which, word, ws_header);
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

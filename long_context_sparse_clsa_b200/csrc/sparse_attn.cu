@@ -585,7 +585,7 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
     }
 #undef CLSA_ATTN_F32
   }
-  launches_add(1);
+  launches_add(1, s);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.nsplit == 1) return e;
   const int rows_total = sh.L * sh.B * sh.Hq;
@@ -597,7 +597,7 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
     if (sh.d == 128) attn_combine_kernel<float, 128><<<cg, 256, 0, s>>>(p);
     else attn_combine_kernel<float, 64><<<cg, 256, 0, s>>>(p);
   }
-  launches_add(1);
+  launches_add(1, s);
   return cudaGetLastError();
 }
 

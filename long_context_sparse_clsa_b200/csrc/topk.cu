@@ -11,6 +11,7 @@
 //
 // The C CTAs of one row meet at four barriers (group_barrier: bounded wait,
 // reusable state).  C > 1 requires a cooperative launch; C == 1 rows need none.
+#include <atomic>
 #include "common.cuh"
 #include "kernels.h"
 
@@ -261,12 +262,18 @@ struct TopkLaunchCfg {
 };
 
 TopkLaunchCfg topk_cfg(int B, int n_max) {
-  static int per_sm = -1;
-  if (per_sm < 0) {
+  // resident CTAs per SM, per device (0: not yet queried; a benign race stores the same value)
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> per_sm_dev[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  int per_sm = per_sm_dev[dev].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
     int v = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, topk_kernel, kThreads, 0) != cudaSuccess || v < 1)
       v = 1;
     per_sm = v;
+    per_sm_dev[dev].store(v, std::memory_order_relaxed);
   }
   const int resident = per_sm * device_info().sm_count;
   int C = (n_max + 1023) / 1024;
@@ -298,7 +305,7 @@ cudaError_t launch_topk(const float* scores, const int32_t* seq_lens, int B, int
   cudaError_t e;
   if (C > 1) e = cudaLaunchCooperativeKernel((const void*)topk_kernel, grid, dim3(kThreads), args, 0, s);
   else e = cudaLaunchKernel((const void*)topk_kernel, grid, dim3(kThreads), args, 0, s);
-  launches_add(1);
+  launches_add(1, s);
   return e;
 }
 

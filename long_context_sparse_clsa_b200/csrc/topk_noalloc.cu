@@ -13,6 +13,10 @@
 // call first clears the part it uses (error word, histograms, barrier state)
 // with cudaMemsetAsync on the caller's stream.  Calls whose work overlaps on
 // the GPU (different streams, or different host threads) race on the array.
+//
+// The looked-up address belongs to the device's primary context.  A process that
+// destroys that context (cudaDeviceReset) must not call this entry point on that
+// device again: the cached address would no longer be mapped.
 #include <mutex>
 
 #include "common.cuh"
@@ -54,7 +58,7 @@ cudaError_t scratch_address(void** out) {
 extern "C" clsa_status clsa_topk_noalloc(const float* scores, const int32_t* seq_lens, int B, int n_max, int k,
                                          int32_t* idx, int32_t* count, void* stream) {
   using namespace clsa;
-  launches_reset();
+  CallScope scope(stream);
   if (!scores || !seq_lens || !idx || !count || B < 1 || n_max < 1 || k < 1) return CLSA_ERR_INVALID_ARG;
   if (k > 4096) return CLSA_ERR_UNSUPPORTED;
   for (const void* p : {(const void*)scores, (const void*)seq_lens, (const void*)idx, (const void*)count})
