@@ -511,6 +511,19 @@ def run_clsa(args):
     if st[0] != "CLSA_OK":
         raise RuntimeError(f"device error during the end-to-end timing: {st}")
 
+    # selection path of one extra step, read from the library's phase trace: CTAs whose group
+    # resolved the TopK from the candidate windows, and CTAs whose group took the whole-row path
+    sel_path = None
+    if launches_per_step == 1:
+        os.environ["CLSA_TRACE"] = "1"
+        clsa.decode_step_args(args_sets[0], ws)
+        torch.cuda.synchronize()
+        del os.environ["CLSA_TRACE"]
+        tr = clsa.fused_decode_trace(ws)
+        used = (tr[:, 0] > 0) & ((tr[:, 31] & 0xFFFFFFFF) > 0)
+        fast = int(((tr[:, 31] >> 32) > 0)[used].sum())
+        sel_path = {"ctas_window_path": fast, "ctas_whole_row_path": int(used.sum()) - fast}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, threads, note = time_oracle(inp, w, args.cpu_sample_steps)
@@ -541,6 +554,7 @@ def run_clsa(args):
         "e2e": {"value": replicas.job_rate(world, B, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "launch": e2e_launch},
         "gpu_launches": launches_per_step * args.steps,
+        "selection": sel_path,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
     }

@@ -181,6 +181,15 @@ class Workspace:
         return STATUS.get(code, str(code)), detail.value
 
 
+def fused_decode_trace(ws: Workspace):
+    """Diagnostics of the fused decode step: the per-CTA phase stamps the last step wrote into
+    ``ws`` when the library ran with CLSA_TRACE=1 in the environment (int64 [256][64]:
+    globaltimer ns per phase; a row whose slot 0 is 0 belongs to no CTA of that step).
+    Slot 31 holds the CTA's candidate slot count, plus 2^32 when the candidate windows decided
+    the TopK (0 there: the group took the whole-row selection)."""
+    return ws.buf[256:256 + 256 * 64 * 8].view(torch.int64).view(256, 64).cpu()
+
+
 # ---------------------------------------------------------------------------- calls
 
 def index_scores(q_idx, k_idx, seq_lens, scores=None):

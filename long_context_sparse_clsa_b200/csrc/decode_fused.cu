@@ -16,26 +16,32 @@
 //     (L2-resident), and feed a 12-bit key histogram of the slice.
 //  2. Candidates.  From its own histogram a CTA picks the bound E: the lowest bin edge
 //     with at most win of its tokens at or above it.  It writes those tokens, in token
-//     order, to its window of the candidate list, and E beside them.  No CTA waits
-//     for another before this point.
-//  3. One barrier for the group.  Every CTA then resolves the exact TopK from the
-//     candidate list by itself (a linear-key histogram and an exact rank count in the
-//     boundary bin; ties to the earlier list position = lower token index).  The
-//     result is the TopK of the row iff every CTA's bound E is at or below the k_eff-th
-//     candidate key (a token left out of a window scores below its E); otherwise, or
-//     with too few candidates, the same selection runs digit by digit over the whole
-//     row of scores.  The selected tokens are ranked in ascending token order; each
-//     CTA writes its share of idx and keeps the tokens of its attention unit.
+//     order, to its window of the candidate list, and adds its histogram bins at or
+//     above E into the group's coarse histogram in global memory (L2 reductions), with
+//     E and its largest key folded into group maxima.  No CTA waits for another before
+//     this point.
+//  3. One barrier for the group.  Every CTA then reads the coarse histogram between the
+//     largest bound E_max and the largest key.  It counts every token of those bins (each
+//     CTA added all its bins at or above its own E <= E_max), so it gives the boundary
+//     bin of the k_eff-th key and the count above it; only the candidates of that bin are
+//     histogrammed again (12 more key bits), and the few keys of the boundary sub-bin
+//     are ranked exactly (ties to the earlier list position = lower token index).  If
+//     fewer than k_eff tokens lie at or above E_max, or the sub-bin holds heavy ties,
+//     the same selection runs digit by digit over the whole row of scores.  Selected
+//     tokens are ranked in ascending token order from per-window counts; each CTA
+//     writes its own window's share of idx and keeps the tokens of its attention unit.
 //  4. Attention.  A unit is (KV head g, split s of the selected ranks); its rows
 //     are all L*G (layer, query head) pairs of head g, so every selected K/V row is
 //     read once for all layers.  tcgen05.mma bf16 -> fp32 in TMEM over 64-token
 //     chunks (S = Q K^T, then P V with V as an MN-major operand), online softmax in
 //     exp2 with the output accumulated in registers.
-//  5. Splits of one head meet at a barrier and merge with the log-sum-exp rule.
+//  5. Each split publishes its partial with a flag; the splits of one head merge each
+//     other's partials (log-sum-exp rule) as their flags appear.
 //
 // Every wait is bounded (kWaitLimitNs); running out records CLSA_ERR_TIMEOUT.
 #include <atomic>
 #include <cmath>
+#include <cstdio>
 #include <cstdlib>
 
 #include "common.cuh"
@@ -63,13 +69,20 @@ constexpr int kMaxDevices = 64;       // host-side per-device state
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// per-row global state (u32 words)
-constexpr int kRowBound = 0;                      // [kMaxGroups] each CTA's candidate bound E (key)
-constexpr int kRowMax = kMaxGroups;               // [kMaxGroups] an upper bound on each CTA's largest key
-constexpr int kRowBar = kTauBins + 256 + 32;      // row-group barrier state [2]
-constexpr int kRowCnt = kTauBins + 256 + 64;      // [kMaxGroups] candidate count per CTA
-constexpr int kRowHeadBar = kRowCnt + kMaxGroups; // [Hkv][2] head-group barrier states (<= 64 heads)
-constexpr int kRowWords = kRowHeadBar + 128;
+// per-row global state (u32 words).  The group histogram of 16-bit key bins has two
+// copies: launch e of a row uses copy e & 1 and the bin-range words of slot e & 3; at its
+// start it clears the bins copy (e - 1) & 1 had touched (range slot (e - 1) & 3) and zeroes
+// slot (e + 1) & 3, so no CTA clears shared state at the end of a launch.  e is the row's
+// own counter (the last CTA of the launch adds one for every row it processed).
+constexpr int kH16Bits = 16;
+constexpr int kH16Bins = 1 << kH16Bits;
+constexpr int kRowEpoch = 0;                      // the row's launch counter
+constexpr int kRowRange = 4;                      // [4][4] per epoch slot: E_max, key max, (kH16Bins - 1 - lowest bin), -
+constexpr int kRowBar = 32;                       // row-group barrier state [2]
+constexpr int kRowFlag = 256;                     // [kMaxGroups] per CTA of the group: its split partial
+                                                  // is written (the row's launch counter + 1)
+constexpr int kRowH16 = 512;                      // [2][kH16Bins] group histograms of the 16-bit key bins
+constexpr int kRowWords = kRowH16 + 2 * kH16Bins;
 
 struct FusedParams {
   const __nv_bfloat16* q_idx;
@@ -93,9 +106,11 @@ struct FusedParams {
   unsigned long long* trace;  // [gridDim][16] globaltimer stamps per phase, or null
   int B, n_max, k, L, Hq, Hkv, G, rows, nsplit_max;
   float scale_log2;
+  float pf_mult;       // K/V rows of a CTA's likely-selected tokens are prefetched into L2:
+  uint32_t pf_add;     // its top pf_mult * e + pf_add tokens (to the key-bin granularity)
 };
 
-constexpr int kTraceSlots = 32;
+constexpr int kTraceSlots = 64;
 __device__ __forceinline__ void stamp(const FusedParams& p, int phase) {
   if (p.trace && threadIdx.x == 0) {
     p.trace[blockIdx.x * kTraceSlots + phase] = globaltimer_ns();
@@ -120,19 +135,24 @@ struct Smem {
   uint32_t tmem_base;
   int abort_flag;
   uint32_t tau_key;
-  int all_selected;
-  int ctot, fast;        // candidate count; candidates held in shared memory
   uint32_t theta, ties_needed;
   int sel_bin;
   uint32_t sel_above;
   uint32_t warp_tot[kWarps];
   uint32_t warp_tot2[kWarps + 1];
   int seg_off[kMaxGroups + 1];
+  int seg_cnt[kMaxGroups];
+  uint32_t b16, above16, m16;
+  int sel_ok;
+  int leave_last;
+  uint32_t live_rows[4];                // rows with tokens (the fused path takes B <= 128)
+  __align__(16) uint32_t row_hdr[20];   // the row's epoch and range slots (async copy at entry)
+  uint32_t grp_emax, grp_kmax;
   __align__(16) uint32_t hist[kBins];
-  uint32_t red_min[kWarps], red_max[kWarps];
+  uint32_t red_max[kWarps];
   uint32_t theta_key, theta_pos;
   int list_n;
-  uint32_t slice_max, emax, kmax, pf_key;
+  uint32_t slice_max, pf_key;
   union {                          // slice scores until the candidates are out, then the
     float score[kMaxUnitTok];      // boundary-bin list of the selection, then unit tokens
     int unit_tok[kMaxUnitTok];
@@ -230,6 +250,24 @@ __device__ __forceinline__ uint32_t block_flag_scan(bool flag, uint32_t* warp_to
   return before;
 }
 
+// Exclusive prefix of v over the block in thread order with a single barrier: every warp
+// reads the 16 warp totals itself (redux).  wt [kWarps] must not be written again until a
+// later barrier has passed (alternate two arrays between back-to-back calls).
+__device__ __forceinline__ uint32_t block_excl_scan1(uint32_t v, uint32_t* wt, uint32_t* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wt[w] = incl;
+  __syncthreads();
+  const uint32_t t = lane < kWarps ? wt[lane] : 0u;
+  *total = __reduce_add_sync(0xffffffffu, t);
+  return __reduce_add_sync(0xffffffffu, lane < w ? t : 0u) + incl - v;
+}
+
 // histogram increment (plain shared atomics measured ~9x faster here than warp aggregation)
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) { atomicAdd(&hist[bin], 1u); }
 
@@ -286,15 +324,19 @@ __device__ void select_bin_wide(Smem& sm, const uint32_t* hist, int nbins, uint3
 // ---------------------------------------------------------------------------
 // work partition (computed identically by every CTA from seq_lens)
 // ---------------------------------------------------------------------------
-__device__ void make_plan(const FusedParams& p, Plan& pl) {
+// live: bit b set for every row with tokens (rows < 128)
+__device__ void make_plan(const FusedParams& p, Plan& pl, uint32_t* live) {
   const int ncta = gridDim.x;
   long long total = 0;
   int nb = 0;
+#pragma unroll 1
+  for (int w = 0; w < 4; ++w) live[w] = 0u;
 #pragma unroll 1
   for (int b = 0; b < p.B; ++b) {
     const int len = max(0, min(p.seq_lens[b], p.n_max));
     total += len;
     nb += len > 0;
+    if (len > 0) live[b >> 5] |= 1u << (b & 31);
   }
   pl.b = -1;
   if (nb == 0) return;
@@ -315,11 +357,11 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
       const int chunk = (len + Cb - 1) / Cb;
       pl.r0 = min(len, pl.c * chunk);
       pl.r1 = min(len, pl.r0 + chunk);
-      // window: the expected share e = k_eff / C_b of the TopK per CTA plus 6 sqrt(e) + 4
-      // (a CTA holding more TopK tokens than its window sends the group to the whole-row
-      // path); all windows of the group fit kCandCap
+      // window: 1.5 e + 4 sqrt(e) + 4 slots for the expected share e = k_eff / C_b of the
+      // TopK per CTA (a CTA holding more TopK tokens than its window sends the group to
+      // the whole-row path); all windows of the group fit kCandCap
       const float e = (float)pl.keff / (float)Cb;
-      const int wn = ((int)ceilf(e + 6.f * sqrtf(e) + 4.f) + 3) & ~3;
+      const int wn = ((int)ceilf(1.5f * e + 4.f * sqrtf(e) + 4.f) + 3) & ~3;
       pl.win = max(4, min(wn, (kCandCap / Cb) & ~3));
       break;
     }
@@ -346,23 +388,54 @@ __device__ void make_plan(const FusedParams& p, Plan& pl) {
 }
 
 // The count-barrier words are zeroed by the last CTA to leave them: every CTA counts
-// itself in p.leave right after its last count barrier (leave_issue) and reads the
-// old count only at its end (leave_finish), so no barrier waits on that atomic.  The
+// itself in p.leave right after its last count barrier and its last read of the group
+// state (leave_issue) and reads the old count only at its end (leave_finish), so no
+// barrier waits on that atomic.  The
 // CTA that saw gridDim.x - 1 runs after every CTA has stopped polling, and the next
 // launch starts from zeroed words.
+// A relaxed add: the CTA does not wait for it (an acquire here would hold the whole CTA for
+// an L2 round trip); its old value is read only at the end, in leave_finish.
 __device__ __forceinline__ uint32_t leave_issue(const FusedParams& p) {
   return threadIdx.x == 0 ? atomicAdd(p.leave, 1u) : 0u;
 }
-__device__ __forceinline__ void leave_finish(const FusedParams& p, uint32_t old) {
-  if (threadIdx.x != 0 || old != gridDim.x - 1) return;
-#pragma unroll 1
-  for (int b = 0; b < p.B; ++b) {
+__device__ __forceinline__ void red_max_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Called by every thread of the CTA.  The last CTA to leave returns the barrier words to
+// zero and advances the launch counter of every row it processed (a row with tokens).
+__device__ void leave_finish(const FusedParams& p, Smem& sm, uint32_t old) {
+  if (threadIdx.x == 0) sm.leave_last = old == gridDim.x - 1;
+  __syncthreads();
+  if (!sm.leave_last) return;
+  for (int b = threadIdx.x; b < p.B; b += kThreads) {
     uint32_t* rw = p.row_ws + (size_t)b * kRowWords;
     rw[kRowBar] = 0u;
-#pragma unroll 1
-    for (int g = 0; g < p.Hkv; ++g) rw[kRowHeadBar + 2 * g] = 0u;
+    if ((sm.live_rows[b >> 5] >> (b & 31)) & 1u) red_add_gpu(rw + kRowEpoch, 1u);
   }
-  *p.leave = 0u;
+  if (threadIdx.x == 0) *p.leave = 0u;
+}
+
+// The row's header (launch counter and range slots) into shared memory by async copies
+// (5 x 16 bytes), issued with the first copies of the launch; read after the scan.
+__device__ __forceinline__ void load_row_header(const FusedParams& p, Smem& sm, int b) {
+  if (threadIdx.x < 5) cp_async_16(sm.row_hdr + 4 * threadIdx.x, p.row_ws + (size_t)b * kRowWords + 4 * threadIdx.x, 16);
+  cp_async_commit();
+}
+
+// Launch e of a row: clear the bins launch e - 1 touched in the other histogram copy (the
+// group's CTAs share the range), and zero the range slot of launch e + 1.
+__device__ void clear_previous_copy(const FusedParams& p, const Smem& sm, const Plan& pl) {
+  uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
+  const uint32_t e = sm.row_hdr[kRowEpoch];
+  const uint32_t* pr = sm.row_hdr + kRowRange + ((e - 1u) & 3u) * 4;
+  const int lo = kH16Bins - 1 - (int)pr[2], hi = (int)(pr[1] >> (32 - kH16Bits));
+  uint32_t* old = rw + kRowH16 + ((e - 1u) & 1u) * kH16Bins;
+  for (int i = lo + pl.c * kThreads + (int)threadIdx.x; i <= hi; i += pl.Cb * kThreads) old[i] = 0u;
+  if (pl.c == 0 && threadIdx.x < 4) rw[kRowRange + ((e + 1u) & 3u) * 4 + threadIdx.x] = 0u;
 }
 
 template <int DIDX>
@@ -460,6 +533,8 @@ __device__ __forceinline__ void scan_rows(const FusedParams& p, Smem& sm, uint32
   cp_async_wait<0>();
 }
 
+__device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, unsigned char* sQa);
+
 // this thread's 16-byte chunk of q_idx[b] (the chunk its scan lane multiplies)
 template <int DIDX>
 __device__ __forceinline__ uint4 load_q_chunk(const FusedParams& p, int b) {
@@ -469,8 +544,10 @@ __device__ __forceinline__ uint4 load_q_chunk(const FusedParams& p, int b) {
 // started: the stream was begun by scan_start at entry, and qv holds load_q_chunk of the
 // sequence (both issued before the plan, so their latency overlaps it)
 template <int DIDX>
+// sQa: the attention unit's Q tile is loaded right behind the first stages of the stream
+// (null: this CTA attends nothing)
 __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigned char* ring, bool hist,
-                           bool started, uint4 qv) {
+                           bool started, uint4 qv, unsigned char* sQa) {
   const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   const int nrows = pl.r1 - pl.r0;
   const __nv_bfloat16* src = p.k_idx + ((size_t)pl.b * p.n_max + pl.r0) * DIDX;
@@ -483,7 +560,11 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigne
     unpack_bf16x2(qv.z, q[4], q[5]);
     unpack_bf16x2(qv.w, q[6], q[7]);
   }
-  if (!started) scan_start<DIDX>(reinterpret_cast<uint4*>(ring), src, 0, nrows);
+  if (!started) {
+    load_row_header(p, sm, pl.b);
+    scan_start<DIDX>(reinterpret_cast<uint4*>(ring), src, 0, nrows);
+  }
+  if (sQa) load_q_tile(p, pl.b, pl.unit_g0, sQa);
   stamp(p, 24);
   for (int i = threadIdx.x; i < kTauBins; i += kThreads) th[i] = 0;
   __syncthreads();
@@ -497,20 +578,26 @@ __device__ bool scan_slice(const FusedParams& p, Smem& sm, uint32_t* th, unsigne
 // ---------------------------------------------------------------------------
 // phase 2: candidate bound tau from the group histogram, candidate segment
 // ---------------------------------------------------------------------------
-__device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
+constexpr int kCandRun = 8;  // tokens per thread per pass of the candidate writer (4096 per pass)
+
+__device__ void write_candidates(const FusedParams& p, Smem& sm, const uint32_t* th) {
   const Plan pl = sm.plan;  // a copy: loops below store to shared memory
   uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
+  const uint32_t epoch = sm.row_hdr[kRowEpoch];
+  uint32_t* h16 = rw + kRowH16 + (epoch & 1u) * kH16Bins;
+  uint32_t* rng = rw + kRowRange + (epoch & 3u) * 4;
   // The local bound E: the lower edge of the lowest 12-bit key bin such that the slice
-  // holds at most win tokens at or above it (E = 0: every token).  Thread t sums the
+  // holds at most win tokens at or above it (E = 0: every token).  Thread t holds the
   // eight bins 4088 - 8t .. 4095 - 8t; one scan from the top finds the bin.
+  const int hi = kTauBins - 8 * threadIdx.x;  // this thread's bins: [hi - 8, hi)
+  uint32_t h[8], local = 0;
   {
-    const int hi = kTauBins - 8 * threadIdx.x;  // this thread's bins: [hi - 8, hi)
-    uint32_t h[8], local = 0;
+    const uint4 x0 = *reinterpret_cast<const uint4*>(th + hi - 8), x1 = *reinterpret_cast<const uint4*>(th + hi - 4);
+    h[0] = x0.x, h[1] = x0.y, h[2] = x0.z, h[3] = x0.w, h[4] = x1.x, h[5] = x1.y, h[6] = x1.z, h[7] = x1.w;
+  }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      h[i] = th[hi - 8 + i];
-      local += h[i];
-    }
+  for (int i = 0; i < 8; ++i) local += h[i];
+  {
     uint32_t top = 0;  // 1 + the highest non-empty bin of this thread's run (0: none)
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -518,12 +605,13 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
     top = __reduce_max_sync(0xffffffffu, top);
     if ((threadIdx.x & 31) == 0) sm.red_max[threadIdx.x >> 5] = top;
     uint32_t total;
-    const uint32_t before = block_scan(local, sm.warp_tot, &total);  // tokens in higher bins (syncs)
-    if (threadIdx.x == 0) {
-      uint32_t t = 0;
-      for (int w2 = 0; w2 < kWarps; ++w2) t = max(t, sm.red_max[w2]);
+    const uint32_t before = block_excl_scan1(local, sm.warp_tot, &total);  // tokens in higher bins
+    stamp(p, 42);
+    if (threadIdx.x < 32) {  // warp 0: the slice's highest non-empty bin (redux over the warp maxima)
+      const uint32_t m = __reduce_max_sync(0xffffffffu, threadIdx.x < kWarps ? sm.red_max[threadIdx.x] : 0u);
       // the upper edge of the highest non-empty bin bounds every key of the slice
-      sm.slice_max = t == 0 ? 0u : (t >= (uint32_t)kTauBins ? 0xFFFFFFFFu : (t << (32 - kTauBits)) - 1u);
+      if (threadIdx.x == 0)
+        sm.slice_max = m == 0 ? 0u : (m >= (uint32_t)kTauBins ? 0xFFFFFFFFu : (m << (32 - kTauBits)) - 1u);
     }
     const uint32_t win = (uint32_t)pl.win;
     if (threadIdx.x == 0 && total <= win) sm.tau_key = 0u;
@@ -539,8 +627,8 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
         acc += h[i];
       }
     }
-    // the prefetch bound: the same rule for ~1.5 e + 8 tokens (the likely selected ones)
-    const uint32_t w2 = min(win, (uint32_t)ceilf(1.5f * (float)pl.keff / (float)pl.Cb) + 8u);
+    // the prefetch bound: the same rule for the likely selected tokens
+    const uint32_t w2 = min(win, (uint32_t)ceilf(p.pf_mult * (float)pl.keff / (float)pl.Cb) + p.pf_add);
     if (threadIdx.x == 0 && total <= w2) sm.pf_key = 0u;
     if (before <= w2 && before + local > w2) {
       uint32_t acc = before;
@@ -556,41 +644,56 @@ __device__ void write_candidates(const FusedParams& p, Smem& sm, uint32_t* th) {
     }
   }
   __syncthreads();
+  stamp(p, 43);
   const uint32_t tau = sm.tau_key, pf = sm.pf_key;
-  // this CTA's tokens with key >= tau, in token order, to its window of win slots
+  // This CTA's tokens with key >= tau, in token order, to its window of win slots; each one
+  // adds 1 to its 16-bit bin of the group histogram.  Thread t takes a contiguous run of
+  // the pass's tokens (all its keys loaded before any store), one block scan places them.
   const float* gsc = p.scores + (size_t)pl.b * p.n_max + pl.r0;
   const int n = pl.r1 - pl.r0;
   const bool on_chip = n <= kMaxUnitTok;
   uint32_t* ck = p.cand_key + (size_t)pl.b * kCandCap + (size_t)pl.c * pl.win;
   int32_t* ct = p.cand_tok + (size_t)pl.b * kCandCap + (size_t)pl.c * pl.win;
   uint32_t written = 0;
+  int pass = 0;
 #pragma unroll 1
-  for (int base = 0; base < n; base += kThreads) {
-    const int j = base + threadIdx.x;
-    uint32_t key = 0;
-    bool f = false;
-    if (j < n) {
-      key = float_key(on_chip ? sm.score[j] : __ldcg(gsc + j));
-      f = key >= tau;
-    }
+  for (int base = 0; base < n; base += kThreads * kCandRun, ++pass) {
+    const int nb = min(n - base, kThreads * kCandRun);
+    const int run = (nb + kThreads - 1) / kThreads;
+    const int j0 = base + (int)threadIdx.x * run, j1 = min(j0 + run, base + nb);
+    uint32_t m = 0;  // bit u: token j0 + u is a candidate
+#pragma unroll 1
+    for (int j = j0; j < j1; ++j)
+      m |= (uint32_t)(float_key(on_chip ? sm.score[j] : __ldcg(gsc + j)) >= tau) << (j - j0);
     uint32_t tot;
-    const uint32_t pos = written + block_flag_scan(f, sm.warp_tot2, &tot);
-    if (f && pos < (uint32_t)pl.win) {
-      __stcg(ck + pos, key);
-      __stcg(ct + pos, pl.r0 + j);
-      if (key >= pf) {  // a likely TopK token: its K and V rows (all heads) into L2 now
-        const size_t row = ((size_t)pl.b * p.n_max + pl.r0 + j) * p.Hkv * kD;
-        bulk_prefetch_l2(p.K + row, (uint32_t)(p.Hkv * kD * 2));
-        bulk_prefetch_l2(p.V + row, (uint32_t)(p.Hkv * kD * 2));
+    const uint32_t pos0 = written + block_excl_scan1((uint32_t)__popc(m), (pass & 1) ? sm.warp_tot : sm.warp_tot2, &tot);
+    stamp(p, 44);
+    uint32_t pos = pos0;
+#pragma unroll 1
+    while (m != 0u) {
+      const int j = j0 + __ffs(m) - 1;
+      m &= m - 1u;
+      if (pos < (uint32_t)pl.win) {
+        const uint32_t key = float_key(on_chip ? sm.score[j] : __ldcg(gsc + j));
+        const int tok = pl.r0 + j;
+        __stcg(ck + pos, key);
+        __stcg(ct + pos, tok);
+        red_add_gpu(h16 + (key >> (32 - kH16Bits)), 1u);
+        if (key >= pf) {  // a likely TopK token: its K and V rows (all heads) into L2 now
+          const size_t row = ((size_t)pl.b * p.n_max + tok) * p.Hkv * kD;
+          bulk_prefetch_l2(p.K + row, (uint32_t)(p.Hkv * kD * 2));
+          bulk_prefetch_l2(p.V + row, (uint32_t)(p.Hkv * kD * 2));
+        }
       }
+      ++pos;
     }
     written += tot;
   }
   for (int i = (int)written + threadIdx.x; i < pl.win; i += kThreads) __stcg(ck + i, 0u);  // empty slots
-  if (threadIdx.x == 0) {
-    __stcg(rw + kRowCnt + pl.c, written);  // <= win by the choice of the bound
-    __stcg(rw + kRowBound + pl.c, tau);
-    __stcg(rw + kRowMax + pl.c, sm.slice_max);
+  if (threadIdx.x == 0) {  // E and the key bound into the group maxima, the lowest bin touched
+    red_max_gpu(rng + 0, tau);
+    red_max_gpu(rng + 1, sm.slice_max);
+    if (tau != 0xFFFFFFFFu) red_max_gpu(rng + 2, (uint32_t)(kH16Bins - 1 - (int)(tau >> (32 - kH16Bits))));
   }
 }
 
@@ -682,147 +785,193 @@ __device__ void compact_selected(const FusedParams& p, Smem& sm, const CandSrc& 
 }
 
 // ---------------------------------------------------------------------------
-// phase 3 (fast path): candidates on chip.  One histogram over 2048 bins that are
-// linear in key space between the smallest and the largest candidate key, a
-// two-sync search for the boundary bin, then an exact rank count inside that bin
-// (key descending, list position = token order ascending).  theta is the
-// (key, position) pair of the k_eff-th candidate.  False if the boundary bin holds
-// more than 1024 candidates (then the generic digit-by-digit path runs).
+// phase 3 (fast path): the candidate windows of the group are landing in shared memory
+// (skey: keys back to back in CTA order, each window in token order, empty slots key 0).
+//   a. E_max, the key bound and the group histogram of 16-bit key bins between them (one
+//      round trip: the 512 bins above this CTA's own bound, which hold that range unless
+//      it is wider) give the bin B holding the k_eff-th key and the count above it;
+//   b. thread t holds a contiguous run of slots in registers; the keys of bin B are listed;
+//   c. each listed key is ranked exactly (key descending, slot ascending = token
+//      ascending): theta is the (key, slot) of the k_eff-th;
+//   d. the selected slots are ranked in slot order = ascending token order by one block
+//      scan of the per-thread counts; the CTA keeps its unit's tokens and writes idx for
+//      its own window.
+// Returns false when the windows cannot decide (fewer than k_eff tokens at or above
+// E_max, or more than 1024 keys in bin B): the whole-row path runs.
 // ---------------------------------------------------------------------------
-__device__ bool select_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, int P, uint32_t keff,
-                                  uint32_t emax, uint32_t kmax) {
-  if (kmax < emax) return false;
-  for (int i = threadIdx.x; i < 4096; i += kThreads) sm.hist[i] = 0;
-  if (threadIdx.x == 0) sm.list_n = 0;
-  __syncthreads();
-  // stage A: 2048 linear bins over [E_max, kmax]; keys below E_max cannot be selected
-  int shift = 0;
-  while (((kmax - emax) >> shift) >= 2048u) ++shift;
-#pragma unroll 1
-  for (int i0 = threadIdx.x; i0 < P; i0 += 8 * kThreads) {  // 8 keys loaded before any atomic
-    uint32_t k[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) k[u] = i0 + u * kThreads < P ? skey[i0 + u * kThreads] : 0u;
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (k[u] >= emax && k[u] != 0u) atomicAdd(&sm.hist[(k[u] - emax) >> shift], 1u);
+__device__ bool select_windows(const FusedParams& p, Smem& sm, const uint32_t* rw, const uint32_t* skey,
+                               const int32_t* stok, int P) {
+  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
+  const uint32_t keff = (uint32_t)pl.keff;
+  const uint32_t epoch = sm.row_hdr[kRowEpoch];
+  const uint32_t* h16 = rw + kRowH16 + (epoch & 1u) * kH16Bins;
+  const uint32_t* rng = rw + kRowRange + (epoch & 3u) * 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    sm.sel_ok = 0;
+    sm.list_n = 0;
   }
-  __syncthreads();
-  stamp(p, 19);
-  select_bin_wide(sm, sm.hist, 2048, keff);
-  const int T = sm.sel_bin;
-  if (T < 0) return false;                  // fewer than k_eff keys >= E_max: not exact
-  uint32_t need = keff - sm.sel_above;  // rank (1-based) inside bin T
-  const uint32_t loT = emax + ((uint32_t)T << shift);
-  const uint32_t hiT = T == 2047 ? kmax : loT + (1u << shift) - 1u;  // bin T = [loT, hiT]
-  uint32_t lo2 = loT, hi2 = hiT;  // the keys ranked exactly: bin T, or its stage-B sub-bin
-  uint32_t m = sm.hist[T];
-  if (m > 64u) {
-    // stage B (a crowded bin only): 2048 sub-bins of bin T
-    const int shift2 = max(0, shift - 11);
-    uint32_t* hist2 = sm.hist + 2048;
-#pragma unroll 1
-    for (int i0 = threadIdx.x; i0 < P; i0 += 8 * kThreads) {
-      uint32_t k[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) k[u] = i0 + u * kThreads < P ? skey[i0 + u * kThreads] : 0u;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (k[u] >= loT && k[u] <= hiT && k[u] != 0u) atomicAdd(&hist2[(k[u] - loT) >> shift2], 1u);
-    }
+  const uint32_t emax = __ldcg(rng), kmax = __ldcg(rng + 1);
+  int top = (int)(sm.tau_key >> (32 - kH16Bits)) + kThreads - 1;  // this CTA's bound <= E_max
+  int bin = top - (int)threadIdx.x;
+  uint32_t v = bin < kH16Bins ? __ldcg(h16 + bin) : 0u;
+  if (emax == 0xFFFFFFFFu || kmax < emax) {
+    cp_async_wait<1>();
     __syncthreads();
-    select_bin_wide(sm, hist2, 2048, need);
-    const int T2 = sm.sel_bin;
-    need -= sm.sel_above;  // rank inside sub-bin T2
-    m = hist2[T2];
-    lo2 = loT + ((uint32_t)T2 << shift2);
-    hi2 = min(hiT, lo2 + (1u << shift2) - 1u);
+    return false;
   }
-  if (m > 1024u) return false;  // heavy ties: the digit-by-digit path
-  stamp(p, 20);
-  stamp(p, 21);
-  // the keys of that bin (few) with their list positions
+  const int lo = (int)(emax >> (32 - kH16Bits)), hi = (int)(kmax >> (32 - kH16Bits));
+  uint32_t acc = 0;  // keys in the bins above the current run of 512
+  int pass = 0;
+  if (hi > top) {  // a range wider than the speculative run: runs of 512 from the top
+    top = hi;
+    bin = top - (int)threadIdx.x;
+    v = __ldcg(h16 + bin);
+  }
 #pragma unroll 1
-  for (int i0 = threadIdx.x; i0 < P; i0 += 8 * kThreads) {
-    uint32_t k[8];
+  for (;; ++pass) {
+    const uint32_t x = bin >= lo && bin <= hi ? v : 0u;
+    uint32_t tot;
+    const uint32_t before = acc + block_excl_scan1(x, (pass & 1) ? sm.warp_tot2 : sm.warp_tot, &tot);
+    if (before < keff && keff <= before + x) {
+      sm.b16 = (uint32_t)bin;
+      sm.above16 = before;
+      sm.m16 = x;
+      sm.sel_ok = 1;
+    }
+    if (pass == 0) cp_async_wait<1>();  // the window keys (the tokens may still be in flight)
+    __syncthreads();
+    if (sm.sel_ok || top - kThreads < lo) break;
+    acc += tot;
+    top -= kThreads;
+    bin = top - (int)threadIdx.x;
+    v = bin >= 0 ? __ldcg(h16 + bin) : 0u;
+  }
+  stamp(p, 4);
+  if (!sm.sel_ok || sm.m16 > 1024u) return false;  // too few keys at or above E_max / heavy ties
+  const uint32_t b16 = sm.b16, need = keff - sm.above16, m = sm.m16;
+  // b. thread t takes the contiguous slots [t seg, t seg + seg) of the concatenated windows,
+  //    four at a time (16-byte loads, a rolled loop: few instructions per slot); the keys of
+  //    bin B go to the list.  Empty slots (key 0) never fall in bin B: B >= the bin of E_max,
+  //    and every finite score has a key above 0x007FFFFF.
+  const int seg = ((P + kThreads - 1) / kThreads + 3) & ~3;
+  const int s0 = (int)threadIdx.x * seg, s1 = min(s0 + seg, P);
+  uint32_t inb = 0;   // bit u: slot s0 + u is in bin B (seg <= 32)
+  uint32_t above = 0; // slots of this thread in bins above B (all of them selected)
+  {
+#pragma unroll 1
+    for (int u = 0; s0 + u < s1; u += 4) {
+      const uint4 x = *reinterpret_cast<const uint4*>(skey + s0 + u);
+      const uint32_t b0 = x.x >> (32 - kH16Bits), b1 = x.y >> (32 - kH16Bits), b2 = x.z >> (32 - kH16Bits),
+                     b3 = x.w >> (32 - kH16Bits);
+      inb |= (uint32_t)(b0 == b16) << u | (uint32_t)(b1 == b16) << (u + 1) | (uint32_t)(b2 == b16) << (u + 2) |
+             (uint32_t)(b3 == b16) << (u + 3);
+      above += (uint32_t)(b0 > b16) + (uint32_t)(b1 > b16) + (uint32_t)(b2 > b16) + (uint32_t)(b3 > b16);
+    }
+    const uint32_t n = (uint32_t)__popc(inb);
+    if (__any_sync(0xffffffffu, n != 0u)) {  // warp-aggregated: one list reservation per warp
+      uint32_t pre = n;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) k[u] = i0 + u * kThreads < P ? skey[i0 + u * kThreads] : 0u;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (k[u] >= lo2 && k[u] <= hi2 && k[u] != 0u) {
-        const int q = atomicAdd(&sm.list_n, 1);
-        sm.list_key[q] = k[u];
-        sm.list_pos[q] = i0 + u * kThreads;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += y;
+      }
+      int base = 0;
+      if (lane == 31) base = atomicAdd(&sm.list_n, (int)pre);
+      base = __shfl_sync(0xffffffffu, base, 31) + (int)(pre - n);
+      uint32_t mm = inb;
+#pragma unroll 1
+      while (mm != 0u) {
+        const int u = __ffs(mm) - 1;
+        mm &= mm - 1u;
+        if (base < 1024) {
+          sm.list_key[base] = skey[s0 + u];
+          sm.list_pos[base] = s0 + u;
+        }
+        ++base;
       }
     }
   }
   __syncthreads();
-  stamp(p, 22);
-  for (int e = threadIdx.x; e < (int)m; e += kThreads) {  // rank inside the sub-bin
-    const uint32_t ke = sm.list_key[e];
-    const int pe = sm.list_pos[e];
+  stamp(p, 19);
+  if ((uint32_t)sm.list_n != m) {  // the windows disagree with the group histogram: cannot happen
+    if (threadIdx.x == 0) record_error(p.ws_header, CLSA_ERR_BAD_INDEX, -3);
+    return false;
+  }
+  // c. exact rank inside bin B: eight threads per listed key, each comparing it with every
+  //    eighth key, then a three-step shuffle sum
+#pragma unroll 1
+  for (int e0 = 0; e0 < (int)m; e0 += kThreads / 8) {
+    const int e = e0 + (threadIdx.x >> 3), part = threadIdx.x & 7;
+    const bool live = e < (int)m;
+    const uint32_t ke = live ? sm.list_key[e] : 0u;
+    const int pe = live ? sm.list_pos[e] : 0;
     uint32_t r = 0;
-    for (int f = 0; f < (int)m; ++f) {
+#pragma unroll 1
+    for (int f = part; f < (int)m; f += 8) {
       const uint32_t kf = sm.list_key[f];
-      r += kf > ke || (kf == ke && sm.list_pos[f] < pe);
+      const int pf = sm.list_pos[f];
+      r += kf > ke || (kf == ke && pf < pe);
     }
-    if (r == need - 1) {
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    r += __shfl_xor_sync(0xffffffffu, r, 2);
+    r += __shfl_xor_sync(0xffffffffu, r, 4);
+    if (live && part == 0 && r == need - 1) {
       sm.theta_key = ke;
       sm.theta_pos = (uint32_t)pe;
     }
   }
   __syncthreads();
-  return true;
-}
-
-// selected iff key > theta_key, or key == theta_key at a position <= theta_pos.
-// Each thread owns a contiguous odd-length run (bank-conflict free), reads its keys
-// eight at a time into registers, keeps a bitmask of its selected slots, and after
-// one block scan visits only the selected ones.
-__device__ void compact_candidates(const FusedParams& p, Smem& sm, const uint32_t* skey, const int32_t* stok,
-                                   int P) {
-  const Plan pl = sm.plan;  // a copy: loops below store to shared memory
+  stamp(p, 20);
+  // d. rank the selected slots (key > theta_key, or key == theta_key at a slot <= theta_pos) in
+  //    slot order = ascending token order: one block scan over the per-thread counts (the
+  //    slots above bin B, plus this thread's selected slots of bin B)
   const uint32_t tk = sm.theta_key, tp = sm.theta_pos;
-  int run = (P + kThreads - 1) / kThreads;
-  run += (run & 1) ^ 1;
-  const int a = threadIdx.x * run;
-  uint64_t sel = 0;
-  for (int c0 = 0; c0 < run; c0 += 8) {
-    uint32_t k[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = a + c0 + u;
-      k[u] = (c0 + u < run && i < P) ? skey[i] : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (k[u] > tk || (k[u] == tk && (uint32_t)(a + c0 + u) <= tp)) sel |= 1ull << (c0 + u);
-  }
-  stamp(p, 25);
-  uint32_t tot;
-  uint32_t rank = block_scan((uint32_t)__popcll(sel), sm.warp_tot, &tot);
-  stamp(p, 26);
-  int32_t* out = p.idx + (size_t)pl.b * p.k;
-  // 8 slots at a time: their tokens loaded together, each selected slot's rank from a
-  // popcount of the selected slots before it (no serial chain through the slots)
+  uint32_t cnt = above;
+  {
+    uint32_t mm = inb;
 #pragma unroll 1
-  for (int c0 = 0; c0 < run; c0 += 8) {
-    const uint32_t m8 = (uint32_t)(sel >> c0) & 0xffu;
-    if (m8 == 0u) continue;
-    int32_t t[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) t[u] = (m8 >> u) & 1u ? stok[a + c0 + u] : 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if ((m8 >> u) & 1u) {
-        const int r = (int)rank + __popc(m8 & ((1u << u) - 1u));
-        if (r >= pl.tok0 && r < pl.tok1) sm.unit_tok[r - pl.tok0] = t[u];
-        if (t[u] >= pl.r0 && t[u] < pl.r1 && r < pl.keff) out[r] = t[u];
+    while (mm != 0u) {
+      const int u = __ffs(mm) - 1;
+      mm &= mm - 1u;
+      const uint32_t k = skey[s0 + u];
+      cnt += k > tk || (k == tk && (uint32_t)(s0 + u) <= tp);
+    }
+  }
+  uint32_t tot;
+  stamp(p, 32);
+  cp_async_wait<0>();  // the window tokens (visible to all after the scan's barrier)
+  int r = (int)block_excl_scan1(cnt, sm.warp_tot2, &tot);
+  stamp(p, 33);
+  if (threadIdx.x == 0 && tot != keff) record_error(p.ws_header, CLSA_ERR_BAD_INDEX, -2);
+  // e. the unit's tokens (ranks [tok0, tok1)) and idx for this CTA's own window: only the
+  //    threads whose ranks meet the unit's range or whose slots meet the own window
+  const int own0 = pl.c * pl.win, own1 = own0 + pl.win;
+  int32_t* out = p.idx + (size_t)pl.b * p.k;
+  const bool in_unit = r < pl.tok1 && r + (int)cnt > pl.tok0, in_own = s0 < own1 && s1 > own0;
+  if (cnt != 0u && (in_unit || in_own)) {
+#pragma unroll 1
+    for (int u = 0; s0 + u < s1; u += 4) {
+      const uint4 x = *reinterpret_cast<const uint4*>(skey + s0 + u);
+      const int sl = s0 + u;
+      uint32_t m4 = (uint32_t)(x.x > tk || (x.x == tk && (uint32_t)sl <= tp)) |
+                    (uint32_t)(x.y > tk || (x.y == tk && (uint32_t)(sl + 1) <= tp)) << 1 |
+                    (uint32_t)(x.z > tk || (x.z == tk && (uint32_t)(sl + 2) <= tp)) << 2 |
+                    (uint32_t)(x.w > tk || (x.w == tk && (uint32_t)(sl + 3) <= tp)) << 3;
+#pragma unroll 1
+      while (m4 != 0u) {
+        const int q = sl + __ffs(m4) - 1;
+        m4 &= m4 - 1u;
+        const int t = stok[q];
+        if (r >= pl.tok0 && r < pl.tok1) sm.unit_tok[r - pl.tok0] = t;
+        if (q >= own0 && q < own1 && r < pl.keff) out[r] = t;
+        ++r;
       }
     }
-    rank += (uint32_t)__popc(m8);
   }
+  stamp(p, 34);
   __syncthreads();
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -868,12 +1017,13 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* q) {
 
 // Q rows of head g in the 128-byte-swizzle K-major layout (two 64-column atoms)
 __device__ __forceinline__ void load_q_tile(const FusedParams& p, int b, int g, unsigned char* sQa) {
-#pragma unroll 1
+  const float invG = 1.f / (float)p.G;  // floor((r + 0.5) / G) in fp32 is exact for r < 2^12
+#pragma unroll
   for (int v = threadIdx.x; v < kMaxRows * 16; v += kThreads) {
     const int r = v >> 4, c = v & 15;
     unsigned char* dst = sQa + (c >> 3) * kQAtom + tc::sw128_offset(r, c & 7);
     if (r < p.rows) {
-      const int l = r / p.G, h = g * p.G + r % p.G;
+      const int l = (int)(((float)r + 0.5f) * invG), h = g * p.G + (r - l * p.G);
       cp_async_16(dst, p.Q + (((size_t)l * p.B + b) * p.Hq + h) * kD + c * 8, 16);
     } else {
       *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
@@ -937,6 +1087,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
       load_kv_chunk<TOK>(p, sm, b, g, pl.len, c, ntok, kv + c * 2 * SH::kKVTile, kv + c * 2 * SH::kKVTile + SH::kKVTile);
     cp_async_commit();
   }
+  stamp(p, 35);
   const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
   const bool live = q4 * 32 < p.rows;  // warp-uniform: rows of this lane quarter exist
   float o[32];
@@ -980,6 +1131,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
       if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 30);
       dead = true;
     }
+    if (c == 0) stamp(p, 36);
     tc::fence_after_sync();
     // the scores are read from TMEM twice (for the row max, then for P) rather than held
     // across the exchange: registers stay within budget for 32 columns
@@ -999,6 +1151,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
       sm.cm[cg * kMaxRows + row] = cmx * p.scale_log2;  // scale > 0: the max commutes
     }
     __syncthreads();
+    if (c == 0) stamp(p, 37);
     float alpha = 1.f;
     if (live) {
       const float mn = fmaxf(fmaxf(m, fmaxf(sm.cm[row], sm.cm[kMaxRows + row])),
@@ -1035,6 +1188,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
+    if (c == 0) stamp(p, 38);
     if (threadIdx.x == 0) {
       // O_c = P_c V_c, then S of the next chunk into the other S buffer
       tc::fence_after_sync();
@@ -1049,6 +1203,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
       if (lane == 0) record_error(p.ws_header, CLSA_ERR_TIMEOUT, 31);
       dead = true;
     }
+    if (c == 0) stamp(p, 39);
     tc::fence_after_sync();
     if (live && !dead) {
       uint32_t v[32];
@@ -1098,6 +1253,11 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
 #pragma unroll 1
     for (int i = threadIdx.x; i < p.rows * (kD / 4); i += kThreads)
       __stcg(op + i, *reinterpret_cast<const float4*>(stg + (i / (kD / 4)) * kOPitch + 4 * (i % (kD / 4))));
+    // the partial is complete: the CTA's barrier orders every thread's stores before the
+    // release that publishes its flag (the row's launch counter + 1)
+    __syncthreads();
+    if (threadIdx.x == 0)
+      st_release_gpu(p.row_ws + (size_t)b * kRowWords + kRowFlag + pl.c, sm.row_hdr[kRowEpoch] + 1u);
   }
   stamp(p, 12);
   __syncthreads();  // cm / cl and the tiles are free for the next unit
@@ -1105,10 +1265,12 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
 
 // ---------------------------------------------------------------------------
 // phase 5: merge the nsplit partials of head g for rows r = split, split + nsplit, ...
-// The partial vectors of those rows are staged in shared memory by 16-byte copies, all
-// in flight at once (one L2 round trip per batch of 128), while the (m, l) pairs give
-// each row M = max m and den = sum 2^(m - M) l; then one warp per row sums its splits
-// in split order (the same order every call: the result is deterministic).
+// Warp w waits for the flag of split w (w + 16, ...) and at once issues the 16-byte copies
+// of that split's partial rows and reads its (m, l) pairs, so the copies of the early
+// splits overlap the wait for the late ones.  Each row's M = max m and den = sum 2^(m - M) l
+// come from all pairs; then one warp per row sums its splits in split order (the same
+// order every call: the result is deterministic).  Splits are staged in batches that fit
+// the staging region (one batch at the workloads' shapes).
 // ---------------------------------------------------------------------------
 __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan pl, int g) {
   stamp(p, 18);
@@ -1117,39 +1279,59 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
   const int nr = (p.rows - pl.split + ns - 1) / ns;
   if (nr <= 0) return;
   const size_t cta0 = (size_t)pl.start + (size_t)g * ns;  // CTA holding split 0 of head g
-  const int npair = nr * ns;                              // pair t: row ri = t / ns, split t % ns
-  constexpr int kPB = 128;                                // pairs per batch: 64 KiB staged
-  float4* stg = reinterpret_cast<float4*>(big);           // [kPB][32]
-  float4* acc = stg + kPB * 32;                           // [nr][32] (nr <= kMaxRows: 64 KiB)
-  auto issue = [&](int t0) {
-    const int nb = min(kPB, npair - t0);
-    #pragma unroll 1
-    for (int x = threadIdx.x; x < nb * 32; x += kThreads) {
-      const int t = t0 + x / 32, ri = t / ns, s2 = t % ns;
-      cp_async_16(stg + x, p.Op + ((cta0 + s2) * p.rows + pl.split + ri * ns) * kD + (x % 32) * 4, 16);
+  const uint32_t* flags = p.row_ws + (size_t)pl.b * kRowWords + kRowFlag + (size_t)g * ns;
+  const uint32_t tag = sm.row_hdr[kRowEpoch] + 1u;
+  constexpr int kMaxPairs = 224;                          // 112 KiB of staged partial rows
+  float4* stg = reinterpret_cast<float4*>(big);           // [pairs of the batch][32]
+  const int sb = max(1, min(ns, kMaxPairs / nr));         // splits per batch
+  bool dead = false;
+  // (m, l) of every pair first (the flags of all splits), then the first batch's rows
+  auto wait_flag = [&](int s2) {  // warp-wide; false on timeout
+    uint32_t ok = 1;
+    if (lane == 0) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (ld_acquire_gpu(flags + s2) != tag) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          record_error(p.ws_header, CLSA_ERR_TIMEOUT, 2);
+          ok = 0;
+          break;
+        }
+      }
     }
-    cp_async_commit();
+    __syncwarp();  // lane 0's acquire orders the warp's loads below
+    return __shfl_sync(0xffffffffu, ok, 0) != 0u;
   };
-  issue(0);
-  #pragma unroll 1
-  for (int t = threadIdx.x; t < npair; t += kThreads) {
-    const int ri = t / ns, s2 = t % ns;
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
-    sm.cm[t] = ml.x;
-    sm.cl[t] = ml.y;
+  auto issue_rows = [&](int s2, int s_lo) {
+    for (int ri = 0; ri < nr; ++ri)
+      cp_async_16(stg + ((s2 - s_lo) * nr + ri) * 32 + lane,
+                  p.Op + ((cta0 + s2) * p.rows + pl.split + ri * ns) * kD + lane * 4, 16);
+  };
+#pragma unroll 1
+  for (int s2 = warp; s2 < ns; s2 += kWarps) {
+    if (!wait_flag(s2)) {
+      dead = true;
+      continue;
+    }
+    for (int ri = lane; ri < nr; ri += 32) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
+      sm.cm[ri * ns + s2] = ml.x;
+      sm.cl[ri * ns + s2] = ml.y;
+    }
+    if (s2 < sb) issue_rows(s2, 0);
   }
-  #pragma unroll 1
-  for (int i = threadIdx.x; i < nr * 32; i += kThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  cp_async_commit();
+  if (dead) sm.abort_flag = 1;
   __syncthreads();
   stamp(p, 17);
+  if (sm.abort_flag) return;
   // per row: M, den, and each split's weight 2^(m - M) in place of its m
-  #pragma unroll 1
+#pragma unroll 1
   for (int ri = warp; ri < nr; ri += kWarps) {
     float M = -INFINITY, den = 0.f;
-    #pragma unroll 1
+#pragma unroll 1
     for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, sm.cm[ri * ns + s2]);
     M = warp_max(M);
-    #pragma unroll 1
+#pragma unroll 1
     for (int s2 = lane; s2 < ns; s2 += 32) {
       const float wgt = M == -INFINITY ? 0.f : exp2f(sm.cm[ri * ns + s2] - M);
       den = fmaf(wgt, sm.cl[ri * ns + s2], den);
@@ -1161,47 +1343,56 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
       sm.rowD[ri] = den;
     }
   }
-  #pragma unroll 1
-  for (int t0 = 0; t0 < npair; t0 += kPB) {
-    if (t0 > 0) issue(t0);
-    cp_async_wait<0>();
-    __syncthreads();  // this batch (and, first time, every row's M) is visible
-    const int nb = min(kPB, npair - t0);
-    #pragma unroll 1
-    for (int ri = warp; ri < nr; ri += kWarps) {
-      const int s_lo = max(0, t0 - ri * ns), s_hi = min(ns, t0 + nb - ri * ns);
-      if (s_lo >= s_hi) continue;
-      float4 a = acc[ri * 32 + lane];
-      // the splits in order (a fixed summation order: deterministic); unrolled so the
-      // staged loads overlap
-      #pragma unroll 6
-      for (int s2 = s_lo; s2 < s_hi; ++s2) {
-        const int t = ri * ns + s2;
-        const float w = sm.cm[t];
-        const float4 v = stg[(t - t0) * 32 + lane];
-        a.x = fmaf(w, v.x, a.x);
-        a.y = fmaf(w, v.y, a.y);
-        a.z = fmaf(w, v.z, a.z);
-        a.w = fmaf(w, v.w, a.w);
-      }
-      acc[ri * 32 + lane] = a;
+  // one warp per row accumulates its splits in order (lane: 4 of the 128 columns)
+  float4 acc[(kMaxRows + kWarps - 1) / kWarps];
+#pragma unroll
+  for (int i = 0; i < (kMaxRows + kWarps - 1) / kWarps; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+  for (int s_lo = 0; s_lo < ns; s_lo += sb) {
+    const int s_hi = min(ns, s_lo + sb);
+    if (s_lo > 0) {  // later batches: the flags were seen above
+      __syncthreads();  // the previous batch is consumed
+#pragma unroll 1
+      for (int s2 = s_lo + warp; s2 < s_hi; s2 += kWarps) issue_rows(s2, s_lo);
+      cp_async_commit();
     }
-    __syncthreads();  // before the next batch overwrites the stage
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < (kMaxRows + kWarps - 1) / kWarps; ++i) {
+      const int ri = warp + i * kWarps;
+      if (ri < nr) {
+        float4 a = acc[i];
+#pragma unroll 6
+        for (int s2 = s_lo; s2 < s_hi; ++s2) {
+          const float w = sm.cm[ri * ns + s2];
+          const float4 v = stg[((s2 - s_lo) * nr + ri) * 32 + lane];
+          a.x = fmaf(w, v.x, a.x);
+          a.y = fmaf(w, v.y, a.y);
+          a.z = fmaf(w, v.z, a.z);
+          a.w = fmaf(w, v.w, a.w);
+        }
+        acc[i] = a;
+      }
+    }
   }
-  #pragma unroll 1
-  for (int ri = warp; ri < nr; ri += kWarps) {
-    const int r = pl.split + ri * ns;
-    const float den = sm.rowD[ri], M = sm.rowM[ri];
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const float4 a = acc[ri * 32 + lane];
-    const int l = r / p.G, h = g * p.G + r % p.G;
-    __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
-    uint2 wv;
-    wv.x = pack_bf16x2(a.x * inv, a.y * inv);
-    wv.y = pack_bf16x2(a.z * inv, a.w * inv);
-    *reinterpret_cast<uint2*>(out) = wv;
-    if (p.lse && lane == 0)
-      p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+#pragma unroll
+  for (int i = 0; i < (kMaxRows + kWarps - 1) / kWarps; ++i) {
+    const int ri = warp + i * kWarps;
+    if (ri < nr) {
+      const int r = pl.split + ri * ns;
+      const float den = sm.rowD[ri], M = sm.rowM[ri];
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const float4 a = acc[i];
+      const int l = r / p.G, h = g * p.G + r % p.G;
+      __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
+      uint2 wv;
+      wv.x = pack_bf16x2(a.x * inv, a.y * inv);
+      wv.y = pack_bf16x2(a.z * inv, a.w * inv);
+      *reinterpret_cast<uint2*>(out) = wv;
+      if (p.lse && lane == 0)
+        p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+    }
   }
 }
 
@@ -1233,12 +1424,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
       pre_r0 = min(len, (int)blockIdx.x * chunk);
       pre_r1 = min(len, pre_r0 + chunk);
       pre_q = load_q_chunk<DIDX>(p, 0);  // ahead of the K_idx stream (it would queue behind it)
+      load_row_header(p, sm, 0);
       scan_start<DIDX>(reinterpret_cast<uint4*>(big), p.k_idx + (size_t)pre_r0 * DIDX, 0, pre_r1 - pre_r0);
       pre = true;
     }
   }
   if (threadIdx.x == 0) {
-    make_plan(p, sm.plan);
+    make_plan(p, sm.plan, sm.live_rows);
     sm.abort_flag = 0;
   }
   __syncthreads();
@@ -1260,10 +1452,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     }
   }
   if (pl.b < 0) {
-    leave_finish(p, leave_issue(p));
+    leave_finish(p, sm, leave_issue(p));
     return;
   }
-  const bool head_bar = pl.nsplit > 1 && pl.nunits_here > 0;  // the split combine waits on the head's splits
+  const bool merge = pl.nsplit > 1 && pl.nunits_here > 0;  // this CTA merges split partials of its head
   uint32_t left = 0;
   if (pl.c == 0) {
     for (int i = pl.keff + threadIdx.x; i < p.k; i += kThreads) p.idx[(size_t)pl.b * p.k + i] = -1;
@@ -1280,12 +1472,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
 
   const bool all_sel = pl.keff == pl.len;
   stamp(p, 23);
-  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel, pre, pre_q)) return;
-  if (pl.nunits_here > 0) load_q_tile(p, pl.b, pl.unit_g0, sQa);  // lands during the selection
+  if (!scan_slice<DIDX>(p, sm, sm.hist, big, !all_sel, pre, pre_q, pl.nunits_here > 0 ? sQa : nullptr)) return;
+  clear_previous_copy(p, sm, pl);
   stamp(p, 1);
 
   if (all_sel) {  // every token is selected: rank = token index
-    if (!head_bar) left = leave_issue(p);
+    left = leave_issue(p);
     int32_t* out = p.idx + (size_t)pl.b * p.k;
     for (int j = pl.r0 + threadIdx.x; j < pl.r1; j += kThreads) out[j] = j;
     for (int i = threadIdx.x; i < pl.tok1 - pl.tok0; i += kThreads) sm.unit_tok[i] = pl.tok0 + i;
@@ -1295,65 +1487,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     stamp(p, 2);
     uint32_t* rw = p.row_ws + (size_t)pl.b * kRowWords;
     if (!count_barrier(rw + kRowBar, pl.Cb, p.ws_header, 1)) return;
-    if (!head_bar) left = leave_issue(p);
     stamp(p, 3);
     // the group's windows (back to back, token order, empty slots key 0) to shared
-    // memory in 16-byte copies, all in flight while the group totals are reduced
+    // memory in 16-byte copies: keys first, then tokens (needed only for the ranking)
     uint32_t* skey = reinterpret_cast<uint32_t*>(big);
     int32_t* stok = reinterpret_cast<int32_t*>(big + kCandCap * 4);
     const int nslot = pl.Cb * pl.win;  // a multiple of 4
     {
       const uint4* gk = reinterpret_cast<const uint4*>(p.cand_key + (size_t)pl.b * kCandCap);
       const uint4* gt = reinterpret_cast<const uint4*>(p.cand_tok + (size_t)pl.b * kCandCap);
-      for (int i = threadIdx.x; i < nslot / 4; i += kThreads) {
-        cp_async_16(skey + 4 * i, gk + i, 16);
-        cp_async_16(stok + 4 * i, gt + i, 16);
-      }
+      for (int i = threadIdx.x; i < nslot / 4; i += kThreads) cp_async_16(skey + 4 * i, gk + i, 16);
       cp_async_commit();
-      // candidate total, the largest bound E_max and the largest key bound over the group
-      const bool mine = threadIdx.x < pl.Cb;
-      const uint32_t v = mine ? __ldcg(rw + kRowCnt + threadIdx.x) : 0u;
-      const uint32_t e = mine ? __ldcg(rw + kRowBound + threadIdx.x) : 0u;
-      const uint32_t x = mine ? __ldcg(rw + kRowMax + threadIdx.x) : 0u;
-      const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-      const uint32_t vs = __reduce_add_sync(0xffffffffu, v), es = __reduce_max_sync(0xffffffffu, e),
-                     xs = __reduce_max_sync(0xffffffffu, x);
-      if (lane == 0) {
-        sm.warp_tot[w] = vs;
-        sm.red_min[w] = es;
-        sm.red_max[w] = xs;
-      }
+      for (int i = threadIdx.x; i < nslot / 4; i += kThreads) cp_async_16(stok + 4 * i, gt + i, 16);
+      cp_async_commit();
+    }
+    const bool done = select_windows(p, sm, rw, skey, stok, nslot);
+    // past the row barrier: the last CTA to leave may reset its word
+    left = leave_issue(p);
+    stamp(p, 5);
+    if (!done) {  // too few candidates at or above E_max, or a boundary sub-bin of heavy ties:
+              // digit-by-digit select over the whole row
       cp_async_wait<0>();
       __syncthreads();
-      const uint32_t total = __reduce_add_sync(0xffffffffu, lane < kWarps ? sm.warp_tot[lane] : 0u);
-      const uint32_t emax = __reduce_max_sync(0xffffffffu, lane < kWarps ? sm.red_min[lane] : 0u);
-      const uint32_t kmax = __reduce_max_sync(0xffffffffu, lane < kWarps ? sm.red_max[lane] : 0u);
-      if (threadIdx.x == 0) {
-        sm.ctot = nslot;
-        sm.fast = total >= (uint32_t)pl.keff;  // too few candidates: whole-row path
-        sm.emax = emax;
-        sm.kmax = kmax;
-      }
-      __syncthreads();
-    }
-    stamp(p, 4);
-    bool done = false;
-    if (sm.fast) {
-      // exact iff every CTA's unpublished tokens (keys below its bound E) lie strictly
-      // below the k_eff-th candidate key, i.e. iff at least k_eff candidates have keys
-      // >= E_max (checked inside)
-      done = select_candidates(p, sm, skey, sm.ctot, (uint32_t)pl.keff, sm.emax, sm.kmax);
-      stamp(p, 5);
-      if (done) compact_candidates(p, sm, skey, stok, sm.ctot);
-    }
-    if (!done) {  // too few candidates, a bound above the boundary, or a boundary bin of
-                  // heavy ties: digit-by-digit select over the whole row
       CandSrc src{skey, stok, p.scores + (size_t)pl.b * p.n_max, false};
       resolve_theta(sm, src, pl.len, (uint32_t)pl.keff, p.ws_header);
-      stamp(p, 5);
       compact_selected(p, sm, src, pl.len);
     }
-    if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + 31] = (unsigned long long)sm.ctot | ((unsigned long long)sm.fast << 32);
+    if (p.trace && threadIdx.x == 0) p.trace[blockIdx.x * kTraceSlots + 31] = (unsigned long long)nslot | ((unsigned long long)done << 32);
   }
   stamp(p, 6);
 
@@ -1385,14 +1545,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     if (threadIdx.x < 32) tc::tmem_dealloc(tmem, kTmemCols);
   }
   stamp(p, 7);
-  if (head_bar) {
-    uint32_t* hb = p.row_ws + (size_t)pl.b * kRowWords + kRowHeadBar + 2 * pl.unit_g0;
-    if (!count_barrier(hb, pl.nsplit, p.ws_header, 2)) return;
-    left = leave_issue(p);
+  if (merge) {
     stamp(p, 8);
     combine_head(p, sm, big, pl, pl.unit_g0);
   }
-  leave_finish(p, left);
+  leave_finish(p, sm, left);
   stamp(p, 9);
 }
 
@@ -1501,6 +1658,16 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   p.rows = a->L * p.G;
   p.nsplit_max = std::max(1, cfg.ncta / a->Hkv);
   p.scale_log2 = scale * kLog2e;
+  p.pf_mult = 1.5f;
+  p.pf_add = 8u;
+  if (const char* pf = std::getenv("CLSA_PREFETCH")) {  // "mult,add" (tuning)
+    float m = 0.f;
+    unsigned ad = 0;
+    if (std::sscanf(pf, "%f,%u", &m, &ad) == 2) {
+      p.pf_mult = m;
+      p.pf_add = ad;
+    }
+  }
   p.ws_header = ws_header;
   char* w = static_cast<char*>(ws_body);
   const char* tr = std::getenv("CLSA_TRACE");
