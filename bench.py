@@ -55,7 +55,7 @@ def parse():
                     help="between steps: rotate through input sets larger than L2 (default), or flush L2")
     ap.add_argument("--sets", type=int, default=6, help="input sets rotated through (--l2 rotate)")
     ap.add_argument("--variant", default="clsa",
-                    choices=["clsa", "per_layer_routing", "yoco_dense", "standard", "distill_target"],
+                    choices=["clsa", "per_layer_routing", "yoco_dense", "standard", "distill_target", "attention_mass"],
                     help="a comparison system built from the library's calls (one GPU; not the default line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-steps", type=int, default=2)
@@ -165,7 +165,9 @@ class ClockSampler:
 # ------------------------------------------------------------------ CPU oracle timing
 
 def time_oracle(inp, w, steps: int):
-    """Run the oracle's decode step on the host cores; returns (s per step, threads, note)."""
+    """Run the oracle's decode step on the host cores, once with its BLAS pool limited to one
+    thread and once with one thread per core this process may use (os.sched_getaffinity).
+    Returns (s per step all-cores, cores, s per step single-thread, note)."""
     from oracle import clsa_oracle as O
     # the cache is upcast once (state a real decoder keeps resident); each sample step
     # re-scores, re-selects and attends
@@ -174,16 +176,24 @@ def time_oracle(inp, w, steps: int):
     Kf = inp.f32("K").astype(np.float64)
     Vf = inp.f32("V").astype(np.float64)
     Qf = inp.f32("Q").astype(np.float64)
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        O.decode_step(qf, kf, Kf, Vf, Qf, inp.seq_lens, w.k)
-    dt = (time.perf_counter() - t0) / steps
-    try:  # threads of the BLAS pool the oracle's matrix products ran on
-        from threadpoolctl import threadpool_info
-        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
-    return dt, threads, f"{steps} full decode step(s) of {w.name} (B={w.B}, n={w.n_max})"
+    cores = len(os.sched_getaffinity(0))
+
+    def run(n):
+        t0 = time.perf_counter()
+        for _ in range(n):
+            O.decode_step(qf, kf, Kf, Vf, Qf, inp.seq_lens, w.k)
+        return (time.perf_counter() - t0) / n
+
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            dt1 = run(1)
+        with threadpool_limits(limits=cores):
+            dt = run(steps)
+    except Exception:  # no control over the BLAS pool: one measurement as it stands
+        dt = run(steps)
+        dt1 = None
+    return dt, cores, dt1, f"{steps} full decode step(s) of {w.name} (B={w.B}, n={w.n_max}); single-thread: 1 step"
 
 
 # ------------------------------------------------------------------ main paths
@@ -197,16 +207,15 @@ def run_reference(args):
     w = WORKLOADS[args.workload]
     inp = make_inputs(w)
     steps = max(1, min(args.steps, args.cpu_sample_steps))
-    for _ in range(min(args.warmup, 1)):
-        time_oracle(inp, w, 1)
-    dt, threads, note = time_oracle(inp, w, steps)
+    dt, threads, dt1, note = time_oracle(inp, w, steps)
     v = w.B / dt
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
             "warmup": min(args.warmup, 1), "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "B": w.B, "n": w.n_max, "k": w.k, "L": w.L, "Hq": w.Hq,
                        "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note,
+                             "single_thread_value": (w.B / dt1) if dt1 else None},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -378,12 +387,13 @@ def run_clsa(args):
     KS = torch.empty(B, k, w.Hkv, d, dtype=dv["K"].dtype, device=dev)
     VS = torch.empty_like(KS)
 
-    def timed(fn, reps=50):
+    def timed(fn, reps=50, flush=True):
         fn()
         torch.cuda.synchronize()
         tot = 0.0
         for _ in range(reps):
-            flush_l2()
+            if flush:
+                flush_l2()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -404,6 +414,10 @@ def run_clsa(args):
     O1 = torch.empty_like(Q1)
     kern["sparse_attn_one_layer"] = timed(
         lambda: clsa.sparse_attn(Q1, KS, VS, out["count"], ws=attn_ws, O=O1, want_lse=False))
+    # the model-faithful per-layer call with the step's gathered K_S/V_S still in L2 (a model
+    # runs the layers back to back on the one selection): no flush between calls
+    kern["sparse_attn_one_layer_l2_resident"] = timed(
+        lambda: clsa.sparse_attn(Q1, KS, VS, out["count"], ws=attn_ws, O=O1, want_lse=False), flush=False)
 
     hbm, bf16, peak_kind = peaks()
     if launches_per_step == 1:
@@ -526,8 +540,9 @@ def run_clsa(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, threads, note = time_oracle(inp, w, args.cpu_sample_steps)
-        cpu = {"value": w.B / dt, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note}
+        dt, threads, dt1, note = time_oracle(inp, w, args.cpu_sample_steps)
+        cpu = {"value": w.B / dt, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note,
+               "single_thread_value": (w.B / dt1) if dt1 else None}
 
     replicas.finish(world)
     if rank != 0:
@@ -579,6 +594,24 @@ class _DistillStep:
         return clsa.last_launch_count()
 
 
+class _MassStep:
+    """The attention-mass coverage as one timed step (preallocated outputs and workspace)."""
+
+    def __init__(self, Q, K, lse_sparse, seq_lens):
+        from long_context_sparse_clsa_b200 import clsa
+        import torch
+        self.args = (Q, K, lse_sparse, seq_lens)
+        L, B, Hq, d = Q.shape
+        self.ws = clsa.Workspace(clsa.load_library().clsa_attention_mass_workspace_size(B, K.shape[1], L, Hq,
+                                                                                        K.shape[2], d))
+        self.mass = torch.empty(L, B, Hq, dtype=torch.float32, device=Q.device)
+
+    def step(self) -> int:
+        from long_context_sparse_clsa_b200 import clsa
+        clsa.attention_mass(*self.args, ws=self.ws, mass=self.mass, want_lse_all=False)
+        return clsa.last_launch_count()
+
+
 def run_variant(args):
     """Time a comparison system of the pages' ablation (per-layer routing, YOCO only,
     standard attention) on the same workload, built from the library's own calls."""
@@ -625,6 +658,12 @@ def run_variant(args):
         sysm = baselines.YocoDense(dv["K"], dv["V"], dv["Q"], dv["seq_lens"], Ob)
         step_bytes_ = 2 * sum(lens) * Hkv * d * eb + qo_bytes
         note = "every layer dense over the one shared cache (one call, the L*G rows of a head read each row once)"
+    elif args.variant == "attention_mass":
+        r = clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], dv["seq_lens"], k)
+        sysm = _MassStep(dv["Q"], dv["K"], r["lse"], dv["seq_lens"])
+        # the cache's K once, Q once, the selection's lse in and the mass out
+        step_bytes_ = sum(lens) * Hkv * d * eb + qo_bytes // 2 + 2 * L * B * Hq * 4
+        note = "share of the dense softmax mass on the selection: one lse pass over K, merged with the step's lse"
     elif args.variant == "distill_target":
         sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
         sysm = _DistillStep(dv["Q"], dv["K"], sc, dv["seq_lens"])

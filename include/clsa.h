@@ -148,6 +148,29 @@ CLSA_API clsa_status clsa_sparse_attn(const void* Q, const void* K_S, const void
                              void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Attention-mass coverage of the shared selection                            */
+/* ------------------------------------------------------------------------ */
+/* picx.dev CLSA summary, Attention Sparsity Analysis: the share of each layer's
+ * dense softmax mass that the selected tokens hold,
+ *   mass[l][b][h] = sum_{j in S_b} softmax_j(Q^(l)[b,h] K[b]^T * scale)
+ *                 = exp(lse_S[l][b][h] - lse_all[l][b][h]),
+ * with lse_S the lse the decode step returned for the selection (clsa_decode_step's
+ * `lse` output) and lse_all the lse over every one of the len_b cached rows.
+ * Q [L][B][Hq][d], K [B][n_max][Hkv][d] in dt; lse_sparse [L][B][Hq] fp32 (natural
+ * log); seq_lens [B] device int32.  mass [L][B][Hq] fp32 out (0 where either lse is
+ * -inf); lse_all [L][B][Hq] fp32 out, may be NULL.  Query head h reads KV head
+ * h / (Hq / Hkv); scale <= 0 selects 1/sqrt(d).  V is not read (the lse does not use
+ * it).  bf16 with d = 128 streams K once on the tensor cores (per-split row max and
+ * sum, then one merge in split order: deterministic), 2 launches; other shapes take
+ * the row lse from the split-k attention kernel.  Caller-owned workspace of
+ * clsa_attention_mass_workspace_size bytes; errors as above. */
+CLSA_API size_t clsa_attention_mass_workspace_size(int B, int n_max, int L, int Hq, int Hkv, int d);
+CLSA_API clsa_status clsa_attention_mass(const void* Q, const void* K, const float* lse_sparse,
+                                         const int32_t* seq_lens, int B, int n_max, int L, int Hq, int Hkv,
+                                         int d, float scale, clsa_dtype dt, float* mass, float* lse_all,
+                                         void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Distillation target of the shared indexer (forward only)                   */
 /* ------------------------------------------------------------------------ */
 /* picx.dev CLSA summary, Methodology > Architecture Overview, multi-layer

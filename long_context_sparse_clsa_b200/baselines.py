@@ -93,17 +93,11 @@ class StandardAttention:
 
 
 def attention_mass(Q, K, V, seq_lens, lse_sparse, scale: float = 0.0, ws=None):
-    """Share of the dense softmax mass on the selected rows, per (layer, sequence, head).
-
-    lse_sparse [L][B][Hq]: the lse the decode step returned (softmax over S); the dense
-    lse over every cached row comes from one clsa_sparse_attn call with the cache as
-    K_S/V_S.  Returns (mass [L][B][Hq] fp32, lse_all).  The pages' figure (~80 % at 2048 of
-    32K tokens) needs trained weights; on synthetic N(0, 1) inputs the indexer keys are
+    """Share of the dense softmax mass on the selected rows, per (layer, sequence, head):
+    clsa_attention_mass (one streaming pass over K for the dense lse; V is not needed).
+    Returns (mass [L][B][Hq] fp32, lse_all).  The pages' figure (~80 % at 2048 of 32K
+    tokens) needs trained weights; on synthetic N(0, 1) inputs the indexer keys are
     independent of K, so the share is close to |S| / n.
     """
-    import torch
-    L, B, Hq, d = Q.shape
-    O = torch.empty_like(Q)
-    lse_all = torch.empty(L, B, Hq, dtype=torch.float32, device=Q.device)
-    clsa.sparse_attn(Q, K, V, seq_lens, scale, ws=ws, O=O, lse=lse_all)
-    return torch.exp(lse_sparse - lse_all), lse_all
+    del V  # the lse over the cache does not depend on V
+    return clsa.attention_mass(Q, K, lse_sparse, seq_lens, scale, ws=ws)

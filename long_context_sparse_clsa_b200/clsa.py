@@ -26,7 +26,8 @@ EXPORTS = [
     "clsa_index_scores", "clsa_topk_workspace_size", "clsa_topk", "clsa_topk_noalloc",
     "clsa_gather_kv_workspace_size",
     "clsa_gather_kv", "clsa_sparse_attn_workspace_size", "clsa_sparse_attn",
-    "clsa_distill_workspace_size", "clsa_distill_target",
+    "clsa_distill_workspace_size", "clsa_distill_target", "clsa_attention_mass_workspace_size",
+    "clsa_attention_mass",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
     "clsa_prefill_chunk", "clsa_workspace_size", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
     "clsa_selftest_timeout", "clsa_version", "clsa_last_launch_count", "clsa_time_next_call",
@@ -83,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_sparse_attn": (S, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp,
                                  _sz, _vp]),
         "clsa_distill_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+        "clsa_attention_mass_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+        "clsa_attention_mass": (S, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
         "clsa_distill_target": (S, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz, _vp]),
         "clsa_decode_workspace_size": (_sz, [ctypes.POINTER(DecodeArgs)]),
         "clsa_decode_step": (S, [ctypes.POINTER(DecodeArgs), _vp, _sz, _vp]),
@@ -269,6 +272,24 @@ def decode_args(q_idx, k_idx, K, V, Q, seq_lens, k, O, idx, count, scores=None, 
 
 def decode_workspace_size(args: DecodeArgs) -> int:
     return load_library().clsa_decode_workspace_size(ctypes.byref(args))
+
+
+def attention_mass(Q, K, lse_sparse, seq_lens, scale: float = 0.0, ws: Optional[Workspace] = None,
+                   mass=None, lse_all=None, want_lse_all: bool = True):
+    """Share of the dense softmax mass on the selection (see clsa.h): returns (mass, lse_all),
+    both fp32 [L][B][Hq]; lse_sparse is the decode step's lse output."""
+    lib = load_library()
+    L, B, Hq, d = Q.shape
+    _, n_max, Hkv, _ = K.shape
+    need = lib.clsa_attention_mass_workspace_size(B, n_max, L, Hq, Hkv, d)
+    ws = (ws or Workspace(need)).ensure(need)
+    if mass is None:
+        mass = torch.empty(L, B, Hq, dtype=torch.float32, device=Q.device)
+    if lse_all is None and want_lse_all:
+        lse_all = torch.empty(L, B, Hq, dtype=torch.float32, device=Q.device)
+    _check(lib.clsa_attention_mass(_p(Q), _p(K), _p(lse_sparse), _p(seq_lens), B, n_max, L, Hq, Hkv, d, scale,
+                                   _dt(K), _p(mass), _p(lse_all), ws.ptr, ws.nbytes, _stream()), "clsa_attention_mass")
+    return mass, lse_all
 
 
 def distill_target(Q, K, scores, seq_lens, scale: float = 0.0, ws: Optional[Workspace] = None,

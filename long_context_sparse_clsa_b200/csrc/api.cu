@@ -312,6 +312,29 @@ clsa_status clsa_distill_target(const void* Q, const void* K, const float* score
                                   kl, w, w + kWsHeader, static_cast<cudaStream_t>(stream)));
 }
 
+size_t clsa_attention_mass_workspace_size(int B, int n_max, int L, int Hq, int Hkv, int d) {
+  if (check_attn(B, n_max, L, Hq, Hkv, d, CLSA_BF16, kMaxDirectK) != CLSA_OK) return 0;
+  return kWsHeader + std::max(attention_mass_ws_bytes(B, n_max, L, Hq, Hkv, d, CLSA_BF16),
+                              attention_mass_ws_bytes(B, n_max, L, Hq, Hkv, d, CLSA_F32));
+}
+
+clsa_status clsa_attention_mass(const void* Q, const void* K, const float* lse_sparse, const int32_t* seq_lens, int B,
+                                int n_max, int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* mass,
+                                float* lse_all, void* ws, size_t ws_bytes, void* stream) {
+  CallScope scope(stream);
+  clsa_status st = check_attn(B, n_max, L, Hq, Hkv, d, dt, kMaxDirectK);
+  if (st != CLSA_OK) return st;
+  if (!Q || !K || !lse_sparse || !seq_lens || !mass) return CLSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned4(lse_sparse) || !aligned4(seq_lens) || !aligned4(mass) ||
+      (lse_all && !aligned4(lse_all)))
+    return CLSA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < clsa_attention_mass_workspace_size(B, n_max, L, Hq, Hkv, d) || !aligned16(ws))
+    return CLSA_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  return from_cuda(launch_attention_mass(Q, K, lse_sparse, seq_lens, B, n_max, L, Hq, Hkv, d, resolve_scale(scale, d),
+                                         dt, mass, lse_all, w, w + kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
 size_t clsa_decode_workspace_size(const clsa_decode_args* a) {
   if (check_decode(a) != CLSA_OK) return 0;
   return decode_layout(a).total;

@@ -244,4 +244,48 @@ cudaError_t launch_distill(const void* Q, const void* K, const float* scores, co
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Attention-mass coverage for the shapes the tensor-core pass does not take (fp32, d = 64):
+// the row lse over each sequence's cache from the split-k attention kernel (K stands in for
+// V: the lse does not use V; the output is discarded), then mass = exp(lse_S - lse_all).
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void mass_from_lse_kernel(const float* __restrict__ lse_sparse, const float* __restrict__ lse_all, int n,
+                                     float* __restrict__ mass) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float ls = lse_sparse[i], la = lse_all[i];
+  mass[i] = (la == -INFINITY || ls == -INFINITY) ? 0.f : expf(ls - la);
+}
+}  // namespace
+
+size_t attention_mass_ws_bytes(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dtype dt) {
+  if (distill_tc_supported(B, n_max, L, Hq, Hkv, d, dt)) return attention_mass_tc_ws_bytes(B, n_max, L, Hq, Hkv);
+  AttnShape sh{B, n_max, L, Hq, Hkv, d, dt, false, n_max, 0};
+  size_t off = 0;
+  off += align_up((size_t)L * B * Hq * d * (dt == CLSA_BF16 ? 2 : 4), 256);  // discarded attention output
+  off += align_up((size_t)L * B * Hq * 4, 256);                              // row lse
+  off += attn_ws_bytes(sh);
+  return off;
+}
+
+cudaError_t launch_attention_mass(const void* Q, const void* K, const float* lse_sparse, const int32_t* lens, int B,
+                                  int n_max, int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* mass,
+                                  float* lse_all, void* ws_header, void* ws, cudaStream_t s) {
+  if (distill_tc_supported(B, n_max, L, Hq, Hkv, d, dt))
+    return launch_attention_mass_tc(Q, K, lse_sparse, lens, B, n_max, L, Hq, Hkv, scale, mass, lse_all, ws_header, ws, s);
+  char* w = static_cast<char*>(ws);
+  void* O = w;
+  w += align_up((size_t)L * B * Hq * d * (dt == CLSA_BF16 ? 2 : 4), 256);
+  float* lse_row = lse_all ? lse_all : reinterpret_cast<float*>(w);
+  w += align_up((size_t)L * B * Hq * 4, 256);
+  AttnShape sh{B, n_max, L, Hq, Hkv, d, dt, false, n_max, 0};
+  cudaError_t e = launch_sparse_attn(sh, Q, K, K, nullptr, lens, scale, O, lse_row, ws_header, w, s);
+  if (e != cudaSuccess) return e;
+  const int n = L * B * Hq;
+  mass_from_lse_kernel<<<(n + 255) / 256, 256, 0, s>>>(lse_sparse, lse_row, n, mass);
+  launches_add(1, s);
+  return cudaGetLastError();
+}
+
 }  // namespace clsa

@@ -505,4 +505,71 @@ cudaError_t launch_distill_tc(const void* Q, const void* K, const float* scores,
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Attention-mass coverage: the share of each row's dense softmax mass that the selection S
+// holds, mass = sum_{j in S} softmax_j = exp(lse_S - lse_all).  lse_all over the whole
+// cache is pass 1 of the distillation kernel (per unit row: max and sum of 2^(s scale
+// log2 e) over its token split); this kernel merges the splits in split order and takes
+// lse_S from the decode step's lse output.
+// ---------------------------------------------------------------------------
+namespace {
+
+__global__ void __launch_bounds__(128) attn_mass_kernel(const float* __restrict__ pm, const float* __restrict__ pl,
+                                                        const float* __restrict__ lse_sparse, int B, int L, int Hq,
+                                                        int Hkv, int G, int Lg, int nlg, int nsplit,
+                                                        float* __restrict__ mass, float* __restrict__ lse_all) {
+  pdl_enter();
+  int u = blockIdx.x;  // (b, g, layer group), the order of distill_tc_kernel's units / nsplit
+  const int lg = u % nlg;
+  u /= nlg;
+  const int g = u % Hkv, b = u / Hkv;
+  const int r = threadIdx.x;
+  const int rows = min(Lg, L - lg * Lg) * G;
+  if (r >= rows) return;
+  const size_t unit0 = ((size_t)blockIdx.x * nsplit) * 128 + r;
+  float M = -INFINITY;
+  for (int x = 0; x < nsplit; ++x) M = fmaxf(M, pm[unit0 + (size_t)x * 128]);
+  float S = 0.f;
+  if (M != -INFINITY)
+    for (int x = 0; x < nsplit; ++x) S += pl[unit0 + (size_t)x * 128] * exp2f(pm[unit0 + (size_t)x * 128] - M);
+  const float la = S > 0.f ? (M + log2f(S)) * 0.6931471805599453f : -INFINITY;  // natural log
+  const int l = lg * Lg + r / G, h = g * G + r % G;
+  const size_t o = ((size_t)l * B + b) * Hq + h;
+  const float ls = lse_sparse[o];
+  mass[o] = (la == -INFINITY || ls == -INFINITY) ? 0.f : expf(ls - la);
+  if (lse_all) lse_all[o] = la;
+}
+
+}  // namespace
+
+size_t attention_mass_tc_ws_bytes(int B, int n_max, int L, int Hq, int Hkv) {
+  const DTPlan pl = dt_plan(B, n_max, L, Hq, Hkv);
+  return 2 * align_up((size_t)pl.units * 128 * 4, 256);
+}
+
+cudaError_t launch_attention_mass_tc(const void* Q, const void* K, const float* lse_sparse, const int32_t* lens, int B,
+                                     int n_max, int L, int Hq, int Hkv, float scale, float* mass, float* lse_all,
+                                     void* ws_header, void* ws, cudaStream_t s) {
+  const DTPlan pl = dt_plan(B, n_max, L, Hq, Hkv);
+  char* w = static_cast<char*>(ws);
+  float* pm = reinterpret_cast<float*>(w);
+  w += align_up((size_t)pl.units * 128 * 4, 256);
+  float* plsum = reinterpret_cast<float*>(w);
+  CUtensorMap tk;
+  if (!make_tmap_bf16_2d(&tk, K, (uint64_t)B * n_max, (uint64_t)Hkv * kHd, (uint64_t)Hkv * kHd * 2, kTokT, 64))
+    return cudaErrorInvalidValue;
+  DTParams p{static_cast<const __nv_bfloat16*>(Q), lens, pm, plsum, nullptr, ws_header, B, n_max, L, Hq, Hkv,
+             pl.G, pl.Lg, pl.nlg, pl.nsplit, pl.chunk, scale * 1.4426950408889634f};
+  cudaError_t e = cudaFuncSetAttribute(distill_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kDTSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(distill_tc_kernel<1>, dim3(pl.units), dim3(kDThreads), kDTSmemBytes, s, tk, p);
+  if (e == cudaSuccess)
+    e = launch_pdl(attn_mass_kernel, dim3(B * Hkv * pl.nlg), dim3(128), 0, s, (const float*)pm, (const float*)plsum,
+                   lse_sparse, B, L, Hq, Hkv, pl.G, pl.Lg, pl.nlg, pl.nsplit, mass, lse_all);
+  if (e != cudaSuccess) return e;
+  launches_add(2, s);
+  return cudaGetLastError();
+}
+
 }  // namespace clsa

@@ -82,6 +82,16 @@ cudaError_t launch_distill_tc(const void* Q, const void* K, const float* scores,
                               int L, int Hq, int Hkv, float scale, float* abar, float* kl, void* ws_header, void* ws,
                               cudaStream_t s);
 
+// ----- attention-mass coverage: exp(lse_S - lse_all) per (layer, sequence, query head) -----
+size_t attention_mass_ws_bytes(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dtype dt);
+cudaError_t launch_attention_mass(const void* Q, const void* K, const float* lse_sparse, const int32_t* lens, int B,
+                                  int n_max, int L, int Hq, int Hkv, int d, float scale, clsa_dtype dt, float* mass,
+                                  float* lse_all, void* ws_header, void* ws, cudaStream_t s);
+size_t attention_mass_tc_ws_bytes(int B, int n_max, int L, int Hq, int Hkv);
+cudaError_t launch_attention_mass_tc(const void* Q, const void* K, const float* lse_sparse, const int32_t* lens, int B,
+                                     int n_max, int L, int Hq, int Hkv, float scale, float* mass, float* lse_all,
+                                     void* ws_header, void* ws, cudaStream_t s);
+
 // ----- failure-detection self-test (a wait that runs out and reports) ------------
 cudaError_t launch_selftest_timeout(int which, void* ws_header, void* ws_body, cudaStream_t s);
 

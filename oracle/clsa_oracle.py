@@ -262,6 +262,29 @@ def prefill_chunk(q_idx, k_idx, K, V, Q, n: int, k: int,
 # distillation target of the shared indexer (forward only)
 # --------------------------------------------------------------------------
 
+def attention_mass(Q, K, idx, count, seq_lens, scale: Optional[float] = None):
+    """Attention-mass coverage (picx.dev CLSA summary, Attention Sparsity Analysis): for each
+    layer l, sequence b and query head h, the share of the dense softmax over the len_b cached
+    rows that falls on the selected rows idx[b, :count[b]].  Query head h reads KV head
+    h // (Hq / Hkv).  Q [L][B][Hq][d], K [B][n_max][Hkv][d]; float64 [L][B][Hq], 0 for a
+    sequence with no tokens.
+    """
+    Qf, Kf = _f64(Q), _f64(K)
+    L, B, Hq, _ = Qf.shape
+    G = Hq // Kf.shape[2]
+    out = np.zeros((L, B, Hq))
+    for b in range(B):
+        n, c = int(seq_lens[b]), int(count[b])
+        if n == 0 or c == 0:
+            continue
+        sel = np.asarray(idx[b, :c], dtype=np.int64)
+        for l in range(L):
+            for h in range(Hq):
+                w, _ = attention_weights(Qf[l, b, h], Kf[b, :n, h // G], scale)
+                out[l, b, h] = w[sel].sum()
+    return out
+
+
 def distill_target(Q, K, I, seq_lens, scale: Optional[float] = None):
     """Per decode query b: Abar_b = mean over every (layer, query head) of that head's
     softmax over the len_b cached tokens (query head h reads KV head h // (Hq / Hkv)),

@@ -454,3 +454,43 @@ def test_distill_invariances():
     A3, kl3 = O.distill_target(Q3, K, I, lens)
     np.testing.assert_allclose(A3, A, rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(kl3, kl, rtol=1e-10)
+
+
+# --------------------------------------------------------------------- attention-mass coverage
+# picx.dev CLSA summary, Attention Sparsity Analysis: the share of the dense softmax mass on S
+
+def test_attention_mass_against_torch_softmax_and_closed_forms():
+    rng = np.random.default_rng(17)
+    L, B, Hq, Hkv, d, n = 2, 2, 4, 2, 16, 40
+    Q = rng.standard_normal((L, B, Hq, d))
+    K = rng.standard_normal((B, n, Hkv, d))
+    lens = np.array([n, 23])
+    idx = np.full((B, 10), -1)
+    count = np.array([10, 7])
+    for b in range(B):
+        idx[b, :count[b]] = np.sort(rng.choice(lens[b], count[b], replace=False))
+    got = O.attention_mass(Q, K, idx, count, lens)
+    # an independent route: torch's float64 softmax over the whole row, summed over S
+    for l in range(L):
+        for b in range(B):
+            for h in range(Hq):
+                s = torch.tensor(K[b, :lens[b], h // 2] @ Q[l, b, h] / math.sqrt(d))
+                p = torch.softmax(s, dim=0).numpy()
+                assert abs(got[l, b, h] - p[idx[b, :count[b]]].sum()) < 1e-12
+    assert np.all((got > 0) & (got < 1))
+    # every row selected: the whole mass
+    full = np.tile(np.arange(n), (B, 1))
+    np.testing.assert_allclose(O.attention_mass(Q, K, full, lens, lens), 1.0, atol=1e-12)
+    # equal keys: the mass is the selected fraction |S| / n
+    Ke = np.repeat(K[:, :1], n, axis=1)
+    np.testing.assert_allclose(O.attention_mass(Q, Ke, idx, count, lens)[:, 0], count[0] / n, atol=1e-12)
+    np.testing.assert_allclose(O.attention_mass(Q, Ke, idx, count, lens)[:, 1], count[1] / lens[1], atol=1e-12)
+    # one dominant key: ~1 when it is selected, ~0 when not
+    Kd = K.copy()
+    j = int(idx[0, 0])
+    Kd[0, j, :] = 60 * Q[0, 0, 0] / np.linalg.norm(Q[0, 0, 0])
+    assert O.attention_mass(Q, Kd, idx, count, lens)[0, 0, 0] > 1 - 1e-9
+    other = np.array([[k for k in range(n) if k != j][:10], idx[1]])
+    assert O.attention_mass(Q, Kd, other, count, lens)[0, 0, 0] < 1e-9
+    # an empty sequence: 0
+    assert np.all(O.attention_mass(Q, K, idx, np.array([0, 7]), np.array([0, 23]))[:, 0] == 0)
