@@ -394,6 +394,10 @@ def run_clsa(args):
         for _ in range(reps):
             if flush:
                 flush_l2()
+            # a device-side wait ahead of the first event keeps the stream busy while the
+            # host issues the call, so the events bracket the device work, not the host's
+            # argument marshalling
+            torch.cuda._sleep(200_000)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()

@@ -69,6 +69,12 @@ size_t attn_ws_bytes(const AttnShape& sh);
 cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
                                const int32_t* idx, const int32_t* count, float scale, void* O, float* lse,
                                void* ws_header, void* attn_ws, cudaStream_t s);
+// the same attention on tcgen05 (bf16, d = 128, rows <= 128); partials as the split-k path's
+bool sparse_attn_tc_supported(const AttnShape& sh, const AttnPlan& pl, const void* Q, const void* K, const void* V,
+                              const void* O);
+cudaError_t launch_sparse_attn_tc(const AttnShape& sh, const AttnPlan& pl, const void* Q, const void* Kc,
+                                  const void* Vc, const int32_t* idx, const int32_t* count, float scale_log2, void* O,
+                                  float* lse, float* Op, float* Mp, float* Lp, void* ws_header, cudaStream_t s);
 
 // ----- distillation target (forward): Abar and KL(Abar || softmax(I)) ----------------
 size_t distill_ws_bytes(int B, int n_max, int L, int Hq, int Hkv, int d, clsa_dtype dt);

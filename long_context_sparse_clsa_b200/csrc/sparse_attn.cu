@@ -437,6 +437,12 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
+  // one warp per output row.  The split partials of a row are independent loads: lane s
+  // reads split s's max and row sum, and the outputs go in batches of 8 splits whose loads
+  // are all issued before any is used (one L2 round trip per batch, not per split).
+  constexpr int CPL = D / 32;  // output columns per lane: 4 (D = 128) or 2 (D = 64)
+  constexpr int kBatch = 8;
+  pdl_enter();  // launched programmatically behind the attention kernel: its partials first
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= p.L * p.B * p.Hq) return;
@@ -447,20 +453,48 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
   const int r = (l % p.Lg) * p.G + h % p.G;
   const size_t base = (((size_t)b * p.Hkv + g) * p.nlg + lgrp) * p.nsplit * p.rows + r;
   float M = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.Mp[base + (size_t)s * p.rows]);
-  constexpr int CPL = D / 32;
+  for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, p.Mp[base + (size_t)s * p.rows]);
+  M = warp_max(M);
   float acc[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
   float den = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < p.nsplit; ++s) {
-      const size_t pi = base + (size_t)s * p.rows;
-      const float w = exp2f(p.Mp[pi] - M);
-      den = fmaf(w, p.Lp[pi], den);
+    for (int s0 = 0; s0 < p.nsplit; s0 += 32) {
+      const int ns = min(32, p.nsplit - s0);
+      float wl = 0.f;  // weight 2^(m_s - M) of split s0 + lane
+      if (lane < ns) {
+        const size_t pi = base + (size_t)(s0 + lane) * p.rows;
+        wl = exp2f(p.Mp[pi] - M);
+        den = fmaf(wl, p.Lp[pi], den);
+      }
+      for (int j0 = 0; j0 < ns; j0 += kBatch) {
+        float o[kBatch][CPL];
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[c] = fmaf(w, p.Op[pi * D + lane * CPL + c], acc[c]);
+        for (int u = 0; u < kBatch; ++u) {
+          const float* src = p.Op + (base + (size_t)(s0 + min(j0 + u, ns - 1)) * p.rows) * D + lane * CPL;
+          if constexpr (CPL == 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+            o[u][0] = v.x;
+            o[u][1] = v.y;
+            o[u][2] = v.z;
+            o[u][3] = v.w;
+          } else {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+            o[u][0] = v.x;
+            o[u][1] = v.y;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          float w = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
+          w = j0 + u < ns ? w : 0.f;  // past the last split: the clamped reload counts 0
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[c] = fmaf(w, o[u][c], acc[c]);
+        }
+      }
     }
+    den = warp_sum(den);
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   T* out = static_cast<T*>(p.O) + (((size_t)l * p.B + b) * p.Hq + h) * D;
@@ -543,7 +577,10 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
   }
   dim3 grid(pl.nsplit, sh.Hkv, sh.B * pl.nlg);
   cudaError_t e = cudaSuccess;
-  if (sh.dt == CLSA_BF16) {
+  const bool tc5 = sparse_attn_tc_supported(sh, pl, Q, Kc, Vc, O);
+  if (tc5) {  // counts its own launch
+    e = launch_sparse_attn_tc(sh, pl, Q, Kc, Vc, idx, count, p.scale_log2, O, lse, p.Op, p.Mp, p.Lp, ws_header, s);
+  } else if (sh.dt == CLSA_BF16) {
     const int NW = (pl.rows + 15) / 16;
     const bool two = NW <= 6;  // two CTAs per SM fit
     // the split's token list lives in shared memory only when gathering by index
@@ -585,20 +622,20 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
     }
 #undef CLSA_ATTN_F32
   }
-  launches_add(1, s);
+  if (!tc5) launches_add(1, s);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.nsplit == 1) return e;
   const int rows_total = sh.L * sh.B * sh.Hq;
   dim3 cg((rows_total + 7) / 8);
   if (sh.dt == CLSA_BF16) {
-    if (sh.d == 128) attn_combine_kernel<__nv_bfloat16, 128><<<cg, 256, 0, s>>>(p);
-    else attn_combine_kernel<__nv_bfloat16, 64><<<cg, 256, 0, s>>>(p);
+    if (sh.d == 128) e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 128>, cg, dim3(256), 0, s, p);
+    else e = launch_pdl(attn_combine_kernel<__nv_bfloat16, 64>, cg, dim3(256), 0, s, p);
   } else {
-    if (sh.d == 128) attn_combine_kernel<float, 128><<<cg, 256, 0, s>>>(p);
-    else attn_combine_kernel<float, 64><<<cg, 256, 0, s>>>(p);
+    if (sh.d == 128) e = launch_pdl(attn_combine_kernel<float, 128>, cg, dim3(256), 0, s, p);
+    else e = launch_pdl(attn_combine_kernel<float, 64>, cg, dim3(256), 0, s, p);
   }
   launches_add(1, s);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace clsa

@@ -1,7 +1,7 @@
 """Run one stage of the CLSA path on a named workload, for profilers.
 
     python -m long_context_sparse_clsa_b200.profile_cases --stage decode_step \
-        [--workload decode128k] [--reps 3] [--batch B] [--rows T]
+        [--workload decode128k] [--reps 3] [--batch B] [--rows T] [--layers L]
 
 Stages: index_scores, topk, gather_kv, sparse_attn, decode_step, prefill_chunk, distill_target.
 Inputs are the seeded synthetic workloads of ``inputs.py``; ``--batch`` replaces
@@ -26,6 +26,8 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--batch", type=int, default=0)
     ap.add_argument("--rows", type=int, default=0, help="prefill rows T (default: the workload's)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="sparse_attn: attend with the first LAYERS layers' queries (default: all)")
     a = ap.parse_args()
     w = WORKLOADS[a.workload]
     if a.batch:
@@ -40,12 +42,13 @@ def main():
         sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
         idx, cnt = clsa.topk(sc, dv["seq_lens"], w.k)
         KS, VS = clsa.gather_kv(dv["K"], dv["V"], idx, cnt)
+        Qa = dv["Q"][:a.layers].contiguous() if a.layers else dv["Q"]
         dws = clsa.Workspace(clsa.load_library().clsa_distill_workspace_size(w.B, w.n_max, w.L, w.Hq, w.Hkv, w.d))
         fns = {
             "index_scores": lambda: clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"], sc),
             "topk": lambda: clsa.topk(sc, dv["seq_lens"], w.k, idx=idx, count=cnt),
             "gather_kv": lambda: clsa.gather_kv(dv["K"], dv["V"], idx, cnt, K_S=KS, V_S=VS),
-            "sparse_attn": lambda: clsa.sparse_attn(dv["Q"], KS, VS, cnt),
+            "sparse_attn": lambda: clsa.sparse_attn(Qa, KS, VS, cnt),
             "decode_step": lambda: clsa.decode_step(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"],
                                                     dv["seq_lens"], w.k),
             "distill_target": lambda: clsa.distill_target(dv["Q"], dv["K"], sc, dv["seq_lens"], ws=dws),

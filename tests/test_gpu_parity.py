@@ -152,6 +152,63 @@ def test_sparse_attn(name, L):
     assert max_abs(got_lse[fin], want_lse[fin]) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse[fin]).max())
 
 
+@pytest.mark.parametrize("layers", ["all", "one"])
+def test_sparse_attn_full_size(layers):
+    """decode128k through the stage calls, as the per-kernel timings run them: gathered
+    compact K_S/V_S, then clsa_sparse_attn over all 24 layers or over one layer (the
+    model-faithful per-layer call); every head of the first and last layers against the
+    oracle, with the LSE."""
+    w = WORKLOADS["decode128k"]
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    idx, cnt = clsa.topk(sc, dv["seq_lens"], w.k)
+    KS, VS = clsa.gather_kv(dv["K"], dv["V"], idx, cnt)
+    Q = dv["Q"] if layers == "all" else dv["Q"][-1:].contiguous()
+    out, lse = clsa.sparse_attn(Q, KS, VS, cnt)
+    torch.cuda.synchronize()
+    i_np, c_np = idx.cpu().numpy(), cnt.cpu().numpy()
+    got, got_lse = tensor_f64(out), tensor_f64(lse)
+    # the oracle over the selected rows only (its gather, then its attention)
+    c = int(c_np[0])
+    sel = i_np[0, :c]
+    Kc, Vc = inp.K[:, sel], inp.V[:, sel]
+    ic = np.arange(c, dtype=np.int64)[None]
+    ls = (0, w.L - 1) if layers == "all" else (w.L - 1,)
+    for l in ls:
+        want, want_lse = O.sparse_attention(inp.Q[l:l + 1], Kc, Vc, ic, c_np)
+        lq = l if layers == "all" else 0
+        assert max_abs(got[lq], want[0]) <= TOL[w.dtype], l
+        assert max_abs(got_lse[lq], want_lse[0]) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse).max()), l
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_sparse_attn_growing_scores(dtype):
+    """Scores that grow along the selection by far more than 2^8 per 64-token chunk: the
+    tensor-core kernel's reference max must move and its running output be rescaled
+    (the f32 kernel is the control).  Ragged counts, one empty sequence, several splits."""
+    rng = np.random.default_rng(11)
+    B, k, L, Hq, Hkv, d = 3, 700, 3, 32, 8, 128
+    K = rng.standard_normal((B, k, Hkv, d))
+    K *= (1.0 + np.arange(k) / 40.0)[None, :, None, None]  # |scores| ~ 1 .. 18 sigma
+    V = rng.standard_normal((B, k, Hkv, d))
+    Q = rng.standard_normal((L, B, Hq, d))
+    cnt = np.array([700, 0, 333], dtype=np.int32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    # the oracle sees the values the device holds
+    Kd, Vd, Qd = (torch.tensor(a, dtype=tdt, device="cuda") for a in (K, V, Q))
+    out, lse = clsa.sparse_attn(Qd, Kd, Vd, torch.tensor(cnt, device="cuda"))
+    torch.cuda.synchronize()
+    Kh, Vh, Qh = (tensor_f64(t) for t in (Kd, Vd, Qd))
+    idx = np.tile(np.arange(k, dtype=np.int64), (B, 1))
+    want, want_lse = O.sparse_attention(Qh, Kh, Vh, idx, cnt)
+    assert max_abs(tensor_f64(out), want) <= TOL[dtype]
+    got_lse = tensor_f64(lse)
+    fin = np.isfinite(want_lse)
+    assert (np.isneginf(got_lse) == ~fin).all()
+    assert max_abs(got_lse[fin], want_lse[fin]) <= LSE_TOL[dtype] * (1 + np.abs(want_lse[fin]).max())
+
+
 # ----------------------------------------------------------------------- A5 decode step
 
 @pytest.mark.parametrize("name", list(CASES))
