@@ -224,7 +224,7 @@ clsa_status clsa_index_scores(const void* q_idx, const void* k_idx, const int32_
   if (!dims_ok(d_idx)) return CLSA_ERR_UNSUPPORTED;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned4(seq_lens) || !aligned4(scores))
     return CLSA_ERR_INVALID_ARG;
-  return from_cuda(launch_index_scores(q_idx, k_idx, seq_lens, B, n_max, d_idx, dt, scores,
+  return from_cuda(launch_index_scores(q_idx, k_idx, seq_lens, B, n_max, d_idx, dt, scores, nullptr,
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -351,7 +351,7 @@ clsa_status clsa_decode_step(const clsa_decode_args* a, void* ws, size_t ws_byte
   if (lay.fused) return from_cuda(launch_decode_fused(a, resolve_scale(a->scale, a->d), w, w + kWsHeader, s));
   float* scores = a->scores ? a->scores : reinterpret_cast<float*>(w + lay.scores);
   cudaError_t e = launch_index_scores(a->q_idx, a->k_idx, a->seq_lens, a->B, a->n_max, a->d_idx, a->dtype,
-                                      scores, s);
+                                      scores, w, s);
   if (e != cudaSuccess) return CLSA_ERR_CUDA;
   e = launch_topk(scores, a->seq_lens, a->B, a->n_max, a->k, a->idx, a->count, w, w + lay.topk, s);
   if (e != cudaSuccess) return CLSA_ERR_CUDA;

@@ -3,7 +3,8 @@
 // layers gather KV by the shared index; here the gather happens once for all).
 //
 // One warp per selected token copies its K and V rows (Hkv * d * elem bytes,
-// contiguous in the [n][Hkv][d] cache) with 16-byte loads and stores.  An index
+// contiguous in the [n][Hkv][d] cache) with 16-byte loads and stores, up to 4 K and 4 V
+// loads per lane in flight before the stores (a 4 KiB bf16 row pair per warp at once).  An index
 // outside [0, n_max) is never dereferenced: the row is zero-filled and
 // CLSA_ERR_BAD_INDEX (detail = b * 2^32 + i) is recorded.
 #include "common.cuh"
@@ -35,11 +36,26 @@ __global__ void __launch_bounds__(256) gather_kv_kernel(const uint4* __restrict_
   }
   const uint4* sk = K + ((size_t)b * n_max + t) * row_vec;
   const uint4* sv = V + ((size_t)b * n_max + t) * row_vec;
-  for (int c = lane; c < row_vec; c += 32) {
-    const uint4 a = ld_stream_v4(sk + c);
-    const uint4 v = ld_stream_v4(sv + c);
-    dk[c] = a;
-    dv[c] = v;
+  // every load of a batch is issued before its stores: 2 kU 16-byte loads in flight per lane
+  constexpr int kU = 4;
+  for (int c0 = lane; c0 < row_vec; c0 += 32 * kU) {
+    uint4 a[kU], v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < row_vec) {
+        a[u] = ld_stream_v4(sk + c);
+        v[u] = ld_stream_v4(sv + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < row_vec) {
+        dk[c] = a[u];
+        dv[c] = v[u];
+      }
+    }
   }
 }
 

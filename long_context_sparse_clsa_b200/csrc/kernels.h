@@ -28,8 +28,10 @@ void launches_add(int n, cudaStream_t s);
 int launches_get();
 
 // ----- indexer scan (routing equation, scores) ------------------------------
+// ws_header: the call's error word (a bounded wait that runs out records CLSA_ERR_TIMEOUT), or null
 cudaError_t launch_index_scores(const void* q_idx, const void* k_idx, const int32_t* seq_lens, int B,
-                                int n_max, int d_idx, clsa_dtype dt, float* scores, cudaStream_t s);
+                                int n_max, int d_idx, clsa_dtype dt, float* scores, void* ws_header,
+                                cudaStream_t s);
 
 // ----- exact radix top-k -----------------------------------------------------
 size_t topk_ws_bytes(int B, int n_max, int k);

@@ -437,11 +437,11 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const AttnParams p) {
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
-  // one warp per output row.  The split partials of a row are independent loads: lane s
-  // reads split s's max and row sum, and the outputs go in batches of 8 splits whose loads
-  // are all issued before any is used (one L2 round trip per batch, not per split).
+  // one warp per output row.  Every load of a group of 32 splits is issued before any is
+  // used: lane s reads split s's max and row sum, and every lane its columns of all the
+  // group's partial outputs, so a row costs one L2 round trip per 32 splits (the reductions
+  // over the lanes follow in registers).
   constexpr int CPL = D / 32;  // output columns per lane: 4 (D = 128) or 2 (D = 64)
-  constexpr int kBatch = 8;
   pdl_enter();  // launched programmatically behind the attention kernel: its partials first
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -452,49 +452,52 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
   const int g = h / p.G, lgrp = l / p.Lg;
   const int r = (l % p.Lg) * p.G + h % p.G;
   const size_t base = (((size_t)b * p.Hkv + g) * p.nlg + lgrp) * p.nsplit * p.rows + r;
-  float M = -INFINITY;
-  for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, p.Mp[base + (size_t)s * p.rows]);
-  M = warp_max(M);
   float acc[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
-  float den = 0.f;
-  if (M != -INFINITY) {
-    for (int s0 = 0; s0 < p.nsplit; s0 += 32) {
-      const int ns = min(32, p.nsplit - s0);
-      float wl = 0.f;  // weight 2^(m_s - M) of split s0 + lane
-      if (lane < ns) {
-        const size_t pi = base + (size_t)(s0 + lane) * p.rows;
-        wl = exp2f(p.Mp[pi] - M);
-        den = fmaf(wl, p.Lp[pi], den);
-      }
-      for (int j0 = 0; j0 < ns; j0 += kBatch) {
-        float o[kBatch][CPL];
+  float M = -INFINITY, den = 0.f;
+  for (int s0 = 0; s0 < p.nsplit; s0 += 32) {
+    const int ns = min(32, p.nsplit - s0);
+    float ml = -INFINITY, ll = 0.f;  // split s0 + lane
+    if (lane < ns) {
+      const size_t pi = base + (size_t)(s0 + lane) * p.rows;
+      ml = __ldcg(p.Mp + pi);
+      ll = __ldcg(p.Lp + pi);
+    }
+    float o[32][CPL];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          const float* src = p.Op + (base + (size_t)(s0 + min(j0 + u, ns - 1)) * p.rows) * D + lane * CPL;
-          if constexpr (CPL == 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-            o[u][0] = v.x;
-            o[u][1] = v.y;
-            o[u][2] = v.z;
-            o[u][3] = v.w;
-          } else {
-            const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
-            o[u][0] = v.x;
-            o[u][1] = v.y;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          float w = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
-          w = j0 + u < ns ? w : 0.f;  // past the last split: the clamped reload counts 0
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) acc[c] = fmaf(w, o[u][c], acc[c]);
-        }
+    for (int u = 0; u < 32; ++u) {
+      const float* src = p.Op + (base + (size_t)(s0 + min(u, ns - 1)) * p.rows) * D + lane * CPL;
+      if constexpr (CPL == 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+        o[u][0] = v.x;
+        o[u][1] = v.y;
+        o[u][2] = v.z;
+        o[u][3] = v.w;
+      } else {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+        o[u][0] = v.x;
+        o[u][1] = v.y;
       }
     }
-    den = warp_sum(den);
+    // merge this group into the running (M, den, acc)
+    const float Mg = warp_max(ml);
+    const float Mn = fmaxf(M, Mg);
+    if (Mn != -INFINITY) {
+      const float a = exp2f(M - Mn);  // 0 on the first group with a finite max
+      const float wl = exp2f(ml - Mn);
+      den = den * a + warp_sum(wl * ll);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[c] *= a;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        float w = __shfl_sync(0xffffffffu, wl, u);
+        w = u < ns ? w : 0.f;  // past the last split: the clamped reload counts 0
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[c] = fmaf(w, o[u][c], acc[c]);
+      }
+      M = Mn;
+    }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   T* out = static_cast<T*>(p.O) + (((size_t)l * p.B + b) * p.Hq + h) * D;
