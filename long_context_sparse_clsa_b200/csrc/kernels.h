@@ -71,6 +71,13 @@ size_t attn_ws_bytes(const AttnShape& sh);
 cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
                                const int32_t* idx, const int32_t* count, float scale, void* O, float* lse,
                                void* ws_header, void* attn_ws, cudaStream_t s);
+// few rows per KV head (bf16, L * G <= 16, d = 64 or 128): CUDA cores, splits merged in-kernel;
+// false if the shape is outside it.  The plan it fills is the one plan_attention returns.
+bool sparse_attn_rows_plan(const AttnShape& sh, int sm_count, AttnPlan* pl);
+cudaError_t launch_sparse_attn_rows(const AttnShape& sh, const AttnPlan& pl, const void* Q, const void* Kc,
+                                    const void* Vc, const int32_t* idx, const int32_t* count, float scale_log2,
+                                    void* O, float* lse, float* Op, float* Mp, float* Lp, uint32_t* counter,
+                                    void* ws_header, cudaStream_t s);
 // the same attention on tcgen05 (bf16, d = 128, rows <= 128); partials as the split-k path's
 bool sparse_attn_tc_supported(const AttnShape& sh, const AttnPlan& pl, const void* Q, const void* K, const void* V,
                               const void* O);

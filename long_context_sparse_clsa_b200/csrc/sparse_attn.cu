@@ -507,6 +507,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
     p.lse[((size_t)l * p.B + b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
 }
 
+bool aligned16_(const void* a) { return reinterpret_cast<uintptr_t>(a) % 16 == 0; }
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -516,6 +518,7 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 AttnPlan plan_attention(const AttnShape& sh) {
   AttnPlan pl{};
+  if (sparse_attn_rows_plan(sh, device_info().sm_count, &pl)) return pl;
   const int G = sh.Hq / sh.Hkv;
   const int max_rows = sh.dt == CLSA_BF16 ? 128 : 32;
   int Lg = std::max(1, std::min(sh.L, max_rows / G));
@@ -539,7 +542,9 @@ size_t attn_ws_bytes(const AttnShape& sh) {
   const AttnPlan pl = plan_attention(sh);
   if (pl.nsplit == 1) return 0;
   const size_t n = (size_t)sh.B * sh.Hkv * pl.nlg * pl.nsplit * pl.rows;
-  return align_up(n * sh.d * sizeof(float), 256) + 2 * align_up(n * sizeof(float), 256);
+  // split partials (output, max, sum), then one arrival counter per (b, KV head, layer group)
+  return align_up(n * sh.d * sizeof(float), 256) + 2 * align_up(n * sizeof(float), 256) +
+         align_up((size_t)sh.B * sh.Hkv * pl.nlg * sizeof(uint32_t), 256);
 }
 
 cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
@@ -569,6 +574,7 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
   p.O = O;
   p.lse = lse;
   p.ws_header = ws_header;
+  uint32_t* counter = nullptr;
   if (pl.nsplit > 1) {
     const size_t n = (size_t)sh.B * sh.Hkv * pl.nlg * pl.nsplit * pl.rows;
     char* w = static_cast<char*>(attn_ws);
@@ -577,7 +583,14 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
     p.Mp = reinterpret_cast<float*>(w);
     w += align_up(n * sizeof(float), 256);
     p.Lp = reinterpret_cast<float*>(w);
+    w += align_up(n * sizeof(float), 256);
+    counter = reinterpret_cast<uint32_t*>(w);
   }
+  AttnPlan rp{};
+  if (sparse_attn_rows_plan(sh, device_info().sm_count, &rp) && aligned16_(Q) && aligned16_(Kc) && aligned16_(Vc) &&
+      aligned16_(O))
+    return launch_sparse_attn_rows(sh, pl, Q, Kc, Vc, idx, count, p.scale_log2, O, lse, p.Op, p.Mp, p.Lp, counter,
+                                   ws_header, s);
   dim3 grid(pl.nsplit, sh.Hkv, sh.B * pl.nlg);
   cudaError_t e = cudaSuccess;
   const bool tc5 = sparse_attn_tc_supported(sh, pl, Q, Kc, Vc, O);

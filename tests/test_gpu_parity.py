@@ -182,13 +182,15 @@ def test_sparse_attn_full_size(layers):
         assert max_abs(got_lse[lq], want_lse[0]) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse).max()), l
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_sparse_attn_growing_scores(dtype):
+@pytest.mark.parametrize("dtype,L", [("bf16", 3), ("bf16", 6), ("f32", 3)])
+def test_sparse_attn_growing_scores(dtype, L):
     """Scores that grow along the selection by far more than 2^8 per 64-token chunk: the
-    tensor-core kernel's reference max must move and its running output be rescaled
-    (the f32 kernel is the control).  Ragged counts, one empty sequence, several splits."""
+    tensor-core kernel's reference max must move and its running output be rescaled (L = 6:
+    24 rows per KV head), the few-rows kernel's splits merge across very different maxima
+    (L = 3: 12 rows), the f32 kernel is the control.  Ragged counts, one empty sequence,
+    several splits."""
     rng = np.random.default_rng(11)
-    B, k, L, Hq, Hkv, d = 3, 700, 3, 32, 8, 128
+    B, k, Hq, Hkv, d = 3, 700, 32, 8, 128
     K = rng.standard_normal((B, k, Hkv, d))
     K *= (1.0 + np.arange(k) / 40.0)[None, :, None, None]  # |scores| ~ 1 .. 18 sigma
     V = rng.standard_normal((B, k, Hkv, d))
