@@ -230,12 +230,13 @@ __global__ void __launch_bounds__(kThreadsTC, 2) attn_tc_kernel(const TCParams p
     const uint32_t ts = tl + (uint32_t)(kTok * (c & 1) + kNpt * cg);
     const int nv = ntok - (c * kTok + kNpt * cg);  // valid columns of this thread
     const bool full = nv >= kNpt;  // warp-uniform: every column of this thread is a token
-    uint32_t v[kNpt];  // the scores, held across the row-max exchange
+    uint32_t v[kNpt];  // the scores, held until P is final
+    float lmx = -INFINITY;  // this thread's max of its columns (log2 units)
     if (live) {
-      float cmx = -INFINITY;
       if (!dead) {
         tc::ld_32x32b_x32(ts, v);
         tc::ld_wait();
+        float cmx = -INFINITY;
         if (full) {
 #pragma unroll
           for (int j = 0; j < kNpt; j += 2) cmx = fmaxf(cmx, fmaxf(__uint_as_float(v[j]), __uint_as_float(v[j + 1])));
@@ -244,44 +245,17 @@ __global__ void __launch_bounds__(kThreadsTC, 2) attn_tc_kernel(const TCParams p
           for (int j = 0; j < kNpt; ++j)
             if (j < nv) cmx = fmaxf(cmx, __uint_as_float(v[j]));
         }
+        lmx = cmx * p.scale_log2;  // scale > 0: the max commutes
       } else {
 #pragma unroll
         for (int j = 0; j < kNpt; ++j) v[j] = 0xff800000u;  // -inf: P = 0
       }
-      cm[cg * kM + row] = cmx * p.scale_log2;  // scale > 0: the max commutes
     }
-    __syncthreads();
-    if (live) {
-      const float mn = fmaxf(cm[row], cm[kM + row]);
-      if (c == 0) {
-        m = mn;
-      } else {
-        // both threads of a row take the same decision; the TMEM load / store is
-        // .sync.aligned, so a warp with any rescaled row runs it in every lane (alpha = 1
-        // for the others)
-        const bool up = mn > m + kTau;
-        if (__any_sync(0xffffffffu, up)) {
-          const float alpha = up ? fast_exp2(m - mn) : 1.f;
-          if (up) {
-            m = mn;
-            lp *= alpha;
-          }
-          if (!dead) {  // P V of the previous chunk has completed (waited below)
-#pragma unroll 1
-            for (int h2 = 0; h2 < 2; ++h2) {
-              uint32_t w[32];
-              tc::ld_32x32b_x32(to + (uint32_t)(32 * h2), w);
-              tc::ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(__uint_as_float(w[j]) * alpha);
-              tc::st_32x32b_x32(to + (uint32_t)(32 * h2), w);
-            }
-            tc::st_wait();
-          }
-        }
-      }
+    const int lim = full ? kNpt : nv;  // columns at or past lim are not tokens: P = 0
+    // P of this thread's columns against the row's reference max m, into shared memory; the
+    // row sum of those columns is returned
+    auto write_p = [&]() -> float {
       float rs = 0.f;
-      const int lim = full ? kNpt : nv;  // columns at or past lim are not tokens: P = 0
 #pragma unroll
       for (int q = 0; q < kNpt / 8; ++q) {
         uint32_t pw[4];
@@ -301,12 +275,52 @@ __global__ void __launch_bounds__(kThreadsTC, 2) attn_tc_kernel(const TCParams p
         if (row < rows8)
           *reinterpret_cast<uint4*>(sP + tc::sw128_offset(row, (kNpt * cg) / 8 + q)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
       }
-      lp += rs;
-    }
+      return rs;
+    };
+    // Common case: no column of the thread lies more than 2^kTau above its row's reference max,
+    // and P goes out against that max with no exchange.  The first chunk (no max yet) and a
+    // column above the bound anywhere in the CTA take the exchange below (both threads of a row
+    // then agree on the row's new max and rewrite their P); the vote rides on the barrier that
+    // precedes the MMA issue anyway.
+    const bool need = live && (c == 0 || lmx > m + kTau);
+    float rs = 0.f;
+    if (live && !need) rs = write_p();
     if (c + 1 < nch) cp_async_wait<0>();  // chunk c + 1 landed
     fence_proxy_async_smem();
     tc::fence_before_sync();
-    __syncthreads();
+    if (__syncthreads_or(need)) {
+      if (live) cm[cg * kM + row] = lmx;
+      __syncthreads();
+      if (live) {
+        const float mn = fmaxf(cm[row], cm[kM + row]);
+        const bool up = c == 0 || mn > m + kTau;  // the same in both threads of the row
+        if (c > 0 && __any_sync(0xffffffffu, up)) {
+          // TMEM load / store are .sync.aligned: every lane of the warp (alpha = 1 if not up)
+          const float alpha = up ? fast_exp2(m - mn) : 1.f;
+          if (!dead) {  // P V of the previous chunk has completed (waited below)
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+              uint32_t w[32];
+              tc::ld_32x32b_x32(to + (uint32_t)(32 * h2), w);
+              tc::ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(__uint_as_float(w[j]) * alpha);
+              tc::st_32x32b_x32(to + (uint32_t)(32 * h2), w);
+            }
+            tc::st_wait();
+          }
+          if (up) lp *= alpha;
+        }
+        if (up) {
+          m = mn;
+          rs = write_p();
+        }
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncthreads();
+    }
+    lp += rs;
     if (threadIdx.x == 0) {
       tc::fence_after_sync();
       const uint32_t vb = smem_u32(kv + (c & 1) * kStageBytes + kKVTile);
