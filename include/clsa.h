@@ -38,8 +38,10 @@
  *              matching *_workspace_size function returns.  It must be zeroed
  *              once before first use (clsa_workspace_init) and again after any
  *              call reported CLSA_ERR_TIMEOUT; the kernels leave it clean after
- *              a successful call.  One workspace must not be used by two calls
- *              that can run at the same time.
+ *              a successful call.  Clean means clean for the entry point and
+ *              sizes that last used it: before handing a workspace to another
+ *              entry point or other sizes, zero it again.  One workspace must not
+ *              be used by two calls that can run at the same time.
  * Errors.      Argument errors return before anything is launched.  Errors the
  *              kernels detect (an out-of-range index, a wait that ran out)
  *              are recorded in the workspace and read with

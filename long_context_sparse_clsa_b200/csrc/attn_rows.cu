@@ -3,15 +3,17 @@
 //   O^(l)[b, h] = softmax(Q^(l)[b, h] K_S^T * scale) V_S
 // (picx.dev CLSA summary, Methodology > Architecture Overview, per-layer equation).
 //
-// With 4 query rows per KV head the products are a few hundred thousand multiply-adds per
-// CTA, too small to keep a tensor-core pipeline busy; the time is the latency of moving
-// K_S/V_S in and the result out.  So the kernel runs on the CUDA cores and is built to take
-// few dependent round trips:
-//   1. one CTA per (token split, KV head, sequence): its Q rows and its <= 128 selected K/V
-//      rows land in shared memory in one wave of 16-byte async copies;
-//   2. scores (one thread per token and four rows), the split's row max and sum, P V
-//      (one thread per four columns and two rows), all from shared memory;
-//   3. the split's unnormalised output, max and sum go to the split partials; the CTA that
+// With 4 query rows per KV head the products are a handful of 16 x 8 x 16 tiles per CTA: a
+// tcgen05 pipeline (TMEM allocation, 128-row tiles, commit round trips) would only add
+// latency, and the time is the latency of moving K_S/V_S in and the result out.  So the
+// tiles run on warp-level mma.sync (bf16 in, fp32 out, operands by ldmatrix) and the kernel
+// is built to take few dependent round trips:
+//   1. one CTA per (token split, KV head, sequence): its Q rows (zero-padded to 16) and its
+//      <= 128 selected K/V rows land in shared memory in one wave of 16-byte async copies;
+//   2. warp w: S for tokens [16 w, 16 w + 16); the split's row max and row sum through
+//      shared memory; P as bf16 in shared memory;
+//   3. warp w: P V for output columns [16 w, 16 w + 16) over all the split's tokens;
+//   4. the split's unnormalised output, max and sum go to the split partials; the CTA that
 //      arrives last at its (sequence, head) counter merges the splits with the log-sum-exp
 //      rule, writes O and the LSE, and returns the counter to zero.
 // No second kernel, no grid barrier.  Index checks and counters as in the other paths.
@@ -51,12 +53,13 @@ struct RowsParams {
 
 template <int D>
 struct RowsSmem {
-  static constexpr int KSTR = D + 8;  // padded K row (elements): conflict-free row-per-lane reads
-  __nv_bfloat16 K[kMaxTokR][KSTR];
-  __nv_bfloat16 V[kMaxTokR][D];
-  __nv_bfloat16 Q[kMaxRowsR][D];
-  float S[kMaxRowsR][kMaxTokR];     // scores, then P
-  float m[kMaxRowsR], l[kMaxRowsR];
+  static constexpr int STR = D + 8;   // padded bf16 row: conflict-free ldmatrix
+  static constexpr int PSTR = kMaxTokR + 8;
+  __nv_bfloat16 K[kMaxTokR][STR];
+  __nv_bfloat16 V[kMaxTokR][STR];
+  __nv_bfloat16 Q[kMaxRowsR][STR];  // rows >= R are zero
+  __nv_bfloat16 P[kMaxRowsR][PSTR];
+  float red_m[kThreadsR / 32][kMaxRowsR], red_l[kThreadsR / 32][kMaxRowsR];
   float w[kMaxSplitR][kMaxRowsR];   // merge weights
   float inv[kMaxRowsR];
   int tok[kMaxTokR];
@@ -83,17 +86,22 @@ __global__ void __launch_bounds__(kThreadsR) attn_rows_kernel(const RowsParams p
     if (!ok) record_error(p.ws_header, CLSA_ERR_BAD_INDEX, ((long long)b << 32) | (unsigned)(t0 + i));
     sm.tok[i] = ok ? tk : -1;
   }
-  for (int v = tid; v < R * VPR; v += kThreadsR) {  // row r = (layer r / G, head g * G + r % G)
+  for (int v = tid; v < kMaxRowsR * VPR; v += kThreadsR) {  // row r = (layer r / G, head g * G + r % G)
     const int r = v / VPR, c = v % VPR;
-    const int l = r / p.G, h = g * p.G + r % p.G;
-    cp_async_16(&sm.Q[r][c * 8], p.Q + (((size_t)l * p.B + b) * p.Hq + h) * D + c * 8, 16);
+    if (r < R) {
+      const int l = r / p.G, h = g * p.G + r % p.G;
+      cp_async_16(&sm.Q[r][c * 8], p.Q + (((size_t)l * p.B + b) * p.Hq + h) * D + c * 8, 16);
+    } else {
+      *reinterpret_cast<uint4*>(&sm.Q[r][c * 8]) = make_uint4(0u, 0u, 0u, 0u);  // padding rows: S = 0
+    }
   }
   __syncthreads();  // tokens visible
+  const int nt16 = (ntok + 15) & ~15;  // the MMAs read whole 16-token tiles: the rest zero-filled
   const size_t gstride = (size_t)p.Hkv * D;
   const size_t gbase = (size_t)b * (size_t)p.kv_bstride * gstride + (size_t)g * D;
-  for (int v = tid; v < ntok * VPR; v += kThreadsR) {
+  for (int v = tid; v < nt16 * VPR; v += kThreadsR) {
     const int i = v / VPR, c = v % VPR;
-    const int tk = sm.tok[i];
+    const int tk = i < ntok ? sm.tok[i] : -1;
     const size_t off = tk >= 0 ? gbase + (size_t)tk * gstride + c * 8 : 0;
     cp_async_16(&sm.K[i][c * 8], p.K + off, tk >= 0 ? 16 : 0);
     cp_async_16(&sm.V[i][c * 8], p.V + off, tk >= 0 ? 16 : 0);
@@ -102,123 +110,147 @@ __global__ void __launch_bounds__(kThreadsR) attn_rows_kernel(const RowsParams p
   cp_async_wait<0>();
   __syncthreads();
 
-  // ---- 2a. scores: thread = (token t, rows rg, rg + 4, rg + 8, rg + 12) --------------------
-  {
-    const int t = tid & 63;   // 64 tokens per pass
-    const int rg = tid >> 6;                   // 0..3
+  // ---- 2. S = Q K^T: warp w takes tokens [16 w, 16 w + 16) (mma.sync m16n8k16, fp32) ------
+  const int gid = lane >> 2, tig = lane & 3, mi = lane >> 3;
+  float sc[2][4];  // rows gid, gid + 8; tokens 16 w + 8 nt + 2 tig + (e & 1)
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+  if (16 * warp < nt16) {
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t qa[4], k0, k1, k2, k3;
+      ldmatrix_x4(qa[0], qa[1], qa[2], qa[3], &sm.Q[(lane & 7) + 8 * (mi & 1)][ks * 16 + 8 * (mi >> 1)]);
+      ldmatrix_x4(k0, k1, k2, k3, &sm.K[16 * warp + 8 * (mi >> 1) + (lane & 7)][ks * 16 + 8 * (mi & 1)]);
+      mma_bf16_16816(sc[0], qa, k0, k1);
+      mma_bf16_16816(sc[1], qa, k2, k3);
+    }
+  }
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int t = 16 * warp + 8 * nt + 2 * tig + (e & 1);
+      sc[nt][e] = t < ntok ? sc[nt][e] * p.scale_log2 : -INFINITY;
+    }
+    mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+    mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+  }
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  if (tig == 0) {
+    sm.red_m[warp][gid] = mx0;
+    sm.red_m[warp][gid + 8] = mx1;
+  }
+  __syncthreads();
+  float M0 = -INFINITY, M1 = -INFINITY;  // the split's row maxima (log2 units)
+#pragma unroll
+  for (int w2 = 0; w2 < kThreadsR / 32; ++w2) {
+    M0 = fmaxf(M0, sm.red_m[w2][gid]);
+    M1 = fmaxf(M1, sm.red_m[w2][gid + 8]);
+  }
+  const float r0 = M0 == -INFINITY ? 0.f : M0, r1 = M1 == -INFINITY ? 0.f : M1;
+  float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const float a0 = exp2f(sc[nt][0] - r0), a1 = exp2f(sc[nt][1] - r0);
+    const float b0 = exp2f(sc[nt][2] - r1), b1 = exp2f(sc[nt][3] - r1);
+    l0 += a0 + a1;
+    l1 += b0 + b1;
+    const int t = 16 * warp + 8 * nt + 2 * tig;
+    if (t < kMaxTokR) {
+      *reinterpret_cast<uint32_t*>(&sm.P[gid][t]) = pack_bf16x2(a0, a1);
+      *reinterpret_cast<uint32_t*>(&sm.P[gid + 8][t]) = pack_bf16x2(b0, b1);
+    }
+  }
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  if (tig == 0) {
+    sm.red_l[warp][gid] = l0;
+    sm.red_l[warp][gid + 8] = l1;
+  }
+  __syncthreads();  // P and the partial row sums complete
+
+  // ---- 3. O = P V: warp w takes output columns [16 w, 16 w + 16) over all tokens ----------
+  float o[2][4];
+#pragma unroll
+  for (int nd = 0; nd < 2; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+  const bool pv = 16 * warp < D;
+  if (pv) {
 #pragma unroll 1
-    for (int tb = 0; tb < ntok; tb += 64) {
-      const int tt = tb + t;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      if (tt < ntok) {
-#pragma unroll 4
-        for (int c = 0; c < VPR; ++c) {
-          const uint4 kv = *reinterpret_cast<const uint4*>(&sm.K[tt][c * 8]);
-          float kf[8];
-          unpack_bf16x2(kv.x, kf[0], kf[1]);
-          unpack_bf16x2(kv.y, kf[2], kf[3]);
-          unpack_bf16x2(kv.z, kf[4], kf[5]);
-          unpack_bf16x2(kv.w, kf[6], kf[7]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = rg + 4 * j;
-            if (r < R) {
-              const uint4 qv = *reinterpret_cast<const uint4*>(&sm.Q[r][c * 8]);  // broadcast
-              float qf[8];
-              unpack_bf16x2(qv.x, qf[0], qf[1]);
-              unpack_bf16x2(qv.y, qf[2], qf[3]);
-              unpack_bf16x2(qv.z, qf[4], qf[5]);
-              unpack_bf16x2(qv.w, qf[6], qf[7]);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) acc[j] = fmaf(qf[e], kf[e], acc[j]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = rg + 4 * j;
-        if (r < R && tt < kMaxTokR) sm.S[r][tt] = tt < ntok ? acc[j] * p.scale_log2 : -INFINITY;
-      }
+    for (int kk = 0; kk < nt16 / 16; ++kk) {
+      uint32_t pa[4], v0, v1, v2, v3;
+      ldmatrix_x4(pa[0], pa[1], pa[2], pa[3], &sm.P[(lane & 7) + 8 * (mi & 1)][kk * 16 + 8 * (mi >> 1)]);
+      ldmatrix_x4_trans(v0, v1, v2, v3, &sm.V[kk * 16 + 8 * (mi & 1) + (lane & 7)][16 * warp + 8 * (mi >> 1)]);
+      mma_bf16_16816(o[0], pa, v0, v1);
+      mma_bf16_16816(o[1], pa, v2, v3);
     }
   }
-  __syncthreads();
-
-  // ---- 2b. row max / exponentials / sum: warp w takes rows w and w + 8 ---------------------
-  for (int r = warp; r < R; r += kThreadsR / 32) {
-    float mx = -INFINITY;
-    for (int t = lane; t < ntok; t += 32) mx = fmaxf(mx, sm.S[r][t]);
-    mx = warp_max(mx);
-    float s = 0.f;
-    for (int t = lane; t < ntok; t += 32) {
-      const float e = exp2f(sm.S[r][t] - mx);
-      sm.S[r][t] = e;
-      s += e;
-    }
-    s = warp_sum(s);
-    if (lane == 0) {
-      sm.m[r] = ntok > 0 ? mx : -INFINITY;
-      sm.l[r] = s;
-    }
-  }
-  __syncthreads();
-
-  // ---- 2c. P V: thread = (4 columns cq, rows rr and rr + 8) --------------------------------
-  constexpr int NQ = D / 4;               // column quads: 32 (D = 128) or 16 (D = 64)
-  constexpr int RPT = kThreadsR / NQ;     // row slots per pass: 8 or 16
-  const int cq = tid % NQ, rr = tid / NQ;
-  float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 4
-  for (int t = 0; t < ntok; ++t) {
-    const uint2 vv = *reinterpret_cast<const uint2*>(&sm.V[t][cq * 4]);
-    float vf[4];
-    unpack_bf16x2(vv.x, vf[0], vf[1]);
-    unpack_bf16x2(vv.y, vf[2], vf[3]);
+  float L0 = 0.f, L1 = 0.f;  // the split's row sums
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int r = rr + RPT * j;
-      if (r < R) {
-        const float pr = sm.S[r][t];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[j][e] = fmaf(pr, vf[e], o[j][e]);
-      }
-    }
+  for (int w2 = 0; w2 < kThreadsR / 32; ++w2) {
+    L0 += sm.red_l[w2][gid];
+    L1 += sm.red_l[w2][gid + 8];
   }
-
-  auto store_out = [&](int r, const float* v4, float scale) {  // O row r, columns cq * 4 ..
+  // this thread's outputs: rows gid (e < 2) and gid + 8, columns 16 w + 8 nd + 2 tig + (e & 1)
+  auto out_row = [&](int r) -> __nv_bfloat16* {
     const int l = r / p.G, h = g * p.G + r % p.G;
-    __nv_bfloat16* dst = p.O + (((size_t)l * p.B + b) * p.Hq + h) * D + cq * 4;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v4[0] * scale, v4[1] * scale),
-                                                pack_bf16x2(v4[2] * scale, v4[3] * scale));
+    return p.O + (((size_t)l * p.B + b) * p.Hq + h) * D;
   };
-  auto store_lse = [&](int r, float m2, float s) {
+  auto store_lse = [&](int r, float m2, float s2) {
     if (!p.lse) return;
     const int l = r / p.G, h = g * p.G + r % p.G;
-    p.lse[((size_t)l * p.B + b) * p.Hq + h] = s > 0.f ? (m2 + log2f(s)) * kLn2R : -INFINITY;
+    p.lse[((size_t)l * p.B + b) * p.Hq + h] = s2 > 0.f ? (m2 + log2f(s2)) * kLn2R : -INFINITY;
   };
 
   if (p.nsplit == 1) {  // the CTA holds the whole selection: final rows
+    if (pv) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int r = rr + RPT * j;
-      if (r < R) store_out(r, o[j], sm.l[r] > 0.f ? 1.f / sm.l[r] : 0.f);
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = gid + 8 * hf;
+        if (r >= R) continue;
+        const float Ls = hf ? L1 : L0;
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        __nv_bfloat16* dst = out_row(r);
+#pragma unroll
+        for (int nd = 0; nd < 2; ++nd)
+          *reinterpret_cast<uint32_t*>(dst + 16 * warp + 8 * nd + 2 * tig) =
+              pack_bf16x2(o[nd][2 * hf] * inv, o[nd][2 * hf + 1] * inv);
+      }
     }
-    if (tid < R) store_lse(tid, sm.m[tid], sm.l[tid]);
+    if (warp == 0 && tig == 0) {
+      if (gid < R) store_lse(gid, M0, L0);
+      if (gid + 8 < R) store_lse(gid + 8, M1, L1);
+    }
     return;
   }
 
-  // ---- 3. split partials, then the last CTA of (b, g) merges -------------------------------
+  // ---- 4. split partials, then the last CTA of (b, g) merges -------------------------------
   const size_t ub = ((size_t)b * p.Hkv + g) * p.nsplit;  // this (b, g)'s first split
+  if (pv) {
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int r = rr + RPT * j;
-    if (r < R)
-      __stcg(reinterpret_cast<float4*>(p.Op + ((ub + split) * R + r) * D + cq * 4),
-             make_float4(o[j][0], o[j][1], o[j][2], o[j][3]));
+    for (int hf = 0; hf < 2; ++hf) {
+      const int r = gid + 8 * hf;
+      if (r >= R) continue;
+      float* dst = p.Op + ((ub + split) * R + r) * D + 16 * warp + 2 * tig;
+#pragma unroll
+      for (int nd = 0; nd < 2; ++nd) __stcg(reinterpret_cast<float2*>(dst + 8 * nd), make_float2(o[nd][2 * hf], o[nd][2 * hf + 1]));
+    }
   }
-  if (tid < R) {
-    __stcg(p.Mp + (ub + split) * R + tid, sm.m[tid]);
-    __stcg(p.Lp + (ub + split) * R + tid, sm.l[tid]);
+  if (warp == 0 && tig == 0) {
+    const float mm0 = ntok > 0 ? M0 : -INFINITY, mm1 = ntok > 0 ? M1 : -INFINITY;
+    if (gid < R) {
+      __stcg(p.Mp + (ub + split) * R + gid, mm0);
+      __stcg(p.Lp + (ub + split) * R + gid, L0);
+    }
+    if (gid + 8 < R) {
+      __stcg(p.Mp + (ub + split) * R + gid + 8, mm1);
+      __stcg(p.Lp + (ub + split) * R + gid + 8, L1);
+    }
   }
   __threadfence();  // this thread's partial stores are visible at GPU scope ...
   __syncthreads();  // ... for every thread of the CTA before the arrival
@@ -229,6 +261,13 @@ __global__ void __launch_bounds__(kThreadsR) attn_rows_kernel(const RowsParams p
   __syncthreads();
   if (!sm.last) return;
   __threadfence();  // the other splits' partials, published before their arrivals
+  constexpr int NQ = D / 4;            // column quads: 32 (D = 128) or 16 (D = 64)
+  constexpr int RPT = kThreadsR / NQ;  // row slots per pass: 8 or 16
+  const int cq = tid % NQ, rr = tid / NQ;
+  auto store_out = [&](int r, const float* v4, float scale) {  // O row r, columns cq * 4 ..
+    *reinterpret_cast<uint2*>(out_row(r) + cq * 4) = make_uint2(pack_bf16x2(v4[0] * scale, v4[1] * scale),
+                                                                pack_bf16x2(v4[2] * scale, v4[3] * scale));
+  };
 
   // merge weights: M_r = max_s m_s, w_s = 2^(m_s - M_r), den_r = sum_s w_s l_s.  Warp r takes
   // row r: lane s holds splits s and s + 32 (one round trip for every split's max and sum)
@@ -298,7 +337,9 @@ bool sparse_attn_rows_plan(const AttnShape& sh, int sm_count, AttnPlan* pl) {
   const int G = sh.Hq / sh.Hkv;
   if (sh.L * G > kMaxRowsR) return false;
   const long long units = (long long)sh.B * sh.Hkv;
-  const long long target = 2LL * std::max(sm_count, 1);
+  // about one CTA per SM: splits of up to 128 tokens (fewer splits to merge beat more CTAs
+  // in flight: 7.7 vs 9.2 us per one-layer call at 128K)
+  const long long target = std::max(sm_count, 1);
   const int ns0 = (int)std::max(1LL, (target + units - 1) / units);
   int chunk = (sh.k + ns0 - 1) / ns0;
   chunk = std::min(kMaxTokR, (chunk + 63) / 64 * 64);

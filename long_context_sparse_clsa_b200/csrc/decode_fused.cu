@@ -340,13 +340,20 @@ __device__ void make_plan(const FusedParams& p, Plan& pl, uint32_t* live) {
   }
   pl.b = -1;
   if (nb == 0) return;
-  const int spare = ncta - nb;
+  // A sequence's CTAs scan its slice (work in proportion to its length) and then attend: Hkv
+  // head units of k_eff tokens whatever its length.  With fewer than Hkv CTAs a CTA runs
+  // several head units one after the other, so with several sequences each gets Hkv CTAs
+  // first (when the grid has them) and the rest in proportion to its length; a lone sequence
+  // takes the whole grid.
+  const bool grouped = nb >= 2 && ncta >= p.Hkv * nb;
+  const int base = grouped ? p.Hkv : 1;
+  const int spare = ncta - base * nb;
   int start = 0;
 #pragma unroll 1
   for (int b = 0; b < p.B; ++b) {
     const int len = max(0, min(p.seq_lens[b], p.n_max));
     if (len == 0) continue;
-    const int Cb = 1 + (int)((long long)spare * len / total);
+    const int Cb = base + (int)((long long)spare * len / total);
     if ((int)blockIdx.x < start + Cb) {
       pl.b = b;
       pl.start = start;

@@ -538,13 +538,16 @@ AttnPlan plan_attention(const AttnShape& sh) {
   return pl;
 }
 
+size_t attn_counter_bytes(const AttnShape& sh) { return align_up((size_t)sh.B * sh.Hkv * sizeof(uint32_t), 256); }
+
 size_t attn_ws_bytes(const AttnShape& sh) {
   const AttnPlan pl = plan_attention(sh);
   if (pl.nsplit == 1) return 0;
   const size_t n = (size_t)sh.B * sh.Hkv * pl.nlg * pl.nsplit * pl.rows;
-  // split partials (output, max, sum), then one arrival counter per (b, KV head, layer group)
-  return align_up(n * sh.d * sizeof(float), 256) + 2 * align_up(n * sizeof(float), 256) +
-         align_up((size_t)sh.B * sh.Hkv * pl.nlg * sizeof(uint32_t), 256);
+  // one arrival counter per (b, KV head) first, at an offset no plan changes (so calls of other
+  // shapes on the same workspace never write over them), then the split partials (output, max,
+  // sum)
+  return attn_counter_bytes(sh) + align_up(n * sh.d * sizeof(float), 256) + 2 * align_up(n * sizeof(float), 256);
 }
 
 cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* Kc, const void* Vc,
@@ -578,13 +581,13 @@ cudaError_t launch_sparse_attn(const AttnShape& sh, const void* Q, const void* K
   if (pl.nsplit > 1) {
     const size_t n = (size_t)sh.B * sh.Hkv * pl.nlg * pl.nsplit * pl.rows;
     char* w = static_cast<char*>(attn_ws);
+    counter = reinterpret_cast<uint32_t*>(w);
+    w += attn_counter_bytes(sh);
     p.Op = reinterpret_cast<float*>(w);
     w += align_up(n * sh.d * sizeof(float), 256);
     p.Mp = reinterpret_cast<float*>(w);
     w += align_up(n * sizeof(float), 256);
     p.Lp = reinterpret_cast<float*>(w);
-    w += align_up(n * sizeof(float), 256);
-    counter = reinterpret_cast<uint32_t*>(w);
   }
   AttnPlan rp{};
   if (sparse_attn_rows_plan(sh, device_info().sm_count, &rp) && aligned16_(Q) && aligned16_(Kc) && aligned16_(Vc) &&

@@ -182,6 +182,33 @@ def test_sparse_attn_full_size(layers):
         assert max_abs(got_lse[lq], want_lse[0]) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse).max()), l
 
 
+def test_sparse_attn_workspace_reuse_is_clean():
+    """One workspace through per-layer calls (the in-kernel split merge and its arrival
+    counters), an all-layer call (split partials and the combine) and per-layer calls again:
+    every repeat is bit-identical to the first, so each call left the workspace clean."""
+    w = CASES["d32k_small"]
+    inp, dv = _inputs("d32k_small")
+    sc = clsa.index_scores(dv["q_idx"], dv["k_idx"], dv["seq_lens"])
+    idx, cnt = clsa.topk(sc, dv["seq_lens"], w.k)
+    KS, VS = clsa.gather_kv(dv["K"], dv["V"], idx, cnt)
+    Qall = torch.cat([dv["Q"]] * 8)  # 24 layers: 96 rows per KV head, the tensor-core kernel
+    lib = clsa.load_library()
+    ws = clsa.Workspace(max(lib.clsa_sparse_attn_workspace_size(w.B, w.k, L, w.Hq, w.Hkv, w.d) for L in (1, 24)))
+    outs = []
+    for Q in (dv["Q"][:1], Qall, dv["Q"][:1], Qall, dv["Q"][1:2]):
+        o, l = clsa.sparse_attn(Q.contiguous(), KS, VS, cnt, ws=ws)
+        outs.append((o.clone(), l.clone()))
+    torch.cuda.synchronize()
+    assert ws.status()[0] == "CLSA_OK"
+    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+    assert torch.equal(outs[1][0], outs[3][0]) and torch.equal(outs[1][1], outs[3][1])
+    # layer 1 alone equals layer 1 of the all-layer call, against the oracle too
+    i_np, c_np = idx.cpu().numpy(), cnt.cpu().numpy()
+    want, _ = O.sparse_attention(inp.Q[1:2], inp.K, inp.V, i_np, c_np)
+    assert max_abs(tensor_f64(outs[4][0][0]), want[0]) <= TOL[w.dtype]
+    assert max_abs(tensor_f64(outs[1][0][1]), want[0]) <= TOL[w.dtype]
+
+
 @pytest.mark.parametrize("dtype,L", [("bf16", 3), ("bf16", 6), ("f32", 3)])
 def test_sparse_attn_growing_scores(dtype, L):
     """Scores that grow along the selection by far more than 2^8 per 64-token chunk: the
