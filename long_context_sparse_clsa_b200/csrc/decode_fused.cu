@@ -1097,9 +1097,6 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
   stamp(p, 35);
   const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
   const bool live = q4 * 32 < p.rows;  // warp-uniform: rows of this lane quarter exist
-  float o[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) o[j] = 0.f;
   float m = -INFINITY, lp = 0.f;
   bool dead = false;
   // S = Q K_c^T into TMEM columns [TOK (c & 1), +TOK); issued by thread 0
@@ -1140,39 +1137,28 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
     }
     if (c == 0) stamp(p, 36);
     tc::fence_after_sync();
-    // the scores are read from TMEM twice (for the row max, then for P) rather than held
-    // across the exchange: registers stay within budget for 32 columns
     const uint32_t ts = tl + (uint32_t)(TOK * (c & 1) + NPT * cg);
     const int t0 = c * TOK + NPT * cg;
     const int nv = ntok - t0;  // valid columns of this thread (may be <= 0 or > NPT)
+    uint32_t v[NPT];           // the scores, held until P is final
+    float lmx = -INFINITY;     // this thread's max of its columns (log2 units)
     if (live) {
-      uint32_t v[NPT];
-      float cmx = -INFINITY;
       if (!dead) {
         tmem_ld_row<NPT>(ts, v);
         tc::ld_wait();
+        float cmx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < NPT; ++j)
           if (j < nv) cmx = fmaxf(cmx, __uint_as_float(v[j]));
-      }
-      sm.cm[cg * kMaxRows + row] = cmx * p.scale_log2;  // scale > 0: the max commutes
-    }
-    __syncthreads();
-    if (c == 0) stamp(p, 37);
-    float alpha = 1.f;
-    if (live) {
-      const float mn = fmaxf(fmaxf(m, fmaxf(sm.cm[row], sm.cm[kMaxRows + row])),
-                             fmaxf(sm.cm[2 * kMaxRows + row], sm.cm[3 * kMaxRows + row]));
-      alpha = fast_exp2(m - mn);  // m = -inf on the first chunk: 0
-      m = mn;
-      uint32_t v[NPT];
-      if (!dead) {
-        tmem_ld_row<NPT>(ts, v);
-        tc::ld_wait();
+        lmx = cmx * p.scale_log2;  // scale > 0: the max commutes
       } else {
 #pragma unroll
         for (int j = 0; j < NPT; ++j) v[j] = 0xff800000u;  // -inf: P = 0
       }
+    }
+    // P of this thread's columns against the row's reference max m, into shared memory; the
+    // sum of those columns is returned
+    auto write_p = [&]() -> float {
       float rs = 0.f;
 #pragma unroll
       for (int q = 0; q < NPT / 8; ++q) {  // 8 tokens = one 16-byte chunk of the P row
@@ -1180,8 +1166,8 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int j0 = 8 * q + 2 * j;
-          const float a = j0 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -mn)) : 0.f;
-          const float e = j0 + 1 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -mn)) : 0.f;
+          const float a = j0 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -m)) : 0.f;
+          const float e = j0 + 1 < nv ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -m)) : 0.f;
           rs += a + e;
           pw[j] = pack_bf16x2(a, e);
         }
@@ -1189,20 +1175,62 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
         *reinterpret_cast<uint4*>(sP + (ch >> 3) * SH::kPAtom + tc::sw128_offset(row, ch & 7)) =
             make_uint4(pw[0], pw[1], pw[2], pw[3]);
       }
-      lp = lp * alpha + rs;
-    }
+      return rs;
+    };
+    // The output accumulates in TMEM (P V with accumulate).  P is taken against a reference max
+    // m that moves only when a column exceeds it by more than 2^kTau: then the row's TMEM output
+    // and sum are scaled by 2^(m_old - m_new) once.  In the common case a thread writes its P at
+    // once; the first chunk, or a column above the bound anywhere in the CTA, takes the row-max
+    // exchange (voted on the barrier that precedes the MMA issue anyway), after which the
+    // threads of a row whose max moved rewrite their P.
+    constexpr float kTau = 8.f;
+    const bool need = live && (c == 0 || lmx > m + kTau);
+    float rs = 0.f;
+    if (live && !need) rs = write_p();
     if (SH::kStages == 3 && c + 1 < nch) cp_async_wait<1>();  // chunk c + 1 landed (c + 2 may be in flight)
     fence_proxy_async_smem();
     tc::fence_before_sync();
-    __syncthreads();
+    if (__syncthreads_or(need)) {
+      if (live) sm.cm[cg * kMaxRows + row] = lmx;
+      __syncthreads();
+      if (c == 0) stamp(p, 37);
+      if (live) {
+        const float mn = fmaxf(fmaxf(sm.cm[row], sm.cm[kMaxRows + row]),
+                               fmaxf(sm.cm[2 * kMaxRows + row], sm.cm[3 * kMaxRows + row]));
+        const bool up = c == 0 || mn > m + kTau;  // the same in the four threads of the row
+        if (c > 0 && __any_sync(0xffffffffu, up)) {
+          // TMEM load / store are .sync.aligned: every lane of the warp (alpha = 1 if not up);
+          // P V of the previous chunk has completed (waited below)
+          const float alpha = up ? fast_exp2(m - mn) : 1.f;
+          if (!dead) {
+            uint32_t w[32];
+            tc::ld_32x32b_x32(tl + 128u + (uint32_t)(32 * cg), w);
+            tc::ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(__uint_as_float(w[j]) * alpha);
+            tc::st_32x32b_x32(tl + 128u + (uint32_t)(32 * cg), w);
+            tc::st_wait();
+          }
+          if (up) lp *= alpha;
+        }
+        if (up) {
+          m = mn;
+          rs = write_p();
+        }
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      __syncthreads();
+    }
+    lp += rs;
     if (c == 0) stamp(p, 38);
     if (threadIdx.x == 0) {
-      // O_c = P_c V_c, then S of the next chunk into the other S buffer
+      // O += P_c V_c, then S of the next chunk into the other S buffer
       tc::fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < TOK / 16; ++ks)
         tc::mma_bf16(tmem + 128u, tc::sw128_desc(smem_u32(sP) + (ks >> 2) * SH::kPAtom + (ks & 3) * 32),
-                     tc::sw128_desc_mn(smem_u32(sV) + ks * 16 * 128, SH::kKVAtom), kIdescPV, ks > 0);
+                     tc::sw128_desc_mn(smem_u32(sV) + ks * 16 * 128, SH::kKVAtom), kIdescPV, c > 0 || ks > 0);
       tc::mma_commit(&sm.bar_o);
       if (c + 1 < nch) issue_qk(c + 1);
     }
@@ -1212,16 +1240,20 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
     }
     if (c == 0) stamp(p, 39);
     tc::fence_after_sync();
-    if (live && !dead) {
-      uint32_t v[32];
-      tc::ld_32x32b_x32(tl + 128u + (uint32_t)(32 * cg), v);
-      tc::ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) o[j] = fmaf(o[j], alpha, __uint_as_float(v[j]));
-    }
-    tc::fence_before_sync();  // O_c is read before the next chunk's P barrier lets P V overwrite it
     ++it;
   }
+  // the unit's output rows from TMEM (every lane of a live warp: the load is .sync.aligned)
+  float o[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) o[j] = 0.f;
+  if (live && !dead && nch > 0) {
+    uint32_t w[32];
+    tc::ld_32x32b_x32(tl + 128u + (uint32_t)(32 * cg), w);
+    tc::ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(w[j]);
+  }
+  tc::fence_before_sync();  // the TMEM output is read before the next unit's first P V overwrites it
   cp_async_wait<0>();  // no copy of this unit outlives it (the trailing groups are empty)
   stamp(p, 11);
 

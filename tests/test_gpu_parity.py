@@ -34,6 +34,9 @@ CASES = {
     "tiny": WORKLOADS["tiny"],
     "d32k_small": scaled("decode32k", n_max=8192 + 77, k=512, L=3),
     "ragged_small": scaled("ragged16", B=5, n_max=6000, lens=(0, 6000), k=700, L=2, seed=3),
+    # more sequences than the grid has groups of Hkv CTAs for: the fused step's proportional
+    # split, where a CTA attends several head units one after the other
+    "ragged_b24": scaled("ragged16", B=24, n_max=3000, lens=(1, 3000), k=300, L=2, seed=4),
     "bf16_d64": scaled("decode32k", n_max=3000, d_idx=64, d=64, k=300, L=2, Hq=8, Hkv=2, plant=0.0),
     "f32_d128": scaled("tiny", n_max=2500, d_idx=128, d=128, k=333, L=2, Hq=6, Hkv=3, seed=5),
 }
