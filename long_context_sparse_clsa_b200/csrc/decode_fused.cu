@@ -342,18 +342,45 @@ __device__ void make_plan(const FusedParams& p, Plan& pl, uint32_t* live) {
   if (nb == 0) return;
   // A sequence's CTAs scan its slice (work in proportion to its length) and then attend: Hkv
   // head units of k_eff tokens whatever its length.  With fewer than Hkv CTAs a CTA runs
-  // several head units one after the other, so with several sequences each gets Hkv CTAs
-  // first (when the grid has them) and the rest in proportion to its length; a lone sequence
-  // takes the whole grid.
+  // several head units one after the other.  So with several sequences (when the grid has
+  // Hkv CTAs for each) a sequence whose length share of the grid falls below Hkv CTAs is
+  // pinned at Hkv, and the others share the remaining CTAs in proportion to their lengths
+  // (re-split while new sequences pin: each pass pins one or more, or stops); then every
+  // unpinned share is at least Hkv.  Otherwise CTAs go one per sequence plus the rest in
+  // proportion to length; a lone sequence takes the whole grid.
   const bool grouped = nb >= 2 && ncta >= p.Hkv * nb;
-  const int base = grouped ? p.Hkv : 1;
-  const int spare = ncta - base * nb;
+  uint64_t pin0 = 0u, pin1 = 0u;  // pinned sequences (bit b of pin0, or b - 64 of pin1)
+  auto pinned = [&](int b) { return ((b < 64 ? pin0 >> b : pin1 >> (b - 64)) & 1u) != 0u; };
+  long long tot2 = total;  // length of the unpinned sequences
+  int rem = ncta;          // CTAs they share
+  if (grouped) {
+#pragma unroll 1
+    for (int round = 0; round < nb; ++round) {
+      bool changed = false;
+#pragma unroll 1
+      for (int b = 0; b < p.B; ++b) {
+        const int len = max(0, min(p.seq_lens[b], p.n_max));
+        if (len == 0 || pinned(b)) continue;
+        if ((long long)rem * len < (long long)p.Hkv * tot2) {
+          if (b < 64) pin0 |= 1ull << b;
+          else pin1 |= 1ull << (b - 64);
+          rem -= p.Hkv;
+          tot2 -= len;
+          changed = true;
+        }
+      }
+      if (!changed) break;
+    }
+  }
+  const int spare = ncta - nb;
   int start = 0;
 #pragma unroll 1
   for (int b = 0; b < p.B; ++b) {
     const int len = max(0, min(p.seq_lens[b], p.n_max));
     if (len == 0) continue;
-    const int Cb = base + (int)((long long)spare * len / total);
+    const int Cb = !grouped ? 1 + (int)((long long)spare * len / total)
+                   : pinned(b) ? p.Hkv
+                                                      : (int)((long long)rem * len / tot2);
     if ((int)blockIdx.x < start + Cb) {
       pl.b = b;
       pl.start = start;
