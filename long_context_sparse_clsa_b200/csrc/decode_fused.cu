@@ -1104,7 +1104,7 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&v)[N]) {
 // only for a unit of at most 128 tokens (one chunk).
 template <int TOK>
 __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, unsigned char* kv, int g, int ntok,
-                            bool q_loaded, uint32_t tmem, uint32_t& it) {
+                            bool q_loaded, bool kv0_issued, uint32_t tmem, uint32_t& it) {
   using SH = AttnShape<TOK>;
   constexpr int NPT = SH::kPerThread;
   const Plan pl = sm.plan;  // a copy: loops below store to shared memory
@@ -1117,6 +1117,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
   const int nch = (ntok + TOK - 1) / TOK;
 #pragma unroll 1
   for (int c = 0; c < 2; ++c) {
+    if (c == 0 && kv0_issued) continue;  // the caller issued chunk 0 as its own group
     if (c < nch && c < SH::kStages)
       load_kv_chunk<TOK>(p, sm, b, g, pl.len, c, ntok, kv + c * 2 * SH::kKVTile, kv + c * 2 * SH::kKVTile + SH::kKVTile);
     cp_async_commit();
@@ -1378,12 +1379,13 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
       dead = true;
       continue;
     }
+    // the rows' async copies first: the (m, l) loads below stall the warp until they return
+    if (s2 < sb) issue_rows(s2, 0);
     for (int ri = lane; ri < nr; ri += 32) {
       const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
       sm.cm[ri * ns + s2] = ml.x;
       sm.cl[ri * ns + s2] = ml.y;
     }
-    if (s2 < sb) issue_rows(s2, 0);
   }
   cp_async_commit();
   if (dead) sm.abort_flag = 1;
@@ -1586,6 +1588,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
   // ---- attention units (TMEM held only for this phase: no return path in between)
   if (pl.nunits_here > 0) {
     const int ntok = pl.tok1 - pl.tok0;
+    unsigned char* kv = align1024(big);  // the windows are dead past the ranking
+    // the first unit's first K/V chunk goes out now, so that its gather overlaps the TMEM
+    // allocation and the barrier below (attend_unit then skips it)
+    if (ntok > 0) {
+      if (ntok <= 128) load_kv_chunk<128>(p, sm, pl.b, pl.unit_g0, pl.len, 0, ntok, kv, kv + AttnShape<128>::kKVTile);
+      else load_kv_chunk<64>(p, sm, pl.b, pl.unit_g0, pl.len, 0, ntok, kv, kv + AttnShape<64>::kKVTile);
+    }
+    cp_async_commit();
     if (threadIdx.x < 32) {
       tc::tmem_alloc(&sm.tmem_base, kTmemCols);
       tc::tmem_relinquish();
@@ -1599,12 +1609,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const FusedPa
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
-    unsigned char* kv = align1024(big);
     uint32_t it = 0;
     for (int u = 0; u < pl.nunits_here; ++u) {
       const int g = pl.unit_g0 + u * pl.unit_step;
-      if (ntok <= 128) attend_unit<128>(p, sm, sQa, kv, g, ntok, u == 0, tmem, it);
-      else attend_unit<64>(p, sm, sQa, kv, g, ntok, u == 0, tmem, it);
+      if (ntok <= 128) attend_unit<128>(p, sm, sQa, kv, g, ntok, u == 0, u == 0, tmem, it);
+      else attend_unit<64>(p, sm, sQa, kv, g, ntok, u == 0, u == 0, tmem, it);
     }
     tc::fence_before_sync();
     __syncthreads();
