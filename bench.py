@@ -796,6 +796,18 @@ def run_prefill(args):
             chunk()
             torch.cuda.synchronize()
             per_launch.append(timer.times_ms())
+        # the attention stage alone on the chunk's selection: per row (mode 0, the chunk's own)
+        # and key-centric row pairs over the union of their selections (mode 1)
+        attn_modes = {}
+        for mode in (0, 1):
+            ts = []
+            for _ in range(4):
+                timer.arm()
+                clsa._check(lib.clsa_prefill_attention(ctypes.byref(a), mode, ws.ptr, ws.nbytes, clsa._stream()),
+                            "clsa_prefill_attention")
+                torch.cuda.synchronize()
+                ts.append(timer.times_ms()[0])
+            attn_modes["per_row" if mode == 0 else "key_centric_pairs"] = statistics.median(ts[1:])
     st = ws.status()
     if st[0] != "CLSA_OK":
         raise RuntimeError(f"device error during timing: {st}")
@@ -824,7 +836,8 @@ def run_prefill(args):
                      "useful_flops_per_launch": useful, "us_per_launch": route_ms * 1e3},
         "launch_ms_median": [statistics.median(x) for x in zip(*per_launch)],
         "attention": {"kernel": "last launch of the chunk", "ms": attn_ms,
-                      "useful_tflops": attn_flops / (attn_ms * 1e-3) / 1e12},
+                      "useful_tflops": attn_flops / (attn_ms * 1e-3) / 1e12,
+                      "stage_alone_ms": attn_modes},
         "gpu_launches": launches * steps,
         "clocks": clk.summary(),
     }

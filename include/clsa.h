@@ -240,6 +240,19 @@ typedef struct clsa_prefill_args {
 CLSA_API size_t clsa_prefill_workspace_size(const clsa_prefill_args* a);
 CLSA_API clsa_status clsa_prefill_chunk(const clsa_prefill_args* a, void* ws, size_t ws_bytes, void* stream);
 
+/* The attention stage of a prefill chunk alone: the per-layer equation for every new row
+ * over the selection already in a->idx / a->count (as clsa_prefill_chunk writes them:
+ * ascending token order per row), writing a->O and a->lse.  q_idx and k_idx are not read.
+ * mode 0: each row on its own (what clsa_prefill_chunk runs).
+ * mode 1: key-centric.  Rows go in pairs (t, t + 1); a pair fetches each K/V row of the
+ *   union of its two selections once and scores it against both rows' queries, each row
+ *   keeping only the tokens it selected (an implementation choice, not on the pages; the
+ *   results equal mode 0's up to the fp32 summation order).  bf16, d = 128, k <= 4096;
+ *   other shapes return CLSA_ERR_UNSUPPORTED.
+ * Workspace: clsa_prefill_workspace_size(a) bytes, zeroed as usual; errors as above. */
+CLSA_API clsa_status clsa_prefill_attention(const clsa_prefill_args* a, int mode, void* ws, size_t ws_bytes,
+                                            void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Helpers                                                                    */
 /* ------------------------------------------------------------------------ */

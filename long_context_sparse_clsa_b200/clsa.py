@@ -29,7 +29,7 @@ EXPORTS = [
     "clsa_distill_workspace_size", "clsa_distill_target", "clsa_attention_mass_workspace_size",
     "clsa_attention_mass",
     "clsa_decode_workspace_size", "clsa_decode_step", "clsa_prefill_workspace_size",
-    "clsa_prefill_chunk", "clsa_workspace_size", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
+    "clsa_prefill_chunk", "clsa_prefill_attention", "clsa_workspace_size", "clsa_workspace_init", "clsa_read_device_status", "clsa_status_string",
     "clsa_selftest_timeout", "clsa_version", "clsa_last_launch_count", "clsa_time_next_call",
     "clsa_timed_event_count",
 ]
@@ -91,6 +91,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "clsa_decode_step": (S, [ctypes.POINTER(DecodeArgs), _vp, _sz, _vp]),
         "clsa_prefill_workspace_size": (_sz, [ctypes.POINTER(PrefillArgs)]),
         "clsa_prefill_chunk": (S, [ctypes.POINTER(PrefillArgs), _vp, _sz, _vp]),
+        "clsa_prefill_attention": (S, [ctypes.POINTER(PrefillArgs), _i, _vp, _sz, _vp]),
         "clsa_workspace_size": (_sz, [_i, _vp]),
         "clsa_workspace_init": (S, [_vp, _sz, _vp]),
         "clsa_read_device_status": (S, [_vp, _vp, ctypes.POINTER(ctypes.c_int64)]),
@@ -385,6 +386,23 @@ def prefill_chunk(q_idx, k_idx, K, V, Q, k, scale: float = 0.0, ws: Optional[Wor
            "clsa_prefill_chunk")
     out["ws"] = ws
     return out
+
+
+def prefill_attention(q_idx, k_idx, K, V, Q, k, idx, count, mode: int = 0, scale: float = 0.0,
+                      ws: Optional[Workspace] = None, O=None, lse=None, want_lse: bool = True):
+    """The attention stage of a prefill chunk over a selection already in idx / count (as
+    prefill_chunk returns it).  mode 0: per row; mode 1: key-centric row pairs."""
+    T = q_idx.shape[0]
+    L, _, Hq, d = Q.shape
+    O = O if O is not None else torch.empty_like(Q)
+    if want_lse and lse is None:
+        lse = torch.empty(L, T, Hq, dtype=torch.float32, device=K.device)
+    a = prefill_args(q_idx, k_idx, K, V, Q, k, O, idx, count, lse, scale)
+    need = prefill_workspace_size(a)
+    ws = (ws or Workspace(need)).ensure(need)
+    _check(load_library().clsa_prefill_attention(ctypes.byref(a), int(mode), ws.ptr, ws.nbytes, _stream()),
+           "clsa_prefill_attention")
+    return O, lse
 
 
 def to_device(inp, device="cuda"):

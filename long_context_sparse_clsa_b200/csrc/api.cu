@@ -394,4 +394,23 @@ clsa_status clsa_prefill_chunk(const clsa_prefill_args* a, void* ws, size_t ws_b
   return run_prefill(a, w, w + kWsHeader, static_cast<cudaStream_t>(stream));
 }
 
+clsa_status clsa_prefill_attention(const clsa_prefill_args* a, int mode, void* ws, size_t ws_bytes, void* stream) {
+  CallScope scope(stream);
+  if (!a || (mode != 0 && mode != 1)) return CLSA_ERR_INVALID_ARG;
+  clsa_status st = check_attn(a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype);
+  if (st != CLSA_OK) return st;
+  if (a->dtype != CLSA_BF16) return CLSA_ERR_UNSUPPORTED;
+  if (a->n < 1 || a->T < 1 || a->T > a->n) return CLSA_ERR_INVALID_ARG;
+  if (!dims_ok(a->d_idx)) return CLSA_ERR_UNSUPPORTED;
+  if (!a->K || !a->V || !a->Q || !a->O || !a->idx || !a->count) return CLSA_ERR_INVALID_ARG;
+  for (const void* p : {a->K, a->V, a->Q, (const void*)a->O})
+    if (!aligned16(p)) return CLSA_ERR_INVALID_ARG;
+  if (!aligned4(a->idx) || !aligned4(a->count) || (a->lse && !aligned4(a->lse))) return CLSA_ERR_INVALID_ARG;
+  if (mode == 1 && !prefill_attn_pair_supported(a)) return CLSA_ERR_UNSUPPORTED;
+  const size_t need = clsa_prefill_workspace_size(a);
+  if (!ws || need == 0 || ws_bytes < need || !aligned16(ws)) return CLSA_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  return run_prefill_attention(a, mode, w, w + kWsHeader, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -133,7 +133,13 @@ cudaError_t launch_prefill_route(const clsa_prefill_args* a, void* ws_header, vo
 // per-row sparse attention of a prefill chunk on tcgen05 (bf16, d = 128); else the split-k kernel
 bool prefill_attn_tc_supported(const clsa_prefill_args* a);
 cudaError_t launch_prefill_attn_tc(const clsa_prefill_args* a, float scale, void* ws_header, cudaStream_t s);
+// key-centric prefill attention: pairs of new rows over the union of their selections (tcgen05)
+bool prefill_attn_pair_supported(const clsa_prefill_args* a);
+cudaError_t launch_prefill_attn_pair(const clsa_prefill_args* a, float scale, void* ws_header, cudaStream_t s);
 size_t prefill_ws_bytes(const clsa_prefill_args* a);
 clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_body, cudaStream_t s);
+// the attention stage alone over a->idx / a->count: mode 0 per row, mode 1 key-centric row pairs
+clsa_status run_prefill_attention(const clsa_prefill_args* a, int mode, void* ws_header, void* ws_body,
+                                  cudaStream_t s);
 
 }  // namespace clsa

@@ -208,8 +208,19 @@ clsa_status run_prefill(const clsa_prefill_args* a, void* ws_header, void* ws_bo
     e = launch_topk(scores, nullptr, a->T, a->n, a->k, a->idx, a->count, ws_header, w + lay.topk, s, a->n - a->T);
     if (e != cudaSuccess) return CLSA_ERR_CUDA;
   }
+  return run_prefill_attention(a, 0, ws_header, ws_body, s);
+}
+
+clsa_status run_prefill_attention(const clsa_prefill_args* a, int mode, void* ws_header, void* ws_body,
+                                  cudaStream_t s) {
+  const PrefillLayout lay = prefill_layout(a);
+  char* w = static_cast<char*>(ws_body);
   const float scale = a->scale > 0.f ? a->scale : 1.0f / sqrtf((float)a->d);
-  if (prefill_attn_tc_supported(a)) {
+  cudaError_t e;
+  if (mode == 1) {
+    if (!prefill_attn_pair_supported(a)) return CLSA_ERR_UNSUPPORTED;
+    e = launch_prefill_attn_pair(a, scale, ws_header, s);
+  } else if (prefill_attn_tc_supported(a)) {
     e = launch_prefill_attn_tc(a, scale, ws_header, s);
   } else {
     AttnShape sh{a->T, a->k, a->L, a->Hq, a->Hkv, a->d, a->dtype, true, a->n, 0};

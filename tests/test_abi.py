@@ -93,6 +93,16 @@ def test_prefill_rejects_bad_args(lib):
     assert lib.clsa_prefill_chunk(ctypes.byref(a), p, 1 << 30, NULL) == 2   # fp32 prefill unsupported
 
 
+def test_prefill_attention_rejects_bad_args(lib):
+    p = ctypes.c_void_p(16)
+    a = clsa.PrefillArgs(1, 100, 50, 128, 16, 1, 8, 2, 64, 0.0, p, p, p, p, p, p, p, p, NULL)
+    assert lib.clsa_prefill_attention(None, 0, p, 1 << 30, NULL) == 1
+    assert lib.clsa_prefill_attention(ctypes.byref(a), 2, p, 1 << 30, NULL) == 1    # no mode 2
+    assert lib.clsa_prefill_attention(ctypes.byref(a), 1, p, 1 << 30, NULL) == 2    # key-centric: d = 128 only
+    a.T = 200                                                                         # T > n
+    assert lib.clsa_prefill_attention(ctypes.byref(a), 0, p, 1 << 30, NULL) == 1
+
+
 def test_oracle_is_not_imported_by_the_product():
     pkg = os.path.join(ROOT, "long_context_sparse_clsa_b200")
     for dirpath, _, files in os.walk(pkg):

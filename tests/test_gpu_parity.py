@@ -371,6 +371,38 @@ def test_prefill_full_size_sampled():
     _prefill_check(w, [0, 1, 2047, 2048, 4095])
 
 
+@pytest.mark.parametrize("name,kw,rows", [
+    ("prefill4k_corr", dict(n_max=3000, T=301, k=256, L=2), None),    # correlated rows: a small union; odd T
+    ("prefill4k", dict(n_max=3000, T=300, k=256, L=2), None),         # independent rows: a large union
+    # k_eff = 1 .. k: pairs of unequal sizes
+    ("prefill4k", dict(n_max=700, T=700, k=300, L=5), [0, 1, 2, 62, 63, 64, 65, 127, 128, 299, 300, 511, 698, 699]),
+    # two layer groups
+    ("prefill4k_corr", dict(n_max=1500, T=200, k=160, L=45, Hq=16, Hkv=4), list(range(0, 200, 7)) + [199]),
+])
+def test_prefill_attention_key_centric(name, kw, rows):
+    """clsa_prefill_attention mode 1 (row pairs over the union of their selections) on the
+    selection clsa_prefill_chunk made: every row against the oracle's per-row attention, and
+    against mode 0 on the same selection."""
+    w = scaled(name, **kw)
+    inp = make_inputs(w)
+    dv = clsa.to_device(inp)
+    r = clsa.prefill_chunk(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], w.k)
+    o1, l1 = clsa.prefill_attention(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], w.k, r["idx"], r["count"],
+                                    mode=1)
+    o0, l0 = clsa.prefill_attention(dv["q_idx"], dv["k_idx"], dv["K"], dv["V"], dv["Q"], w.k, r["idx"], r["count"],
+                                    mode=0)
+    torch.cuda.synchronize()
+    assert r["ws"].status()[0] == "CLSA_OK"
+    assert torch.equal(o0, r["O"]) and torch.equal(l0, r["lse"])  # mode 0 is the chunk's own attention
+    i_np, c_np = r["idx"].cpu().numpy(), r["count"].cpu().numpy()
+    rows = rows or list(range(w.T))
+    want, want_lse = O.prefill_attention(inp.Q, inp.K, inp.V, i_np[rows], c_np[rows], rows)
+    assert max_abs(tensor_f64(o1)[:, rows], want) <= TOL[w.dtype]
+    got_lse = tensor_f64(l1)[:, rows]
+    assert max_abs(got_lse, want_lse) <= LSE_TOL[w.dtype] * (1 + np.abs(want_lse).max())
+    assert max_abs(tensor_f64(o1), tensor_f64(o0)) <= TOL[w.dtype]  # every row
+
+
 # ----------------------------------------------------------------------- fused vs four-kernel plan
 
 def _decode(dv, w, plan, monkeypatch, **kw):
