@@ -366,6 +366,15 @@ def test_prefill_layer_groups():
     _prefill_check(w, list(range(0, 200, 7)) + [199])
 
 
+@pytest.mark.parametrize("kw", [dict(L=2, Hq=8, Hkv=2),     # 8 rows per KV head: the few-rows kernel
+                                dict(L=6, Hq=16, Hkv=4)])   # 24 rows per KV head: the mma.sync kernel
+def test_prefill_head_dim_64(kw):
+    """d = 64 (the tensor-core attention takes d = 128 only): prefill rows through the
+    other attention kernels, gathering from the one shared cache."""
+    w = scaled("prefill4k", n_max=2000, T=150, k=200, d=64, **kw)
+    _prefill_check(w, list(range(0, 150, 3)) + [149])
+
+
 def test_prefill_full_size_sampled():
     w = WORKLOADS["prefill4k"]
     _prefill_check(w, [0, 1, 2047, 2048, 4095])
