@@ -107,7 +107,8 @@ def profile_traffic(kernel: str, workload: str, src_files):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi streaming its clocks every 100 ms while the timed region runs."""
+    """nvidia-smi streaming its clocks every 25 ms while the timed region runs (started half a
+    second ahead, so that the stream is flowing when the region starts)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -127,11 +128,11 @@ class ClockSampler:
     def __enter__(self):
         try:
             self._p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                        "--format=csv,noheader,nounits", "-lms", "100"],
+                                        "--format=csv,noheader,nounits", "-lms", "25"],
                                        stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
-            time.sleep(0.3)
+            time.sleep(0.5)
         except Exception:
             self._p = None
         return self
