@@ -100,7 +100,7 @@ struct FusedParams {
   uint32_t* leave;     // CTAs of this launch past their last count barrier
   uint32_t* cand_key;  // [B][kCandCap]  candidate keys, the group's windows back to back (0 = empty slot)
   int32_t* cand_tok;   // [B][kCandCap]
-  float* Op;           // [gridDim][rows][D]  split partials, one slot per CTA
+  __nv_bfloat16* Op;   // [gridDim][rows][D]  split partials (unnormalised), one slot per CTA
   float* Ml;           // [gridDim][rows][2]
   void* ws_header;
   unsigned long long* trace;  // [gridDim][16] globaltimer stamps per phase, or null
@@ -1028,10 +1028,10 @@ __device__ bool select_windows(const FusedParams& p, Smem& sm, const uint32_t* r
 // ---------------------------------------------------------------------------
 constexpr uint32_t kQAtom = kMaxRows * 128;          // 16 KiB
 constexpr uint32_t kTmemCols = 256;                  // S at [0, 128), O_c at [128, 256)
-constexpr int kOPitch = kD + 4;                      // staged partial row, floats
+constexpr int kOPitch = kD + 8;                      // staged partial row, bf16 (272 bytes)
 constexpr uint32_t kIdescPV = tc::idesc_bf16_f32(kMaxRows, kD) | (1u << 16);  // B (V) MN-major
 static_assert(2 * kQAtom + 1024 <= kSmemQ, "Q tile exceeds its region");
-static_assert(kMaxRows * kOPitch * 4 + 1024 <= kSmemBig, "partial staging exceeds big");
+static_assert(kMaxRows * kOPitch * 2 + 1024 <= kSmemBig, "partial staging exceeds big");
 
 template <int TOK>
 struct AttnShape {
@@ -1306,20 +1306,23 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
     }
   }
   if (pl.nsplit > 1) {
-    // this CTA's partial rows are one contiguous block of p.Op: stage them in shared
-    // memory (row pitch kOPitch floats: conflict-free 16-byte stores down a column),
-    // then write the block with whole-line stores
-    float* stg = reinterpret_cast<float*>(kv);
-    float4* srow = reinterpret_cast<float4*>(stg + row * kOPitch + 32 * cg);
+    // this CTA's partial rows are one contiguous block of p.Op, in bf16 (the merge sums them
+    // in fp32; a partial's rounding is 2^-9 of its own size): stage them in shared memory
+    // (row pitch kOPitch bf16: conflict-free 16-byte stores down a column), then write the
+    // block with whole-line stores
+    __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(kv);
+    uint4* srow = reinterpret_cast<uint4*>(stg + row * kOPitch + 32 * cg);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) srow[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+    for (int j = 0; j < 4; ++j)
+      srow[j] = make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
+                           pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
     if (cg == 0 && row < p.rows)
       __stcg(reinterpret_cast<float2*>(p.Ml + ((size_t)blockIdx.x * p.rows + row) * 2), make_float2(m, ls));
     __syncthreads();
-    float4* op = reinterpret_cast<float4*>(p.Op + (size_t)blockIdx.x * p.rows * kD);
+    uint4* op = reinterpret_cast<uint4*>(p.Op + (size_t)blockIdx.x * p.rows * kD);
 #pragma unroll 1
-    for (int i = threadIdx.x; i < p.rows * (kD / 4); i += kThreads)
-      __stcg(op + i, *reinterpret_cast<const float4*>(stg + (i / (kD / 4)) * kOPitch + 4 * (i % (kD / 4))));
+    for (int i = threadIdx.x; i < p.rows * (kD / 8); i += kThreads)
+      __stcg(op + i, *reinterpret_cast<const uint4*>(stg + (i / (kD / 8)) * kOPitch + 8 * (i % (kD / 8))));
     // the partial is complete: the CTA's barrier orders every thread's stores before the
     // release that publishes its flag (the row's launch counter + 1)
     __syncthreads();
@@ -1348,8 +1351,8 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
   const size_t cta0 = (size_t)pl.start + (size_t)g * ns;  // CTA holding split 0 of head g
   const uint32_t* flags = p.row_ws + (size_t)pl.b * kRowWords + kRowFlag + (size_t)g * ns;
   const uint32_t tag = sm.row_hdr[kRowEpoch] + 1u;
-  constexpr int kMaxPairs = 224;                          // 112 KiB of staged partial rows
-  float4* stg = reinterpret_cast<float4*>(big);           // [pairs of the batch][32]
+  constexpr int kMaxPairs = 448;                          // 112 KiB of staged partial rows
+  __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(big);  // [pairs of the batch][kD]
   const int sb = max(1, min(ns, kMaxPairs / nr));         // splits per batch
   bool dead = false;
   // (m, l) of every pair first (the flags of all splits), then the first batch's rows
@@ -1368,10 +1371,12 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
     __syncwarp();  // lane 0's acquire orders the warp's loads below
     return __shfl_sync(0xffffffffu, ok, 0) != 0u;
   };
-  auto issue_rows = [&](int s2, int s_lo) {
-    for (int ri = 0; ri < nr; ++ri)
-      cp_async_16(stg + ((s2 - s_lo) * nr + ri) * 32 + lane,
-                  p.Op + ((cta0 + s2) * p.rows + pl.split + ri * ns) * kD + lane * 4, 16);
+  auto issue_rows = [&](int s2, int s_lo) {  // 16 lanes per 256-byte row, two rows at a time
+    for (int e = lane; e < nr * 16; e += 32) {
+      const int ri = e >> 4, q = e & 15;
+      cp_async_16(stg + ((s2 - s_lo) * nr + ri) * kD + q * 8,
+                  p.Op + ((cta0 + s2) * p.rows + pl.split + ri * ns) * kD + q * 8, 16);
+    }
   };
 #pragma unroll 1
   for (int s2 = warp; s2 < ns; s2 += kWarps) {
@@ -1434,11 +1439,14 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
 #pragma unroll 6
         for (int s2 = s_lo; s2 < s_hi; ++s2) {
           const float w = sm.cm[ri * ns + s2];
-          const float4 v = stg[((s2 - s_lo) * nr + ri) * 32 + lane];
-          a.x = fmaf(w, v.x, a.x);
-          a.y = fmaf(w, v.y, a.y);
-          a.z = fmaf(w, v.z, a.z);
-          a.w = fmaf(w, v.w, a.w);
+          const uint2 vv = *reinterpret_cast<const uint2*>(stg + ((s2 - s_lo) * nr + ri) * kD + lane * 4);
+          float v0, v1, v2, v3;
+          unpack_bf16x2(vv.x, v0, v1);
+          unpack_bf16x2(vv.y, v2, v3);
+          a.x = fmaf(w, v0, a.x);
+          a.y = fmaf(w, v1, a.y);
+          a.z = fmaf(w, v2, a.z);
+          a.w = fmaf(w, v3, a.w);
         }
         acc[i] = a;
       }
@@ -1758,7 +1766,7 @@ cudaError_t launch_decode_fused(const clsa_decode_args* a, float scale, void* ws
   w += align_up((size_t)a->B * kCandCap * 4, 256);
   p.cand_tok = reinterpret_cast<int32_t*>(w);
   w += align_up((size_t)a->B * kCandCap * 4, 256);
-  p.Op = reinterpret_cast<float*>(w);
+  p.Op = reinterpret_cast<__nv_bfloat16*>(w);
   w += align_up((size_t)cfg.ncta * p.rows * kD * 4, 256);
   p.Ml = reinterpret_cast<float*>(w);
   const size_t smem = smem_bytes();
