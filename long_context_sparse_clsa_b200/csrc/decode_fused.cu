@@ -101,7 +101,7 @@ struct FusedParams {
   uint32_t* cand_key;  // [B][kCandCap]  candidate keys, the group's windows back to back (0 = empty slot)
   int32_t* cand_tok;   // [B][kCandCap]
   __nv_bfloat16* Op;   // [gridDim][rows][D]  split partials (unnormalised), one slot per CTA
-  float* Ml;           // [gridDim][rows][2]
+  float* Ml;           // [gridDim][rows][4]  (m, l, -, -): one 16-byte slot per row
   void* ws_header;
   unsigned long long* trace;  // [gridDim][16] globaltimer stamps per phase, or null
   int B, n_max, k, L, Hq, Hkv, G, rows, nsplit_max;
@@ -162,7 +162,6 @@ struct Smem {
     };
   };
   float cm[512], cl[512];          // split-combine staging (m, l per row x split)
-  float rowM[kMaxRows], rowD[kMaxRows];  // split-combine: max and denominator per row
 };
 // dynamic shared memory: [Smem][sQ: kMaxRows x kSTR bf16][big: 128 KiB, reused by phase]
 constexpr size_t kSmemQ = (size_t)kMaxRows * kSTR * 2;
@@ -1317,7 +1316,7 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
       srow[j] = make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
                            pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
     if (cg == 0 && row < p.rows)
-      __stcg(reinterpret_cast<float2*>(p.Ml + ((size_t)blockIdx.x * p.rows + row) * 2), make_float2(m, ls));
+      __stcg(reinterpret_cast<float4*>(p.Ml + ((size_t)blockIdx.x * p.rows + row) * 4), make_float4(m, ls, 0.f, 0.f));
     __syncthreads();
     uint4* op = reinterpret_cast<uint4*>(p.Op + (size_t)blockIdx.x * p.rows * kD);
 #pragma unroll 1
@@ -1335,12 +1334,12 @@ __device__ void attend_unit(const FusedParams& p, Smem& sm, unsigned char* sQa, 
 
 // ---------------------------------------------------------------------------
 // phase 5: merge the nsplit partials of head g for rows r = split, split + nsplit, ...
-// Warp w waits for the flag of split w (w + 16, ...) and at once issues the 16-byte copies
-// of that split's partial rows and reads its (m, l) pairs, so the copies of the early
-// splits overlap the wait for the late ones.  Each row's M = max m and den = sum 2^(m - M) l
-// come from all pairs; then one warp per row sums its splits in split order (the same
-// order every call: the result is deterministic).  Splits are staged in batches that fit
-// the staging region (one batch at the workloads' shapes).
+// Warp w waits for the flag of split w (w + 16, ...) and at once issues the async copies
+// of that split's partial rows and (m, l) pairs, then goes on to its next flag, so the
+// copies of the early splits overlap the wait for the late ones.  Then one warp per row
+// takes M = max m and den = sum 2^(m - M) l over the splits and sums the split rows in
+// split order (the same order every call: the result is deterministic).  The code is
+// rolled: it runs once per launch, so its size is instruction fetches on the critical path.
 // ---------------------------------------------------------------------------
 __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big, const Plan pl, int g) {
   stamp(p, 18);
@@ -1351,11 +1350,13 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
   const size_t cta0 = (size_t)pl.start + (size_t)g * ns;  // CTA holding split 0 of head g
   const uint32_t* flags = p.row_ws + (size_t)pl.b * kRowWords + kRowFlag + (size_t)g * ns;
   const uint32_t tag = sm.row_hdr[kRowEpoch] + 1u;
-  constexpr int kMaxPairs = 448;                          // 112 KiB of staged partial rows
-  __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(big);  // [pairs of the batch][kD]
-  const int sb = max(1, min(ns, kMaxPairs / nr));         // splits per batch
+  // Every (row, split) pair of the head is staged at once: nr * ns <= rows + ns - 1.
+  constexpr int kMaxPairs = kMaxRows + kMaxGroups - 1;
+  static_assert(kMaxPairs * kD * 2 + kMaxPairs * 16 <= (int)kSmemBig, "merge staging exceeds big");
+  static_assert(kMaxPairs <= 512, "split weights exceed sm.cm");
+  __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(big);  // [split][row][kD]
+  float4* mls = reinterpret_cast<float4*>(big + (size_t)kMaxPairs * kD * sizeof(__nv_bfloat16));  // [row][split]
   bool dead = false;
-  // (m, l) of every pair first (the flags of all splits), then the first batch's rows
   auto wait_flag = [&](int s2) {  // warp-wide; false on timeout
     uint32_t ok = 1;
     if (lane == 0) {
@@ -1371,105 +1372,68 @@ __device__ void combine_head(const FusedParams& p, Smem& sm, unsigned char* big,
     __syncwarp();  // lane 0's acquire orders the warp's loads below
     return __shfl_sync(0xffffffffu, ok, 0) != 0u;
   };
-  auto issue_rows = [&](int s2, int s_lo) {  // 16 lanes per 256-byte row, two rows at a time
-    for (int e = lane; e < nr * 16; e += 32) {
-      const int ri = e >> 4, q = e & 15;
-      cp_async_16(stg + ((s2 - s_lo) * nr + ri) * kD + q * 8,
-                  p.Op + ((cta0 + s2) * p.rows + pl.split + ri * ns) * kD + q * 8, 16);
-    }
-  };
 #pragma unroll 1
   for (int s2 = warp; s2 < ns; s2 += kWarps) {
     if (!wait_flag(s2)) {
       dead = true;
       continue;
     }
-    // the rows' async copies first: the (m, l) loads below stall the warp until they return
-    if (s2 < sb) issue_rows(s2, 0);
-    for (int ri = lane; ri < nr; ri += 32) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.Ml + ((cta0 + s2) * p.rows + pl.split + ri * ns) * 2));
-      sm.cm[ri * ns + s2] = ml.x;
-      sm.cl[ri * ns + s2] = ml.y;
+    const size_t src_row = (cta0 + s2) * p.rows + pl.split;  // row ri of the split: src_row + ri * ns
+#pragma unroll 1
+    for (int e = lane; e < nr * 16; e += 32) {  // 16 lanes per 256-byte row
+      const int ri = e >> 4, q = e & 15;
+      cp_async_16(stg + (s2 * nr + ri) * kD + q * 8, p.Op + (src_row + (size_t)ri * ns) * kD + q * 8, 16);
     }
+#pragma unroll 1
+    for (int ri = lane; ri < nr; ri += 32) cp_async_16(mls + ri * ns + s2, p.Ml + (src_row + (size_t)ri * ns) * 4, 16);
   }
   cp_async_commit();
+  cp_async_wait<0>();  // no copy outlives an abort below
   if (dead) sm.abort_flag = 1;
   __syncthreads();
   stamp(p, 17);
   if (sm.abort_flag) return;
-  // per row: M, den, and each split's weight 2^(m - M) in place of its m
 #pragma unroll 1
   for (int ri = warp; ri < nr; ri += kWarps) {
     float M = -INFINITY, den = 0.f;
 #pragma unroll 1
-    for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, sm.cm[ri * ns + s2]);
+    for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, mls[ri * ns + s2].x);
     M = warp_max(M);
 #pragma unroll 1
     for (int s2 = lane; s2 < ns; s2 += 32) {
-      const float wgt = M == -INFINITY ? 0.f : exp2f(sm.cm[ri * ns + s2] - M);
-      den = fmaf(wgt, sm.cl[ri * ns + s2], den);
+      const float4 ml = mls[ri * ns + s2];
+      const float wgt = M == -INFINITY ? 0.f : exp2f(ml.x - M);
+      den = fmaf(wgt, ml.y, den);
       sm.cm[ri * ns + s2] = wgt;
     }
     den = warp_sum(den);
-    if (lane == 0) {
-      sm.rowM[ri] = M;
-      sm.rowD[ri] = den;
+    __syncwarp();  // the row's weights are visible to the whole warp
+    // lane: 4 of the 128 columns
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int s2 = 0; s2 < ns; ++s2) {
+      const float w = sm.cm[ri * ns + s2];
+      const uint2 vv = *reinterpret_cast<const uint2*>(stg + (s2 * nr + ri) * kD + lane * 4);
+      float v0, v1, v2, v3;
+      unpack_bf16x2(vv.x, v0, v1);
+      unpack_bf16x2(vv.y, v2, v3);
+      a.x = fmaf(w, v0, a.x);
+      a.y = fmaf(w, v1, a.y);
+      a.z = fmaf(w, v2, a.z);
+      a.w = fmaf(w, v3, a.w);
     }
+    const int r = pl.split + ri * ns;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const int l = r / p.G, h = g * p.G + r % p.G;
+    __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
+    uint2 wv;
+    wv.x = pack_bf16x2(a.x * inv, a.y * inv);
+    wv.y = pack_bf16x2(a.z * inv, a.w * inv);
+    *reinterpret_cast<uint2*>(out) = wv;
+    if (p.lse && lane == 0)
+      p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
   }
-  // one warp per row accumulates its splits in order (lane: 4 of the 128 columns)
-  float4 acc[(kMaxRows + kWarps - 1) / kWarps];
-#pragma unroll
-  for (int i = 0; i < (kMaxRows + kWarps - 1) / kWarps; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-  for (int s_lo = 0; s_lo < ns; s_lo += sb) {
-    const int s_hi = min(ns, s_lo + sb);
-    if (s_lo > 0) {  // later batches: the flags were seen above
-      __syncthreads();  // the previous batch is consumed
-#pragma unroll 1
-      for (int s2 = s_lo + warp; s2 < s_hi; s2 += kWarps) issue_rows(s2, s_lo);
-      cp_async_commit();
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < (kMaxRows + kWarps - 1) / kWarps; ++i) {
-      const int ri = warp + i * kWarps;
-      if (ri < nr) {
-        float4 a = acc[i];
-#pragma unroll 6
-        for (int s2 = s_lo; s2 < s_hi; ++s2) {
-          const float w = sm.cm[ri * ns + s2];
-          const uint2 vv = *reinterpret_cast<const uint2*>(stg + ((s2 - s_lo) * nr + ri) * kD + lane * 4);
-          float v0, v1, v2, v3;
-          unpack_bf16x2(vv.x, v0, v1);
-          unpack_bf16x2(vv.y, v2, v3);
-          a.x = fmaf(w, v0, a.x);
-          a.y = fmaf(w, v1, a.y);
-          a.z = fmaf(w, v2, a.z);
-          a.w = fmaf(w, v3, a.w);
-        }
-        acc[i] = a;
-      }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < (kMaxRows + kWarps - 1) / kWarps; ++i) {
-    const int ri = warp + i * kWarps;
-    if (ri < nr) {
-      const int r = pl.split + ri * ns;
-      const float den = sm.rowD[ri], M = sm.rowM[ri];
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-      const float4 a = acc[i];
-      const int l = r / p.G, h = g * p.G + r % p.G;
-      __nv_bfloat16* out = p.O + (((size_t)l * p.B + pl.b) * p.Hq + h) * kD + lane * 4;
-      uint2 wv;
-      wv.x = pack_bf16x2(a.x * inv, a.y * inv);
-      wv.y = pack_bf16x2(a.z * inv, a.w * inv);
-      *reinterpret_cast<uint2*>(out) = wv;
-      if (p.lse && lane == 0)
-        p.lse[((size_t)l * p.B + pl.b) * p.Hq + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
-    }
-  }
+  stamp(p, 46);
 }
 
 // ---------------------------------------------------------------------------
@@ -1679,7 +1643,7 @@ size_t fused_decode_ws_bytes(const clsa_decode_args* a) {
   off += align_up(((size_t)a->B * kRowWords + 1) * 4, 256);    // row state, leave count
   off += 2 * align_up((size_t)a->B * kCandCap * 4, 256);  // candidate windows
   off += align_up((size_t)cfg.ncta * rows * kD * 4, 256);      // split partials
-  off += align_up((size_t)cfg.ncta * rows * 2 * 4, 256);
+  off += align_up((size_t)cfg.ncta * rows * 4 * 4, 256);     // split (m, l), 16-byte slots
   return off;
 }
 
