@@ -34,7 +34,7 @@
 //     are all L*G (layer, query head) pairs of head g, so every selected K/V row is
 //     read once for all layers.  tcgen05.mma bf16 -> fp32 in TMEM over 64-token
 //     chunks (S = Q K^T, then P V with V as an MN-major operand), online softmax in
-//     exp2 with the output accumulated in registers.
+//     exp2 with the output accumulated in TMEM (rescaled only when the max jumps).
 //  5. Each split publishes its partial with a flag; the splits of one head merge each
 //     other's partials (log-sum-exp rule) as their flags appear.
 //
@@ -1019,7 +1019,7 @@ __device__ bool select_windows(const FusedParams& p, Smem& sm, const uint32_t* r
 //   O_c = P_c V_c      P_c (bf16) in shared memory (A, K-major), V_c as the MN-major B
 //                      operand straight from its row-major [token][d] tile;
 //                      M128 N128 (K = TOK tokens) -> TMEM columns [128, 256)
-//   o = o 2^(m_old - m) + O_c   in registers, 32 of the d columns per thread
+//   O += P_c V_c in TMEM; O and l are rescaled by 2^(m_old - m) only when m jumps
 // The S MMAs of chunk c + 1 are issued right behind the P V MMAs of chunk c (S is
 // double-buffered in TMEM).  K/V chunks are gathered by 16-byte async copies into the
 // 128-byte-swizzle layout, two chunks ahead.  Each tcgen05.mma costs tens of cycles to
