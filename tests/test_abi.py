@@ -103,6 +103,58 @@ def test_prefill_attention_rejects_bad_args(lib):
     assert lib.clsa_prefill_attention(ctypes.byref(a), 0, p, 1 << 30, NULL) == 1
 
 
+def test_gather_kv_rejects_bad_args(lib):
+    p, q = ctypes.c_void_p(16), ctypes.c_void_p(18)
+    ws = ctypes.c_void_p(256)
+    ok = [p, p, p, p, 1, 64, 8, 2, 128, 1, p, p, ws, 1 << 20, NULL]
+
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.clsa_gather_kv(*a)
+    assert call(a0=NULL) == 1                  # no K
+    assert call(a4=0) == 1                     # B = 0
+    assert call(a9=7) == 1                     # no such dtype
+    assert call(a8=96) == 2                    # d not 64 / 128
+    assert call(a6=5000) == 2                  # k above 4096
+    assert call(a0=q) == 1                     # K not 16-byte aligned
+    assert call(a2=ctypes.c_void_p(18)) == 1   # idx not 4-byte aligned
+    assert call(a12=NULL) == 3                 # no workspace
+    assert call(a13=8) == 3                    # workspace below its header
+
+
+@pytest.mark.parametrize("name", ["clsa_distill_target", "clsa_attention_mass"])
+def test_distill_and_mass_reject_bad_args(lib, name):
+    p, q = ctypes.c_void_p(16), ctypes.c_void_p(18)
+    ws = ctypes.c_void_p(256)
+    # Q, K, scores | lse_sparse, seq_lens, B, n_max, L, Hq, Hkv, d, scale, dt, out, out2, ws, ws_bytes, stream
+    ok = [p, p, p, p, 1, 1024, 2, 8, 2, 128, 0.0, 1, p, p, ws, 1 << 30, NULL]
+    fn = getattr(lib, name)
+
+    def call(**kw):
+        a = list(ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return fn(*a)
+    assert call(a4=0) == 1                     # B = 0
+    assert call(a11=7) == 1                    # no such dtype
+    assert call(a8=3) == 2                     # Hq not a multiple of Hkv
+    assert call(a9=80) == 2                    # d not 64 / 128
+    assert call(a0=NULL) == 1                  # no Q
+    assert call(a1=q) == 1                     # K not 16-byte aligned
+    assert call(a3=ctypes.c_void_p(18)) == 1   # seq_lens not 4-byte aligned
+
+
+def test_topk_noalloc_rejects_bad_args(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.clsa_topk_noalloc(NULL, p, 1, 16, 4, p, p, NULL) == 1                  # no scores
+    assert lib.clsa_topk_noalloc(p, p, 1, 16, 0, p, p, NULL) == 1                     # k = 0
+    assert lib.clsa_topk_noalloc(p, p, 0, 16, 4, p, p, NULL) == 1                     # B = 0
+    assert lib.clsa_topk_noalloc(p, p, 1, 16, 5000, p, p, NULL) == 2                  # k above 4096
+    assert lib.clsa_topk_noalloc(p, p, 1, 16, 4, ctypes.c_void_p(18), p, NULL) == 1   # idx misaligned
+
+
 def test_oracle_is_not_imported_by_the_product():
     pkg = os.path.join(ROOT, "long_context_sparse_clsa_b200")
     for dirpath, _, files in os.walk(pkg):
