@@ -839,7 +839,7 @@ __device__ bool select_windows(const FusedParams& p, Smem& sm, const uint32_t* r
   const uint32_t epoch = sm.row_hdr[kRowEpoch];
   const uint32_t* h16 = rw + kRowH16 + (epoch & 1u) * kH16Bins;
   const uint32_t* rng = rw + kRowRange + (epoch & 3u) * 4;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     sm.sel_ok = 0;
     sm.list_n = 0;
