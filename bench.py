@@ -41,9 +41,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "CLSA decode step µs & tokens/s at 128K ctx; achieved HBM GB/s vs roofline"
 UNIT = "tokens/s"
+DATA = "synthetic (seeded N(0,1), 1% planted index keys)"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
@@ -59,7 +60,7 @@ def parse():
                     help="a comparison system built from the library's calls (one GPU; not the default line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-steps", type=int, default=2)
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ------------------------------------------------------------------ algorithmic bytes
@@ -197,26 +198,95 @@ def time_oracle(inp, w, steps: int):
     return dt, cores, dt1, f"{steps} full decode step(s) of {w.name} (B={w.B}, n={w.n_max}); single-thread: 1 step"
 
 
+# ------------------------------------------------------------------ the decode line's config
+
+def kidx_nbytes(w) -> int:
+    return w.B * w.n_max * w.d_idx * w.elem_bytes
+
+
+def rotation_sets(args, kidx_bytes: int) -> int:
+    """Input sets rotated through between steps: with --l2 rotate at least two, and at least
+    twice L2 in K_idx alone; one set with --l2 flush."""
+    if args.l2 != "rotate":
+        return 1
+    return max(2, min(max(1, args.sets), 16), int(np.ceil(2 * 126e6 / kidx_bytes)))
+
+
+def decode_config(w, args, world: int, graphs_ok: bool, kb: int = 0) -> dict:
+    """The ``config`` of the decode line (kb: bytes of one K_idx set, by default from the
+    workload's shape); the reference arm prints the same one."""
+    kb = kb or kidx_nbytes(w)
+    R = rotation_sets(args, kb)
+    return {"workload": w.name, "B": w.B, "n": w.n_max, "d_idx": w.d_idx, "k": w.k, "L": w.L,
+            "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "parallelism": f"replicas x{world}",
+            "l2": (f"inputs larger than L2: {R} rotating K_idx sets ({R * kb / 2**20:.0f} MiB, row "
+                   f"permutations of the seeded cache), step i uses set i % {R}; no flush"
+                   if args.l2 == "rotate" else
+                   "flushed before every step (512 MiB write + read-back, outside the timed events)"),
+            "launch": (f"cuda graph ({R} steps per graph, one per input set)" if graphs_ok and
+                       args.l2 == "rotate" else "cuda graph" if graphs_ok else "eager")}
+
+
 # ------------------------------------------------------------------ main paths
 
 def run_reference(args):
+    """The oracle on the host cores, on the decode line's metric, unit and config: W warm-up
+    and exactly K timed steps, each a bounded sample of one decode step.  Step i runs the
+    routing in full (scores over the whole cache, then the TopK) and the attention of KV head
+    g = i mod Hkv (its G query heads in every layer, the oracle given that head's slice of
+    the cache); the attention time is scaled by Hkv, the heads being alike in shape and work."""
     from long_context_sparse_clsa_b200 import replicas
     rank, world, _ = replicas.env_ranks()
     if rank != 0:  # rank 0 alone times the oracle; the other ranks exit without work
         return
     from long_context_sparse_clsa_b200.inputs import WORKLOADS, make_inputs
-    w = WORKLOADS[args.workload]
+    from oracle import clsa_oracle as O
+    if args.workload.startswith("prefill"):
+        raise SystemExit("--impl reference times the decode workloads")
+    w = replicas.rank_workload(WORKLOADS[args.workload], 0, world)
     inp = make_inputs(w)
-    steps = max(1, min(args.steps, args.cpu_sample_steps))
-    dt, threads, dt1, note = time_oracle(inp, w, steps)
+    # the cache is upcast once (state a real decoder keeps resident)
+    qf = inp.f32("q_idx").astype(np.float64)
+    kf = inp.f32("k_idx").astype(np.float64)
+    Kf = inp.f32("K").astype(np.float64)
+    Vf = inp.f32("V").astype(np.float64)
+    Qf = inp.f32("Q").astype(np.float64)
+    cores = len(os.sched_getaffinity(0))
+    warmup = max(args.warmup, 3)
+    G = w.Hq // w.Hkv
+
+    def sample(i: int):
+        g = i % w.Hkv
+        t0 = time.perf_counter()
+        I = O.index_scores(qf, kf, inp.seq_lens)
+        idx, count = O.topk_select(I, inp.seq_lens, w.k)
+        t1 = time.perf_counter()
+        O.sparse_attention(Qf[:, :, g * G:(g + 1) * G], Kf[:, :, g:g + 1], Vf[:, :, g:g + 1], idx, count)
+        return t1 - t0, time.perf_counter() - t1
+
+    import contextlib
+    with contextlib.ExitStack() as stack:
+        try:
+            from threadpoolctl import threadpool_limits
+            stack.enter_context(threadpool_limits(limits=cores))
+        except Exception:  # no control over the BLAS pool: it runs as it stands
+            pass
+        for i in range(warmup):
+            sample(i)
+        route = attn = 0.0
+        for i in range(args.steps):
+            a, b = sample(warmup + i)
+            route += a
+            attn += b
+    dt = (route + attn * w.Hkv) / args.steps
     v = w.B / dt
-    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
-            "warmup": min(args.warmup, 1), "ms_per_step": dt * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "n": w.n_max, "k": w.k, "L": w.L, "Hq": w.Hq,
-                       "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": note,
-                             "single_thread_value": (w.B / dt1) if dt1 else None},
+    note = (f"each step: the routing of {w.name} (B={w.B}, n={w.n_max}) in full and the attention of one "
+            f"of its {w.Hkv} KV heads in turn (all {w.L} layers), scaled by {w.Hkv}")
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": warmup, "ms_per_step": dt * 1e3, "us_per_step": dt * 1e6, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA, "impl": "reference",
+            "config": decode_config(w, args, world, graphs_ok=not args.no_graph),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": note},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -264,9 +334,7 @@ def run_clsa(args):
     # and K/V rows from HBM while the kernel code stays cached; with --l2 flush, one set
     # and a 512 MiB write + read-back before every step.
     kidx_bytes = dv["k_idx"].numel() * dv["k_idx"].element_size()
-    R = 1
-    if args.l2 == "rotate":  # at least two sets, and at least twice L2 in K_idx alone
-        R = max(2, min(max(1, args.sets), 16), int(np.ceil(2 * 126e6 / kidx_bytes)))
+    R = rotation_sets(args, kidx_bytes)
     gen = torch.Generator(device="cpu").manual_seed(1234 + rank)
     kidx_sets = [dv["k_idx"]]
     for r in range(1, R):
@@ -578,15 +646,8 @@ def run_clsa(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-        "data": "synthetic (seeded N(0,1), 1% planted index keys)",
-        "config": {"workload": w.name, "B": w.B, "n": w.n_max, "d_idx": w.d_idx, "k": w.k, "L": w.L,
-                   "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "parallelism": f"replicas x{world}",
-                   "l2": (f"inputs larger than L2: {R} rotating K_idx sets ({R * kidx_bytes / 2**20:.0f} MiB, row "
-                          f"permutations of the seeded cache), step i uses set i % {R}; no flush"
-                          if args.l2 == "rotate" else
-                          "flushed before every step (512 MiB write + read-back, outside the timed events)"),
-                   "launch": (f"cuda graph ({R} steps per graph, one per input set)" if graphs is not None and
-                              args.l2 == "rotate" else "cuda graph" if graphs is not None else "eager")},
+        "data": DATA,
+        "config": decode_config(w, args, world, graphs_ok=graphs is not None, kb=kidx_bytes),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": dom_bytes, "us_per_launch": dom_us},

@@ -5,7 +5,6 @@ arm's rule that only rank 0 times the oracle."""
 import io
 import os
 import socket
-import types
 from contextlib import redirect_stdout
 
 import numpy as np
@@ -75,8 +74,27 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     import bench
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("WORLD_SIZE", "2")
-    args = types.SimpleNamespace(workload="tiny", steps=1, warmup=0, gpus=2, cpu_sample_steps=1)
+    args = bench.parse(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--gpus", "2"])
     out = io.StringIO()
     with redirect_stdout(out):
         assert bench.run_reference(args) is None
     assert out.getvalue() == ""
+
+
+def test_reference_arm_line_matches_the_decode_line():
+    """The reference arm times exactly K steps after W warm-up steps and reports the decode
+    line's metric, unit, direction and config."""
+    import json
+    import bench
+    args = bench.parse(["--impl", "reference", "--workload", "tiny", "--steps", "4", "--warmup", "3"])
+    out = io.StringIO()
+    with redirect_stdout(out):
+        bench.run_reference(args)
+    line = json.loads(out.getvalue())
+    w = WORKLOADS["tiny"]
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["higher_is_better"] is True and line["data"] == bench.DATA
+    assert line["steps"] == 4 and line["warmup"] == 3
+    assert line["config"] == bench.decode_config(w, args, 1, graphs_ok=True)
+    assert line["value"] > 0 and line["value"] == pytest.approx(w.B / (line["ms_per_step"] * 1e-3))
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
