@@ -206,10 +206,16 @@ def kidx_nbytes(w) -> int:
 
 def rotation_sets(args, kidx_bytes: int) -> int:
     """Input sets rotated through between steps: with --l2 rotate at least two, and at least
-    twice L2 in K_idx alone; one set with --l2 flush."""
+    twice L2 in K_idx alone; one set with --l2 flush.  Above that minimum, the smallest count
+    (up to 32) that divides K: the timed steps are then whole replays of the R-step graph,
+    with no single-step graphs at the end (each graph launch restarts the launch pipeline)."""
     if args.l2 != "rotate":
         return 1
-    return max(2, min(max(1, args.sets), 16), int(np.ceil(2 * 126e6 / kidx_bytes)))
+    r_min = max(2, min(max(1, args.sets), 16), int(np.ceil(2 * 126e6 / kidx_bytes)))
+    for r in range(r_min, max(r_min, 32) + 1):
+        if args.steps % r == 0:
+            return r
+    return r_min
 
 
 def decode_config(w, args, world: int, graphs_ok: bool, kb: int = 0) -> dict:

@@ -98,3 +98,14 @@ def test_reference_arm_line_matches_the_decode_line():
     assert line["config"] == bench.decode_config(w, args, 1, graphs_ok=True)
     assert line["value"] > 0 and line["value"] == pytest.approx(w.B / (line["ms_per_step"] * 1e-3))
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_rotation_sets_divide_the_timed_steps():
+    import bench
+    kb = WORKLOADS["decode128k"].B * WORKLOADS["decode128k"].n_max * 128 * 2   # 32 MiB: at least 8 sets
+    for steps, want in [(1000, 8), (20, 10), (50, 10), (200, 8), (7, 8), (31, 31), (37, 8)]:
+        assert bench.rotation_sets(bench.parse(["--steps", str(steps)]), kb) == want, steps
+    assert bench.rotation_sets(bench.parse(["--steps", "20", "--l2", "flush"]), kb) == 1
+    big = 64 << 20                                                              # the --sets minimum, 6
+    for steps, want in [(20, 10), (1000, 8), (12, 6), (5, 6)]:
+        assert bench.rotation_sets(bench.parse(["--steps", str(steps)]), big) == want, steps
