@@ -80,32 +80,3 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
         assert bench.run_reference(args) is None
     assert out.getvalue() == ""
 
-
-def test_reference_arm_line_matches_the_decode_line():
-    """The reference arm times exactly K steps after W warm-up steps and reports the decode
-    line's metric, unit, direction and config."""
-    import json
-    import bench
-    args = bench.parse(["--impl", "reference", "--workload", "tiny", "--steps", "4", "--warmup", "3"])
-    out = io.StringIO()
-    with redirect_stdout(out):
-        bench.run_reference(args)
-    line = json.loads(out.getvalue())
-    w = WORKLOADS["tiny"]
-    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
-    assert line["higher_is_better"] is True and line["data"] == bench.DATA
-    assert line["steps"] == 4 and line["warmup"] == 3
-    assert line["config"] == bench.decode_config(w, args, 1, graphs_ok=True)
-    assert line["value"] > 0 and line["value"] == pytest.approx(w.B / (line["ms_per_step"] * 1e-3))
-    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
-
-
-def test_rotation_sets_divide_the_timed_steps():
-    import bench
-    kb = WORKLOADS["decode128k"].B * WORKLOADS["decode128k"].n_max * 128 * 2   # 32 MiB: at least 8 sets
-    for steps, want in [(1000, 8), (20, 10), (50, 10), (200, 8), (7, 8), (31, 31), (37, 8)]:
-        assert bench.rotation_sets(bench.parse(["--steps", str(steps)]), kb) == want, steps
-    assert bench.rotation_sets(bench.parse(["--steps", "20", "--l2", "flush"]), kb) == 1
-    big = 64 << 20                                                              # the --sets minimum, 6
-    for steps, want in [(20, 10), (1000, 8), (12, 6), (5, 6)]:
-        assert bench.rotation_sets(bench.parse(["--steps", str(steps)]), big) == want, steps
