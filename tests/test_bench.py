@@ -59,3 +59,20 @@ def test_committed_profiles_match_the_kernel_sources():
         assert t is not None and t > 0, wl
     scan = ["long_context_sparse_clsa_b200/csrc/index_scores.cu", "long_context_sparse_clsa_b200/csrc/common.cuh"]
     assert bench.profile_traffic("index_scores_kernel", "decode128k", scan) is not None
+
+
+def test_profile_summaries_are_short_text_with_their_commands():
+    """Every summary under profiles/ is a few KB of text that gives the ncu command behind it,
+    and every ncu command there leaves the clocks alone."""
+    import os
+    import re
+    root = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles")
+    names = sorted(os.listdir(root))
+    assert names and all(n.endswith((".txt", ".md")) for n in names)
+    for n in names:
+        text = open(os.path.join(root, n)).read()
+        assert len(text.encode()) < 16384, n
+        cmds = [m.group(0) for m in re.finditer(r"ncu (?:\\\n#?|[^\n])*", text) if "--" in m.group(0)]
+        assert cmds, n
+        for c in cmds:
+            assert "--clock-control none" in c, (n, c)
